@@ -1,0 +1,265 @@
+"""FP64 CPU oracle for LUT-GEMM over binary-coding-quantised (BCQ) weights.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import or call this module.  The product
+path (the CUDA library and its Python binding) never imports it, and this
+module imports nothing from the product: the two share no code.  Inputs come
+from ``bcq_synth`` (random draws only).
+
+What it computes, and where the pages say so
+--------------------------------------------
+Source pages: "LUT-GEMM -- paper by Park et al. (2022), ICLR 2024" (Elamur
+card; sections *Summary*, *Interesting ideas*) and the pith.science card of the
+same paper (abstract).
+
+* BCQ format (Summary; Interesting ideas, "Lookup tables instead of
+  multiplications"): a weight row is a sum of q binary {-1,+1} vectors, each
+  with a scale.  Scales are group-wise (Summary; "Group size as a separate
+  hyper-parameter"): W[j,k] = sum_i alpha[i, k//g, j] * beta[i, j, k].
+* Uniform quantisation is a special case of BCQ (Summary; "One format for many
+  schemes").  The pages give no formula; the closed form used here is derived in
+  ``uniform_to_bcq``.  It needs a per-group offset term (off[k//g, j]).
+* The product y = W x is what LUT-GEMM returns "with no dequantization"
+  (Summary): the lookup form is an exact regrouping of this sum, so the oracle's
+  reference result is the plain dequantise-then-matmul in FP64
+  (``bcq_matmul``).  ``lut_matmul`` writes the lookup regrouping out plainly so
+  the identity itself can be pinned.
+* Lookup table (Interesting ideas): for a run of mu = 8 activations, the 256
+  possible signed sums are computed once; T[p] = sum_t (2*bit_t(p) - 1) * x_t.
+
+Readings where the pages are silent (each also listed in the design notes):
+
+* bit t of a table index / packed byte stands for activation 8c + t (LSB
+  first); bit value 1 means beta = +1.
+* plane i (0-based) of a converted uniform weight is bit i of the integer code.
+* the packed weight layout is this library's own tiled layout; it is defined
+  in ``include/lutgemm.h`` and re-implemented here from that text
+  (``pack_bcq`` / ``unpack_bcq``).
+
+Parity status: every public function here is pinned by
+``tests/test_oracle_pins.py`` against brute force, closed forms, special cases
+or hand-derived fixtures (tests/golden).  None is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+MU = 8            # activations per lookup-table run (256-entry tables)
+SLICE = 1024      # inputs per slice of the packed layout
+TILE_ROWS = 32    # rows per row tile of the packed layout
+PIECE = 128       # inputs per 16-byte lane piece of the packed layout
+BLOCK_BYTES = 4096
+
+__all__ = [
+    "lut_table", "dequantize_bcq", "bcq_matmul", "lut_matmul",
+    "packed_nbytes", "pack_bcq", "unpack_bcq", "unpack_rows",
+    "uniform_to_bcq", "uniform_dequant", "bcq_matmul_rows",
+]
+
+
+# ---------------------------------------------------------------------------
+# Lookup table (Interesting ideas: "the possible sums of activation
+# sub-vectors can be computed once and then simply looked up").
+# ---------------------------------------------------------------------------
+def lut_table(xchunk) -> np.ndarray:
+    """All 256 signed sums of one run of 8 activations, in FP64.
+
+    T[p] = sum_{t=0..7} (2*bit_t(p) - 1) * x[t], bit t of p being (p >> t) & 1.
+    """
+    x = np.asarray(xchunk, dtype=np.float64).reshape(MU)
+    p = np.arange(256)
+    bits = (p[:, None] >> np.arange(MU)[None, :]) & 1          # [256, 8]
+    signs = 2.0 * bits.astype(np.float64) - 1.0
+    return signs @ x
+
+
+# ---------------------------------------------------------------------------
+# BCQ dequantisation and the plain product (Summary; Interesting ideas).
+# ---------------------------------------------------------------------------
+def dequantize_bcq(signs, alpha, g: int, offset=None) -> np.ndarray:
+    """W[j,k] = sum_i alpha[i, k//g, j] * signs[i, j, k] (+ offset[k//g, j]), FP64 [m][n].
+
+    signs: [q][m][n] of -1/+1; alpha: [q][n/g][m] (fp16 or wider);
+    offset: [n/g][m] or None (pure BCQ).
+    """
+    s = np.asarray(signs)
+    q, m, n = s.shape
+    a = np.asarray(alpha, dtype=np.float64)
+    assert a.shape == (q, n // g, m), (a.shape, (q, n // g, m))
+    W = np.zeros((m, n), dtype=np.float64)
+    for i in range(q):
+        a_rows = np.repeat(a[i], g, axis=0).T          # [m][n]: alpha of (row, input)
+        W += a_rows * s[i].astype(np.float64)
+    if offset is not None:
+        o = np.asarray(offset, dtype=np.float64)
+        assert o.shape == (n // g, m)
+        W += np.repeat(o, g, axis=0).T
+    return W
+
+
+def bcq_matmul(x, signs, alpha, g: int, offset=None) -> np.ndarray:
+    """y[b, j] = sum_k W[j, k] * x[b, k] with W from ``dequantize_bcq``; FP64 [batch][m]."""
+    W = dequantize_bcq(signs, alpha, g, offset)
+    xx = np.asarray(x, dtype=np.float64)
+    return xx @ W.T
+
+
+def bcq_matmul_rows(x, signs_rows, alpha_rows, g: int, offset_rows=None) -> np.ndarray:
+    """``bcq_matmul`` restricted to a subset of output rows.
+
+    signs_rows: [q][r][n]; alpha_rows: [q][n/g][r]; offset_rows: [n/g][r] or None.
+    Returns [batch][r].  Used to check sampled outputs of large problems.
+    """
+    return bcq_matmul(x, signs_rows, alpha_rows, g, offset_rows)
+
+
+def lut_matmul(x, signs, alpha, g: int, offset=None) -> np.ndarray:
+    """The lookup-table regrouping of ``bcq_matmul``, written out plainly (FP64).
+
+    For every batch column b and run c of 8 inputs, the 256-entry table
+    T = lut_table(x[b, 8c:8c+8]) is built once; each plane-row then reads one
+    entry, indexed by the byte of its 8 sign bits (bit t = 1 iff sign = +1),
+    and scales it by the alpha of the run's group.  The offset of a converted
+    uniform weight multiplies the group's activation sum.  Requires g % 8 == 0.
+    """
+    s = np.asarray(signs)
+    q, m, n = s.shape
+    assert n % MU == 0 and g % MU == 0 and n % g == 0
+    a = np.asarray(alpha, dtype=np.float64)
+    xx = np.asarray(x, dtype=np.float64)
+    batch = xx.shape[0]
+    weights = (1 << np.arange(MU)).astype(np.int64)
+    y = np.zeros((batch, m), dtype=np.float64)
+    for b in range(batch):
+        for c in range(n // MU):
+            T = lut_table(xx[b, MU * c: MU * c + MU])
+            G = (MU * c) // g
+            for i in range(q):
+                bits = (s[i, :, MU * c: MU * c + MU] > 0).astype(np.int64)   # [m][8]
+                idx = bits @ weights                                           # [m]
+                y[b] += a[i, G, :] * T[idx]
+        if offset is not None:
+            o = np.asarray(offset, dtype=np.float64)
+            for G in range(n // g):
+                y[b] += o[G, :] * xx[b, G * g:(G + 1) * g].sum()
+    return y
+
+
+# ---------------------------------------------------------------------------
+# Packed layout (library-defined; re-implemented from the header's text).
+#
+#   n_s = ceil(n / 1024) slices, m_t = ceil(m / 32) row tiles.
+#   The buffer is n_s * m_t * q blocks of 4096 bytes; block (s, R, i) starts at
+#   byte ((s * m_t + R) * q + i) * 4096.
+#   In that block, byte U*512 + l*16 + j (U < 8, l < 32, j < 16) holds the
+#   8 sign bits of row r = 32*R + l, plane i, inputs
+#   k = 1024*s + 128*P + 8*c + t (bit t, LSB first), where
+#   P = U xor (4 * (l // 16)) and c = j xor (l % 16).
+#   A bit is 1 iff the sign is +1; bits of rows >= m or inputs >= n are 0.
+# ---------------------------------------------------------------------------
+def packed_nbytes(q: int, m: int, n: int) -> int:
+    return math.ceil(n / SLICE) * math.ceil(m / TILE_ROWS) * q * BLOCK_BYTES
+
+
+def _piece_and_run(U: int, l: int, j: int):
+    """(P, c): which 128-input piece and which 8-input run byte (U, l, j) holds."""
+    return U ^ (4 * (l // 16)), j ^ (l % 16)
+
+
+def pack_bcq(signs) -> np.ndarray:
+    """int8 signs [q][m][n] (-1/+1) -> packed uint8 buffer of ``packed_nbytes`` bytes."""
+    s = np.asarray(signs)
+    q, m, n = s.shape
+    if not np.all((s == 1) | (s == -1)):
+        raise ValueError("signs must be -1 or +1")
+    ns, mt = math.ceil(n / SLICE), math.ceil(m / TILE_ROWS)
+    bits = np.zeros((q, mt * TILE_ROWS, ns * SLICE), dtype=np.uint8)
+    bits[:, :m, :n] = (s > 0)
+    # bits_r[i, R, l, s, k_in_slice]
+    bits_r = bits.reshape(q, mt, TILE_ROWS, ns, SLICE)
+    out = np.zeros((ns, mt, q, 8, TILE_ROWS, 16), dtype=np.uint8)
+    for U in range(8):
+        for l in range(TILE_ROWS):
+            for j in range(16):
+                P, c = _piece_and_run(U, l, j)
+                k0 = PIECE * P + MU * c
+                byte = np.zeros((q, mt, ns), dtype=np.uint8)
+                for t in range(MU):
+                    byte |= (bits_r[:, :, l, :, k0 + t] << t).astype(np.uint8)
+                out[:, :, :, U, l, j] = byte.transpose(2, 1, 0)
+    return out.reshape(-1)
+
+
+def unpack_bcq(packed, q: int, m: int, n: int) -> np.ndarray:
+    """Inverse of ``pack_bcq``: packed bytes -> int8 signs [q][m][n]."""
+    return unpack_rows(packed, q, m, n, np.arange(m))
+
+
+def unpack_rows(packed, q: int, m: int, n: int, rows) -> np.ndarray:
+    """Signs [q][len(rows)][n] of the given output rows, read from a packed buffer."""
+    pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    assert pk.size == packed_nbytes(q, m, n)
+    ns, mt = math.ceil(n / SLICE), math.ceil(m / TILE_ROWS)
+    blocks = pk.reshape(ns, mt, q, 8, TILE_ROWS, 16)
+    rows = np.asarray(rows, dtype=np.int64)
+    out_bits = np.zeros((q, rows.size, ns * SLICE), dtype=np.uint8)
+    for ri, r in enumerate(rows):
+        R, l = divmod(int(r), TILE_ROWS)
+        for U in range(8):
+            for j in range(16):
+                P, c = _piece_and_run(U, l, j)
+                k0 = PIECE * P + MU * c
+                byte = blocks[:, R, :, U, l, j]          # [ns][q]
+                for t in range(MU):
+                    bit = (byte >> t) & 1                 # [ns][q]
+                    out_bits[:, ri, np.arange(ns) * SLICE + k0 + t] = bit.T
+    bits = out_bits[:, :, :n]
+    return (bits.astype(np.int8) * 2 - 1)
+
+
+# ---------------------------------------------------------------------------
+# Uniform quantisation rewritten as BCQ (Summary; Interesting ideas, "One
+# format for many schemes").  The pages state that the rewrite exists but give
+# no formula.  Derivation used here:
+#   w = s * (c - z), c = sum_{i=0}^{q-1} 2^i * b_i with b_i in {0,1}.
+#   With beta_i = 2*b_i - 1:  b_i = (beta_i + 1)/2, so
+#   c = sum_i 2^(i-1) * beta_i + (2^q - 1)/2.
+#   Hence w = sum_i (s * 2^(i-1)) * beta_i + s * ((2^q - 1)/2 - z):
+#   alpha_i = s * 2^(i-1) (plane i = bit i of c, 0-based) and
+#   offset  = s * ((2^q - 1)/2 - z).
+# ---------------------------------------------------------------------------
+def uniform_to_bcq(codes, scale, zero, q: int, g: int):
+    """Rewrite a uniform q-bit weight as BCQ.
+
+    codes uint8 [m][n] in [0, 2^q); scale fp16 [n/g][m]; zero uint8 [n/g][m]
+    in [0, 2^q).  Returns (signs int8 [q][m][n], alpha fp16 [q][n/g][m],
+    offset fp32 [n/g][m]).  alpha_i = RNE_fp16(s * 2^(i-1)) (exact unless s*2^-1
+    is an fp16 subnormal with its last bit set); offset = s * ((2^q-1)/2 - z),
+    exact in fp32 (an 11-bit significand times a half-integer below 2^q).
+    """
+    c = np.asarray(codes, dtype=np.int64)
+    z = np.asarray(zero, dtype=np.int64)
+    s64 = np.asarray(scale, dtype=np.float16).astype(np.float64)
+    m, n = c.shape
+    top = 1 << q
+    if c.min(initial=0) < 0 or c.max(initial=0) >= top:
+        raise ValueError("codes must lie in [0, 2^q)")
+    if z.min(initial=0) < 0 or z.max(initial=0) >= top:
+        raise ValueError("zero-points must lie in [0, 2^q)")
+    signs = np.empty((q, m, n), dtype=np.int8)
+    alpha = np.empty((q,) + s64.shape, dtype=np.float16)
+    for i in range(q):
+        signs[i] = (((c >> i) & 1) * 2 - 1).astype(np.int8)
+        alpha[i] = (s64 * (2.0 ** (i - 1))).astype(np.float16)
+    offset = (s64 * ((top - 1) / 2.0 - z)).astype(np.float32)
+    return signs, alpha, offset
+
+
+def uniform_dequant(codes, scale, zero, g: int) -> np.ndarray:
+    """The plain uniform dequantisation w[j,k] = s[k//g, j] * (c[j,k] - z[k//g, j]) in FP64."""
+    c = np.asarray(codes, dtype=np.float64)
+    s = np.repeat(np.asarray(scale, dtype=np.float16).astype(np.float64), g, axis=0).T
+    z = np.repeat(np.asarray(zero, dtype=np.float64), g, axis=0).T
+    return s * (c - z)
