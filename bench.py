@@ -1,0 +1,415 @@
+"""Benchmark: LUT-GEMM microseconds per matmul and achieved HBM GB/s at batch 1.
+
+One step is one pass over the linears of an OPT-175B-shaped decoder layer
+(QKV 36864x12288, out-proj 12288x12288, FC1 49152x12288, FC2 12288x49152) with
+q = 3 BCQ planes, g = 128, batch 1: four lutgemm_run calls.  Weights are
+synthetic (uniform random sign bits, |N(0, 0.02)| fp16 scales, x ~ N(0, 1)),
+drawn by bcq_synth; the step's working set (765 MB) is far larger than the
+126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lutgemm|reference]
+
+N > 1 runs under torchrun: every rank runs its own layer (independent weights,
+no data-path collective: weak scaling); the timed region is bracketed by a
+barrier and device synchronisation and its length is the max over ranks.
+"--impl reference" times the FP64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import bcq_synth as S  # noqa: E402
+from weight_only_quantized_bcq_b200.roofline import algorithmic_bytes  # noqa: E402
+
+METRIC = "LUT-GEMM µs/matmul and achieved HBM GB/s (fraction of B200 peak) at batch 1"
+WORKLOAD = "opt175b_layer"
+DATASHEET_GBS = 8000.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def _kernel_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_hash: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches this kernel source."""
+    path = os.path.join(ROOT, "profiles", "lut_gemm_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_hash") != kernel_hash:
+        return None
+    return d.get("dram_bytes_per_launch_avg")
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons read through NVML every millisecond while
+    the timed region runs (reads only; no GPU setting is touched)."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, torch_index: int, period_s: float = 0.001):
+        self.torch_index = torch_index
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+
+    def _handle(self, nv):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.torch_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.torch_index)
+
+    def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nvml = nv
+            self.h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM))
+            self._thread = threading.Thread(target=self._loop, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._nvml = None
+        return self
+
+    def _loop(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((float(mhz), int(mask)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+        if self._nvml is not None:
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return None
+        nv = self._nvml or __import__("pynvml")
+        reasons = set()
+        for _, mask in self.samples:
+            for name, const in self.REASONS:
+                if mask & int(getattr(nv, const, 0)):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml, 1 ms"}
+
+
+# ---------------------------------------------------------------------------
+# Workload
+# ---------------------------------------------------------------------------
+def make_layer(q: int, batch: int, seed: int, device, only=None):
+    """Packed planes, scales and inputs of the four linears, resident on `device`."""
+    from weight_only_quantized_bcq_b200 import lutgemm
+    w = S.WORKLOADS[WORKLOAD]
+    gen = S.generator(seed)
+    mats = []
+    for sh in w.shapes:
+        if only and sh.name != only:
+            continue
+        nbytes = lutgemm.packed_bytes(q, sh.m, sh.n)
+        packed = S.draw_random_bytes(gen, nbytes).to(device)
+        alpha = S.draw_alpha(gen, q, sh.m, sh.n, w.g, w.alpha_sigma).to(device)
+        x_host = S.draw_x(gen, batch, sh.n).pin_memory()
+        mats.append({
+            "name": sh.name, "m": sh.m, "n": sh.n, "packed": packed, "alpha": alpha,
+            "x_host": x_host, "x": x_host.to(device),
+            "y": torch.empty((batch, sh.m), dtype=torch.float32, device=device),
+            "y_host": torch.empty((batch, sh.m), dtype=torch.float32).pin_memory(),
+            "ws": lutgemm.new_workspace(sh.m, sh.n, batch, q, w.g, device=device),
+            "bytes": algorithmic_bytes(sh.m, sh.n, q, w.g, batch),
+        })
+    return mats, w.g
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_lutgemm(args):
+    from weight_only_quantized_bcq_b200 import lutgemm
+    world, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    q, batch = args.q, args.batch
+    mats, g = make_layer(q, batch, seed=S.WORKLOADS[WORKLOAD].seed + 1000 * rank, device=device,
+                         only=args.only)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        for i, mt in enumerate(mats):
+            if events is not None:
+                events[i][0].record(stream)
+            lutgemm.run(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"],
+                        workspace=mt["ws"], stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    def e2e_step():
+        for mt in mats:
+            mt["x"].copy_(mt["x_host"], non_blocking=True)
+            lutgemm.run(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"],
+                        workspace=mt["ws"], stream=stream)
+            mt["y_host"].copy_(mt["y"], non_blocking=True)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+
+    # Device-resident timing: K steps, CUDA events around the whole region and
+    # around every launch (same stream).
+    per_launch = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+                   for _ in mats] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier()
+        t0.record(stream)
+        for k in range(args.steps):
+            step(per_launch[k])
+        t1.record(stream)
+        barrier()
+    region_ms = max_over_ranks(t0.elapsed_time(t1))
+    launch_ms = [[per_launch[k][i][0].elapsed_time(per_launch[k][i][1]) for i in range(len(mats))]
+                 for k in range(args.steps)]
+
+    # End to end through the public API: per step, pinned x -> device, the four
+    # runs, y -> pinned host; all inside the timed region.
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+
+    step_bytes = sum(mt["bytes"] for mt in mats)
+    total_bytes = step_bytes * args.steps * world
+    value = total_bytes / (region_ms * 1e-3) / 1e9
+    e2e_gbs = total_bytes / (e2e_ms * 1e-3) / 1e9
+    kern_ms_total = sum(sum(r) for r in launch_ms)
+    achieved = step_bytes * args.steps / (kern_ms_total * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    khash = _kernel_hash()
+    us_per = {mt["name"]: 1e3 * statistics.median([launch_ms[k][i] for k in range(args.steps)])
+              for i, mt in enumerate(mats)}
+    gbs_per = {mt["name"]: mt["bytes"] / (us_per[mt["name"]] * 1e-6) / 1e9 for mt in mats}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(region_ms / args.steps, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {
+                "workload": "OPT-175B decoder-layer linears (QKV 36864x12288, out 12288x12288, "
+                            f"FC1 49152x12288, FC2 12288x49152), BCQ q={q}, g={g}, batch {batch}",
+                "q": q, "g": g, "batch": batch,
+                "bytes_per_step": step_bytes,
+                "l2": "no flush: each step streams 765 MB (> 126 MB L2) of distinct weights",
+                "parallelism": "replicas" if world == 1 else f"replicas{world} (one layer per GPU)",
+                "only": args.only,
+            },
+            "us_per_matmul": {k: round(v, 2) for k, v in us_per.items()},
+            "gbs_per_matmul": {k: round(v, 1) for k, v in gbs_per.items()},
+            "frac_of_datasheet_8tbs": round(value / world / DATASHEET_GBS, 4),
+            "roofline": {
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": _traffic(khash),
+                "peak_kind": peak_kind, "kernel": "lut_gemm_kernel", "kernel_hash": khash,
+            },
+            "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
+                    "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
+            "gpu_launches": len(mats) * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(q, batch, args.cpu_rows)
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# The FP64 oracle on the host cores, on a bounded sample of the same workload.
+# ---------------------------------------------------------------------------
+def _oracle_sample(q: int, batch: int, rows_per_matrix: int, seed: int):
+    """Timed oracle work on `rows_per_matrix` sampled rows of each of the four linears.
+
+    Returns (seconds, algorithmic bytes of the sampled rows)."""
+    import numpy as np
+    from oracle import bcq_oracle as O
+    w = S.WORKLOADS[WORKLOAD]
+    rng = np.random.default_rng(seed)
+    secs, nbytes = 0.0, 0
+    for sh in w.shapes:
+        gen = S.generator(seed * 31 + sh.m)
+        mt = -(-sh.m // 32)
+        # Only the row tiles the sample touches are drawn: rows 32*R + l.
+        tiles = np.sort(rng.choice(mt, size=max(1, rows_per_matrix // 32), replace=False))
+        m_s = 32 * tiles.size
+        packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m_s, sh.n)).numpy()
+        alpha = S.draw_alpha(gen, q, m_s, sh.n, w.g, w.alpha_sigma).numpy()
+        x = S.draw_x(gen, batch, sh.n).numpy()
+        t = time.perf_counter()
+        signs = O.unpack_bcq(packed, q, m_s, sh.n)
+        y = O.bcq_matmul(x, signs, alpha, w.g)
+        secs += time.perf_counter() - t
+        assert np.all(np.isfinite(y))
+        nbytes += algorithmic_bytes(m_s, sh.n, q, w.g, batch)
+    return secs, nbytes
+
+
+def cpu_baseline(q: int, batch: int, rows: int):
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        secs, nbytes = _oracle_sample(q, batch, rows, seed=7)
+    return {"value": round(nbytes / secs / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(secs, 2),
+            "sample": f"{rows} rows of each of the 4 layer linears (q={q}, g=128, batch {batch}): "
+                      "oracle unpack + FP64 dequantise + matmul, one thread"}
+
+
+def run_reference(args):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return
+    q, batch = args.q, args.batch
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=1)
+    for k in range(args.warmup):
+        _oracle_sample(q, batch, args.ref_rows, seed=100 + k)
+    secs, nbytes = 0.0, 0
+    for k in range(args.steps):
+        s, b = _oracle_sample(q, batch, args.ref_rows, seed=200 + k)
+        secs += s
+        nbytes += b
+    value = nbytes / secs / 1e9
+    sample = (f"{args.ref_rows} rows of each of the 4 layer linears per step (q={q}, g=128, batch {batch}): "
+              "oracle unpack + FP64 dequantise + matmul, one thread")
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "OPT-175B decoder-layer linears (QKV 36864x12288, out 12288x12288, "
+                               f"FC1 49152x12288, FC2 12288x49152), BCQ q={q}, g=128, batch {batch}",
+                   "q": q, "g": 128, "batch": batch, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["lutgemm", "reference"], default="lutgemm")
+    ap.add_argument("--q", type=int, default=3)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--cpu-rows", type=int, default=512, help="rows per linear in the CPU baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=64, help="rows per linear per step of --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
+                    help="time one linear of the layer only (profiling)")
+    args = ap.parse_args()
+    # At least three untimed warm-up steps, whatever the caller asks for.
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_lutgemm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * lutgemm.h -- C ABI of a B200 (sm_100a) LUT-GEMM library for weights stored
+ * in binary-coding quantisation (BCQ).
+ *
+ * What the library computes (source: "LUT-GEMM -- paper by Park et al. (2022),
+ * ICLR 2024", Elamur card, sections Summary and Interesting ideas; pith.science
+ * card of the same paper, abstract):
+ *
+ *   A BCQ weight matrix W (m outputs x n inputs) is a sum of q binary planes,
+ *   each scaled per group of g consecutive inputs:
+ *       W[j,k] = sum_{i<q} alpha[i][k/g][j] * beta[i][j][k] (+ offset[k/g][j]),
+ *   beta in {-1,+1}.  The product y = W x is formed without dequantising W:
+ *   for every run of 8 activations the 256 possible signed sums are put in a
+ *   table once, and each plane-row reads the entry indexed by its 8 sign bits
+ *   ("Lookup tables instead of multiplications").  Uniform quantisation is
+ *   rewritten as BCQ plus a per-group offset, so one kernel serves both
+ *   (Summary; "One format for many schemes").  q and g are independent
+ *   parameters ("Group size as a separate hyper-parameter").
+ *
+ * Conventions shared by every call
+ *   - Every buffer is caller-owned and caller-allocated.  The library
+ *     allocates nothing and keeps no state between calls, except that the
+ *     workspace of lutgemm_run must be zero-filled once before its first use
+ *     and is left zero-filled again by every call that returns LUTGEMM_OK.
+ *   - "dev" pointers are CUDA device pointers on the current device; fp16
+ *     values are passed as their raw 16-bit patterns (uint16_t).
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All device work is enqueued on it and is asynchronous.
+ *   - Arguments are validated before anything is enqueued: a status other
+ *     than LUTGEMM_OK means no work was enqueued (LUTGEMM_ERR_CUDA: the launch
+ *     itself failed, as reported by cudaGetLastError).
+ *   - Values that can only be checked on the device (a sign that is not +-1,
+ *     a code or zero-point >= 2^q) are reported through an optional
+ *     device int32 *status_flags: the kernel ORs LUTGEMM_FLAG_* bits into it.
+ *     Read it after synchronising the stream; pass NULL to skip reporting.
+ *
+ * Packed bit-plane layout (produced by lutgemm_pack_bcq and
+ * lutgemm_uniform_to_bcq, consumed by lutgemm_run).  The pages do not fix a
+ * layout; this one lets each GPU lane read 16 contiguous bytes per step and
+ * makes the table reads of a warp fall in 32 distinct shared-memory banks.
+ *   n_s = ceil(n/1024) slices of 1024 inputs, m_t = ceil(m/32) row tiles.
+ *   The buffer holds n_s * m_t * q blocks of 4096 bytes; block (s, R, i)
+ *   starts at byte ((s * m_t + R) * q + i) * 4096.
+ *   In block (s, R, i), byte U*512 + l*16 + j  (U < 8, l < 32, j < 16) holds
+ *   the 8 sign bits of row r = 32*R + l, plane i, inputs
+ *   k = 1024*s + 128*P + 8*c + t for t = 0..7 (bit t, least significant
+ *   first), where P = U xor (4 * (l / 16)) and c = j xor (l % 16).
+ *   A bit is 1 iff beta = +1.  Bits of rows r >= m or inputs k >= n are 0.
+ *
+ * Other layouts (row-major, innermost last):
+ *   signs  int8   [q][m][n]     each -1 or +1
+ *   codes  uint8  [m][n]        uniform codes in [0, 2^q)
+ *   scale  fp16   [n/g][m]      uniform scale s
+ *   zero   uint8  [n/g][m]      uniform integer zero-point z in [0, 2^q)
+ *   alpha  fp16   [q][n/g][m]   group-wise plane scales
+ *   offset fp32   [n/g][m]      group offsets of converted uniform weights
+ *   x      fp16   [batch][n]
+ *   y      fp32 (or fp16 with LUTGEMM_Y_F16) [batch][m]
+ */
+#ifndef LUTGEMM_H
+#define LUTGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every int-valued call. */
+#define LUTGEMM_OK             0
+#define LUTGEMM_ERR_NULL       1  /* a required pointer is NULL */
+#define LUTGEMM_ERR_SHAPE      2  /* m, n, batch < 1; q not in [1,8]; n%8, g%8 or n%g != 0 */
+#define LUTGEMM_ERR_ALIGN      3  /* a pointer is not aligned as its call requires */
+#define LUTGEMM_ERR_WORKSPACE  4  /* workspace smaller than lutgemm_workspace_size() */
+#define LUTGEMM_ERR_VALUE      5  /* a host-checkable value is out of range */
+#define LUTGEMM_ERR_CUDA       6  /* a CUDA runtime call or launch failed */
+
+/* Bits OR-ed into *status_flags by device-side value checks. */
+#define LUTGEMM_FLAG_BAD_SIGN  1  /* lutgemm_pack_bcq: a sign was neither -1 nor +1 */
+#define LUTGEMM_FLAG_BAD_CODE  2  /* lutgemm_uniform_to_bcq: a code >= 2^q */
+#define LUTGEMM_FLAG_BAD_ZERO  4  /* lutgemm_uniform_to_bcq: a zero-point >= 2^q */
+
+/* Flags of lutgemm_run. */
+#define LUTGEMM_Y_F16          1u /* write y as fp16 (round to nearest even of the fp32 sum) */
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+int lutgemm_version(void);
+
+/* Static English text for a status code (never NULL). */
+const char* lutgemm_status_string(int status);
+
+/* Bytes of the packed bit-plane buffer for (q, m, n):
+ * ceil(n/1024) * ceil(m/32) * q * 4096.  Returns 0 for invalid shapes.
+ * Pure host function. */
+size_t lutgemm_packed_bytes(int q, int m, int n);
+
+/* Bytes of the lutgemm_run workspace (split-K partial sums and per-row-tile
+ * arrival counters).  Returns 0 for invalid shapes.  Pure host function. */
+size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g);
+
+/* Pack q planes of +-1 signs into the packed bit-plane layout above.
+ * Defines the BCQ binary planes of the LUT-GEMM card (Summary; Interesting
+ * ideas: weights are binary +-1 vectors with scales).
+ *   signs        dev int8 [q][m][n], 8-byte aligned, each -1 or +1
+ *   q, m, n      1 <= q <= 8, m >= 1, n >= 8, n % 8 == 0
+ *   packed       dev, lutgemm_packed_bytes(q,m,n) bytes, 16-byte aligned;
+ *                every byte is written (padding bits 0)
+ *   status_flags dev int32 or NULL; LUTGEMM_FLAG_BAD_SIGN is OR-ed in if a
+ *                sign is neither -1 nor +1 (its bit is then written as
+ *                1 iff the value is > 0)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN or ERR_CUDA. */
+int lutgemm_pack_bcq(const int8_t* signs, int q, int m, int n,
+                     uint8_t* packed, int32_t* status_flags, void* stream);
+
+/* Rewrite a uniform q-bit weight w = s * (c - z) as BCQ plus a group offset
+ * (LUT-GEMM card, Summary and "One format for many schemes": uniform
+ * quantisation is a special case of BCQ; the pages give no formula).  With
+ * c = sum_i 2^i b_i and beta_i = 2 b_i - 1:
+ *     plane i = bit i of c,   alpha_i = s * 2^(i-1),
+ *     offset  = s * ((2^q - 1)/2 - z),
+ * so sum_i alpha_i beta_i + offset = s * (c - z).  alpha_i is rounded to
+ * fp16 (nearest even; exact unless s/2 is an fp16 subnormal with its last bit
+ * set); offset is exact in fp32.
+ *   codes        dev uint8 [m][n], 8-byte aligned, each < 2^q
+ *   scale        dev fp16 [n/g][m]
+ *   zero         dev uint8 [n/g][m], each < 2^q
+ *   q, m, n, g   1 <= q <= 8, m >= 1, n % 8 == 0, g % 8 == 0, n % g == 0
+ *   packed       dev, lutgemm_packed_bytes(q,m,n) bytes, 16-byte aligned
+ *   alpha        dev fp16 [q][n/g][m] (output)
+ *   offset       dev fp32 [n/g][m] (output), 4-byte aligned
+ *   status_flags dev int32 or NULL; LUTGEMM_FLAG_BAD_CODE / _BAD_ZERO are
+ *                OR-ed in for out-of-range codes / zero-points (the values
+ *                are then used modulo 2^q)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN or ERR_CUDA. */
+int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
+                           const uint8_t* zero, int q, int m, int n, int g,
+                           uint8_t* packed, uint16_t* alpha, float* offset,
+                           int32_t* status_flags, void* stream);
+
+/* y = W x for a BCQ weight, through per-8-activation lookup tables, with no
+ * dequantisation (LUT-GEMM card, Summary and "Lookup tables instead of
+ * multiplications"; pith.science abstract).  For each batch column b and each
+ * slice of 1024 inputs, tables T[c][p] = sum_{t<8} (2*bit_t(p) - 1) * x[b][8c+t]
+ * are built in fp32 in shared memory; each plane-row adds T[c][byte] over the
+ * runs of a group, scales the sum by alpha (and adds offset * sum of the
+ * group's x for converted uniform weights), and the per-slice partial sums
+ * are reduced in a fixed order, so repeated calls give identical bits.
+ *   m, n, batch, q, g  m >= 1, batch >= 1, 1 <= q <= 8, n % 8 == 0,
+ *                      g % 8 == 0, n % g == 0
+ *   packed     dev, packed layout above, 16-byte aligned
+ *   alpha      dev fp16 [q][n/g][m], 2-byte aligned
+ *   offset     dev fp32 [n/g][m] or NULL (pure BCQ), 4-byte aligned
+ *   x          dev fp16 [batch][n], 16-byte aligned
+ *   y          dev [batch][m] fp32 (4-byte aligned) or, with LUTGEMM_Y_F16,
+ *              fp16 (2-byte aligned); fully overwritten
+ *   flags      0 or LUTGEMM_Y_F16
+ *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
+ *              16-byte aligned, zero-filled before its first use; left
+ *              zero-filled by every successful call.  Calls that share a
+ *              workspace must not overlap on the device.
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE or
+ * ERR_CUDA. */
+int lutgemm_run(int m, int n, int batch, int q, int g,
+                const uint8_t* packed, const uint16_t* alpha,
+                const float* offset, const uint16_t* x, void* y,
+                unsigned flags, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LUTGEMM_H */

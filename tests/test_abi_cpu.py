@@ -1,0 +1,146 @@
+"""CPU checks of the C-ABI library: it builds, loads, exports every declared
+symbol, and its host-side logic (sizes, argument validation) is right.  No call
+here reaches a CUDA kernel: every invalid argument is rejected before launch.
+"""
+from __future__ import annotations
+
+import math
+import os
+import re
+
+import pytest
+
+from oracle import bcq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lutgemm.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from weight_only_quantized_bcq_b200 import build, lutgemm
+    build.build()
+    return lutgemm
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lutgemm_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("lutgemm_pack_bcq", "lutgemm_uniform_to_bcq", "lutgemm_run",
+                 "lutgemm_packed_bytes", "lutgemm_workspace_size", "lutgemm_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    lib = L.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(L):
+    lib = L.lib()
+    assert lib.lutgemm_version() >= 10000
+    for st in range(7):
+        assert len(L.status_string(st)) > 5
+    assert L.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("q,m,n", [(1, 1, 8), (3, 512, 512), (3, 49152, 12288), (2, 33, 1032),
+                                   (8, 100, 5000), (4, 5120, 5120)])
+def test_packed_bytes_matches_oracle(L, q, m, n):
+    assert L.packed_bytes(q, m, n) == O.packed_nbytes(q, m, n)
+
+
+@pytest.mark.parametrize("q,m,n", [(0, 32, 1024), (9, 32, 1024), (3, 0, 1024), (3, 32, 0), (3, 32, 12)])
+def test_packed_bytes_rejects_bad_shapes(L, q, m, n):
+    assert L.packed_bytes(q, m, n) == 0
+
+
+def test_workspace_size(L):
+    m, n, b = 49152, 12288, 1
+    ns, mt = math.ceil(n / 1024), math.ceil(m / 32)
+    part = b * ns * mt * 32 * 4
+    cnt = b * mt * 4
+    rup = lambda v: (v + 255) // 256 * 256
+    assert L.workspace_size(m, n, b, 3, 128) == rup(part) + rup(cnt) + 256   # + status word
+    assert L.workspace_size(m, n, 0, 3, 128) == 0
+    assert L.workspace_size(m, n, 1, 3, 100) == 0          # g % 8 != 0
+    assert L.workspace_size(m, 12288, 1, 3, 5000) == 0     # n % g != 0
+
+
+FAKE = 1 << 20           # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _run(L, m=64, n=1024, batch=1, q=3, g=128, packed=FAKE, alpha=FAKE, offset=None, x=FAKE, y=FAKE,
+         flags=0, ws=FAKE, ws_bytes=None):
+    lib = L.lib()
+    if ws_bytes is None:
+        ws_bytes = 1 << 30
+    return lib.lutgemm_run(m, n, batch, q, g, packed, alpha, offset, x, y, flags, ws, ws_bytes, None)
+
+
+def test_run_rejects_null(L):
+    assert _run(L, packed=None) == L.ERR_NULL
+    assert _run(L, alpha=None) == L.ERR_NULL
+    assert _run(L, x=None) == L.ERR_NULL
+    assert _run(L, y=None) == L.ERR_NULL
+    assert _run(L, ws=None) == L.ERR_NULL
+
+
+@pytest.mark.parametrize("kw", [dict(m=0), dict(n=0), dict(n=1028), dict(batch=0), dict(q=0), dict(q=9),
+                                dict(g=100), dict(g=0), dict(n=1024, g=384), dict(n=12)])
+def test_run_rejects_bad_shapes(L, kw):
+    assert _run(L, **kw) == L.ERR_SHAPE
+
+
+def test_run_rejects_misaligned(L):
+    assert _run(L, packed=FAKE + 8) == L.ERR_ALIGN
+    assert _run(L, x=FAKE + 8) == L.ERR_ALIGN
+    assert _run(L, alpha=FAKE + 1) == L.ERR_ALIGN
+    assert _run(L, offset=FAKE + 2) == L.ERR_ALIGN
+    assert _run(L, y=FAKE + 2) == L.ERR_ALIGN
+    assert _run(L, ws=FAKE + 4) == L.ERR_ALIGN
+
+
+def test_run_rejects_bad_flags_and_small_workspace(L):
+    assert _run(L, flags=2) == L.ERR_VALUE
+    need = L.workspace_size(64, 1024, 1, 3, 128)
+    assert _run(L, ws_bytes=need - 1) == L.ERR_WORKSPACE
+
+
+def test_pack_and_convert_validation(L):
+    lib = L.lib()
+    assert lib.lutgemm_pack_bcq(None, 3, 32, 1024, FAKE, None, None) == L.ERR_NULL
+    assert lib.lutgemm_pack_bcq(FAKE, 3, 32, 1020, FAKE, None, None) == L.ERR_SHAPE
+    assert lib.lutgemm_pack_bcq(FAKE + 4, 3, 32, 1024, FAKE, None, None) == L.ERR_ALIGN
+    assert lib.lutgemm_pack_bcq(FAKE, 3, 32, 1024, FAKE + 8, None, None) == L.ERR_ALIGN
+    args = [FAKE, FAKE, FAKE, 4, 32, 1024, 128, FAKE, FAKE, FAKE, None, None]
+    bad = list(args); bad[1] = None
+    assert lib.lutgemm_uniform_to_bcq(*bad) == L.ERR_NULL
+    bad = list(args); bad[6] = 96
+    assert lib.lutgemm_uniform_to_bcq(*bad) == L.ERR_SHAPE
+    bad = list(args); bad[9] = FAKE + 2
+    assert lib.lutgemm_uniform_to_bcq(*bad) == L.ERR_ALIGN
+
+
+def test_product_has_no_cpu_fallback(L, monkeypatch):
+    """Without the library the binding raises instead of computing anything."""
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "LIB_PATH", os.path.join(ROOT, "does-not-exist.so"))
+    with pytest.raises(RuntimeError):
+        L.lib()
+
+
+def test_product_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "weight_only_quantized_bcq_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
+                assert "bcq_oracle" not in text, f

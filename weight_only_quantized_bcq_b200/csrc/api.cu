@@ -1,0 +1,192 @@
+// C ABI of the LUT-GEMM library: argument validation, workspace sizing and
+// kernel launches on the caller's stream.  Declarations and the contract of
+// every call are in include/lutgemm.h.
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "lutgemm.h"
+#include "lutgemm_common.cuh"
+
+namespace lutgemm {
+cudaError_t launch_pack_signs(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* flags,
+                              cudaStream_t stream);
+cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, const uint8_t* zero, int q,
+                                  int m, int n, int g, uint8_t* packed, __half* alpha, float* offset,
+                                  int32_t* flags, cudaStream_t stream);
+}  // namespace lutgemm
+
+namespace {
+
+using namespace lutgemm;
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool valid_matrix(int q, int m, int n) { return q >= 1 && q <= 8 && m >= 1 && n >= 8 && n % 8 == 0; }
+
+bool valid_groups(int n, int g) { return g >= 8 && g % 8 == 0 && n % g == 0; }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Per-device state that is set once: SM count and the shared-memory opt-in of
+// every kernel launched on that device.
+std::mutex g_mutex;
+std::set<std::pair<const void*, int>> g_smem_done;
+int g_sm_count[64] = {0};
+
+cudaError_t device_setup(RunKernel kernel, int* sm_count) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (g_sm_count[dev] == 0) {
+    int v = 0, reserved = 0, optin = 0;
+    err = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (err != cudaSuccess) return err;
+    // The tables sit at a fixed window address above the reserved region.
+    if ((unsigned)reserved > kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
+    g_sm_count[dev] = v;
+  }
+  *sm_count = g_sm_count[dev];
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  if (g_smem_done.find(key) == g_smem_done.end()) {
+    err = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    g_smem_done.insert(key);
+  }
+  return cudaSuccess;
+}
+
+int group_mode(int g) {
+  if (g == 128) return kG128;
+  if (g % 128 == 0) return kG128x;
+  if (g == 64) return kG64;
+  if (g == 8) return kG8;
+  return kGAny;
+}
+
+RunKernel select_kernel(int q, int mode, bool has_offset) {
+  switch (q) {
+    case 1: return run_kernel_q1(mode, has_offset);
+    case 2: return run_kernel_q2(mode, has_offset);
+    case 3: return run_kernel_q3(mode, has_offset);
+    case 4: return run_kernel_q4(mode, has_offset);
+    default: return run_kernel_q8(mode, has_offset);
+  }
+}
+
+// Workspace: [split-K partials | arrival counters | status word], each 256-byte aligned.
+size_t part_bytes(int m, int n, int batch) {
+  return (size_t)batch * ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * kTileRows * sizeof(float);
+}
+
+size_t counter_bytes(int m, int batch) { return (size_t)batch * ceil_div(m, kTileRows) * sizeof(unsigned); }
+
+constexpr size_t kStatusBytes = 256;
+
+}  // namespace
+
+extern "C" {
+
+int lutgemm_version(void) { return kVersion; }
+
+const char* lutgemm_status_string(int status) {
+  switch (status) {
+    case LUTGEMM_OK: return "success";
+    case LUTGEMM_ERR_NULL: return "a required pointer is NULL";
+    case LUTGEMM_ERR_SHAPE: return "invalid shape (need m,n,batch >= 1, 1 <= q <= 8, n%8 == 0, g%8 == 0, n%g == 0)";
+    case LUTGEMM_ERR_ALIGN: return "a pointer is not aligned as the call requires";
+    case LUTGEMM_ERR_WORKSPACE: return "workspace is smaller than lutgemm_workspace_size()";
+    case LUTGEMM_ERR_VALUE: return "an argument value is out of range";
+    case LUTGEMM_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    default: return "unknown status";
+  }
+}
+
+size_t lutgemm_packed_bytes(int q, int m, int n) {
+  if (!valid_matrix(q, m, n)) return 0;
+  return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * q * kBlockBytes;
+}
+
+size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g) {
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return 0;
+  return round_up(part_bytes(m, n, batch), 256) + round_up(counter_bytes(m, batch), 256) + kStatusBytes;
+}
+
+int lutgemm_pack_bcq(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* status_flags,
+                     void* stream) {
+  if (!signs || !packed) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n)) return LUTGEMM_ERR_SHAPE;
+  if (!aligned(signs, 8) || !aligned(packed, 16) || !aligned(status_flags, 4)) return LUTGEMM_ERR_ALIGN;
+  const cudaError_t err =
+      launch_pack_signs(signs, q, m, n, packed, status_flags, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
+int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale, const uint8_t* zero, int q, int m,
+                           int n, int g, uint8_t* packed, uint16_t* alpha, float* offset,
+                           int32_t* status_flags, void* stream) {
+  if (!codes || !scale || !zero || !packed || !alpha || !offset) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g)) return LUTGEMM_ERR_SHAPE;
+  if (!aligned(codes, 8) || !aligned(scale, 2) || !aligned(packed, 16) || !aligned(alpha, 2) ||
+      !aligned(offset, 4) || !aligned(status_flags, 4))
+    return LUTGEMM_ERR_ALIGN;
+  const cudaError_t err = launch_uniform_to_bcq(
+      codes, reinterpret_cast<const __half*>(scale), zero, q, m, n, g, packed,
+      reinterpret_cast<__half*>(alpha), offset, status_flags, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
+int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, const uint16_t* alpha,
+                const float* offset, const uint16_t* x, void* y, unsigned flags, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  if (!packed || !alpha || !x || !y || !workspace) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return LUTGEMM_ERR_SHAPE;
+  if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
+  const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
+  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||
+      !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
+    return LUTGEMM_ERR_ALIGN;
+  if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
+
+  RunParams p;
+  p.packed = packed;
+  p.alpha = reinterpret_cast<const __half*>(alpha);
+  p.offset = offset;
+  p.x = reinterpret_cast<const __half*>(x);
+  p.y = y;
+  p.m = m;
+  p.n = n;
+  p.batch = batch;
+  p.q = q;
+  p.g = g;
+  p.ns = ceil_div(n, kSliceInputs);
+  p.mt = ceil_div(m, kTileRows);
+  p.ng = n / g;
+  p.y_f16 = y_f16 ? 1 : 0;
+  p.total_units = (long long)batch * p.ns * p.mt;
+  char* ws = reinterpret_cast<char*>(workspace);
+  const size_t cnt_off = round_up(part_bytes(m, n, batch), 256);
+  p.part = reinterpret_cast<float*>(ws);
+  p.cnt = reinterpret_cast<unsigned*>(ws + cnt_off);
+  p.status = reinterpret_cast<unsigned*>(ws + cnt_off + round_up(counter_bytes(m, batch), 256));
+
+  const RunKernel kernel = select_kernel(q, group_mode(g), offset != nullptr);
+  int sm_count = 0;
+  if (device_setup(kernel, &sm_count) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  const long long grid = p.total_units < sm_count ? p.total_units : (long long)sm_count;
+  kernel<<<(unsigned)grid, kThreads, kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,157 @@
+// Set-up kernels: pack +-1 planes into the tiled bit-plane layout, and rewrite
+// uniform q-bit weights as BCQ planes, scales and group offsets.
+//
+// Sources: LUT-GEMM card (Elamur), Summary and Interesting ideas ("Lookup
+// tables instead of multiplications": weights are binary +-1 vectors with
+// scales; "One format for many schemes": uniform quantisation is a special
+// case of BCQ).  The layout is defined in include/lutgemm.h.
+//
+// One thread writes one 16-byte lane piece: block (s, R, i), step U, lane l.
+// Byte j of the piece holds inputs 1024 s + 128 P + 8 c .. +7 of row 32R + l
+// with P = U xor 4*(l/16), c = j xor (l%16).  The 8 source bytes of a byte are
+// contiguous, so each is one 8-byte load.
+#include "lutgemm_common.cuh"
+#include "lutgemm.h"
+
+namespace lutgemm {
+
+namespace {
+
+__device__ __forceinline__ int piece_of(int U, int l) { return U ^ (4 * (l >> 4)); }
+__device__ __forceinline__ int run_of(int j, int l) { return j ^ (l & 15); }
+
+// Eight int8 signs -> sign byte (bit t set iff sign t > 0); flags values other than +-1.
+__device__ __forceinline__ uint32_t sign_byte(uint2 v, bool& bad) {
+  uint32_t byte = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const uint32_t w = t < 4 ? v.x : v.y;
+    const int8_t sv = (int8_t)((w >> (8 * (t & 3))) & 0xFFu);
+    bad |= (sv != 1) && (sv != -1);
+    byte |= (uint32_t)(sv > 0) << t;
+  }
+  return byte;
+}
+
+__global__ void pack_signs_kernel(const int8_t* __restrict__ signs, int q, int m, int n, int mt,
+                                  long long nthreads, uint8_t* __restrict__ packed, int32_t* flags) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nthreads) return;
+  const long long blk = tid >> 8;            // block index ((s*mt + R)*q + i)
+  const int within = (int)(tid & 255);
+  const int U = within >> 5, l = within & 31;
+  const int i = (int)(blk % q);
+  const long long sR = blk / q;
+  const int R = (int)(sR % mt);
+  const int s = (int)(sR / mt);
+  const int r = R * kTileRows + l;
+  const int P = piece_of(U, l);
+  uint32_t words[4] = {0u, 0u, 0u, 0u};
+  bool bad = false;
+  if (r < m) {
+    const int8_t* rowp = signs + ((size_t)i * m + r) * (size_t)n;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int k0 = s * kSliceInputs + 128 * P + 8 * run_of(j, l);
+      if (k0 < n) {
+        const uint2 v = *reinterpret_cast<const uint2*>(rowp + k0);
+        words[j >> 2] |= sign_byte(v, bad) << (8 * (j & 3));
+      }
+    }
+  }
+  *reinterpret_cast<uint4*>(packed + blk * kBlockBytes + U * 512 + l * 16) =
+      make_uint4(words[0], words[1], words[2], words[3]);
+  if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_SIGN);
+}
+
+// Plane i of a uniform code is bit i of the code (0-based, least significant first).
+__global__ void pack_codes_kernel(const uint8_t* __restrict__ codes, int q, int m, int n, int mt,
+                                  long long nthreads, uint8_t* __restrict__ packed, int32_t* flags) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nthreads) return;
+  const long long sR = tid >> 8;             // (s*mt + R)
+  const int within = (int)(tid & 255);
+  const int U = within >> 5, l = within & 31;
+  const int R = (int)(sR % mt);
+  const int s = (int)(sR / mt);
+  const int r = R * kTileRows + l;
+  const int P = piece_of(U, l);
+  uint32_t words[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) words[i][k] = 0u;
+  bool bad = false;
+  const uint32_t top_mask = q >= 8 ? 0u : (0xFFu << q) & 0xFFu;
+  if (r < m) {
+    const uint8_t* rowp = codes + (size_t)r * n;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int k0 = s * kSliceInputs + 128 * P + 8 * run_of(j, l);
+      if (k0 < n) {
+        const uint2 v = *reinterpret_cast<const uint2*>(rowp + k0);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const uint32_t code = ((t < 4 ? v.x : v.y) >> (8 * (t & 3))) & 0xFFu;
+          bad |= (code & top_mask) != 0u;
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            words[i][j >> 2] |= ((code >> i) & 1u) << (8 * (j & 3) + t);
+        }
+      }
+    }
+  }
+  for (int i = 0; i < q; ++i) {
+    *reinterpret_cast<uint4*>(packed + (sR * q + i) * kBlockBytes + U * 512 + l * 16) =
+        make_uint4(words[i][0], words[i][1], words[i][2], words[i][3]);
+  }
+  if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_CODE);
+}
+
+// alpha_i = RNE_fp16(s * 2^(i-1)); offset = s * ((2^q - 1)/2 - z), exact in fp32.
+__global__ void uniform_scales_kernel(const __half* __restrict__ scale, const uint8_t* __restrict__ zero,
+                                      int q, long long count, size_t plane_stride,
+                                      __half* __restrict__ alpha, float* __restrict__ offset,
+                                      int32_t* flags) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= count) return;
+  const float sf = __half2float(scale[e]);
+  const int top = 1 << q;
+  const int z = zero[e];
+  if (z >= top && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_ZERO);
+  const int zz = z & (top - 1);
+  for (int i = 0; i < q; ++i) alpha[(size_t)i * plane_stride + e] = __float2half_rn(ldexpf(sf, i - 1));
+  offset[e] = sf * ((float)(top - 1) * 0.5f - (float)zz);
+}
+
+}  // namespace
+
+cudaError_t launch_pack_signs(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* flags,
+                              cudaStream_t stream) {
+  const int mt = (m + kTileRows - 1) / kTileRows;
+  const int ns = (n + kSliceInputs - 1) / kSliceInputs;
+  const long long nthreads = (long long)ns * mt * q * 256;
+  const int block = 256;
+  const long long grid = (nthreads + block - 1) / block;
+  pack_signs_kernel<<<(unsigned)grid, block, 0, stream>>>(signs, q, m, n, mt, nthreads, packed, flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, const uint8_t* zero, int q,
+                                  int m, int n, int g, uint8_t* packed, __half* alpha, float* offset,
+                                  int32_t* flags, cudaStream_t stream) {
+  const int mt = (m + kTileRows - 1) / kTileRows;
+  const int ns = (n + kSliceInputs - 1) / kSliceInputs;
+  const long long nthreads = (long long)ns * mt * 256;
+  const int block = 256;
+  pack_codes_kernel<<<(unsigned)((nthreads + block - 1) / block), block, 0, stream>>>(
+      codes, q, m, n, mt, nthreads, packed, flags);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const long long count = (long long)(n / g) * m;
+  uniform_scales_kernel<<<(unsigned)((count + block - 1) / block), block, 0, stream>>>(
+      scale, zero, q, count, (size_t)count, alpha, offset, flags);
+  return cudaGetLastError();
+}
+
+}  // namespace lutgemm

@@ -1,0 +1,6 @@
+// Instantiations of the LUT-GEMM kernel for q = 1 bit planes.
+#include "lutgemm_run.cuh"
+
+namespace lutgemm {
+RunKernel run_kernel_q1(int mode, bool has_offset) { LUTGEMM_RUN_SELECT(1, false, pipeline_stages(1)) }
+}  // namespace lutgemm

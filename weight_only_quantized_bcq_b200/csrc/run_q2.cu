@@ -1,0 +1,6 @@
+// Instantiations of the LUT-GEMM kernel for q = 2 bit planes.
+#include "lutgemm_run.cuh"
+
+namespace lutgemm {
+RunKernel run_kernel_q2(int mode, bool has_offset) { LUTGEMM_RUN_SELECT(2, false, pipeline_stages(2)) }
+}  // namespace lutgemm

@@ -1,0 +1,144 @@
+"""Thin ctypes binding over ``liblutgemm.so`` (declared in ``include/lutgemm.h``).
+
+The functions here only marshal torch tensors (device memory, the current CUDA
+stream) into the C calls; every step of the computation runs in the library's
+CUDA kernels.  If the library is missing the calls raise: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblutgemm.so")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_VALUE, ERR_CUDA = range(7)
+FLAG_BAD_SIGN, FLAG_BAD_CODE, FLAG_BAD_ZERO = 1, 2, 4
+Y_F16 = 1
+
+_lib = None
+
+_c_int, _c_uint, _c_size, _vp = ctypes.c_int, ctypes.c_uint, ctypes.c_size_t, ctypes.c_void_p
+_SIGNATURES = {
+    "lutgemm_version": ([], _c_int),
+    "lutgemm_status_string": ([_c_int], ctypes.c_char_p),
+    "lutgemm_packed_bytes": ([_c_int, _c_int, _c_int], _c_size),
+    "lutgemm_workspace_size": ([_c_int, _c_int, _c_int, _c_int, _c_int], _c_size),
+    "lutgemm_pack_bcq": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "lutgemm_uniform_to_bcq": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp],
+                               _c_int),
+    "lutgemm_run": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_uint, _vp, _c_size,
+                     _vp], _c_int),
+}
+
+
+class LutgemmError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m weight_only_quantized_bcq_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().lutgemm_status_string(int(status)).decode()
+
+
+def _check(status: int, call: str):
+    if status != OK:
+        raise LutgemmError(status, call)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def packed_bytes(q: int, m: int, n: int) -> int:
+    return int(lib().lutgemm_packed_bytes(q, m, n))
+
+
+def workspace_size(m: int, n: int, batch: int, q: int, g: int) -> int:
+    return int(lib().lutgemm_workspace_size(m, n, batch, q, g))
+
+
+def new_workspace(m: int, n: int, batch: int, q: int, g: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace, as lutgemm_run requires before first use."""
+    nbytes = workspace_size(m, n, batch, q, g)
+    if nbytes == 0:
+        raise ValueError("invalid shape for lutgemm_workspace_size")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def pack_bcq(signs: torch.Tensor, packed: torch.Tensor = None, status_flags: torch.Tensor = None,
+             stream=None) -> torch.Tensor:
+    """int8 signs [q][m][n] (+-1) on the GPU -> packed uint8 planes."""
+    _need(signs, torch.int8, "signs")
+    q, m, n = signs.shape
+    if packed is None:
+        packed = torch.empty(max(packed_bytes(q, m, n), 16), dtype=torch.uint8, device=signs.device)
+    _check(lib().lutgemm_pack_bcq(_ptr(signs), q, m, n, _ptr(packed), _ptr(status_flags), _stream(stream)),
+           "lutgemm_pack_bcq")
+    return packed
+
+
+def uniform_to_bcq(codes: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor, q: int, g: int,
+                   status_flags: torch.Tensor = None, stream=None):
+    """Uniform codes [m][n], scale fp16 [n/g][m], zero uint8 [n/g][m] -> (packed, alpha, offset)."""
+    _need(codes, torch.uint8, "codes")
+    _need(scale, torch.float16, "scale")
+    _need(zero, torch.uint8, "zero")
+    m, n = codes.shape
+    dev = codes.device
+    packed = torch.empty(max(packed_bytes(q, m, n), 16), dtype=torch.uint8, device=dev)
+    alpha = torch.empty((q, n // g, m), dtype=torch.float16, device=dev)
+    offset = torch.empty((n // g, m), dtype=torch.float32, device=dev)
+    _check(lib().lutgemm_uniform_to_bcq(_ptr(codes), _ptr(scale), _ptr(zero), q, m, n, g, _ptr(packed),
+                                        _ptr(alpha), _ptr(offset), _ptr(status_flags), _stream(stream)),
+           "lutgemm_uniform_to_bcq")
+    return packed, alpha, offset
+
+
+def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
+        offset: torch.Tensor = None, y: torch.Tensor = None, workspace: torch.Tensor = None,
+        y_f16: bool = False, stream=None) -> torch.Tensor:
+    """y[b] = W x[b] for a packed BCQ weight W (m x n), computed by lutgemm_run."""
+    _need(packed, torch.uint8, "packed")
+    _need(alpha, torch.float16, "alpha")
+    _need(x, torch.float16, "x")
+    if offset is not None:
+        _need(offset, torch.float32, "offset")
+    batch = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
+    if workspace is None:
+        workspace = new_workspace(m, n, batch, q, g, device=x.device)
+    _check(lib().lutgemm_run(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
+                             Y_F16 if y_f16 else 0, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "lutgemm_run")
+    return y
