@@ -50,27 +50,32 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("lutgemm_common.cuh", "lutgemm_run.cuh")
+
+
 def _kernel_hash() -> str:
+    """Hash of the sources that define lut_gemm_kernel (ncu counters are tied to it)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
-def _traffic(kernel_hash: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if it matches this kernel source."""
+def _traffic(kernel_hash: str, names):
+    """Mean DRAM bytes per launch over the step's linears, from the committed ncu
+    summary; null unless it was taken on this kernel source and covers every linear."""
     path = os.path.join(ROOT, "profiles", "lut_gemm_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
-    if d.get("kernel_hash") != kernel_hash:
+    per = d.get("per_shape_bytes", {})
+    if d.get("kernel_hash") != kernel_hash or not all(n in per for n in names):
         return None
-    return d.get("dram_bytes_per_launch_avg")
+    return sum(per[n] for n in names) / len(names)
 
 
 class ClockSampler:
@@ -300,7 +305,7 @@ def run_lutgemm(args):
             "frac_of_datasheet_8tbs": round(value / world / DATASHEET_GBS, 4),
             "roofline": {
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": _traffic(khash),
+                "frac": round(achieved / peak, 4), "traffic": _traffic(khash, [mt["name"] for mt in mats]),
                 "peak_kind": peak_kind, "kernel": "lut_gemm_kernel", "kernel_hash": khash,
             },
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
