@@ -167,6 +167,34 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
                 unsigned flags, void* workspace, size_t workspace_bytes,
                 void* stream);
 
+/* Bytes of the device scratch array used by lutgemm_run_noalloc (16 MiB). */
+#define LUTGEMM_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* lutgemm_run for callers that cannot allocate device memory.  The paper has
+ * no counterpart to this call; it exists for callers that own no device
+ * allocator: a serving runtime that gave all device memory to its own pool up
+ * front, a plugin or FFI host that hands a kernel only its input and output
+ * tensors, or a latency-critical path where an allocation and its possible
+ * failure are not acceptable.  Such callers cannot supply lutgemm_run's
+ * workspace, so this call takes its split-K scratch from a fixed
+ * LUTGEMM_NOALLOC_SCRATCH_BYTES array in the library's own device memory
+ * (held on every GPU that loads the library until the process exits) and
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   Arguments, layouts and results are those of lutgemm_run, without the
+ *   workspace.  Returns LUTGEMM_ERR_WORKSPACE when the problem needs more
+ *   scratch than the array holds: more than 65536 row-tile counters
+ *   (batch * ceil(m/32)) or more than 16 MiB - 256 KiB - 256 B of partial sums
+ *   (batch * ceil(n/1024) * ceil(m/32) * 128 bytes).  Other statuses as for
+ *   lutgemm_run.
+ *   The first call on a device does a one-time set-up on that device (looks
+ *   up the array's device address and zeroes its counters on `stream`); make
+ *   that first call before any stream capture.  Every call shares the one
+ *   array, so calls that overlap on the GPU race: serialise them. */
+int lutgemm_run_noalloc(int m, int n, int batch, int q, int g,
+                        const uint8_t* packed, const uint16_t* alpha,
+                        const float* offset, const uint16_t* x, void* y,
+                        unsigned flags, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

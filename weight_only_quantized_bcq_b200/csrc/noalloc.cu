@@ -1,0 +1,149 @@
+// lutgemm_run_noalloc: the LUT-GEMM product for callers that cannot allocate
+// device memory.  Some callers own no allocator of their own: a serving
+// runtime that hands all device memory to its own pool up front, a plugin or
+// FFI host that gives a kernel nothing but its input and output tensors, or a
+// latency-critical path where an allocation (and its possible failure) is not
+// acceptable.  They cannot provide the split-K workspace that lutgemm_run
+// needs, so this entry point takes its scratch from a fixed-size array in the
+// library's own device memory instead and allocates nothing.
+//
+// The scratch is a file-scope __device__ array: every GPU on which the library
+// is loaded holds its LUTGEMM_NOALLOC_SCRATCH_BYTES until the process exits.
+// Layout (fixed, independent of the problem size):
+//   [0, 256)              status word (sticky internal-error bits)
+//   [256, 256 + 256 KB)   split-K arrival counters, zero between calls
+//   [256 + 256 KB, end)   split-K partial sums, written before they are read
+// The counters sit at a fixed place so that they are never overlaid by
+// another call's partial sums; the kernel resets every counter it uses, and
+// the first call on a device zeroes them once.  Every call shares the array,
+// so calls that overlap on the GPU (other streams, other host threads) race
+// and must be serialised by the caller.
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "lutgemm.h"
+#include "lutgemm_common.cuh"
+
+namespace {
+
+using namespace lutgemm;
+
+constexpr size_t kScratchBytes = LUTGEMM_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kStatusOff = 0;
+constexpr size_t kCounterOff = 256;
+constexpr size_t kCounterBytes = 256 * 1024;
+constexpr size_t kPartOff = kCounterOff + kCounterBytes;
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+struct DeviceScratch {
+  bool ready = false;
+  unsigned char* base = nullptr;  // device address of g_scratch on this device
+  int sm_count = 0;
+};
+
+std::mutex g_mutex;
+DeviceScratch g_dev[64];
+std::set<std::pair<const void*, int>> g_smem_done;
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+RunKernel pick_kernel(int q, int g, bool has_offset) {
+  const int mode = g == 128 ? kG128 : (g % 128 == 0 ? kG128x : (g == 64 ? kG64 : (g == 8 ? kG8 : kGAny)));
+  switch (q) {
+    case 1: return run_kernel_q1(mode, has_offset);
+    case 2: return run_kernel_q2(mode, has_offset);
+    case 3: return run_kernel_q3(mode, has_offset);
+    case 4: return run_kernel_q4(mode, has_offset);
+    default: return run_kernel_q8(mode, has_offset);
+  }
+}
+
+// Once per device, with that device current: look up the scratch array's
+// device address and zero its status word and counters on the caller's
+// stream (ordered before the first launch).  Then, once per kernel and
+// device, opt the kernel into its shared-memory size.
+cudaError_t prepare(RunKernel kernel, cudaStream_t stream, DeviceScratch* out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceScratch& d = g_dev[dev];
+  if (!d.ready) {
+    void* ptr = nullptr;
+    err = cudaGetSymbolAddress(&ptr, g_scratch);
+    if (err != cudaSuccess) return err;
+    int sms = 0, reserved = 0, optin = 0;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess)
+      return err;
+    if ((err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+      return err;
+    if ((unsigned)reserved > kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
+    err = cudaMemsetAsync(ptr, 0, kPartOff, stream);
+    if (err != cudaSuccess) return err;
+    d.base = static_cast<unsigned char*>(ptr);
+    d.sm_count = sms;
+    d.ready = true;
+  }
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  if (g_smem_done.find(key) == g_smem_done.end()) {
+    err = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    g_smem_done.insert(key);
+  }
+  *out = d;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const uint8_t* packed,
+                                   const uint16_t* alpha, const float* offset, const uint16_t* x, void* y,
+                                   unsigned flags, void* stream) {
+  if (!packed || !alpha || !x || !y) return LUTGEMM_ERR_NULL;
+  if (q < 1 || q > 8 || m < 1 || n < 8 || n % 8 != 0 || g < 8 || g % 8 != 0 || n % g != 0 || batch < 1)
+    return LUTGEMM_ERR_SHAPE;
+  if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
+  const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
+  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||
+      !aligned(y, y_f16 ? 2 : 4))
+    return LUTGEMM_ERR_ALIGN;
+  const int ns = ceil_div(n, kSliceInputs);
+  const int mt = ceil_div(m, kTileRows);
+  const size_t counters = (size_t)batch * mt * sizeof(unsigned);
+  const size_t partials = (size_t)batch * ns * mt * kTileRows * sizeof(float);
+  if (counters > kCounterBytes || partials > kScratchBytes - kPartOff) return LUTGEMM_ERR_WORKSPACE;
+
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const RunKernel kernel = pick_kernel(q, g, offset != nullptr);
+  DeviceScratch d;
+  if (prepare(kernel, st, &d) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+
+  RunParams p;
+  p.packed = packed;
+  p.alpha = reinterpret_cast<const __half*>(alpha);
+  p.offset = offset;
+  p.x = reinterpret_cast<const __half*>(x);
+  p.y = y;
+  p.part = reinterpret_cast<float*>(d.base + kPartOff);
+  p.cnt = reinterpret_cast<unsigned*>(d.base + kCounterOff);
+  p.status = reinterpret_cast<unsigned*>(d.base + kStatusOff);
+  p.m = m;
+  p.n = n;
+  p.batch = batch;
+  p.q = q;
+  p.g = g;
+  p.ns = ns;
+  p.mt = mt;
+  p.ng = n / g;
+  p.y_f16 = y_f16 ? 1 : 0;
+  p.total_units = (long long)batch * ns * mt;
+  const long long grid = p.total_units < d.sm_count ? p.total_units : (long long)d.sm_count;
+  kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}

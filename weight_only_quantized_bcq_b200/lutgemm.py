@@ -31,6 +31,8 @@ _SIGNATURES = {
                                _c_int),
     "lutgemm_run": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_uint, _vp, _c_size,
                      _vp], _c_int),
+    "lutgemm_run_noalloc": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_uint, _vp],
+                            _c_int),
 }
 
 
@@ -141,4 +143,25 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
     _check(lib().lutgemm_run(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
                              Y_F16 if y_f16 else 0, _ptr(workspace), workspace.numel(), _stream(stream)),
            "lutgemm_run")
+    return y
+
+
+def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
+                offset: torch.Tensor = None, y: torch.Tensor = None, y_f16: bool = False,
+                stream=None) -> torch.Tensor:
+    """``run`` through lutgemm_run_noalloc, for callers that cannot allocate a
+    workspace: the library uses its own fixed 16 MiB device scratch instead.
+    Only ``y`` is allocated here, and only when the caller passes none.  Calls
+    that overlap on the GPU share that scratch and race."""
+    _need(packed, torch.uint8, "packed")
+    _need(alpha, torch.float16, "alpha")
+    _need(x, torch.float16, "x")
+    if offset is not None:
+        _need(offset, torch.float32, "offset")
+    batch = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
+    _check(lib().lutgemm_run_noalloc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x),
+                                     _ptr(y), Y_F16 if y_f16 else 0, _stream(stream)),
+           "lutgemm_run_noalloc")
     return y
