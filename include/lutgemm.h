@@ -39,13 +39,16 @@
  * layout; this one lets each GPU lane read 16 contiguous bytes per step and
  * makes the table reads of a warp fall in 32 distinct shared-memory banks.
  *   n_s = ceil(n/1024) slices of 1024 inputs, m_t = ceil(m/32) row tiles.
- *   The buffer holds n_s * m_t * q blocks of 4096 bytes; block (s, R, i)
- *   starts at byte ((s * m_t + R) * q + i) * 4096.
- *   In block (s, R, i), byte U*512 + l*16 + j  (U < 8, l < 32, j < 16) holds
- *   the 8 sign bits of row r = 32*R + l, plane i, inputs
- *   k = 1024*s + 128*P + 8*c + t for t = 0..7 (bit t, least significant
- *   first), where P = U xor (4 * (l / 16)) and c = j xor (l % 16).
+ *   The buffer holds n_s * m_t * 8 * q chunks of 512 bytes; chunk
+ *   (s, R, U, i) (U < 8, plane i < q) starts at byte
+ *   (((s * m_t + R) * 8 + U) * q + i) * 512.
+ *   In chunk (s, R, U, i), byte l*16 + j  (l < 32, j < 16) holds the 8 sign
+ *   bits of row r = 32*R + l, plane i, inputs k = 1024*s + 128*P + 8*c + t
+ *   for t = 0..7 (bit t, least significant first), where
+ *   P = U xor (4 * (l / 16)) and c = j xor (l % 16).
  *   A bit is 1 iff beta = +1.  Bits of rows r >= m or inputs k >= n are 0.
+ *   The q * 4096 bytes of one (slice, row tile) are contiguous, and so are
+ *   the q * 512 bytes a warp reads per step.
  *
  * Other layouts (row-major, innermost last):
  *   signs  int8   [q][m][n]     each -1 or +1
@@ -95,8 +98,9 @@ const char* lutgemm_status_string(int status);
  * Pure host function. */
 size_t lutgemm_packed_bytes(int q, int m, int n);
 
-/* Bytes of the lutgemm_run workspace (split-K partial sums and per-row-tile
- * arrival counters).  Returns 0 for invalid shapes.  Pure host function. */
+/* Bytes of the lutgemm_run workspace (split-K partial sums, per-row-tile
+ * arrival counters, per-slice tile counters and a status word).  Returns 0
+ * for invalid shapes.  Pure host function. */
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g);
 
 /* Pack q planes of +-1 signs into the packed bit-plane layout above.
@@ -183,7 +187,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
  *   Arguments, layouts and results are those of lutgemm_run, without the
  *   workspace.  Returns LUTGEMM_ERR_WORKSPACE when the problem needs more
  *   scratch than the array holds: more than 65536 row-tile counters
- *   (batch * ceil(m/32)) or more than 16 MiB - 256 KiB - 256 B of partial sums
+ *   (batch * ceil(m/32)) or more than 16 MiB - 260 KiB - 256 B of partial sums
  *   (batch * ceil(n/1024) * ceil(m/32) * 128 bytes).  Other statuses as for
  *   lutgemm_run.
  *   The first call on a device does a one-time set-up on that device (looks

@@ -50,7 +50,7 @@ MU = 8            # activations per lookup-table run (256-entry tables)
 SLICE = 1024      # inputs per slice of the packed layout
 TILE_ROWS = 32    # rows per row tile of the packed layout
 PIECE = 128       # inputs per 16-byte lane piece of the packed layout
-BLOCK_BYTES = 4096
+BLOCK_BYTES = 4096  # bytes of one (slice, row tile, plane): 8 chunks of 512
 
 __all__ = [
     "lut_table", "dequantize_bcq", "bcq_matmul", "lut_matmul",
@@ -151,12 +151,11 @@ def lut_matmul(x, signs, alpha, g: int, offset=None) -> np.ndarray:
 # Packed layout (library-defined; re-implemented from the header's text).
 #
 #   n_s = ceil(n / 1024) slices, m_t = ceil(m / 32) row tiles.
-#   The buffer is n_s * m_t * q blocks of 4096 bytes; block (s, R, i) starts at
-#   byte ((s * m_t + R) * q + i) * 4096.
-#   In that block, byte U*512 + l*16 + j (U < 8, l < 32, j < 16) holds the
-#   8 sign bits of row r = 32*R + l, plane i, inputs
-#   k = 1024*s + 128*P + 8*c + t (bit t, LSB first), where
-#   P = U xor (4 * (l // 16)) and c = j xor (l % 16).
+#   The buffer is n_s * m_t * 8 * q chunks of 512 bytes; chunk (s, R, U, i)
+#   starts at byte (((s * m_t + R) * 8 + U) * q + i) * 512.
+#   In that chunk, byte l*16 + j (l < 32, j < 16) holds the 8 sign bits of
+#   row r = 32*R + l, plane i, inputs k = 1024*s + 128*P + 8*c + t (bit t,
+#   LSB first), where P = U xor (4 * (l // 16)) and c = j xor (l % 16).
 #   A bit is 1 iff the sign is +1; bits of rows >= m or inputs >= n are 0.
 # ---------------------------------------------------------------------------
 def packed_nbytes(q: int, m: int, n: int) -> int:
@@ -179,7 +178,7 @@ def pack_bcq(signs) -> np.ndarray:
     bits[:, :m, :n] = (s > 0)
     # bits_r[i, R, l, s, k_in_slice]
     bits_r = bits.reshape(q, mt, TILE_ROWS, ns, SLICE)
-    out = np.zeros((ns, mt, q, 8, TILE_ROWS, 16), dtype=np.uint8)
+    out = np.zeros((ns, mt, 8, q, TILE_ROWS, 16), dtype=np.uint8)
     for U in range(8):
         for l in range(TILE_ROWS):
             for j in range(16):
@@ -188,7 +187,7 @@ def pack_bcq(signs) -> np.ndarray:
                 byte = np.zeros((q, mt, ns), dtype=np.uint8)
                 for t in range(MU):
                     byte |= (bits_r[:, :, l, :, k0 + t] << t).astype(np.uint8)
-                out[:, :, :, U, l, j] = byte.transpose(2, 1, 0)
+                out[:, :, U, :, l, j] = byte.transpose(2, 1, 0)
     return out.reshape(-1)
 
 
@@ -202,7 +201,7 @@ def unpack_rows(packed, q: int, m: int, n: int, rows) -> np.ndarray:
     pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
     assert pk.size == packed_nbytes(q, m, n)
     ns, mt = math.ceil(n / SLICE), math.ceil(m / TILE_ROWS)
-    blocks = pk.reshape(ns, mt, q, 8, TILE_ROWS, 16)
+    chunks = pk.reshape(ns, mt, 8, q, TILE_ROWS, 16)
     rows = np.asarray(rows, dtype=np.int64)
     out_bits = np.zeros((q, rows.size, ns * SLICE), dtype=np.uint8)
     for ri, r in enumerate(rows):
@@ -211,7 +210,7 @@ def unpack_rows(packed, q: int, m: int, n: int, rows) -> np.ndarray:
             for j in range(16):
                 P, c = _piece_and_run(U, l, j)
                 k0 = PIECE * P + MU * c
-                byte = blocks[:, R, :, U, l, j]          # [ns][q]
+                byte = chunks[:, R, U, :, l, j]          # [ns][q]
                 for t in range(MU):
                     bit = (byte >> t) & 1                 # [ns][q]
                     out_bits[:, ri, np.arange(ns) * SLICE + k0 + t] = bit.T

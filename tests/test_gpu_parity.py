@@ -257,9 +257,9 @@ def test_deterministic_and_workspace_reuse(L):
     part = (b * ns * mt * 32 * 4 + 255) // 256 * 256
     cnt = ws[part:part + b * mt * 4].cpu().numpy().view(np.uint32)
     assert not cnt.any()
-    status_off = part + (b * mt * 4 + 255) // 256 * 256
-    assert ws.numel() == status_off + 256
-    assert not ws[status_off:].cpu().numpy().any()
+    tiles_off = part + (b * mt * 4 + 255) // 256 * 256
+    assert ws.numel() == tiles_off + 4096 + 256
+    assert not ws[tiles_off:].cpu().numpy().any()     # tile counters and status word
 
 
 def test_small_workspace_is_rejected(L):

@@ -431,6 +431,15 @@ def test_pack_pins_catch_wrong_run_xor(monkeypatch):
     assert not pin_pack_golden(O.pack_bcq)
 
 
+def test_pack_pins_catch_plane_major_chunk_order():
+    def plane_major(s):
+        q, m, n = s.shape
+        pk = O.pack_bcq(s)
+        ns, mt = -(-n // 1024), -(-m // 32)
+        return pk.reshape(ns, mt, 8, q, 512).transpose(0, 1, 3, 2, 4).reshape(-1)
+    assert not pin_pack_golden(plane_major)
+
+
 def test_pack_pins_catch_msb_first():
     def msb_first(s):
         bits = np.unpackbits(O.pack_bcq(s), bitorder="little")

@@ -52,8 +52,8 @@ cudaError_t device_setup(RunKernel kernel, int* sm_count) {
     if (err != cudaSuccess) return err;
     err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (err != cudaSuccess) return err;
-    // The tables sit at a fixed window address above the reserved region.
-    if ((unsigned)reserved > kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
+    // The tables sit at a fixed window address right after the reserved region.
+    if ((unsigned)reserved != kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
     g_sm_count[dev] = v;
   }
   *sm_count = g_sm_count[dev];
@@ -85,7 +85,8 @@ RunKernel select_kernel(int q, int mode, bool has_offset) {
   }
 }
 
-// Workspace: [split-K partials | arrival counters | status word], each 256-byte aligned.
+// Workspace: [split-K partials | arrival counters | tile counters | status word],
+// each part 256-byte aligned.
 size_t part_bytes(int m, int n, int batch) {
   return (size_t)batch * ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * kTileRows * sizeof(float);
 }
@@ -93,6 +94,7 @@ size_t part_bytes(int m, int n, int batch) {
 size_t counter_bytes(int m, int batch) { return (size_t)batch * ceil_div(m, kTileRows) * sizeof(unsigned); }
 
 constexpr size_t kStatusBytes = 256;
+constexpr size_t kTileCounterBytes = kMaxTileCounters * sizeof(unsigned);
 
 }  // namespace
 
@@ -120,7 +122,8 @@ size_t lutgemm_packed_bytes(int q, int m, int n) {
 
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g) {
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return 0;
-  return round_up(part_bytes(m, n, batch), 256) + round_up(counter_bytes(m, batch), 256) + kStatusBytes;
+  return round_up(part_bytes(m, n, batch), 256) + round_up(counter_bytes(m, batch), 256) + kTileCounterBytes +
+         kStatusBytes;
 }
 
 int lutgemm_pack_bcq(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* status_flags,
@@ -179,13 +182,26 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   const size_t cnt_off = round_up(part_bytes(m, n, batch), 256);
   p.part = reinterpret_cast<float*>(ws);
   p.cnt = reinterpret_cast<unsigned*>(ws + cnt_off);
-  p.status = reinterpret_cast<unsigned*>(ws + cnt_off + round_up(counter_bytes(m, batch), 256));
+  const size_t tile_off = cnt_off + round_up(counter_bytes(m, batch), 256);
+  p.tile_cnt = reinterpret_cast<unsigned*>(ws + tile_off);
+  p.status = reinterpret_cast<unsigned*>(ws + tile_off + kTileCounterBytes);
 
   const RunKernel kernel = select_kernel(q, group_mode(g), offset != nullptr);
   int sm_count = 0;
   if (device_setup(kernel, &sm_count) != cudaSuccess) return LUTGEMM_ERR_CUDA;
-  const long long grid = p.total_units < sm_count ? p.total_units : (long long)sm_count;
-  kernel<<<(unsigned)grid, kThreads, kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  long long grid = 0;
+  choose_launch(sm_count, (long long)batch * p.ns, p.mt, &grid, &p.seg_aligned);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 

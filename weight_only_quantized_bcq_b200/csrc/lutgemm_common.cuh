@@ -25,17 +25,35 @@ constexpr int kHalfTableBytes = 256 * 64 * 4;       // 256 patterns x 64 run col
 constexpr int kTableBytes = 2 * kHalfTableBytes;    // both halves: 128 runs
 
 // Shared-memory map, in absolute addresses of the CTA's shared window.  The
-// tables start at 64 KB, so a table read address is a PRMT result (bytes 0-1:
-// column and pattern, bytes 2-3: zero) plus a compile-time immediate.  The
-// dynamic allocation starts at the window's base R0 (the reserved region,
-// at most a few KB) and is sized to reach kSmemEnd; [R0, 64 KB) is unused.
-constexpr uint32_t kTableBase = 0x10000;
-constexpr uint32_t kMiscBase = kTableBase + kTableBytes;            // run sums for offsets
-constexpr uint32_t kSmemEnd = kMiscBase + 2 * kRunsPerSlice * 4;
-constexpr int kSmemBytes = (int)kSmemEnd;                          // dynamic bytes requested
+// window starts with the 1 KB region the driver reserves on sm_100, so the
+// dynamic allocation begins at 0x400; the tables sit there, at a compile-time
+// address, so a table read is a PRMT result (bytes 0-1: column and pattern,
+// bytes 2-3: zero) plus an immediate.  After them: run sums for offsets, the
+// mbarriers of the weight rings, and one ring of TMA stages per warp.
+constexpr uint32_t kTableBase = 0x400;
+constexpr uint32_t kMiscBase = kTableBase + kTableBytes;           // chunk / run sums (1 KB)
+constexpr uint32_t kBarBase = kMiscBase + 1024;                    // 16 warps x <= 8 stages x 8 B
+constexpr uint32_t kRingBase = kBarBase + 1024;                    // weight rings
+constexpr uint32_t kSmemEnd = kTableBase + 227 * 1024;             // end of a 227 KB allocation
+constexpr uint32_t kRingBytesPerWarp = (kSmemEnd - kRingBase) / kWarps / 512 * 512;
+constexpr int kSmemBytes = (int)(kSmemEnd - kTableBase);           // dynamic bytes requested
 
-// Register pipeline depth: a lane keeps NB steps of loads, NB - 1 in flight.
-constexpr int pipeline_stages(int q) { return q <= 3 ? 4 : 2; }
+// Planes one step of a unit carries; steps per TMA copy (two while a ring of
+// two such copies fits a warp's share); TMA ring stages per warp (at most 8).
+__host__ __device__ constexpr int step_planes(int q) { return q < 4 ? q : 4; }
+__host__ __device__ constexpr int chunk_steps(int q) {
+  return 2u * 2u * 512u * step_planes(q) <= kRingBytesPerWarp ? 2 : 1;
+}
+// Stages fit the warp's share, and at most one unit (8 steps) ahead.
+__host__ __device__ constexpr int ring_stages(int q) {
+  return (int)(kRingBytesPerWarp / (512u * step_planes(q) * chunk_steps(q))) < 8 / chunk_steps(q)
+             ? (int)(kRingBytesPerWarp / (512u * step_planes(q) * chunk_steps(q)))
+             : 8 / chunk_steps(q);
+}
+
+// Per-segment tile counters for dynamic tile assignment (segment-aligned
+// mode); the last entry counts finished CTAs, so that the last one resets all.
+constexpr int kMaxTileCounters = 1024;
 
 // How the group size g maps onto the 128-input pieces a lane walks.
 enum GroupMode : int {
@@ -54,14 +72,74 @@ struct RunParams {
   void* y;                 // [batch][m], fp32 or fp16
   float* part;             // [batch][ns][mt*32] split-K partial sums
   unsigned* cnt;           // [batch][mt] arrival counters (zero between calls)
-  unsigned* status;        // sticky internal-error bits (1: shared window base above kTableBase)
+  unsigned* tile_cnt;      // [segments] tile counters of segment-aligned mode (zero between calls)
+  unsigned* status;        // sticky internal-error bits: 1 shared window base is not kTableBase,
+                           // 2 a weight-ring wait timed out (results invalid)
   int m, n, batch, q, g;
   int ns, mt, ng;
   int y_f16;
+  int seg_aligned;         // 1: CTAs grouped per segment; 0: unit list cut evenly
   long long total_units;   // batch * ns * mt
 };
 
+// Range [begin, end) of units of CTA c out of G: either a share of one
+// segment's row tiles (segment-aligned), or a contiguous cut of the list.
+__host__ __device__ inline void cta_range(long long c, long long G, long long segments, long long mt,
+                                          bool aligned, long long* begin, long long* end) {
+  if (aligned) {
+    const long long z = c * segments / G;
+    const long long c0 = (z * G + segments - 1) / segments, c1 = ((z + 1) * G + segments - 1) / segments;
+    const long long k = c - c0, cz = c1 - c0;
+    *begin = z * mt + k * mt / cz;
+    *end = z * mt + (k + 1) * mt / cz;
+  } else {
+    *begin = c * segments * mt / G;
+    *end = (c + 1) * segments * mt / G;
+  }
+}
+
+// Slowest CTA of the contiguous cut, in unit-times: ceil(units / 16 warps)
+// per segment touched plus a quarter for each table build.
+inline double contiguous_worst(long long G, long long segments, long long mt) {
+  double worst = 0.0;
+  for (long long c = 0; c < G; ++c) {
+    long long b, e;
+    cta_range(c, G, segments, mt, false, &b, &e);
+    double t = 0.0;
+    while (b < e) {
+      const long long seg_end = (b / mt + 1) * mt;
+      const long long k = (e < seg_end ? e : seg_end) - b;
+      t += (double)((k + kWarps - 1) / kWarps) + 0.25;
+      b += k;
+    }
+    if (t > worst) worst = t;
+  }
+  return worst;
+}
+
+// Launch geometry.  Segment-aligned mode gives every segment the same number
+// of CTAs, floor(grid / segments), whose warps share its tiles dynamically;
+// the SMs left over start the next kernel of the stream early (programmatic
+// launch).  It is chosen when its slowest group is no slower than the
+// slowest CTA of the contiguous cut over the full grid.
+inline void choose_launch(long long sms, long long segments, long long mt, long long* grid, int* aligned) {
+  const long long units = segments * mt;
+  const long long g = units < sms ? units : sms;
+  *grid = g;
+  *aligned = 0;
+  if (segments > g || segments > kMaxTileCounters - 1) return;
+  const long long cz = g / segments;
+  const double t_aligned = (double)mt / (double)(cz * kWarps) + 0.25;
+  if (t_aligned <= contiguous_worst(g, segments, mt)) {
+    *grid = cz * segments;
+    *aligned = 1;
+  }
+}
+
 using RunKernel = void (*)(RunParams);
+
+constexpr unsigned kStatusWindow = 1u;
+constexpr unsigned kStatusTimeout = 2u;
 
 RunKernel run_kernel_q1(int mode, bool has_offset);
 RunKernel run_kernel_q2(int mode, bool has_offset);

@@ -8,16 +8,23 @@
 //
 // Design on B200 (148 SMs, 228 KB shared memory per SM, 128 B/clk shared
 // memory bandwidth per SM, HBM3e):
-//   * One persistent 512-thread CTA per SM.  The work is the linear list of
-//     units (batch column, slice, 32-row tile), cut into one contiguous range
-//     per CTA.  A range crosses at most a few (batch column, slice) segments;
-//     the CTA rebuilds the 128 KB fp32 tables of a slice once per segment.
-//   * A warp processes a unit, one output row per lane.  Per step U (8 steps
-//     per unit) a lane reads one 16-byte piece per plane with a streaming
-//     128-bit load; the packed layout makes each warp load 512 contiguous
-//     bytes.  Loads run NB-1 steps ahead in registers, across unit
-//     boundaries; a warp's first loads of a segment are issued before the
-//     table build so that their latency overlaps it.
+//   * One persistent 512-thread CTA per SM.  The work is the list of units
+//     (batch column, slice, 32-row tile).  Either every (batch column, slice)
+//     segment gets its own group of CTAs that share its tiles round-robin, or
+//     the list is cut into one contiguous range per CTA, whichever the host
+//     finds better balanced.  A CTA builds the 128 KB fp32 tables of a slice
+//     once per segment it touches.
+//   * A warp processes a unit, one output row per lane, in 8 steps.  Warp w
+//     takes the CTA's tiles w, w+16, w+32, ... of a segment.
+//   * Weights move by TMA: the q pieces of all 32 lanes of a step are q*512
+//     contiguous bytes of the packed layout, and CH consecutive steps (CH = 2
+//     for q <= 3) are fetched by one cp.async.bulk into a per-warp ring of S
+//     shared-memory stages (one mbarrier each), S copies ahead and across
+//     unit boundaries; a warp's first copies of a segment are issued before
+//     the table build.  Every wait is bounded in time; a timeout sets a
+//     status bit instead of hanging.  At a stage's first step each lane reads
+//     its 16-byte pieces of all the stage's steps (one LDS.128 each) and the
+//     stage is refilled at once, so S copies stay in flight during compute.
 //   * Table reads are conflict-free: at every step the 32 lanes read 32
 //     distinct banks.  Lanes 0-15 and 16-31 walk the 8 pieces of the slice
 //     four apart, and lane l reads the runs of its piece in the order
@@ -26,7 +33,8 @@
 //     256) next to the lane's column byte, one LDS whose immediate carries the
 //     table base, half and band, and one FADD.
 //   * Per-group alpha (and offset) are applied once per piece (g = 128),
-//     per half-piece (g = 64) or per run (other g).
+//     per half-piece (g = 64) or per run (other g); the per-piece values are
+//     prefetched three steps ahead in registers.
 //   * Split-K: each unit stores its fp32 partial.  When a warp has finished
 //     its units of a segment it fences once and bumps the arrival counters of
 //     those row tiles (one lane per tile); the last arrival for a tile (no
@@ -60,12 +68,12 @@ __device__ __forceinline__ void sts_at(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-// 16 bytes of packed planes; each byte is read exactly once, so skip L1.
-__device__ __forceinline__ uint4 ld_stream16(const uint8_t* ptr) {
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(ptr));
+               : "r"(addr)
+               : "memory");
   return v;
 }
 
@@ -77,6 +85,47 @@ __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int k) {
   return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred P;\n mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n selp.u32 %0, 1, 0, P;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier; give up after about one second.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try(bar, parity)) {
+    if (global_ns() - t0 > 1000000000ull) return false;
+  }
+  return true;
+}
+
+// One TMA bulk copy of `bytes` (a multiple of 16) from global memory into this
+// CTA's shared memory, completing on mbarrier `bar`.  The proxy fence orders
+// the warp's earlier generic reads of the stage before the copy overwrites it.
+__device__ __forceinline__ void tma_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // PRMT selector for byte t of a stored word: result byte 0 <- column byte t of
@@ -169,17 +218,29 @@ __device__ __forceinline__ void static_for(std::integer_sequence<int, Is...>, F&
 
 }  // namespace detail
 
-template <int Q, int MODE, bool MULTI, bool HAS_OFF, int NB>
+template <int Q, int MODE, bool MULTI, bool HAS_OFF>
 __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p) {
   using namespace detail;
-  static_assert(NB == 2 || NB == 4 || NB == 8, "pipeline stages must divide the 8 steps of a unit");
+  constexpr int SP = step_planes(MULTI ? 8 : Q);       // planes in one step (<= 4)
+  constexpr int CH = chunk_steps(MULTI ? 8 : Q);       // steps per TMA copy
+  constexpr int S = ring_stages(MULTI ? 8 : Q);        // TMA stages per warp
+  constexpr uint32_t STEP_BYTES = 512u * SP;
+  constexpr uint32_t STAGE_BYTES = STEP_BYTES * CH;
+  static_assert(!MULTI || CH == 1, "plane groups are fetched one step at a time");
+  constexpr int NA = 4;                                // alpha register stages (3 steps ahead)
+  static_assert(S >= 2 && S <= 8, "weight ring of 2..8 stages");
+
   extern __shared__ __align__(16) unsigned char smem[];
+  // Let the next kernel in the stream start on SMs as they free up; it waits
+  // for this grid's completion before touching anything this grid writes.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t r0 = (uint32_t)__cvta_generic_to_shared(smem);
-  if (r0 > kTableBase) {  // uniform over the CTA: the tables would not fit the allocation
-    if (threadIdx.x == 0) atomicOr(p.status, 1u);
+  if (r0 != kTableBase) {  // uniform over the CTA: the map would not match the allocation
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusWindow);
     return;
   }
-  float* const chunk_sum = reinterpret_cast<float*>(smem + (kMiscBase - r0));
+  float* const chunk_sum = reinterpret_cast<float*>(smem + (kMiscBase - kTableBase));
   float* const run_sum = chunk_sum + kRunsPerSlice;
 
   // Runs (8-input table columns) that share one alpha inside a piece.
@@ -208,39 +269,106 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     }
   }
 
+  // This warp's weight ring: S stages of STAGE_BYTES (CH steps), one mbarrier
+  // each.  (st, ph) is the stage to consume next and its phase parity; both
+  // run on across segments.  At a segment boundary every issued copy has been
+  // consumed.
+  const uint32_t ring = kRingBase + (uint32_t)warp * kRingBytesPerWarp;
+  const uint32_t bars = kBarBase + (uint32_t)warp * 64u;
+  if (lane == 0) {
+#pragma unroll
+    for (int st0 = 0; st0 < S; ++st0) mbar_init(bars + 8u * st0);
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncwarp();
+  int st = 0;
+  uint32_t ph = 0;
+  bool failed = false;     // a ring wait timed out: stop streaming, keep taking the CTA barriers
+  int outstanding = 0;     // copies issued and not yet consumed
+
   const int npg = MULTI ? (p.q + 3) >> 2 : 1;
+  const int steps_per_unit = 8 * npg;
   const size_t plane_stride = (size_t)p.ng * (size_t)p.m;
   const uint32_t unit_bytes = (uint32_t)p.q * kBlockBytes;
 
-  const long long total = p.total_units;
-  const long long u_begin = (long long)blockIdx.x * total / gridDim.x;
-  const long long u_end = (long long)(blockIdx.x + 1) * total / gridDim.x;
+  // Work of this CTA.  Segment-aligned: one segment z, whose row tiles its
+  // cz CTAs share round-robin (CTA k takes tiles k, k+cz, ...), so that every
+  // CTA's reads spread over the whole segment.  Otherwise: a contiguous range
+  // [u_begin, u_end) of the unit list, visited segment by segment.
+  const long long Z = (long long)p.batch * p.ns;
+  long long u_begin = 0, u_end = 0, a_seg = 0, a_first = 0, a_stride = 1;
+  if (p.seg_aligned) {
+    // Segment z gets the CTAs c = z, z + Z, z + 2Z, ...: a group spread over
+    // the whole grid rather than a block of neighbouring CTAs.
+    const long long G = gridDim.x, c = blockIdx.x;
+    a_seg = c % Z;
+    a_first = c / Z;
+    a_stride = (G - a_seg + Z - 1) / Z;
+  } else {
+    cta_range(blockIdx.x, gridDim.x, Z, p.mt, false, &u_begin, &u_end);
+  }
 
-  uint4 wb[NB][Q];
-  uint16_t ab[NB][Q][APP];
-  float ob[NB][APP];
+  uint16_t ab[NA][Q][APP];
+  float ob[NA][APP];
+  uint4 wst[CH][SP];       // the pieces of the current ring stage
 
-  for (long long u = u_begin; u < u_end;) {
-    const long long seg = u / p.mt;
+  auto group_size = [&](long long z) { return (long long)((gridDim.x - z + Z - 1) / Z); };
+
+  for (int visit = 0;; ++visit) {
+    // Segment-aligned mode visits the CTA's own segment once; the contiguous
+    // mode visits the segments of its range in order.
+    long long seg, tile_first = 0, tile_stride = 1, tile_count = 0;
+    if (p.seg_aligned) {
+      if (visit > 0) break;
+      seg = a_seg;
+      tile_first = a_first;
+      tile_stride = a_stride;
+      tile_count = a_first < p.mt ? (p.mt - 1 - a_first) / a_stride + 1 : 0;
+    } else {
+      if (u_begin >= u_end) break;
+      seg = u_begin / p.mt;
+      const long long seg_end = min(u_end, (seg + 1) * p.mt);
+      tile_first = u_begin - seg * p.mt;
+      tile_stride = 1;
+      tile_count = seg_end - u_begin;
+      u_begin = seg_end;
+    }
     const int b = (int)(seg / p.ns);
     const int s = (int)(seg - (long long)b * p.ns);
-    const long long seg_first = seg * p.mt;
-    const long long seg_end = min(u_end, seg_first + p.mt);
     const uint8_t* slice_base = p.packed + (size_t)s * p.mt * unit_bytes;
-    const long long first_unit = u + warp;
-    const bool busy = first_unit < seg_end;
+    // This warp's row tiles.  In the contiguous mode: indices warp, warp+16,
+    // ... of the CTA's tiles (tile_first + index * tile_stride).  In
+    // segment-aligned mode the G_z CTAs of a segment take two static tiles per
+    // warp, covering tiles [0, 32 G_z); all further tiles come from the
+    // segment's tile counter, grabbed one tile ahead by lane 0, so the group's
+    // warps share out the rest as they finish.  The last CTA to finish the
+    // kernel resets the counters for the next call.
+    const bool dyn = p.seg_aligned != 0;
+    auto static_tile = [&](int k) -> int {
+      const long long idx = (long long)warp + (long long)k * kWarps;
+      return idx < tile_count ? (int)(tile_first + idx * tile_stride) : -1;
+    };
+    unsigned* const tile_ctr = p.tile_cnt + seg;
+    const long long dyn_base = dyn ? 32 * group_size(seg) : 0;
+    int t_cur = failed ? -1 : static_tile(0);
+    int t_nxt = static_tile(1);
+    const bool busy = t_cur >= 0;
+    constexpr int CPT = 8 / CH;                      // ring chunks per unit and plane group
+    const int chunks_per_unit = CPT * npg;
 
-    // Loads of one step into stage SLOT: the Q 16-byte pieces and, when
-    // prefetched, the alpha (and offset) values the step will need.
-    auto load_step = [&]<int SLOT>(int R_, int pg_, int U_) {
-      const uint8_t* src = slice_base + ((size_t)R_ * p.q + (size_t)pg_ * 4) * kBlockBytes +
-                           U_ * 512 + lane * 16;
-#pragma unroll
-      for (int i = 0; i < Q; ++i) {
-        const bool live = !MULTI || (pg_ * 4 + i < p.q);
-        if (live) wb[SLOT][i] = ld_stream16(src + (size_t)i * kBlockBytes);
-      }
+    // TMA copy of chunk c (steps c*CH .. c*CH+CH-1) of row tile R into ring
+    // stage `stage` (lane 0 only).  The CH steps are contiguous.
+    auto issue = [&](int R_, int c, int stage) {
+      const int pg_ = c / CPT, U_ = (c - pg_ * CPT) * CH;
+      const int planes = MULTI ? min(4, p.q - 4 * pg_) : Q;
+      const uint8_t* src = slice_base + (size_t)R_ * unit_bytes + ((size_t)U_ * p.q + 4 * pg_) * 512;
+      tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * planes * CH, bars + 8u * stage);
+    };
+
+    // Per-piece scales (and offsets) of step j of row tile R into register stage SLOT.
+    auto load_alpha = [&]<int SLOT>(int R_, int j) {
       if constexpr (PRE_ALPHA) {
+        const int pg_ = j >> 3, U_ = j & 7;
         const int row = R_ * kTileRows + lane;
         const int P = U_ ^ (int)(4 * a);
 #pragma unroll
@@ -261,154 +389,272 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
       }
     };
 
-    // The first NB-1 steps of this warp's first unit go out before the tables
-    // are built; they do not touch shared memory.
-    int R = busy ? (int)(first_unit - seg_first) : 0;
-    if (busy)
-      static_for(std::make_integer_sequence<int, NB - 1>{}, [&]<int D>() { load_step.template operator()<D>(R, 0, D); });
+    // The first S copies of the first tile go out before the tables are built.
+    if (busy && lane == 0) {
+      int st2 = st;
+      for (int c = 0; c < S; ++c) {
+        issue(t_cur, c, st2);
+        st2 = st2 + 1 == S ? 0 : st2 + 1;
+      }
+    }
+    if (busy) outstanding = S;
+    // Programmatic dependent launch: everything above reads only the weights.
+    // x, y and the workspace may belong to the previous kernel in the stream,
+    // so wait for it to complete before the first touch (a no-op otherwise).
+    if (visit == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();  // every warp is done with the previous segment's tables
     build_tables<RUN, HAS_OFF>(p, b, s, chunk_sum, run_sum);
 
     if (busy) {
-      long long unit = first_unit;
-      int pg = 0;
-      float yacc = 0.f;
-      while (true) {
-        int next_pg = pg + 1;
-        long long next_unit = unit;
-        if (next_pg >= npg) {
-          next_pg = 0;
-          next_unit = unit + kWarps;
-        }
-        const bool has_next = next_unit < seg_end;
-        const int next_R = has_next ? (int)(next_unit - seg_first) : 0;
-        const int row = R * kTileRows + lane;
+      static_for(std::make_integer_sequence<int, NA - 1>{}, [&]<int D>() {
+        load_alpha.template operator()<D>(t_cur, D);
+      });
+      const int steps_per_unit_ = steps_per_unit;
+      int my_tile = 0;        // lane k holds the tile of this warp's k-th unpublished partial
+      int ntiles = 0;
+      bool more = dyn;        // grabs may still succeed
+      unsigned pend = 0;      // lane 0: raw count returned by the pending grab
 
-        static_for(std::make_integer_sequence<int, 8>{}, [&]<int U>() {
-          constexpr int LU = U + NB - 1;          // step whose loads are issued now
-          if constexpr (LU < 8) load_step.template operator()<LU % NB>(R, pg, LU);
-          else if (has_next) load_step.template operator()<LU % NB>(next_R, next_pg, LU - 8);
-
-          constexpr uint32_t IMM = step_imm<U>();
-          constexpr int u2 = U >> 2;
-          const int P = U ^ (int)(4 * a);
+      // Split-K arrival for the first `n` tiles held in my_tile: one fence for
+      // their partials, then one lane per tile bumps the tile's counter; the
+      // last arrival sums the slices in slice order, writes y and resets it.
+      auto publish = [&](int n) {
+        __threadfence();
+        unsigned prev = 0;
+        if (lane < n) prev = atomicAdd(p.cnt + (size_t)b * p.mt + my_tile, 1u);
+        unsigned last = __ballot_sync(0xffffffffu, lane < n && prev == (unsigned)(p.ns - 1));
+        if (last) __threadfence();
+        // Sum the tiles this warp closed, up to 4 at a time, with the loads of
+        // 4 slices x 4 tiles in flight together (lane = row of the tile).
+        const size_t stride = (size_t)p.mt * kTileRows;
+        while (last) {
+          int Rt[4];
+          int nt = 0;
 #pragma unroll
-          for (int i = 0; i < Q; ++i) {
-            if (MULTI && pg * 4 + i >= p.q) continue;
-            const uint4 w4 = wb[U % NB][i];
-            if constexpr (RUN == 16) {
-              float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-              for (int k = 0; k < 4; ++k) lookup_word<IMM>(word_of(w4, k), colb[u2][k], acc0, acc1);
-              yacc = fmaf(h2f(ab[U % NB][i][0]), acc0 + acc1, yacc);
-            } else if constexpr (RUN == 8) {
-#pragma unroll
-              for (int r = 0; r < 2; ++r) {
-                float acc0 = 0.f, acc1 = 0.f;
-                lookup_word<IMM>(word_of(w4, 2 * r), colb[u2][2 * r], acc0, acc1);
-                lookup_word<IMM>(word_of(w4, 2 * r + 1), colb[u2][2 * r + 1], acc0, acc1);
-                yacc = fmaf(h2f(ab[U % NB][i][r]), acc0 + acc1, yacc);
-              }
-            } else {
-              // One scale per run: group of run c is (1024 s + 8 c) / g.
-              const __half* ap = p.alpha + (size_t)(pg * 4 + i) * plane_stride + row;
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                float v[4];
-                lookup_word_values<IMM>(word_of(w4, k), colb[u2][k], v);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  const int c = 16 * P + ((4 * k + t) ^ (int)lam);
-                  const int G = MODE == kG8 ? 128 * s + c : (s * kSliceInputs + 8 * c) / p.g;
-                  const float al = (row < p.m && G < p.ng) ? h2f(ld_u16(ap + (size_t)G * p.m)) : 0.f;
-                  yacc = fmaf(al, v[t], yacc);
-                }
-              }
+          for (int e = 0; e < 4; ++e) {
+            Rt[e] = -1;
+            if (last) {
+              const int src_lane = __ffs(last) - 1;
+              last &= last - 1;
+              Rt[e] = __shfl_sync(0xffffffffu, my_tile, src_lane);
+              ++nt;
             }
           }
-          // Offset of converted uniform weights: offset[G][row] * (sum of x over the run).
-          if constexpr (HAS_OFF) {
-            if (pg == 0) {
-              if constexpr (RUN >= 8) {
+          float sum[4];
+          const float* col[4];
 #pragma unroll
-                for (int r = 0; r < APP; ++r) {
-                  const int nat = RUN == 16 ? P : 2 * P + (r ^ (int)(lam >> 3));
-                  yacc = fmaf(ob[U % NB][r], run_sum[nat], yacc);
+          for (int e = 0; e < 4; ++e) {
+            sum[e] = 0.f;
+            col[e] = p.part + ((size_t)b * p.ns * p.mt + (Rt[e] < 0 ? Rt[0] : Rt[e])) * kTileRows + lane;
+          }
+          int s2 = 0;
+          for (; s2 + 4 <= p.ns; s2 += 4) {
+            float v[4][4];
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) v[d][e] = e < nt ? __ldcg(col[e] + (size_t)(s2 + d) * stride) : 0.f;
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) sum[e] += v[d][e];
+          }
+          for (; s2 < p.ns; ++s2)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (e < nt) sum[e] += __ldcg(col[e] + (size_t)s2 * stride);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (e >= nt) continue;
+            const int row = Rt[e] * kTileRows + lane;
+            if (row < p.m) {
+              const size_t o = (size_t)b * p.m + row;
+              if (p.y_f16) reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(sum[e]);
+              else reinterpret_cast<float*>(p.y)[o] = sum[e];
+            }
+            if (lane == 0) p.cnt[(size_t)b * p.mt + Rt[e]] = 0u;
+          }
+        }
+      };
+
+      for (int k = 0; !failed; ++k) {
+        // Tile k is t_cur, tile k+1 is t_nxt (or none).  Grab tile k+2 now.
+        const bool grabbing = dyn && more && t_nxt >= 0;
+        if (grabbing && lane == 0) pend = atomicAdd(tile_ctr, 1u);
+        const int R = t_cur;
+        const int row = R * kTileRows + lane;
+        float yacc = 0.f;
+        for (int pg = 0; pg < npg && !failed; ++pg) {
+          static_for(std::make_integer_sequence<int, 8>{}, [&]<int U>() {
+            if (failed) return;
+            const int j = pg * 8 + U;          // step within the unit
+            {
+              const int ja = j + NA - 1;       // alpha three steps ahead
+              if (ja < steps_per_unit_) load_alpha.template operator()<(U + NA - 1) % NA>(t_cur, ja);
+              else if (t_nxt >= 0) load_alpha.template operator()<(U + NA - 1) % NA>(t_nxt, ja - steps_per_unit_);
+            }
+
+            // Pieces of a whole stage (CH steps) come out of the ring at its
+            // first step; the stage is refilled (S copies ahead) right away, so
+            // S full copies are in flight while the steps are computed.
+            if constexpr (U % CH == 0) {
+              const bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8u * st, ph));
+              if (!ok) {
+                failed = true;
+                if (lane == 0) atomicOr(p.status, kStatusTimeout);
+                return;
+              }
+              const uint32_t src = ring + (uint32_t)st * STAGE_BYTES + (uint32_t)lane * 16u;
+#pragma unroll
+              for (int h = 0; h < CH; ++h)
+#pragma unroll
+                for (int i = 0; i < SP; ++i) {
+                  const bool live = !MULTI || (pg * 4 + i < p.q);
+                  wst[h][i] = live ? lds128(src + (uint32_t)h * STEP_BYTES + 512u * i) : make_uint4(0, 0, 0, 0);
+                }
+              __syncwarp();
+              const int cn = j / CH + S;       // chunk to fetch into the freed stage
+              if (cn < chunks_per_unit) {
+                if (lane == 0) issue(t_cur, cn, st);
+              } else if (t_nxt >= 0) {
+                if (lane == 0) issue(t_nxt, cn - chunks_per_unit, st);
+              } else {
+                --outstanding;
+              }
+              st = st + 1 == S ? 0 : st + 1;
+              if (st == 0) ph ^= 1u;
+            }
+            const uint4 (&wv)[SP] = wst[U % CH];
+
+            constexpr uint32_t IMM = step_imm<U>();
+            constexpr int u2 = U >> 2;
+            const int P = U ^ (int)(4 * a);
+#pragma unroll
+            for (int i = 0; i < Q; ++i) {
+              if (MULTI && pg * 4 + i >= p.q) continue;
+              const uint4 w4 = wv[i];
+              if constexpr (RUN == 16) {
+                float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) lookup_word<IMM>(word_of(w4, kk), colb[u2][kk], acc0, acc1);
+                yacc = fmaf(h2f(ab[U % NA][i][0]), acc0 + acc1, yacc);
+              } else if constexpr (RUN == 8) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                  float acc0 = 0.f, acc1 = 0.f;
+                  lookup_word<IMM>(word_of(w4, 2 * r), colb[u2][2 * r], acc0, acc1);
+                  lookup_word<IMM>(word_of(w4, 2 * r + 1), colb[u2][2 * r + 1], acc0, acc1);
+                  yacc = fmaf(h2f(ab[U % NA][i][r]), acc0 + acc1, yacc);
                 }
               } else {
+                // One scale per run: group of run c is (1024 s + 8 c) / g.
+                const __half* ap = p.alpha + (size_t)(pg * 4 + i) * plane_stride + row;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  const int c = 16 * P + (j ^ (int)lam);
-                  const int G = MODE == kG8 ? 128 * s + c : (s * kSliceInputs + 8 * c) / p.g;
-                  const float of = (row < p.m && G < p.ng) ? __ldg(p.offset + (size_t)G * p.m + row) : 0.f;
-                  yacc = fmaf(of, chunk_sum[c], yacc);
+                for (int kk = 0; kk < 4; ++kk) {
+                  float v[4];
+                  lookup_word_values<IMM>(word_of(w4, kk), colb[u2][kk], v);
+#pragma unroll
+                  for (int t = 0; t < 4; ++t) {
+                    const int c = 16 * P + ((4 * kk + t) ^ (int)lam);
+                    const int G = MODE == kG8 ? 128 * s + c : (s * kSliceInputs + 8 * c) / p.g;
+                    const float al = (row < p.m && G < p.ng) ? h2f(ld_u16(ap + (size_t)G * p.m)) : 0.f;
+                    yacc = fmaf(al, v[t], yacc);
+                  }
                 }
               }
             }
-          }
-        });
-
-        if (pg == npg - 1) {
-          // This slice's partial sum of the row tile; published below.
-          p.part[((size_t)((long long)b * p.ns + s) * p.mt + R) * kTileRows + lane] = yacc;
-          yacc = 0.f;
+            // Offset of converted uniform weights: offset[G][row] * (sum of x over the run).
+            if constexpr (HAS_OFF) {
+              if (pg == 0) {
+                if constexpr (RUN >= 8) {
+#pragma unroll
+                  for (int r = 0; r < APP; ++r) {
+                    const int nat = RUN == 16 ? P : 2 * P + (r ^ (int)(lam >> 3));
+                    yacc = fmaf(ob[U % NA][r], run_sum[nat], yacc);
+                  }
+                } else {
+#pragma unroll
+                  for (int jj = 0; jj < 16; ++jj) {
+                    const int c = 16 * P + (jj ^ (int)lam);
+                    const int G = MODE == kG8 ? 128 * s + c : (s * kSliceInputs + 8 * c) / p.g;
+                    const float of = (row < p.m && G < p.ng) ? __ldg(p.offset + (size_t)G * p.m + row) : 0.f;
+                    yacc = fmaf(of, chunk_sum[c], yacc);
+                  }
+                }
+              }
+            }
+          });
         }
-        if (!has_next) break;
-        unit = next_unit;
-        R = next_R;
-        pg = next_pg;
+        if (failed) break;
+        // This slice's partial sum of the row tile; published in batches of 32.
+        p.part[((size_t)((long long)b * p.ns + s) * p.mt + R) * kTileRows + lane] = yacc;
+        if (lane == ntiles) my_tile = R;
+        if (++ntiles == 32) {
+          publish(32);
+          ntiles = 0;
+        }
+
+        // Advance: tile k+2 comes from the grab (dynamic) or the static list.
+        if (t_nxt < 0) break;
+        int t_after = -1;
+        if (dyn) {
+          if (grabbing) {
+            int tile = -1;
+            if (lane == 0) {
+              const long long t = dyn_base + pend;
+              tile = t < p.mt ? (int)t : -1;
+            }
+            t_after = __shfl_sync(0xffffffffu, tile, 0);
+            more = t_after >= 0;
+          }
+        } else {
+          t_after = static_tile(k + 2);
+        }
+        t_cur = t_nxt;
+        t_nxt = t_after;
       }
+      if (!failed && ntiles > 0) publish(ntiles);
+    }
+  }
 
-      // Split-K arrival: one fence for all of this warp's partials, then one
-      // lane per row tile bumps the tile's counter.  The last arrival sums the
-      // slices in slice order, writes y and resets the counter.
+  // Segment-aligned mode: the last CTA to finish resets the tile counters.
+  if (p.seg_aligned) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned* done = p.tile_cnt + (kMaxTileCounters - 1);
       __threadfence();
-      const int nunits = (int)((seg_end - 1 - first_unit) / kWarps) + 1;
-      for (int k0 = 0; k0 < nunits; k0 += 32) {
-        const int k = k0 + lane;
-        int Rk = 0;
-        unsigned prev = 0;
-        if (k < nunits) {
-          Rk = (int)(first_unit + (long long)k * kWarps - seg_first);
-          prev = atomicAdd(p.cnt + (size_t)b * p.mt + Rk, 1u);
-        }
-        unsigned last = __ballot_sync(0xffffffffu, k < nunits && prev == (unsigned)(p.ns - 1));
-        if (last) __threadfence();
-        while (last) {
-          const int src = __ffs(last) - 1;
-          last &= last - 1;
-          const int Rt = __shfl_sync(0xffffffffu, Rk, src);
-          const float* col = p.part + ((size_t)b * p.ns * p.mt + Rt) * kTileRows + lane;
-          float sum = 0.f;
-          for (int s2 = 0; s2 < p.ns; ++s2) sum += __ldcg(col + (size_t)s2 * p.mt * kTileRows);
-          const int row = Rt * kTileRows + lane;
-          if (row < p.m) {
-            const size_t o = (size_t)b * p.m + row;
-            if (p.y_f16) reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(sum);
-            else reinterpret_cast<float*>(p.y)[o] = sum;
-          }
-          if (lane == 0) p.cnt[(size_t)b * p.mt + Rt] = 0u;
-        }
+      if (atomicAdd(done, 1u) == gridDim.x - 1) {
+        for (long long z = 0; z < Z; ++z) p.tile_cnt[z] = 0u;
+        *done = 0u;
       }
     }
-    u = seg_end;
+  }
+
+  // After a timeout, let copies still in flight land before the CTA exits
+  // (each wait bounded again).
+  if (failed) {
+    for (int k = 0; k < outstanding; ++k) {
+      (void)mbar_wait(bars + 8u * st, ph);
+      st = st + 1 == S ? 0 : st + 1;
+      if (st == 0) ph ^= 1u;
+    }
   }
 }
 
-#define LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, OFFv, NBv)                              \
+#define LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, OFFv)                                   \
   switch (mode) {                                                                  \
-    case kG128: return lut_gemm_kernel<Qv, kG128, MULTIv, OFFv, NBv>;              \
-    case kG128x: return lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv, NBv>;            \
-    case kG64: return lut_gemm_kernel<Qv, kG64, MULTIv, OFFv, NBv>;                \
-    case kG8: return lut_gemm_kernel<Qv, kG8, MULTIv, OFFv, NBv>;                  \
-    default: return lut_gemm_kernel<Qv, kGAny, MULTIv, OFFv, NBv>;                 \
+    case kG128: return lut_gemm_kernel<Qv, kG128, MULTIv, OFFv>;                   \
+    case kG128x: return lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv>;                 \
+    case kG64: return lut_gemm_kernel<Qv, kG64, MULTIv, OFFv>;                     \
+    case kG8: return lut_gemm_kernel<Qv, kG8, MULTIv, OFFv>;                       \
+    default: return lut_gemm_kernel<Qv, kGAny, MULTIv, OFFv>;                      \
   }
 
-#define LUTGEMM_RUN_SELECT(Qv, MULTIv, NBv)                                        \
+#define LUTGEMM_RUN_SELECT(Qv, MULTIv)                                             \
   if (has_offset) {                                                                \
-    LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, true, NBv)                                  \
+    LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, true)                                       \
   } else {                                                                         \
-    LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, false, NBv)                                 \
+    LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, false)                                      \
   }
 
 }  // namespace lutgemm

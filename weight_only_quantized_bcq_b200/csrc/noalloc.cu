@@ -11,8 +11,9 @@
 // is loaded holds its LUTGEMM_NOALLOC_SCRATCH_BYTES until the process exits.
 // Layout (fixed, independent of the problem size):
 //   [0, 256)              status word (sticky internal-error bits)
-//   [256, 256 + 256 KB)   split-K arrival counters, zero between calls
-//   [256 + 256 KB, end)   split-K partial sums, written before they are read
+//   [256, +256 KB)        split-K arrival counters, zero between calls
+//   [.., +4 KB)           per-segment tile counters, zero between calls
+//   [.., end)             split-K partial sums, written before they are read
 // The counters sit at a fixed place so that they are never overlaid by
 // another call's partial sums; the kernel resets every counter it uses, and
 // the first call on a device zeroes them once.  Every call shares the array,
@@ -33,7 +34,8 @@ constexpr size_t kScratchBytes = LUTGEMM_NOALLOC_SCRATCH_BYTES;
 constexpr size_t kStatusOff = 0;
 constexpr size_t kCounterOff = 256;
 constexpr size_t kCounterBytes = 256 * 1024;
-constexpr size_t kPartOff = kCounterOff + kCounterBytes;
+constexpr size_t kTileCounterOff = kCounterOff + kCounterBytes;
+constexpr size_t kPartOff = kTileCounterOff + kMaxTileCounters * sizeof(unsigned);
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
@@ -82,7 +84,7 @@ cudaError_t prepare(RunKernel kernel, cudaStream_t stream, DeviceScratch* out) {
       return err;
     if ((err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
       return err;
-    if ((unsigned)reserved > kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
+    if ((unsigned)reserved != kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
     err = cudaMemsetAsync(ptr, 0, kPartOff, stream);
     if (err != cudaSuccess) return err;
     d.base = static_cast<unsigned char*>(ptr);
@@ -132,6 +134,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   p.y = y;
   p.part = reinterpret_cast<float*>(d.base + kPartOff);
   p.cnt = reinterpret_cast<unsigned*>(d.base + kCounterOff);
+  p.tile_cnt = reinterpret_cast<unsigned*>(d.base + kTileCounterOff);
   p.status = reinterpret_cast<unsigned*>(d.base + kStatusOff);
   p.m = m;
   p.n = n;
@@ -143,7 +146,18 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   p.ng = n / g;
   p.y_f16 = y_f16 ? 1 : 0;
   p.total_units = (long long)batch * ns * mt;
-  const long long grid = p.total_units < d.sm_count ? p.total_units : (long long)d.sm_count;
-  kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(p);
+  long long grid = 0;
+  choose_launch(d.sm_count, (long long)batch * ns, mt, &grid, &p.seg_aligned);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }

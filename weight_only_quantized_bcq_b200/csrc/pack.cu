@@ -6,7 +6,7 @@
 // scales; "One format for many schemes": uniform quantisation is a special
 // case of BCQ).  The layout is defined in include/lutgemm.h.
 //
-// One thread writes one 16-byte lane piece: block (s, R, i), step U, lane l.
+// One thread writes one 16-byte lane piece: chunk (s, R, U, i), lane l.
 // Byte j of the piece holds inputs 1024 s + 128 P + 8 c .. +7 of row 32R + l
 // with P = U xor 4*(l/16), c = j xor (l%16).  The 8 source bytes of a byte are
 // contiguous, so each is one 8-byte load.
@@ -37,11 +37,12 @@ __global__ void pack_signs_kernel(const int8_t* __restrict__ signs, int q, int m
                                   long long nthreads, uint8_t* __restrict__ packed, int32_t* flags) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid >= nthreads) return;
-  const long long blk = tid >> 8;            // block index ((s*mt + R)*q + i)
-  const int within = (int)(tid & 255);
-  const int U = within >> 5, l = within & 31;
-  const int i = (int)(blk % q);
-  const long long sR = blk / q;
+  const long long chunk = tid >> 5;          // (((s*mt + R)*8 + U)*q + i)
+  const int l = (int)(tid & 31);
+  const int i = (int)(chunk % q);
+  const long long sRU = chunk / q;
+  const int U = (int)(sRU & 7);
+  const long long sR = sRU >> 3;
   const int R = (int)(sR % mt);
   const int s = (int)(sR / mt);
   const int r = R * kTileRows + l;
@@ -59,8 +60,7 @@ __global__ void pack_signs_kernel(const int8_t* __restrict__ signs, int q, int m
       }
     }
   }
-  *reinterpret_cast<uint4*>(packed + blk * kBlockBytes + U * 512 + l * 16) =
-      make_uint4(words[0], words[1], words[2], words[3]);
+  *reinterpret_cast<uint4*>(packed + chunk * 512 + l * 16) = make_uint4(words[0], words[1], words[2], words[3]);
   if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_SIGN);
 }
 
@@ -69,9 +69,10 @@ __global__ void pack_codes_kernel(const uint8_t* __restrict__ codes, int q, int 
                                   long long nthreads, uint8_t* __restrict__ packed, int32_t* flags) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid >= nthreads) return;
-  const long long sR = tid >> 8;             // (s*mt + R)
-  const int within = (int)(tid & 255);
-  const int U = within >> 5, l = within & 31;
+  const long long sRU = tid >> 5;            // ((s*mt + R)*8 + U)
+  const int l = (int)(tid & 31);
+  const int U = (int)(sRU & 7);
+  const long long sR = sRU >> 3;
   const int R = (int)(sR % mt);
   const int s = (int)(sR / mt);
   const int r = R * kTileRows + l;
@@ -102,7 +103,7 @@ __global__ void pack_codes_kernel(const uint8_t* __restrict__ codes, int q, int 
     }
   }
   for (int i = 0; i < q; ++i) {
-    *reinterpret_cast<uint4*>(packed + (sR * q + i) * kBlockBytes + U * 512 + l * 16) =
+    *reinterpret_cast<uint4*>(packed + (sRU * q + i) * 512 + l * 16) =
         make_uint4(words[i][0], words[i][1], words[i][2], words[i][3]);
   }
   if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_CODE);
