@@ -98,9 +98,9 @@ const char* lutgemm_status_string(int status);
  * Pure host function. */
 size_t lutgemm_packed_bytes(int q, int m, int n);
 
-/* Bytes of the lutgemm_run workspace (split-K partial sums, per-row-tile
- * arrival counters, per-slice tile counters and a status word).  Returns 0
- * for invalid shapes.  Pure host function. */
+/* Bytes of the lutgemm_run workspace (split-K partial sums, per-slice tile
+ * counters and a status word).  Returns 0 for invalid shapes.  Pure host
+ * function. */
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g);
 
 /* Pack q planes of +-1 signs into the packed bit-plane layout above.
@@ -157,7 +157,9 @@ int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
  *   offset     dev fp32 [n/g][m] or NULL (pure BCQ), 4-byte aligned
  *   x          dev fp16 [batch][n], 16-byte aligned
  *   y          dev [batch][m] fp32 (4-byte aligned) or, with LUTGEMM_Y_F16,
- *              fp16 (2-byte aligned); fully overwritten
+ *              fp16 (2-byte aligned); fully overwritten.  For n > 1024 the
+ *   call enqueues two kernels: the lookup kernel writes per-slice partial
+ *   sums to the workspace and a reduce kernel adds them in slice order.
  *   flags      0 or LUTGEMM_Y_F16
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
  *              16-byte aligned, zero-filled before its first use; left
@@ -186,10 +188,9 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
  * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   Arguments, layouts and results are those of lutgemm_run, without the
  *   workspace.  Returns LUTGEMM_ERR_WORKSPACE when the problem needs more
- *   scratch than the array holds: more than 65536 row-tile counters
- *   (batch * ceil(m/32)) or more than 16 MiB - 260 KiB - 256 B of partial sums
- *   (batch * ceil(n/1024) * ceil(m/32) * 128 bytes).  Other statuses as for
- *   lutgemm_run.
+ *   scratch than the array holds: more than 16 MiB - 4 KiB - 256 B of
+ *   split-K partial sums (batch * ceil(n/1024) * ceil(m/32) * 128 bytes when
+ *   n > 1024).  Other statuses as for lutgemm_run.
  *   The first call on a device does a one-time set-up on that device (looks
  *   up the array's device address and zeroes its counters on `stream`); make
  *   that first call before any stream capture.  Every call shares the one

@@ -65,9 +65,8 @@ def test_workspace_size(L):
     m, n, b = 49152, 12288, 1
     ns, mt = math.ceil(n / 1024), math.ceil(m / 32)
     part = b * ns * mt * 32 * 4
-    cnt = b * mt * 4
     rup = lambda v: (v + 255) // 256 * 256
-    assert L.workspace_size(m, n, b, 3, 128) == rup(part) + rup(cnt) + 4096 + 256   # + tile counters, status
+    assert L.workspace_size(m, n, b, 3, 128) == rup(part) + 4096 + 256   # + tile counters, status word
     assert L.workspace_size(m, n, 0, 3, 128) == 0
     assert L.workspace_size(m, n, 1, 3, 100) == 0          # g % 8 != 0
     assert L.workspace_size(m, 12288, 1, 3, 5000) == 0     # n % g != 0

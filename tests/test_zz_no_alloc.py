@@ -11,6 +11,7 @@ to be collected last.
 from __future__ import annotations
 
 import ctypes
+import math
 
 import numpy as np
 import pytest
@@ -87,11 +88,17 @@ def test_noalloc_full_size_layer_linear_twice(L):
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch(L):
+    """Oversized problems are refused before anything is launched.
+
+    The pointers below are a 64-byte dummy, so every case is first checked on
+    the host to need more scratch than the array holds: a call that passed
+    validation would read far past them.
+    """
+    capacity = (16 << 20) - 4096 - 256
     small = torch.zeros(64, dtype=torch.uint8, device=DEV)
     p = ctypes.c_void_p(small.data_ptr())
-    # FC1 at batch 32 needs 75 MB of partial sums: more than the 16 MiB array.
-    st = L.lib().lutgemm_run_noalloc(49152, 12288, 32, 3, 128, p, p, None, p, p, 0, None)
-    assert st == L.ERR_WORKSPACE
-    # Too many row-tile counters (batch * ceil(m/32) > 65536).
-    st = L.lib().lutgemm_run_noalloc(32 * 65537, 8, 1, 1, 8, p, p, None, p, p, 0, None)
-    assert st == L.ERR_WORKSPACE
+    for (m, n, batch) in [(49152, 12288, 32), (12288, 49152, 8), (8192, 28672, 32)]:
+        need = batch * math.ceil(n / 1024) * math.ceil(m / 32) * 32 * 4
+        assert need > capacity, (m, n, batch, need)
+        st = L.lib().lutgemm_run_noalloc(m, n, batch, 3, 128, p, p, None, p, p, 0, None)
+        assert st == L.ERR_WORKSPACE

@@ -85,13 +85,11 @@ RunKernel select_kernel(int q, int mode, bool has_offset) {
   }
 }
 
-// Workspace: [split-K partials | arrival counters | tile counters | status word],
-// each part 256-byte aligned.
+// Workspace: [split-K partials | tile counters | status word], each part
+// 256-byte aligned.
 size_t part_bytes(int m, int n, int batch) {
   return (size_t)batch * ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * kTileRows * sizeof(float);
 }
-
-size_t counter_bytes(int m, int batch) { return (size_t)batch * ceil_div(m, kTileRows) * sizeof(unsigned); }
 
 constexpr size_t kStatusBytes = 256;
 constexpr size_t kTileCounterBytes = kMaxTileCounters * sizeof(unsigned);
@@ -122,8 +120,7 @@ size_t lutgemm_packed_bytes(int q, int m, int n) {
 
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g) {
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return 0;
-  return round_up(part_bytes(m, n, batch), 256) + round_up(counter_bytes(m, batch), 256) + kTileCounterBytes +
-         kStatusBytes;
+  return round_up(part_bytes(m, n, batch), 256) + kTileCounterBytes + kStatusBytes;
 }
 
 int lutgemm_pack_bcq(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* status_flags,
@@ -179,10 +176,8 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   p.y_f16 = y_f16 ? 1 : 0;
   p.total_units = (long long)batch * p.ns * p.mt;
   char* ws = reinterpret_cast<char*>(workspace);
-  const size_t cnt_off = round_up(part_bytes(m, n, batch), 256);
+  const size_t tile_off = round_up(part_bytes(m, n, batch), 256);
   p.part = reinterpret_cast<float*>(ws);
-  p.cnt = reinterpret_cast<unsigned*>(ws + cnt_off);
-  const size_t tile_off = cnt_off + round_up(counter_bytes(m, batch), 256);
   p.tile_cnt = reinterpret_cast<unsigned*>(ws + tile_off);
   p.status = reinterpret_cast<unsigned*>(ws + tile_off + kTileCounterBytes);
 
@@ -202,7 +197,10 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  if (p.ns > 1 && launch_splitk_reduce(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LUTGEMM_ERR_CUDA;
+  return LUTGEMM_OK;
 }
 
 }  // extern "C"

@@ -70,8 +70,7 @@ struct RunParams {
   const float* offset;     // [ng][m] or nullptr
   const __half* x;         // [batch][n]
   void* y;                 // [batch][m], fp32 or fp16
-  float* part;             // [batch][ns][mt*32] split-K partial sums
-  unsigned* cnt;           // [batch][mt] arrival counters (zero between calls)
+  float* part;             // [batch][ns][mt*32] split-K partial sums (ns > 1)
   unsigned* tile_cnt;      // [segments] tile counters of segment-aligned mode (zero between calls)
   unsigned* status;        // sticky internal-error bits: 1 shared window base is not kTableBase,
                            // 2 a weight-ring wait timed out (results invalid)
@@ -137,6 +136,10 @@ inline void choose_launch(long long sms, long long segments, long long mt, long 
 }
 
 using RunKernel = void (*)(RunParams);
+
+// y = sum over slices of the split-K partials (slice order), launched after
+// the run kernel when ns > 1 (programmatic launch: it waits for the run).
+cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream);
 
 constexpr unsigned kStatusWindow = 1u;
 constexpr unsigned kStatusTimeout = 2u;

@@ -35,11 +35,9 @@
 //   * Per-group alpha (and offset) are applied once per piece (g = 128),
 //     per half-piece (g = 64) or per run (other g); the per-piece values are
 //     prefetched three steps ahead in registers.
-//   * Split-K: each unit stores its fp32 partial.  When a warp has finished
-//     its units of a segment it fences once and bumps the arrival counters of
-//     those row tiles (one lane per tile); the last arrival for a tile (no
-//     waiting anywhere) sums the slices in fixed order, writes y and resets
-//     the counter.
+//   * Split-K: each unit stores its fp32 partial; a second, small kernel
+//     (programmatically chained) sums the slices of every row in slice order
+//     and writes y.  With a single slice the run kernel writes y itself.
 #pragma once
 
 #include <utility>
@@ -410,72 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         load_alpha.template operator()<D>(t_cur, D);
       });
       const int steps_per_unit_ = steps_per_unit;
-      int my_tile = 0;        // lane k holds the tile of this warp's k-th unpublished partial
-      int ntiles = 0;
       bool more = dyn;        // grabs may still succeed
       unsigned pend = 0;      // lane 0: raw count returned by the pending grab
-
-      // Split-K arrival for the first `n` tiles held in my_tile: one fence for
-      // their partials, then one lane per tile bumps the tile's counter; the
-      // last arrival sums the slices in slice order, writes y and resets it.
-      auto publish = [&](int n) {
-        __threadfence();
-        unsigned prev = 0;
-        if (lane < n) prev = atomicAdd(p.cnt + (size_t)b * p.mt + my_tile, 1u);
-        unsigned last = __ballot_sync(0xffffffffu, lane < n && prev == (unsigned)(p.ns - 1));
-        if (last) __threadfence();
-        // Sum the tiles this warp closed, up to 4 at a time, with the loads of
-        // 4 slices x 4 tiles in flight together (lane = row of the tile).
-        const size_t stride = (size_t)p.mt * kTileRows;
-        while (last) {
-          int Rt[4];
-          int nt = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            Rt[e] = -1;
-            if (last) {
-              const int src_lane = __ffs(last) - 1;
-              last &= last - 1;
-              Rt[e] = __shfl_sync(0xffffffffu, my_tile, src_lane);
-              ++nt;
-            }
-          }
-          float sum[4];
-          const float* col[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            sum[e] = 0.f;
-            col[e] = p.part + ((size_t)b * p.ns * p.mt + (Rt[e] < 0 ? Rt[0] : Rt[e])) * kTileRows + lane;
-          }
-          int s2 = 0;
-          for (; s2 + 4 <= p.ns; s2 += 4) {
-            float v[4][4];
-#pragma unroll
-            for (int d = 0; d < 4; ++d)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) v[d][e] = e < nt ? __ldcg(col[e] + (size_t)(s2 + d) * stride) : 0.f;
-#pragma unroll
-            for (int d = 0; d < 4; ++d)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) sum[e] += v[d][e];
-          }
-          for (; s2 < p.ns; ++s2)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (e < nt) sum[e] += __ldcg(col[e] + (size_t)s2 * stride);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (e >= nt) continue;
-            const int row = Rt[e] * kTileRows + lane;
-            if (row < p.m) {
-              const size_t o = (size_t)b * p.m + row;
-              if (p.y_f16) reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(sum[e]);
-              else reinterpret_cast<float*>(p.y)[o] = sum[e];
-            }
-            if (lane == 0) p.cnt[(size_t)b * p.mt + Rt[e]] = 0u;
-          }
-        }
-      };
 
       for (int k = 0; !failed; ++k) {
         // Tile k is t_cur, tile k+1 is t_nxt (or none).  Grab tile k+2 now.
@@ -586,12 +520,16 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           });
         }
         if (failed) break;
-        // This slice's partial sum of the row tile; published in batches of 32.
-        p.part[((size_t)((long long)b * p.ns + s) * p.mt + R) * kTileRows + lane] = yacc;
-        if (lane == ntiles) my_tile = R;
-        if (++ntiles == 32) {
-          publish(32);
-          ntiles = 0;
+        // One slice: the row's sum is y.  Several: this slice's partial, summed
+        // over slices by the split-K reduce kernel that follows.
+        if (p.ns == 1) {
+          if (row < p.m) {
+            const size_t o = (size_t)b * p.m + row;
+            if (p.y_f16) reinterpret_cast<__half*>(p.y)[o] = __float2half_rn(yacc);
+            else reinterpret_cast<float*>(p.y)[o] = yacc;
+          }
+        } else {
+          p.part[((size_t)((long long)b * p.ns + s) * p.mt + R) * kTileRows + lane] = yacc;
         }
 
         // Advance: tile k+2 comes from the grab (dynamic) or the static list.
@@ -613,7 +551,6 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         t_cur = t_nxt;
         t_nxt = t_after;
       }
-      if (!failed && ntiles > 0) publish(ntiles);
     }
   }
 

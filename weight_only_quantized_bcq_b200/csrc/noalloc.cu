@@ -11,8 +11,7 @@
 // is loaded holds its LUTGEMM_NOALLOC_SCRATCH_BYTES until the process exits.
 // Layout (fixed, independent of the problem size):
 //   [0, 256)              status word (sticky internal-error bits)
-//   [256, +256 KB)        split-K arrival counters, zero between calls
-//   [.., +4 KB)           per-segment tile counters, zero between calls
+//   [256, +4 KB)          per-segment tile counters, zero between calls
 //   [.., end)             split-K partial sums, written before they are read
 // The counters sit at a fixed place so that they are never overlaid by
 // another call's partial sums; the kernel resets every counter it uses, and
@@ -32,9 +31,7 @@ using namespace lutgemm;
 
 constexpr size_t kScratchBytes = LUTGEMM_NOALLOC_SCRATCH_BYTES;
 constexpr size_t kStatusOff = 0;
-constexpr size_t kCounterOff = 256;
-constexpr size_t kCounterBytes = 256 * 1024;
-constexpr size_t kTileCounterOff = kCounterOff + kCounterBytes;
+constexpr size_t kTileCounterOff = 256;
 constexpr size_t kPartOff = kTileCounterOff + kMaxTileCounters * sizeof(unsigned);
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
@@ -117,9 +114,8 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
     return LUTGEMM_ERR_ALIGN;
   const int ns = ceil_div(n, kSliceInputs);
   const int mt = ceil_div(m, kTileRows);
-  const size_t counters = (size_t)batch * mt * sizeof(unsigned);
   const size_t partials = (size_t)batch * ns * mt * kTileRows * sizeof(float);
-  if (counters > kCounterBytes || partials > kScratchBytes - kPartOff) return LUTGEMM_ERR_WORKSPACE;
+  if (partials > kScratchBytes - kPartOff) return LUTGEMM_ERR_WORKSPACE;
 
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const RunKernel kernel = pick_kernel(q, g, offset != nullptr);
@@ -133,7 +129,6 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   p.x = reinterpret_cast<const __half*>(x);
   p.y = y;
   p.part = reinterpret_cast<float*>(d.base + kPartOff);
-  p.cnt = reinterpret_cast<unsigned*>(d.base + kCounterOff);
   p.tile_cnt = reinterpret_cast<unsigned*>(d.base + kTileCounterOff);
   p.status = reinterpret_cast<unsigned*>(d.base + kStatusOff);
   p.m = m;
@@ -159,5 +154,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  if (p.ns > 1 && launch_splitk_reduce(p, st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  return LUTGEMM_OK;
 }
