@@ -1,7 +1,9 @@
-// Split-K reduction of the LUT-GEMM: y[b][r] = sum over slices s (in order
-// s = 0, 1, ...) of the fp32 partials part[b][s][r], so repeated calls give
-// identical bits.  One thread sums four rows with 16-byte loads, eight slices
-// in flight.  Launched right after the run kernel with programmatic
+// Split-K reduction of the LUT-GEMM: y[b][r] = sum over slices of the fp32
+// partials part[b][s][r], in a fixed order, so repeated calls give identical
+// bits.  A block covers 256/SL row quads (four rows, one 16-byte load); its
+// SL slice lanes per quad each sum a contiguous run of slices in slice order,
+// all loads of a thread in flight at once, and lane 0 then adds the SL lane
+// sums in lane order.  Launched right after the run kernel with programmatic
 // dependent launch: it waits for the run to complete before reading.
 #include "lutgemm_common.cuh"
 
@@ -9,38 +11,53 @@ namespace lutgemm {
 
 namespace {
 
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, void* y, int m, int mt,
-                                                           int ns, int batch, int y_f16) {
+constexpr int kReduceThreads = 256;
+constexpr int kMaxLaneSlices = 8;   // loads of one thread kept in flight together
+
+__global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const float* __restrict__ part, void* y,
+                                                                      int m, int mt, int ns, int batch,
+                                                                      int sl_log2, int y_f16) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float4 lane_sum[kReduceThreads];
+  const int SL = 1 << sl_log2;
+  const int qpb = kReduceThreads >> sl_log2;               // quads per block
   const long long quads = (long long)mt * (kTileRows / 4);
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)batch * quads) return;
-  const int b = (int)(idx / quads);
-  const long long rq = idx - (long long)b * quads;
-  const float4* src = reinterpret_cast<const float4*>(part) + (size_t)b * ns * quads + rq;
+  const long long blocks_per_col = (quads + qpb - 1) / qpb;
+  const int b = (int)(blockIdx.x / blocks_per_col);
+  const long long rq = (blockIdx.x - (long long)b * blocks_per_col) * qpb + (threadIdx.x >> sl_log2);
+  const int sl = threadIdx.x & (SL - 1);
+  const int per = (ns + SL - 1) >> sl_log2;                // slices per lane
+  const int s0 = sl * per, s1 = min(ns, s0 + per);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int s = 0;
-  for (; s + 8 <= ns; s += 8) {
-    float4 v[8];
+  if (rq < quads) {
+    const float4* src = reinterpret_cast<const float4*>(part) + (size_t)b * ns * quads + rq;
+    for (int s = s0; s < s1; s += kMaxLaneSlices) {
+      float4 v[kMaxLaneSlices];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __ldcg(src + (size_t)(s + e) * quads);
+      for (int e = 0; e < kMaxLaneSlices; ++e)
+        v[e] = s + e < s1 ? __ldcg(src + (size_t)(s + e) * quads) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      acc.x += v[e].x;
-      acc.y += v[e].y;
-      acc.z += v[e].z;
-      acc.w += v[e].w;
+      for (int e = 0; e < kMaxLaneSlices; ++e) {
+        acc.x += v[e].x;
+        acc.y += v[e].y;
+        acc.z += v[e].z;
+        acc.w += v[e].w;
+      }
     }
   }
-  for (; s < ns; ++s) {
-    const float4 v = __ldcg(src + (size_t)s * quads);
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
+  lane_sum[threadIdx.x] = acc;
+  __syncthreads();
+  if (sl != 0 || rq >= quads) return;
+  float4 t = lane_sum[threadIdx.x];
+  for (int k = 1; k < SL; ++k) {
+    const float4 u = lane_sum[threadIdx.x + k];
+    t.x += u.x;
+    t.y += u.y;
+    t.z += u.z;
+    t.w += u.w;
   }
-  const float r[4] = {acc.x, acc.y, acc.z, acc.w};
+  const float r[4] = {t.x, t.y, t.z, t.w};
   const long long row0 = rq * 4;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -55,10 +72,15 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 }  // namespace
 
 cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream) {
-  const long long threads = (long long)p.batch * p.mt * (kTileRows / 4);
+  // Slice lanes per quad: 8 when there are at least 8 slices, else the
+  // largest power of two not above ns.
+  const int sl_log2 = p.ns >= 8 ? 3 : (p.ns >= 4 ? 2 : (p.ns >= 2 ? 1 : 0));
+  const int qpb = kReduceThreads >> sl_log2;
+  const long long quads = (long long)p.mt * (kTileRows / 4);
+  const long long blocks = (long long)p.batch * ((quads + qpb - 1) / qpb);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kReduceThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -67,7 +89,7 @@ cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, (const float*)p.part, p.y, p.m, p.mt, p.ns,
-                                       p.batch, p.y_f16);
+                                       p.batch, sl_log2, p.y_f16);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
