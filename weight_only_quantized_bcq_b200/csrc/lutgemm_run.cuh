@@ -18,7 +18,8 @@
 //     takes the CTA's tiles w, w+16, w+32, ... of a segment.
 //   * Weights move by TMA: the q pieces of all 32 lanes of a step are q*512
 //     contiguous bytes of the packed layout, and CH consecutive steps (CH = 2
-//     for q <= 3) are fetched by one cp.async.bulk into a per-warp ring of S
+//     for q <= 3) are fetched by one cp.async.bulk (L2 evict-first: the
+//     weights are read once) into a per-warp ring of S
 //     shared-memory stages (one mbarrier each), S copies ahead and across
 //     unit boundaries; a warp's first copies of a segment are issued before
 //     the table build.  Every wait is bounded in time; a timeout sets a
@@ -115,15 +116,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// L2 policy for the weight stream: every weight byte is read exactly once, so
+// its lines are the first to go, and the scales, inputs and split-K partials
+// keep their place in L2.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // One TMA bulk copy of `bytes` (a multiple of 16) from global memory into this
-// CTA's shared memory, completing on mbarrier `bar`.  The proxy fence orders
-// the warp's earlier generic reads of the stage before the copy overwrites it.
-__device__ __forceinline__ void tma_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+// CTA's shared memory, completing on mbarrier `bar`, with L2 policy `pol`.
+// The proxy fence orders the warp's earlier generic reads of the stage before
+// the copy overwrites it.
+__device__ __forceinline__ void tma_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar, uint64_t pol) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
 }
 
 // PRMT selector for byte t of a stored word: result byte 0 <- column byte t of
@@ -279,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   }
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncwarp();
+  const uint64_t wpol = evict_first_policy();
   int st = 0;
   uint32_t ph = 0;
   bool failed = false;     // a ring wait timed out: stop streaming, keep taking the CTA barriers
@@ -360,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
       const int pg_ = c / CPT, U_ = (c - pg_ * CPT) * CH;
       const int planes = MULTI ? min(4, p.q - 4 * pg_) : Q;
       const uint8_t* src = slice_base + (size_t)R_ * unit_bytes + ((size_t)U_ * p.q + 4 * pg_) * 512;
-      tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * planes * CH, bars + 8u * stage);
+      tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * planes * CH, bars + 8u * stage, wpol);
     };
 
     // Per-piece scales (and offsets) of step j of row tile R into register stage SLOT.
