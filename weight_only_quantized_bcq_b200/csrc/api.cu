@@ -59,6 +59,11 @@ cudaError_t device_setup(RunKernel kernel, int* sm_count) {
   *sm_count = g_sm_count[dev];
   const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
   if (g_smem_done.find(key) == g_smem_done.end()) {
+    // Static shared memory would move the dynamic window off kTableBase.
+    cudaFuncAttributes fa;
+    err = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
+    if (err != cudaSuccess) return err;
+    if (fa.sharedSizeBytes != 0) return cudaErrorInvalidConfiguration;
     err = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;

@@ -240,6 +240,13 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   static_assert(!MULTI || CH == 1, "plane groups are fetched one step at a time");
   constexpr int NA = 4;                                // alpha register stages (3 steps ahead)
   static_assert(S >= 2 && S <= 8, "weight ring of 2..8 stages");
+  constexpr int NPG = MULTI ? 2 : 1;                   // plane groups of a unit
+  // Step of a unit at which the next tile is first needed: the alpha
+  // prefetch reaches it NA-1 steps before the end, the ring refill S stages
+  // before the end.  Three steps cover a tile-counter atomic comfortably.
+  constexpr int NEED = (8 * NPG - (NA - 1)) < ((8 / CH) * NPG - S) * CH ? (8 * NPG - (NA - 1))
+                                                                        : ((8 / CH) * NPG - S) * CH;
+  constexpr bool AHEAD1 = NEED >= 3;
 
   extern __shared__ __align__(16) unsigned char smem[];
   // Let the next kernel in the stream start on SMs as they free up; it waits
@@ -352,9 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     // ... of the CTA's tiles (tile_first + index * tile_stride).  In
     // segment-aligned mode the G_z CTAs of a segment take two static tiles per
     // warp, covering tiles [0, 32 G_z); all further tiles come from the
-    // segment's tile counter, grabbed one tile ahead by lane 0, so the group's
-    // warps share out the rest as they finish.  The last CTA to finish the
-    // kernel resets the counters for the next call.
+    // segment's tile counter (lane 0 grabs), so the group's warps share out
+    // the rest as they finish.  The last CTA to finish the kernel resets the
+    // counters for the next call.
     const bool dyn = p.seg_aligned != 0;
     auto static_tile = [&](int k) -> int {
       const long long idx = (long long)warp + (long long)k * kWarps;
@@ -424,10 +431,22 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
       const int steps_per_unit_ = steps_per_unit;
       bool more = dyn;        // grabs may still succeed
       unsigned pend = 0;      // lane 0: raw count returned by the pending grab
+      bool nxt_pending = false;
 
       for (int k = 0; !failed; ++k) {
-        // Tile k is t_cur, tile k+1 is t_nxt (or none).  Grab tile k+2 now.
-        const bool grabbing = dyn && more && t_nxt >= 0;
+        // Tile k is t_cur.  Tile k+1 is first needed NEED steps into tile k
+        // (alpha prefetch or ring refill).  When that leaves time for the
+        // atomic's round trip, tile k+1 is grabbed now and read at step NEED,
+        // so a warp holds at most one tile that no other warp can take.
+        // Otherwise tile k+1 is already known (t_nxt) and k+2 is grabbed now.
+        bool grabbing;
+        if constexpr (AHEAD1) {
+          t_nxt = (dyn && k >= 1) ? -1 : static_tile(k + 1);
+          grabbing = dyn && more && k >= 1;
+          nxt_pending = grabbing;
+        } else {
+          grabbing = dyn && more && t_nxt >= 0;
+        }
         if (grabbing && lane == 0) pend = atomicAdd(tile_ctr, 1u);
         const int R = t_cur;
         const int row = R * kTileRows + lane;
@@ -436,6 +455,18 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           static_for(std::make_integer_sequence<int, 8>{}, [&]<int U>() {
             if (failed) return;
             const int j = pg * 8 + U;          // step within the unit
+            if constexpr (AHEAD1) {
+              if (j == NEED && nxt_pending) {
+                int tile = -1;
+                if (lane == 0) {
+                  const long long t = dyn_base + pend;
+                  tile = t < p.mt ? (int)t : -1;
+                }
+                t_nxt = __shfl_sync(0xffffffffu, tile, 0);
+                more = t_nxt >= 0;
+                nxt_pending = false;
+              }
+            }
             {
               const int ja = j + NA - 1;       // alpha three steps ahead
               if (ja < steps_per_unit_) load_alpha.template operator()<(U + NA - 1) % NA>(t_cur, ja);
@@ -548,6 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
 
         // Advance: tile k+2 comes from the grab (dynamic) or the static list.
         if (t_nxt < 0) break;
+        if constexpr (AHEAD1) {
+          t_cur = t_nxt;
+          continue;
+        }
         int t_after = -1;
         if (dyn) {
           if (grabbing) {

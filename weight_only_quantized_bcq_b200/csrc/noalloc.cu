@@ -90,6 +90,11 @@ cudaError_t prepare(RunKernel kernel, cudaStream_t stream, DeviceScratch* out) {
   }
   const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
   if (g_smem_done.find(key) == g_smem_done.end()) {
+    // Static shared memory would move the dynamic window off kTableBase.
+    cudaFuncAttributes fa;
+    err = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
+    if (err != cudaSuccess) return err;
+    if (fa.sharedSizeBytes != 0) return cudaErrorInvalidConfiguration;
     err = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
