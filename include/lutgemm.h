@@ -151,7 +151,7 @@ int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
  * group's x for converted uniform weights), and the per-slice partial sums
  * are reduced in a fixed order, so repeated calls give identical bits.
  *   m, n, batch, q, g  m >= 1, batch >= 1, 1 <= q <= 8, n % 8 == 0,
- *                      g % 8 == 0, n % g == 0
+ *                      g % 8 == 0, n % g == 0, batch * ceil(n/1024) < 2^31
  *   packed     dev, packed layout above, 16-byte aligned
  *   alpha      dev fp16 [q][n/g][m], 2-byte aligned
  *   offset     dev fp32 [n/g][m] or NULL (pure BCQ), 4-byte aligned

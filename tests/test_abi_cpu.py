@@ -92,7 +92,9 @@ def test_run_rejects_null(L):
 
 
 @pytest.mark.parametrize("kw", [dict(m=0), dict(n=0), dict(n=1028), dict(batch=0), dict(q=0), dict(q=9),
-                                dict(g=100), dict(g=0), dict(n=1024, g=384), dict(n=12)])
+                                dict(g=100), dict(g=0), dict(n=1024, g=384), dict(n=12),
+                                # batch * ceil(n / 1024) must stay below 2^31
+                                dict(batch=1 << 20, n=1 << 21)])
 def test_run_rejects_bad_shapes(L, kw):
     assert _run(L, **kw) == L.ERR_SHAPE
 

@@ -157,6 +157,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
                 size_t workspace_bytes, void* stream) {
   if (!packed || !alpha || !x || !y || !workspace) return LUTGEMM_ERR_NULL;
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return LUTGEMM_ERR_SHAPE;
+  if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
   if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||

@@ -314,12 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   // cz CTAs share round-robin (CTA k takes tiles k, k+cz, ...), so that every
   // CTA's reads spread over the whole segment.  Otherwise: a contiguous range
   // [u_begin, u_end) of the unit list, visited segment by segment.
-  const long long Z = (long long)p.batch * p.ns;
-  long long u_begin = 0, u_end = 0, a_seg = 0, a_first = 0, a_stride = 1;
+  // Index arithmetic is 32-bit where the host bounds allow it (batch * ns <
+  // 2^31; segment-aligned mode has at most kMaxTileCounters - 1 segments and
+  // one CTA per SM): 64-bit division is a long software sequence.
+  const unsigned Z = (unsigned)p.batch * (unsigned)p.ns;
+  long long u_begin = 0, u_end = 0;
+  unsigned a_seg = 0, a_first = 0, a_stride = 1;
   if (p.seg_aligned) {
     // Segment z gets the CTAs c = z, z + Z, z + 2Z, ...: a group spread over
     // the whole grid rather than a block of neighbouring CTAs.
-    const long long G = gridDim.x, c = blockIdx.x;
+    const unsigned G = gridDim.x, c = blockIdx.x;
     a_seg = c % Z;
     a_first = c / Z;
     a_stride = (G - a_seg + Z - 1) / Z;
@@ -331,29 +335,30 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   float ob[NA][APP];
   uint4 wst[CH][SP];       // the pieces of the current ring stage
 
-  auto group_size = [&](long long z) { return (long long)((gridDim.x - z + Z - 1) / Z); };
+  auto group_size = [&](unsigned z) { return (gridDim.x - z + Z - 1) / Z; };
 
   for (int visit = 0;; ++visit) {
     // Segment-aligned mode visits the CTA's own segment once; the contiguous
     // mode visits the segments of its range in order.
-    long long seg, tile_first = 0, tile_stride = 1, tile_count = 0;
+    unsigned seg, tile_first = 0, tile_stride = 1, tile_count = 0;
     if (p.seg_aligned) {
       if (visit > 0) break;
       seg = a_seg;
       tile_first = a_first;
       tile_stride = a_stride;
-      tile_count = a_first < p.mt ? (p.mt - 1 - a_first) / a_stride + 1 : 0;
+      tile_count = a_first < (unsigned)p.mt ? ((unsigned)p.mt - 1 - a_first) / a_stride + 1 : 0;
     } else {
       if (u_begin >= u_end) break;
-      seg = u_begin / p.mt;
-      const long long seg_end = min(u_end, (seg + 1) * p.mt);
-      tile_first = u_begin - seg * p.mt;
+      const long long sg = u_begin / p.mt;
+      const long long seg_end = min(u_end, (sg + 1) * p.mt);
+      seg = (unsigned)sg;
+      tile_first = (unsigned)(u_begin - sg * p.mt);
       tile_stride = 1;
-      tile_count = seg_end - u_begin;
+      tile_count = (unsigned)(seg_end - u_begin);
       u_begin = seg_end;
     }
-    const int b = (int)(seg / p.ns);
-    const int s = (int)(seg - (long long)b * p.ns);
+    const int b = (int)(seg / (unsigned)p.ns);
+    const int s = (int)(seg - (unsigned)b * (unsigned)p.ns);
     const uint8_t* slice_base = p.packed + (size_t)s * p.mt * unit_bytes;
     // This warp's row tiles.  In the contiguous mode: indices warp, warp+16,
     // ... of the CTA's tiles (tile_first + index * tile_stride).  In
@@ -364,11 +369,11 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     // counters for the next call.
     const bool dyn = p.seg_aligned != 0;
     auto static_tile = [&](int k) -> int {
-      const long long idx = (long long)warp + (long long)k * kWarps;
+      const unsigned idx = (unsigned)warp + (unsigned)k * kWarps;
       return idx < tile_count ? (int)(tile_first + idx * tile_stride) : -1;
     };
     unsigned* const tile_ctr = p.tile_cnt + seg;
-    const long long dyn_base = dyn ? 32 * group_size(seg) : 0;
+    const long long dyn_base = dyn ? 32ll * group_size(seg) : 0;
     int t_cur = failed ? -1 : static_tile(0);
     int t_nxt = static_tile(1);
     const bool busy = t_cur >= 0;

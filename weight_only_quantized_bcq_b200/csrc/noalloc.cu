@@ -112,6 +112,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   if (!packed || !alpha || !x || !y) return LUTGEMM_ERR_NULL;
   if (q < 1 || q > 8 || m < 1 || n < 8 || n % 8 != 0 || g < 8 || g % 8 != 0 || n % g != 0 || batch < 1)
     return LUTGEMM_ERR_SHAPE;
+  if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
   if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||
