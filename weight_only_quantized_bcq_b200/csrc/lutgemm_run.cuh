@@ -35,7 +35,7 @@
 //     table base, half and band, and one FADD.
 //   * Per-group alpha (and offset) are applied once per piece (g = 128),
 //     per half-piece (g = 64) or per run (other g); the per-piece values are
-//     prefetched three steps ahead in registers.
+//     prefetched up to seven steps ahead in registers.
 //   * Split-K: each unit stores its fp32 partial; a second, small kernel
 //     (programmatically chained) sums the slices of every row in slice order
 //     and writes y.  With a single slice the run kernel writes y itself.
@@ -238,15 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr uint32_t STEP_BYTES = 512u * SP;
   constexpr uint32_t STAGE_BYTES = STEP_BYTES * CH;
   static_assert(!MULTI || CH == 1, "plane groups are fetched one step at a time");
-  constexpr int NA = 4;                                // alpha register stages (3 steps ahead)
   static_assert(S >= 2 && S <= 8, "weight ring of 2..8 stages");
   constexpr int NPG = MULTI ? 2 : 1;                   // plane groups of a unit
-  // Step of a unit at which the next tile is first needed: the alpha
-  // prefetch reaches it NA-1 steps before the end, the ring refill S stages
-  // before the end.  Three steps cover a tile-counter atomic comfortably.
-  constexpr int NEED = (8 * NPG - (NA - 1)) < ((8 / CH) * NPG - S) * CH ? (8 * NPG - (NA - 1))
-                                                                        : ((8 / CH) * NPG - S) * CH;
-  constexpr bool AHEAD1 = NEED >= 3;
 
   extern __shared__ __align__(16) unsigned char smem[];
   // Let the next kernel in the stream start on SMs as they free up; it waits
@@ -265,6 +258,18 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr int RUN = (MODE == kG128 || MODE == kG128x) ? 16 : (MODE == kG64 ? 8 : 1);
   constexpr int APP = RUN >= 8 ? 16 / RUN : 1;      // prefetched scales per piece
   constexpr bool PRE_ALPHA = RUN >= 8;
+  // Register stages of prefetched scales: step j's are loaded NA-1 steps
+  // ahead (7 with one scale per piece, 3 with two, to bound registers); the
+  // scales come from HBM and their latency under full load is microseconds.
+  constexpr int NA = APP == 1 ? 8 : 4;
+  static_assert((8 * NPG) % NA == 0, "scale stages must tile the unit");
+  // Step of a unit at which the next tile is first needed: the scale
+  // prefetch reaches it NA-1 steps before the end, the ring refill S stages
+  // before the end.  Three steps cover a tile-counter atomic comfortably.
+  constexpr int NEED_A = PRE_ALPHA ? 8 * NPG - (NA - 1) : 8 * NPG;
+  constexpr int NEED_R = ((8 / CH) * NPG - S) * CH;
+  constexpr int NEED = NEED_A < NEED_R ? NEED_A : NEED_R;
+  constexpr bool AHEAD1 = NEED >= 3;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -473,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
               }
             }
             {
-              const int ja = j + NA - 1;       // alpha three steps ahead
+              const int ja = j + NA - 1;       // scales NA-1 steps ahead
               if (ja < steps_per_unit_) load_alpha.template operator()<(U + NA - 1) % NA>(t_cur, ja);
               else if (t_nxt >= 0) load_alpha.template operator()<(U + NA - 1) % NA>(t_nxt, ja - steps_per_unit_);
             }

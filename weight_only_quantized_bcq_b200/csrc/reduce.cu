@@ -72,9 +72,10 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
 }  // namespace
 
 cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream) {
-  // Slice lanes per quad: 8 when there are at least 8 slices, else the
-  // largest power of two not above ns.
-  const int sl_log2 = p.ns >= 8 ? 3 : (p.ns >= 4 ? 2 : (p.ns >= 2 ? 1 : 0));
+  // Slice lanes per quad: the smallest power of two that leaves each lane at
+  // most two slices, up to 32 lanes.
+  int sl_log2 = 0;
+  while (sl_log2 < 5 && ((p.ns + (1 << sl_log2) - 1) >> sl_log2) > 2) ++sl_log2;
   const int qpb = kReduceThreads >> sl_log2;
   const long long quads = (long long)p.mt * (kTileRows / 4);
   const long long blocks = (long long)p.batch * ((quads + qpb - 1) / qpb);
