@@ -50,6 +50,20 @@
  *   The q * 4096 bytes of one (slice, row tile) are contiguous, and so are
  *   the q * 512 bytes a warp reads per step.
  *
+ * Unit-major scale layout (produced by lutgemm_pack_scales, consumed by
+ * lutgemm_run with LUTGEMM_SCALES_PACKED; only for g % 128 == 0, where every
+ * 128-input piece has one scale per plane).  The pages fix no layout; this
+ * one gives each lane the scales of a whole (slice, row tile) in 16*SP
+ * contiguous bytes, so they arrive in a few 16-byte loads one tile ahead.
+ *   SP = min(q, 4) planes per step, n_pg = ceil(q/4) plane groups.
+ *   Element (s, R, pg, l, U, e) (pg < n_pg, l < 32, U < 8, e < SP) is the
+ *   fp16 at element index ((((s * m_t + R) * n_pg + pg) * 32 + l) * 8 + U) * SP + e
+ *   and holds alpha[4*pg + e][G][32*R + l] with
+ *   G = (1024*s + 128*P) / g, P = U xor (4 * (l / 16)) (the piece lane l
+ *   reads at step U).  It is 0 when 4*pg + e >= q, 32*R + l >= m or
+ *   1024*s + 128*P >= n.  Size: n_s * m_t * n_pg * 512 * SP bytes (equal to
+ *   the [q][n/g][m] array when g == 128, m % 32 == 0 and n % 1024 == 0).
+ *
  * Other layouts (row-major, innermost last):
  *   signs  int8   [q][m][n]     each -1 or +1
  *   codes  uint8  [m][n]        uniform codes in [0, 2^q)
@@ -86,6 +100,7 @@ extern "C" {
 
 /* Flags of lutgemm_run. */
 #define LUTGEMM_Y_F16          1u /* write y as fp16 (round to nearest even of the fp32 sum) */
+#define LUTGEMM_SCALES_PACKED  2u /* alpha is in the unit-major scale layout (g % 128 == 0) */
 
 /* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
 int lutgemm_version(void);
@@ -97,6 +112,11 @@ const char* lutgemm_status_string(int status);
  * ceil(n/1024) * ceil(m/32) * q * 4096.  Returns 0 for invalid shapes.
  * Pure host function. */
 size_t lutgemm_packed_bytes(int q, int m, int n);
+
+/* Bytes of the unit-major scale buffer for (q, m, n, g):
+ * ceil(n/1024) * ceil(m/32) * ceil(q/4) * 512 * min(q, 4).  Returns 0 for
+ * invalid shapes and when g % 128 != 0.  Pure host function. */
+size_t lutgemm_scales_bytes(int q, int m, int n, int g);
 
 /* Bytes of the lutgemm_run workspace (split-K partial sums, per-slice tile
  * counters and a status word).  Returns 0 for invalid shapes.  Pure host
@@ -142,6 +162,19 @@ int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
                            uint8_t* packed, uint16_t* alpha, float* offset,
                            int32_t* status_flags, void* stream);
 
+/* Reorder group-wise plane scales into the unit-major scale layout above
+ * (a data movement only: every output is one input value or 0).  The scales
+ * are those of the BCQ format (LUT-GEMM card, Summary: q binary planes, each
+ * with a scale per group of g inputs).
+ *   alpha        dev fp16 [q][n/g][m], 2-byte aligned
+ *   q, m, n, g   1 <= q <= 8, m >= 1, n % 8 == 0, g % 128 == 0, n % g == 0
+ *   scales       dev, lutgemm_scales_bytes(q,m,n,g) bytes, 16-byte aligned
+ *                (output, fully written)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also for g % 128 != 0),
+ * ERR_ALIGN or ERR_CUDA. */
+int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
+                        uint16_t* scales, void* stream);
+
 /* y = W x for a BCQ weight, through per-8-activation lookup tables, with no
  * dequantisation (LUT-GEMM card, Summary and "Lookup tables instead of
  * multiplications"; pith.science abstract).  For each batch column b and each
@@ -153,14 +186,17 @@ int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
  *   m, n, batch, q, g  m >= 1, batch >= 1, 1 <= q <= 8, n % 8 == 0,
  *                      g % 8 == 0, n % g == 0, batch * ceil(n/1024) < 2^31
  *   packed     dev, packed layout above, 16-byte aligned
- *   alpha      dev fp16 [q][n/g][m], 2-byte aligned
+ *   alpha      dev fp16 [q][n/g][m], 2-byte aligned; with
+ *              LUTGEMM_SCALES_PACKED the lutgemm_pack_scales output instead
+ *              (16-byte aligned; g % 128 == 0), which gives the same bits
  *   offset     dev fp32 [n/g][m] or NULL (pure BCQ), 4-byte aligned
  *   x          dev fp16 [batch][n], 16-byte aligned
  *   y          dev [batch][m] fp32 (4-byte aligned) or, with LUTGEMM_Y_F16,
  *              fp16 (2-byte aligned); fully overwritten.  For n > 1024 the
  *   call enqueues two kernels: the lookup kernel writes per-slice partial
  *   sums to the workspace and a reduce kernel adds them in slice order.
- *   flags      0 or LUTGEMM_Y_F16
+ *   flags      OR of LUTGEMM_Y_F16 and LUTGEMM_SCALES_PACKED; other bits,
+ *              or LUTGEMM_SCALES_PACKED with g % 128 != 0, give ERR_VALUE
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
  *              16-byte aligned, zero-filled before its first use; left
  *              zero-filled by every successful call.  Calls that share a

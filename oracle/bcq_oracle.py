@@ -34,7 +34,8 @@ Readings where the pages are silent (each also listed in the design notes):
 * plane i (0-based) of a converted uniform weight is bit i of the integer code.
 * the packed weight layout is this library's own tiled layout; it is defined
   in ``include/lutgemm.h`` and re-implemented here from that text
-  (``pack_bcq`` / ``unpack_bcq``).
+  (``pack_bcq`` / ``unpack_bcq``).  So is the unit-major scale layout
+  (``pack_scales`` / ``unpack_scales``).
 
 Parity status: every public function here is pinned by
 ``tests/test_oracle_pins.py`` against brute force, closed forms, special cases
@@ -55,6 +56,7 @@ BLOCK_BYTES = 4096  # bytes of one (slice, row tile, plane): 8 chunks of 512
 __all__ = [
     "lut_table", "dequantize_bcq", "bcq_matmul", "lut_matmul",
     "packed_nbytes", "pack_bcq", "unpack_bcq", "unpack_rows",
+    "scales_nbytes", "pack_scales", "unpack_scales",
     "uniform_to_bcq", "uniform_dequant", "bcq_matmul_rows",
 ]
 
@@ -216,6 +218,84 @@ def unpack_rows(packed, q: int, m: int, n: int, rows) -> np.ndarray:
                     out_bits[:, ri, np.arange(ns) * SLICE + k0 + t] = bit.T
     bits = out_bits[:, :, :n]
     return (bits.astype(np.int8) * 2 - 1)
+
+
+# ---------------------------------------------------------------------------
+# Unit-major scale layout (this library's own; defined in include/lutgemm.h).
+# Only for g % 128 == 0.  SP = min(q, 4), n_pg = ceil(q / 4).  Element
+# (s, R, pg, l, U, e) sits at index
+#   ((((s * m_t + R) * n_pg + pg) * 32 + l) * 8 + U) * SP + e
+# and holds alpha[4*pg + e][G][32*R + l], G = (1024*s + 128*P) // g,
+# P = U xor (4 * (l // 16)); 0 when the plane, row or piece is out of range.
+# ---------------------------------------------------------------------------
+def _scale_dims(q: int, m: int, n: int, g: int):
+    if g % PIECE != 0 or n % g != 0:
+        raise ValueError("the unit-major scale layout needs g % 128 == 0 and n % g == 0")
+    return math.ceil(n / SLICE), math.ceil(m / TILE_ROWS), min(q, 4), math.ceil(q / 4)
+
+
+def scales_nbytes(q: int, m: int, n: int, g: int) -> int:
+    ns, mt, sp, npg = _scale_dims(q, m, n, g)
+    return ns * mt * npg * 512 * sp
+
+
+def pack_scales(alpha, g: int) -> np.ndarray:
+    """fp16 alpha [q][n/g][m] -> fp16 unit-major scale buffer (1-D)."""
+    a = np.asarray(alpha, dtype=np.float16)
+    q, ng, m = a.shape
+    n = ng * g
+    ns, mt, sp, npg = _scale_dims(q, m, n, g)
+    out = np.zeros((ns, mt, npg, TILE_ROWS, 8, sp), dtype=np.float16)
+    for s_ in range(ns):
+        for U in range(8):
+            for half in range(2):                       # l // 16
+                P = U ^ (4 * half)
+                k0 = SLICE * s_ + PIECE * P
+                if k0 >= n:
+                    continue                            # piece beyond n: stays 0
+                G = k0 // g
+                for pg in range(npg):
+                    for e in range(sp):
+                        i = 4 * pg + e
+                        if i >= q:
+                            continue                    # padding plane: stays 0
+                        col = np.zeros(mt * TILE_ROWS, dtype=np.float16)
+                        col[:m] = a[i, G, :]
+                        col = col.reshape(mt, TILE_ROWS)
+                        lanes = slice(16 * half, 16 * half + 16)
+                        out[s_, :, pg, lanes, U, e] = col[:, lanes]
+    return out.reshape(-1)
+
+
+def unpack_scales(scales, q: int, m: int, n: int, g: int) -> np.ndarray:
+    """Inverse of ``pack_scales``: fp16 alpha [q][n/g][m] read back from the buffer.
+
+    A group wider than one piece appears once per piece; every copy must agree.
+    """
+    ns, mt, sp, npg = _scale_dims(q, m, n, g)
+    buf = np.asarray(scales, dtype=np.float16).reshape(ns, mt, npg, TILE_ROWS, 8, sp)
+    ng = n // g
+    out = np.full((q, ng, m), np.nan, dtype=np.float64)
+    for s_ in range(ns):
+        for U in range(8):
+            for l in range(TILE_ROWS):
+                P = U ^ (4 * (l // 16))
+                k0 = SLICE * s_ + PIECE * P
+                if k0 >= n:
+                    continue
+                G = k0 // g
+                rows = np.arange(mt) * TILE_ROWS + l
+                ok = rows < m
+                for i in range(q):
+                    v = buf[s_, :, i // 4, l, U, i % 4].astype(np.float64)[ok]
+                    prev = out[i, G, rows[ok]]
+                    seen = ~np.isnan(prev)
+                    if np.any(prev[seen] != v[seen]):
+                        raise ValueError("copies of one group scale disagree")
+                    out[i, G, rows[ok]] = v
+    if np.isnan(out).any():
+        raise ValueError("some scale never appears in the buffer")
+    return out.astype(np.float16)
 
 
 # ---------------------------------------------------------------------------

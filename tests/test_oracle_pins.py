@@ -451,6 +451,116 @@ def test_pack_pins_catch_msb_first():
 # The footprint the card prints (Key points: 347.9 GB -> 65.3 GB, 5.33x) pins
 # the bits-per-weight count used for algorithmic bytes.
 # ---------------------------------------------------------------------------
+# ---------------------------------------------------------------------------
+# Unit-major scale layout: hand-derived positions (tests/golden), round trip,
+# and planted mistakes in the index map.
+# ---------------------------------------------------------------------------
+def _distinct_alpha(q, ng, m):
+    """fp16 scales whose bit patterns are 1, 2, 3, ... (all distinct, none zero)."""
+    bits = np.arange(1, q * ng * m + 1, dtype=np.uint16).reshape(q, ng, m)
+    return bits.view(np.float16)
+
+
+def pin_scales_golden(pack_scales) -> bool:
+    for case in _golden("scales_layout_positions.json")["cases"]:
+        q, m, n, g = case["q"], case["m"], case["n"], case["g"]
+        alpha = _distinct_alpha(q, n // g, m)
+        out = np.asarray(pack_scales(alpha, g), dtype=np.float16).view(np.uint16)
+        if out.size != case["nelem"] or out.size * 2 != O.scales_nbytes(q, m, n, g):
+            return False
+        for e in case["entries"]:
+            want = 0 if e[1] is None else int(alpha.view(np.uint16)[e[1], e[2], e[3]])
+            if int(out[e[0]]) != want:
+                return False
+    return True
+
+
+def test_scales_pins():
+    assert pin_scales_golden(O.pack_scales)
+
+
+@pytest.mark.parametrize("q,m,n,g", [(1, 32, 1024, 128), (3, 40, 2048, 128), (4, 100, 3072, 384),
+                                     (5, 70, 2048, 256), (8, 33, 1152, 128), (2, 33, 640, 128)])
+def test_scales_roundtrip(q, m, n, g):
+    alpha = _distinct_alpha(q, n // g, m)
+    packed = O.pack_scales(alpha, g)
+    assert packed.size * 2 == O.scales_nbytes(q, m, n, g)
+    back = O.unpack_scales(packed, q, m, n, g)
+    assert np.array_equal(back.view(np.uint16), alpha.view(np.uint16))
+    # Every stored value is a scale or padding zero, and each scale is stored
+    # once per piece of its group that lies inside n.
+    vals = packed.view(np.uint16)
+    counts = np.bincount(vals, minlength=alpha.size + 1)
+    assert np.all(counts[1:] == g // 128)
+
+
+def test_scales_reject_groups_below_a_piece():
+    with pytest.raises(ValueError):
+        O.scales_nbytes(3, 32, 1024, 64)
+
+
+def _scales_pieces_not_swapped(alpha, g):
+    """Planted: lanes 16..31 read the same piece as lanes 0..15."""
+    a = np.asarray(alpha, dtype=np.float16)
+    q, ng, m = a.shape
+    n = ng * g
+    ns, mt, sp, npg = math.ceil(n / 1024), math.ceil(m / 32), min(q, 4), math.ceil(q / 4)
+    out = np.zeros((ns, mt, npg, 32, 8, sp), dtype=np.float16)
+    for s_ in range(ns):
+        for U in range(8):
+            k0 = 1024 * s_ + 128 * U
+            if k0 >= n:
+                continue
+            for i in range(q):
+                col = np.zeros(mt * 32, dtype=np.float16)
+                col[:m] = a[i, k0 // g, :]
+                out[s_, :, i // 4, :, U, i % 4] = col.reshape(mt, 32)
+    return out.reshape(-1)
+
+
+def _scales_step_major(alpha, g):
+    """Planted: step outside lane ([..][U][l][e] instead of [..][l][U][e])."""
+    good = O.pack_scales(alpha, g)
+    a = np.asarray(alpha)
+    q, ng, m = a.shape
+    n = ng * g
+    ns, mt, sp, npg = math.ceil(n / 1024), math.ceil(m / 32), min(q, 4), math.ceil(q / 4)
+    return good.reshape(ns, mt, npg, 32, 8, sp).transpose(0, 1, 2, 4, 3, 5).reshape(-1)
+
+
+def _scales_planes_reversed(alpha, g):
+    """Planted: planes stored in reverse order."""
+    return O.pack_scales(np.asarray(alpha)[::-1], g)
+
+
+def _scales_group_per_run(alpha, g):
+    """Planted: group index taken from the run (8 inputs) instead of the piece."""
+    a = np.asarray(alpha, dtype=np.float16)
+    q, ng, m = a.shape
+    n = ng * g
+    ns, mt, sp, npg = math.ceil(n / 1024), math.ceil(m / 32), min(q, 4), math.ceil(q / 4)
+    out = np.zeros((ns, mt, npg, 32, 8, sp), dtype=np.float16)
+    for s_ in range(ns):
+        for U in range(8):
+            for half in range(2):
+                P = U ^ (4 * half)
+                k0 = 1024 * s_ + 8 * P
+                if 1024 * s_ + 128 * P >= n:
+                    continue
+                for i in range(q):
+                    col = np.zeros(mt * 32, dtype=np.float16)
+                    col[:m] = a[i, k0 // g, :]
+                    ln = slice(16 * half, 16 * half + 16)
+                    out[s_, :, i // 4, ln, U, i % 4] = col.reshape(mt, 32)[:, ln]
+    return out.reshape(-1)
+
+
+@pytest.mark.parametrize("mutant", [_scales_pieces_not_swapped, _scales_step_major, _scales_planes_reversed,
+                                    _scales_group_per_run])
+def test_scales_pins_catch_mistakes(mutant):
+    assert not pin_scales_golden(mutant)
+
+
 def test_footprint_matches_printed_ratio():
     from weight_only_quantized_bcq_b200.roofline import bits_per_weight
     gold = _golden("opt175b_footprint.json")
