@@ -221,6 +221,80 @@ def test_full_size_sampled(L, name, m, n, q, g, batch, sigma, outl, seed):
 
 
 # ---------------------------------------------------------------------------
+# Unit-major scales: the packing is bit-exact against the oracle, and a run
+# with packed scales gives the same bits as a run with the [q][n/g][m] array.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("q,m,n,g", [(1, 32, 1024, 128), (3, 40, 2048, 128), (2, 33, 640, 128),
+                                     (4, 100, 3072, 384), (5, 70, 2048, 256), (8, 33, 1152, 128)])
+def test_pack_scales_bit_exact(L, q, m, n, g):
+    alpha = S.draw_alpha(S.generator(300 + q), q, m, n, g, 0.02)
+    scales = L.pack_scales(alpha.to(DEV), m, n, g)
+    torch.cuda.synchronize()
+    want = O.pack_scales(alpha.numpy(), g)
+    assert scales.numel() == want.size
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), want.view(np.uint16))
+
+
+PACKED_CASES = [
+    # q, m, n, g, batch, with_off, y_f16
+    (3, 300, 3072, 128, 1, False, False),
+    (3, 257, 2560, 256, 3, True, False),
+    (1, 64, 1024, 128, 2, False, True),
+    (2, 97, 640, 128, 1, True, False),
+    (4, 130, 4096, 512, 4, False, False),
+    (5, 70, 2048, 256, 1, False, False),
+    (8, 129, 3072, 128, 2, True, True),
+]
+
+
+@pytest.mark.parametrize("q,m,n,g,batch,with_off,y_f16", PACKED_CASES)
+def test_packed_scales_give_identical_bits(L, q, m, n, g, batch, with_off, y_f16):
+    signs, alpha, x = _problem(400 + q + m, q, m, n, g, batch)
+    offset = None
+    if with_off:
+        offset = (torch.randn((n // g, m), generator=S.generator(m + 7)) * 0.05).to(torch.float16).float().to(DEV)
+    packed = L.pack_bcq(signs.to(DEV))
+    a_d, x_d = alpha.to(DEV), x.to(DEV)
+    scales = L.pack_scales(a_d, m, n, g)
+    y_raw = L.run(packed, a_d, x_d, m, n, q, g, offset=offset, y_f16=y_f16)
+    y_pk = L.run(packed, scales, x_d, m, n, q, g, offset=offset, y_f16=y_f16, scales_packed=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y_raw, y_pk)
+    y_ref = O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), g,
+                         None if offset is None else offset.cpu().numpy())
+    if not y_f16:
+        ok, st = compare(y_pk.cpu().numpy(), y_ref, alpha.numpy(), x.numpy(), n)
+        assert ok, st
+
+
+def test_packed_scales_full_size_fc1(L):
+    """OPT-175B FC1 (49152 x 12288, q=3, g=128, batch 1) with packed scales, as
+    the benchmark runs it: sampled rows against the oracle."""
+    m, n, q, g, seed = 49152, 12288, 3, 128, 2
+    gen = S.generator(seed)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n))
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.02)
+    x = S.draw_x(gen, 1, n)
+    scales = L.pack_scales(alpha.to(DEV), m, n, g)
+    y = L.run(packed.to(DEV), scales, x.to(DEV), m, n, q, g, scales_packed=True)
+    torch.cuda.synchronize()
+    rows = _sample_rows(m, seed=seed)
+    s_rows = O.unpack_rows(packed.numpy(), q, m, n, rows)
+    a_rows = alpha.numpy()[:, :, rows]
+    y_ref = O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g)
+    ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_rows, x.numpy(), n)
+    assert ok, st
+
+
+def test_packed_scales_rejected_for_small_groups(L):
+    signs, alpha, x = _problem(88, 3, 64, 1024, 64, 1)
+    packed = L.pack_bcq(signs.to(DEV))
+    with pytest.raises(L.LutgemmError) as e:
+        L.run(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 64, scales_packed=True)
+    assert e.value.status == L.ERR_VALUE
+
+
+# ---------------------------------------------------------------------------
 # Output modes, determinism, workspace contract, streams.
 # ---------------------------------------------------------------------------
 def test_y_f16_is_rounded_fp32(L):

@@ -71,6 +71,19 @@ def test_noalloc_matches_run_on_consecutive_calls(L, q, m, n, g, batch, with_off
         assert ok, st
 
 
+def test_noalloc_with_packed_scales_matches_run(L):
+    """Unit-major scales through the no-alloc call give the bits of lutgemm_run."""
+    q, m, n, g, batch = 3, 300, 3072, 128, 2
+    signs, alpha, x, _ = _inputs(555, q, m, n, g, batch, False)
+    packed = L.pack_bcq(signs.to(DEV))
+    scales = L.pack_scales(alpha.to(DEV), m, n, g)
+    x_d = x.to(DEV)
+    y_run = L.run(packed, scales, x_d, m, n, q, g, scales_packed=True)
+    y = L.run_noalloc(packed, scales, x_d, m, n, q, g, scales_packed=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_run)
+
+
 def test_noalloc_full_size_layer_linear_twice(L):
     """The OPT-175B FC1 shape at batch 1 fits the scratch; two calls in a row."""
     m, n, q, g = 49152, 12288, 3, 128

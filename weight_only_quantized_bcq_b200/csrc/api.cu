@@ -14,6 +14,8 @@ cudaError_t launch_pack_signs(const int8_t* signs, int q, int m, int n, uint8_t*
 cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, const uint8_t* zero, int q,
                                   int m, int n, int g, uint8_t* packed, __half* alpha, float* offset,
                                   int32_t* flags, cudaStream_t stream);
+cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
+                               cudaStream_t stream);
 }  // namespace lutgemm
 
 namespace {
@@ -80,13 +82,13 @@ int group_mode(int g) {
   return kGAny;
 }
 
-RunKernel select_kernel(int q, int mode, bool has_offset) {
+RunKernel select_kernel(int q, int mode, bool has_offset, bool packed) {
   switch (q) {
-    case 1: return run_kernel_q1(mode, has_offset);
-    case 2: return run_kernel_q2(mode, has_offset);
-    case 3: return run_kernel_q3(mode, has_offset);
-    case 4: return run_kernel_q4(mode, has_offset);
-    default: return run_kernel_q8(mode, has_offset);
+    case 1: return run_kernel_q1(mode, has_offset, packed);
+    case 2: return run_kernel_q2(mode, has_offset, packed);
+    case 3: return run_kernel_q3(mode, has_offset, packed);
+    case 4: return run_kernel_q4(mode, has_offset, packed);
+    default: return run_kernel_q8(mode, has_offset, packed);
   }
 }
 
@@ -121,6 +123,21 @@ const char* lutgemm_status_string(int status) {
 size_t lutgemm_packed_bytes(int q, int m, int n) {
   if (!valid_matrix(q, m, n)) return 0;
   return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * q * kBlockBytes;
+}
+
+size_t lutgemm_scales_bytes(int q, int m, int n, int g) {
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g % 128 != 0) return 0;
+  const size_t sp = q < 4 ? (size_t)q : 4u;
+  return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * ceil_div(q, 4) * 512u * sp;
+}
+
+int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g, uint16_t* scales, void* stream) {
+  if (!alpha || !scales) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g % 128 != 0) return LUTGEMM_ERR_SHAPE;
+  if (!aligned(alpha, 2) || !aligned(scales, 16)) return LUTGEMM_ERR_ALIGN;
+  const cudaError_t err = launch_pack_scales(reinterpret_cast<const __half*>(alpha), q, m, n, g, scales,
+                                             reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g) {
@@ -158,10 +175,12 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   if (!packed || !alpha || !x || !y || !workspace) return LUTGEMM_ERR_NULL;
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED)) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
-  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||
-      !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
+  const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
+  if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
+  if (!aligned(packed, 16) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(offset, 4) ||
+      !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
     return LUTGEMM_ERR_ALIGN;
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
 
@@ -187,7 +206,8 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   p.tile_cnt = reinterpret_cast<unsigned*>(ws + tile_off);
   p.status = reinterpret_cast<unsigned*>(ws + tile_off + kTileCounterBytes);
 
-  const RunKernel kernel = select_kernel(q, group_mode(g), offset != nullptr);
+  const RunKernel kernel = select_kernel(q, group_mode(g), offset != nullptr, scales_packed);
+  if (kernel == nullptr) return LUTGEMM_ERR_VALUE;
   int sm_count = 0;
   if (device_setup(kernel, &sm_count) != cudaSuccess) return LUTGEMM_ERR_CUDA;
   long long grid = 0;

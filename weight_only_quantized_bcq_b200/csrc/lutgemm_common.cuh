@@ -144,10 +144,12 @@ cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream);
 constexpr unsigned kStatusWindow = 1u;
 constexpr unsigned kStatusTimeout = 2u;
 
-RunKernel run_kernel_q1(int mode, bool has_offset);
-RunKernel run_kernel_q2(int mode, bool has_offset);
-RunKernel run_kernel_q3(int mode, bool has_offset);
-RunKernel run_kernel_q4(int mode, bool has_offset);
-RunKernel run_kernel_q8(int mode, bool has_offset);   // 5 <= q <= 8, planes in groups of four
+// Kernel for q planes, group mode, offsets on/off and unit-major scales on/off
+// (nullptr for unit-major scales with a mode that has several per piece).
+RunKernel run_kernel_q1(int mode, bool has_offset, bool packed);
+RunKernel run_kernel_q2(int mode, bool has_offset, bool packed);
+RunKernel run_kernel_q3(int mode, bool has_offset, bool packed);
+RunKernel run_kernel_q4(int mode, bool has_offset, bool packed);
+RunKernel run_kernel_q8(int mode, bool has_offset, bool packed);   // 5 <= q <= 8, planes in groups of four
 
 }  // namespace lutgemm

@@ -35,7 +35,9 @@
 //     table base, half and band, and one FADD.
 //   * Per-group alpha (and offset) are applied once per piece (g = 128),
 //     per half-piece (g = 64) or per run (other g); the per-piece values are
-//     prefetched up to seven steps ahead in registers.
+//     prefetched up to seven steps ahead in registers.  With scales in the
+//     unit-major layout (g % 128 == 0), a lane's scales for a whole pass over
+//     a tile are SP 16-byte loads, issued one pass ahead.
 //   * Split-K: each unit stores its fp32 partial; a second, small kernel
 //     (programmatically chained) sums the slices of every row in slice order
 //     and writes y.  With a single slice the run kernel writes y itself.
@@ -229,7 +231,7 @@ __device__ __forceinline__ void static_for(std::integer_sequence<int, Is...>, F&
 
 }  // namespace detail
 
-template <int Q, int MODE, bool MULTI, bool HAS_OFF>
+template <int Q, int MODE, bool MULTI, bool HAS_OFF, bool PK>
 __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p) {
   using namespace detail;
   constexpr int SP = step_planes(MULTI ? 8 : Q);       // planes in one step (<= 4)
@@ -258,6 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr int RUN = (MODE == kG128 || MODE == kG128x) ? 16 : (MODE == kG64 ? 8 : 1);
   constexpr int APP = RUN >= 8 ? 16 / RUN : 1;      // prefetched scales per piece
   constexpr bool PRE_ALPHA = RUN >= 8;
+  // Scales in the unit-major layout: p.alpha holds, for every (slice, row
+  // tile, plane group, lane), the 8 x SP scales of that lane's pass.
+  static_assert(!PK || RUN == 16, "unit-major scales need one scale per piece");
   // Register stages of prefetched scales: step j's are loaded NA-1 steps
   // ahead (7 with one scale per piece, 3 with two, to bound registers); the
   // scales come from HBM and their latency under full load is microseconds.
@@ -268,7 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   // before the end.  Three steps cover a tile-counter atomic comfortably.
   constexpr int NEED_A = PRE_ALPHA ? 8 * NPG - (NA - 1) : 8 * NPG;
   constexpr int NEED_R = ((8 / CH) * NPG - S) * CH;
-  constexpr int NEED = NEED_A < NEED_R ? NEED_A : NEED_R;
+  constexpr int NEED_P = PK ? 8 * (NPG - 1) : 8 * NPG;   // next tile's scales: start of its last pass
+  constexpr int NEED_AR = NEED_A < NEED_R ? NEED_A : NEED_R;
+  constexpr int NEED = NEED_AR < NEED_P ? NEED_AR : NEED_P;
   constexpr bool AHEAD1 = NEED >= 3;
 
   const int lane = threadIdx.x & 31;
@@ -337,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   }
 
   uint16_t ab[NA][Q][APP];
+  uint4 sc_cur[PK ? SP : 1], sc_nxt[PK ? SP : 1];   // unit-major scales of this pass and the next
   float ob[NA][APP];
   uint4 wst[CH][SP];       // the pieces of the current ring stage
 
@@ -408,10 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           else G = 16 * s + 2 * P + (r ^ (int)(lam >> 3));
           const bool ok = row < p.m && G < p.ng;
           const __half* ap = p.alpha + (size_t)G * p.m + row;
+          if constexpr (!PK) {
 #pragma unroll
-          for (int i = 0; i < Q; ++i) {
-            const bool live = !MULTI || (pg_ * 4 + i < p.q);
-            ab[SLOT][i][r] = (ok && live) ? ld_u16(ap + (size_t)(pg_ * 4 + i) * plane_stride) : (uint16_t)0;
+            for (int i = 0; i < Q; ++i) {
+              const bool live = !MULTI || (pg_ * 4 + i < p.q);
+              ab[SLOT][i][r] = (ok && live) ? ld_u16(ap + (size_t)(pg_ * 4 + i) * plane_stride) : (uint16_t)0;
+            }
           }
           if constexpr (HAS_OFF) ob[SLOT][r] = (ok && pg_ == 0) ? __ldg(p.offset + (size_t)G * p.m + row) : 0.f;
         }
@@ -434,7 +444,18 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     __syncthreads();  // every warp is done with the previous segment's tables
     build_tables<RUN, HAS_OFF>(p, b, s, chunk_sum, run_sum);
 
+    // Unit-major scales of pass pg_ of row tile R_ (SP 16-byte loads).
+    auto load_scales = [&](int R_, int pg_, uint4 (&dst)[PK ? SP : 1]) {
+      if constexpr (PK) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.alpha) +
+                           ((((size_t)s * p.mt + R_) * npg + pg_) * kTileRows + lane) * SP;
+#pragma unroll
+        for (int e = 0; e < SP; ++e) dst[e] = __ldg(src + e);
+      }
+    };
+
     if (busy) {
+      load_scales(t_cur, 0, sc_cur);
       static_for(std::make_integer_sequence<int, NA - 1>{}, [&]<int D>() {
         load_alpha.template operator()<D>(t_cur, D);
       });
@@ -476,6 +497,12 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
                 more = t_nxt >= 0;
                 nxt_pending = false;
               }
+            }
+            if constexpr (PK && U == 0) {
+              // Scales of the next pass: this tile's next plane group, or the
+              // next tile's first.
+              if (pg + 1 < npg) load_scales(t_cur, pg + 1, sc_nxt);
+              else if (t_nxt >= 0) load_scales(t_nxt, 0, sc_nxt);
             }
             {
               const int ja = j + NA - 1;       // scales NA-1 steps ahead
@@ -526,7 +553,15 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
                 float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) lookup_word<IMM>(word_of(w4, kk), colb[u2][kk], acc0, acc1);
-                yacc = fmaf(h2f(ab[U % NA][i][0]), acc0 + acc1, yacc);
+                float al;
+                if constexpr (PK) {
+                  const int h = U * SP + i;       // half h of the lane's pass scales (unrolled: constant)
+                  const uint32_t w2 = word_of(sc_cur[h / 8], (h / 2) % 4);
+                  al = h2f((uint16_t)((h & 1) ? (w2 >> 16) : (w2 & 0xffffu)));
+                } else {
+                  al = h2f(ab[U % NA][i][0]);
+                }
+                yacc = fmaf(al, acc0 + acc1, yacc);
               } else if constexpr (RUN == 8) {
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -573,6 +608,10 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
               }
             }
           });
+          if constexpr (PK) {
+#pragma unroll
+            for (int e = 0; e < SP; ++e) sc_cur[e] = sc_nxt[e];
+          }
         }
         if (failed) break;
         // One slice: the row's sum is y.  Several: this slice's partial, summed
@@ -637,13 +676,19 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   }
 }
 
+// Kernel for (mode, offsets, unit-major scales); unit-major scales exist
+// only for the one-scale-per-piece modes (g % 128 == 0).
 #define LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, OFFv)                                   \
   switch (mode) {                                                                  \
-    case kG128: return lut_gemm_kernel<Qv, kG128, MULTIv, OFFv>;                   \
-    case kG128x: return lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv>;                 \
-    case kG64: return lut_gemm_kernel<Qv, kG64, MULTIv, OFFv>;                     \
-    case kG8: return lut_gemm_kernel<Qv, kG8, MULTIv, OFFv>;                       \
-    default: return lut_gemm_kernel<Qv, kGAny, MULTIv, OFFv>;                      \
+    case kG128:                                                                    \
+      return packed ? lut_gemm_kernel<Qv, kG128, MULTIv, OFFv, true>               \
+                    : lut_gemm_kernel<Qv, kG128, MULTIv, OFFv, false>;             \
+    case kG128x:                                                                   \
+      return packed ? lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv, true>              \
+                    : lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv, false>;            \
+    case kG64: return packed ? nullptr : lut_gemm_kernel<Qv, kG64, MULTIv, OFFv, false>; \
+    case kG8: return packed ? nullptr : lut_gemm_kernel<Qv, kG8, MULTIv, OFFv, false>;   \
+    default: return packed ? nullptr : lut_gemm_kernel<Qv, kGAny, MULTIv, OFFv, false>;  \
   }
 
 #define LUTGEMM_RUN_SELECT(Qv, MULTIv)                                             \

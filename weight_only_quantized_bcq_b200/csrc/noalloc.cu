@@ -49,14 +49,14 @@ std::set<std::pair<const void*, int>> g_smem_done;
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-RunKernel pick_kernel(int q, int g, bool has_offset) {
+RunKernel pick_kernel(int q, int g, bool has_offset, bool packed) {
   const int mode = g == 128 ? kG128 : (g % 128 == 0 ? kG128x : (g == 64 ? kG64 : (g == 8 ? kG8 : kGAny)));
   switch (q) {
-    case 1: return run_kernel_q1(mode, has_offset);
-    case 2: return run_kernel_q2(mode, has_offset);
-    case 3: return run_kernel_q3(mode, has_offset);
-    case 4: return run_kernel_q4(mode, has_offset);
-    default: return run_kernel_q8(mode, has_offset);
+    case 1: return run_kernel_q1(mode, has_offset, packed);
+    case 2: return run_kernel_q2(mode, has_offset, packed);
+    case 3: return run_kernel_q3(mode, has_offset, packed);
+    case 4: return run_kernel_q4(mode, has_offset, packed);
+    default: return run_kernel_q8(mode, has_offset, packed);
   }
 }
 
@@ -113,10 +113,12 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   if (q < 1 || q > 8 || m < 1 || n < 8 || n % 8 != 0 || g < 8 || g % 8 != 0 || n % g != 0 || batch < 1)
     return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED)) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
-  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||
-      !aligned(y, y_f16 ? 2 : 4))
+  const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
+  if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
+  if (!aligned(packed, 16) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(offset, 4) ||
+      !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
   const int ns = ceil_div(n, kSliceInputs);
   const int mt = ceil_div(m, kTileRows);
@@ -124,7 +126,8 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   if (partials > kScratchBytes - kPartOff) return LUTGEMM_ERR_WORKSPACE;
 
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const RunKernel kernel = pick_kernel(q, g, offset != nullptr);
+  const RunKernel kernel = pick_kernel(q, g, offset != nullptr, scales_packed);
+  if (kernel == nullptr) return LUTGEMM_ERR_VALUE;
   DeviceScratch d;
   if (prepare(kernel, st, &d) != cudaSuccess) return LUTGEMM_ERR_CUDA;
 

@@ -125,7 +125,58 @@ __global__ void uniform_scales_kernel(const __half* __restrict__ scale, const ui
   offset[e] = sf * ((float)(top - 1) * 0.5f - (float)zz);
 }
 
+// Unit-major scales: one thread per (slice, row tile, plane group, lane)
+// writes that lane's 8 x SP scales (SP 16-byte stores).  Element (U, e) is
+// alpha[4*pg + e][(1024*s + 128*P) / g][32*R + l], P = U xor 4*(l/16), or 0
+// for a plane, row or piece out of range.
+__global__ void pack_scales_kernel(const __half* __restrict__ alpha, int q, int m, int n, int g, int mt,
+                                   int npg, int sp, long long nthreads, uint4* __restrict__ out) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nthreads) return;
+  const int l = (int)(tid & 31);
+  const long long sRp = tid >> 5;            // ((s*mt + R)*npg + pg)
+  const int pg = (int)(sRp % npg);
+  const long long sR = sRp / npg;
+  const int R = (int)(sR % mt);
+  const int s = (int)(sR / mt);
+  const int row = R * kTileRows + l;
+  const int ng = n / g;
+  uint32_t words[16];
+#pragma unroll
+  for (int w = 0; w < 16; ++w) words[w] = 0u;
+#pragma unroll
+  for (int U = 0; U < 8; ++U) {
+    const int P = U ^ (4 * (l >> 4));
+    const int k0 = s * kSliceInputs + 128 * P;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = 4 * pg + e;
+      if (e < sp && i < q && row < m && k0 < n) {
+        const uint32_t h = __ldg(reinterpret_cast<const unsigned short*>(alpha) +
+                                 ((size_t)i * ng + k0 / g) * (size_t)m + row);
+        const int idx = U * sp + e;
+        words[idx >> 1] |= h << (16 * (idx & 1));
+      }
+    }
+  }
+  uint4* dst = out + (size_t)tid * sp;
+  for (int v = 0; v < sp; ++v) dst[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
+}
+
 }  // namespace
+
+cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
+                               cudaStream_t stream) {
+  const int mt = (m + kTileRows - 1) / kTileRows;
+  const int ns = (n + kSliceInputs - 1) / kSliceInputs;
+  const int npg = (q + 3) / 4;
+  const int sp = q < 4 ? q : 4;
+  const long long nthreads = (long long)ns * mt * npg * 32;
+  const int block = 256;
+  pack_scales_kernel<<<(unsigned)((nthreads + block - 1) / block), block, 0, stream>>>(
+      alpha, q, m, n, g, mt, npg, sp, nthreads, reinterpret_cast<uint4*>(scales));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack_signs(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* flags,
                               cudaStream_t stream) {

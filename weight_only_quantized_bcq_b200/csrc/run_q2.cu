@@ -2,5 +2,5 @@
 #include "lutgemm_run.cuh"
 
 namespace lutgemm {
-RunKernel run_kernel_q2(int mode, bool has_offset) { LUTGEMM_RUN_SELECT(2, false) }
+RunKernel run_kernel_q2(int mode, bool has_offset, bool packed) { LUTGEMM_RUN_SELECT(2, false) }
 }  // namespace lutgemm

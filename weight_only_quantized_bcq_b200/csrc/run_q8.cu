@@ -3,5 +3,5 @@
 #include "lutgemm_run.cuh"
 
 namespace lutgemm {
-RunKernel run_kernel_q8(int mode, bool has_offset) { LUTGEMM_RUN_SELECT(4, true) }
+RunKernel run_kernel_q8(int mode, bool has_offset, bool packed) { LUTGEMM_RUN_SELECT(4, true) }
 }  // namespace lutgemm

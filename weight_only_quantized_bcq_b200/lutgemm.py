@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "liblutgemm.so")
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_VALUE, ERR_CUDA = range(7)
 FLAG_BAD_SIGN, FLAG_BAD_CODE, FLAG_BAD_ZERO = 1, 2, 4
 Y_F16 = 1
+SCALES_PACKED = 2
 
 _lib = None
 
@@ -26,6 +27,8 @@ _SIGNATURES = {
     "lutgemm_status_string": ([_c_int], ctypes.c_char_p),
     "lutgemm_packed_bytes": ([_c_int, _c_int, _c_int], _c_size),
     "lutgemm_workspace_size": ([_c_int, _c_int, _c_int, _c_int, _c_int], _c_size),
+    "lutgemm_scales_bytes": ([_c_int, _c_int, _c_int, _c_int], _c_size),
+    "lutgemm_pack_scales": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lutgemm_pack_bcq": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "lutgemm_uniform_to_bcq": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp],
                                _c_int),
@@ -97,6 +100,25 @@ def new_workspace(m: int, n: int, batch: int, q: int, g: int, device=None) -> to
     return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
 
 
+def scales_bytes(q: int, m: int, n: int, g: int) -> int:
+    """Bytes of the unit-major scale buffer (0 when g % 128 != 0 or the shape is invalid)."""
+    return lib().lutgemm_scales_bytes(q, m, n, g)
+
+
+def pack_scales(alpha: torch.Tensor, m: int, n: int, g: int, stream=None) -> torch.Tensor:
+    """fp16 alpha [q][n/g][m] on the GPU -> unit-major scales (fp16, 1-D), for
+    ``run(..., scales_packed=True)``; needs g % 128 == 0."""
+    _need(alpha, torch.float16, "alpha")
+    q = alpha.shape[0]
+    nbytes = scales_bytes(q, m, n, g)
+    if nbytes == 0:
+        raise LutgemmError(ERR_SHAPE, "lutgemm_scales_bytes")
+    scales = torch.empty(nbytes // 2, dtype=torch.float16, device=alpha.device)
+    _check(lib().lutgemm_pack_scales(_ptr(alpha), q, m, n, g, _ptr(scales), _stream(stream)),
+           "lutgemm_pack_scales")
+    return scales
+
+
 def pack_bcq(signs: torch.Tensor, packed: torch.Tensor = None, status_flags: torch.Tensor = None,
              stream=None) -> torch.Tensor:
     """int8 signs [q][m][n] (+-1) on the GPU -> packed uint8 planes."""
@@ -128,8 +150,9 @@ def uniform_to_bcq(codes: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
 
 def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
         offset: torch.Tensor = None, y: torch.Tensor = None, workspace: torch.Tensor = None,
-        y_f16: bool = False, stream=None) -> torch.Tensor:
-    """y[b] = W x[b] for a packed BCQ weight W (m x n), computed by lutgemm_run."""
+        y_f16: bool = False, scales_packed: bool = False, stream=None) -> torch.Tensor:
+    """y[b] = W x[b] for a packed BCQ weight W (m x n), computed by lutgemm_run.
+    With ``scales_packed`` alpha is the output of ``pack_scales``."""
     _need(packed, torch.uint8, "packed")
     _need(alpha, torch.float16, "alpha")
     _need(x, torch.float16, "x")
@@ -140,15 +163,16 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     if workspace is None:
         workspace = new_workspace(m, n, batch, q, g, device=x.device)
+    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0)
     _check(lib().lutgemm_run(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
-                             Y_F16 if y_f16 else 0, _ptr(workspace), workspace.numel(), _stream(stream)),
+                             flags, _ptr(workspace), workspace.numel(), _stream(stream)),
            "lutgemm_run")
     return y
 
 
 def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
                 offset: torch.Tensor = None, y: torch.Tensor = None, y_f16: bool = False,
-                stream=None) -> torch.Tensor:
+                scales_packed: bool = False, stream=None) -> torch.Tensor:
     """``run`` through lutgemm_run_noalloc, for callers that cannot allocate a
     workspace: the library uses its own fixed 16 MiB device scratch instead.
     Only ``y`` is allocated here, and only when the caller passes none.  Calls
@@ -161,7 +185,8 @@ def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: i
     batch = x.shape[0] if x.dim() == 2 else 1
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
+    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0)
     _check(lib().lutgemm_run_noalloc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x),
-                                     _ptr(y), Y_F16 if y_f16 else 0, _stream(stream)),
+                                     _ptr(y), flags, _stream(stream)),
            "lutgemm_run_noalloc")
     return y
