@@ -154,8 +154,12 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # Workload
 # ---------------------------------------------------------------------------
-def make_layer(q: int, batch: int, seed: int, device, only=None):
-    """Packed planes, scales and inputs of the four linears, resident on `device`."""
+def make_layer(q: int, batch: int, seed: int, device, only=None, scales="packed"):
+    """Packed planes, scales and inputs of the four linears, resident on `device`.
+
+    With scales="packed" the [q][n/g][m] scales are reordered once, at load
+    time, into the unit-major layout that lutgemm_run reads with
+    LUTGEMM_SCALES_PACKED (same bytes for g = 128)."""
     from weight_only_quantized_bcq_b200 import lutgemm
     w = S.WORKLOADS[WORKLOAD]
     gen = S.generator(seed)
@@ -166,9 +170,12 @@ def make_layer(q: int, batch: int, seed: int, device, only=None):
         nbytes = lutgemm.packed_bytes(q, sh.m, sh.n)
         packed = S.draw_random_bytes(gen, nbytes).to(device)
         alpha = S.draw_alpha(gen, q, sh.m, sh.n, w.g, w.alpha_sigma).to(device)
+        if scales == "packed":
+            alpha = lutgemm.pack_scales(alpha, sh.m, sh.n, w.g)
         x_host = S.draw_x(gen, batch, sh.n).pin_memory()
         mats.append({
             "name": sh.name, "m": sh.m, "n": sh.n, "packed": packed, "alpha": alpha,
+            "scales_packed": scales == "packed", "launches": 1 + (sh.n > 1024),
             "x_host": x_host, "x": x_host.to(device),
             "y": torch.empty((batch, sh.m), dtype=torch.float32, device=device),
             "y_host": torch.empty((batch, sh.m), dtype=torch.float32).pin_memory(),
@@ -176,6 +183,25 @@ def make_layer(q: int, batch: int, seed: int, device, only=None):
             "bytes": algorithmic_bytes(sh.m, sh.n, q, w.g, batch),
         })
     return mats, w.g
+
+
+def max_over_ranks(dist, v: float, device) -> float:
+    """Largest v over all ranks (every rank gets it); v itself without a process group."""
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(step_bytes: int, steps: int, world: int, region_ms: float) -> float:
+    """Whole-job throughput: every rank's bytes over the slowest rank's time (weak scaling)."""
+    return step_bytes * steps * world / (region_ms * 1e-3) / 1e9
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of rank `rank`'s layer: every rank draws its own weights and inputs."""
+    return S.WORKLOADS[WORKLOAD].seed + 1000 * rank
 
 
 def _dist_env():
@@ -199,8 +225,7 @@ def run_lutgemm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
         pg = dist
     q, batch = args.q, args.batch
-    mats, g = make_layer(q, batch, seed=S.WORKLOADS[WORKLOAD].seed + 1000 * rank, device=device,
-                         only=args.only)
+    mats, g = make_layer(q, batch, seed=rank_seed(rank), device=device, only=args.only, scales=args.scales)
     stream = torch.cuda.current_stream()
 
     def step(events=None):
@@ -208,7 +233,7 @@ def run_lutgemm(args):
             if events is not None:
                 events[i][0].record(stream)
             lutgemm.run(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"],
-                        workspace=mt["ws"], stream=stream)
+                        workspace=mt["ws"], scales_packed=mt["scales_packed"], stream=stream)
             if events is not None:
                 events[i][1].record(stream)
 
@@ -216,7 +241,7 @@ def run_lutgemm(args):
         for mt in mats:
             mt["x"].copy_(mt["x_host"], non_blocking=True)
             lutgemm.run(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"],
-                        workspace=mt["ws"], stream=stream)
+                        workspace=mt["ws"], scales_packed=mt["scales_packed"], stream=stream)
             mt["y_host"].copy_(mt["y"], non_blocking=True)
 
     def barrier():
@@ -224,13 +249,6 @@ def run_lutgemm(args):
         if pg is not None:
             pg.barrier()
         torch.cuda.synchronize()
-
-    def max_over_ranks(v: float) -> float:
-        if pg is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(args.warmup):
         step()
@@ -247,7 +265,7 @@ def run_lutgemm(args):
             step()
         t1.record(stream)
         barrier()
-    region_ms = max_over_ranks(t0.elapsed_time(t1))
+    region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
 
     # Per-linear times: a separate pass with events around every launch (the
     # events serialise the launches, so these are isolated kernel times).
@@ -270,12 +288,11 @@ def run_lutgemm(args):
         e2e_step()
     e1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1), device)
 
     step_bytes = sum(mt["bytes"] for mt in mats)
-    total_bytes = step_bytes * args.steps * world
-    value = total_bytes / (region_ms * 1e-3) / 1e9
-    e2e_gbs = total_bytes / (e2e_ms * 1e-3) / 1e9
+    value = aggregate_gbs(step_bytes, args.steps, world, region_ms)
+    e2e_gbs = aggregate_gbs(step_bytes, args.steps, world, e2e_ms)
     # Every launch in the region is lut_gemm_kernel: its achieved bandwidth is
     # the algorithmic bytes of all launches over the region's device time.
     achieved = step_bytes * args.steps / (region_ms * 1e-3) / 1e9
@@ -305,6 +322,8 @@ def run_lutgemm(args):
                 "q": q, "g": g, "batch": batch,
                 "bytes_per_step": step_bytes,
                 "l2": "no flush: each step streams 765 MB (> 126 MB L2) of distinct weights",
+                "scales": ("unit-major, reordered once at load time (lutgemm_pack_scales)"
+                           if args.scales == "packed" else "[q][n/g][m]"),
                 "parallelism": "replicas" if world == 1 else f"replicas{world} (one layer per GPU)",
                 "only": args.only,
             },
@@ -320,7 +339,8 @@ def run_lutgemm(args):
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
                     "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
-            "gpu_launches": len(mats) * args.steps,
+            # Per lutgemm_run: the lookup kernel, plus the split-K reduce when n > 1024.
+            "gpu_launches": sum(mt["launches"] for mt in mats) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -414,6 +434,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=512, help="rows per linear in the CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="rows per linear per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scales", choices=["packed", "raw"], default="packed",
+                    help="scale layout lutgemm_run reads (packed: unit-major, reordered at load time)")
     ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
                     help="time one linear of the layer only (profiling)")
     args = ap.parse_args()
