@@ -226,7 +226,10 @@ def run_lutgemm(args):
         pg = dist
     q, batch = args.q, args.batch
     mats, g = make_layer(q, batch, seed=rank_seed(rank), device=device, only=args.only, scales=args.scales)
-    stream = torch.cuda.current_stream()
+    # All work goes on one non-default stream (a CUDA graph cannot be captured
+    # on the legacy default stream); it is made current so torch's copies use it.
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
 
     def step(events=None):
         for i, mt in enumerate(mats):
@@ -254,18 +257,36 @@ def run_lutgemm(args):
         step()
     barrier()
 
-    # Device-resident timing: K steps launched back to back (consecutive
-    # launches overlap their ramps by programmatic dependent launch), with
-    # CUDA events on the launching stream around the whole region.
+    # Device-resident timing: K steps back to back (consecutive launches
+    # overlap their ramps by programmatic dependent launch), with CUDA events
+    # on the launching stream around the whole region.  By default the steps
+    # are replayed from a CUDA graph of G steps (the launches of a decode
+    # step, captured once as a serving runtime would), K/G replays.
+    per_graph = 0
+    graph = None
+    if args.graph_steps > 0:
+        per_graph = args.graph_steps if args.steps % args.graph_steps == 0 else 1
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(per_graph):
+                step()
+        graph.replay()  # untimed: uploads the graph and runs its steps once
+        barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clocks:
         barrier()
         t0.record(stream)
-        for _ in range(args.steps):
-            step()
+        if graph is not None:
+            for _ in range(args.steps // per_graph):
+                graph.replay()
+        else:
+            for _ in range(args.steps):
+                step()
         t1.record(stream)
         barrier()
     region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
+    if graph is not None:
+        del graph
 
     # Per-linear times: a separate pass with events around every launch (the
     # events serialise the launches, so these are isolated kernel times).
@@ -324,6 +345,8 @@ def run_lutgemm(args):
                 "l2": "no flush: each step streams 765 MB (> 126 MB L2) of distinct weights",
                 "scales": ("unit-major, reordered once at load time (lutgemm_pack_scales)"
                            if args.scales == "packed" else "[q][n/g][m]"),
+                "launch": (f"CUDA graph of {per_graph} steps, replayed {args.steps // per_graph} times"
+                           if per_graph else "eager launches"),
                 "parallelism": "replicas" if world == 1 else f"replicas{world} (one layer per GPU)",
                 "only": args.only,
             },
@@ -434,6 +457,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=512, help="rows per linear in the CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="rows per linear per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph-steps", type=int, default=10,
+                    help="steps per captured CUDA graph in the timed region (0: eager launches)")
     ap.add_argument("--scales", choices=["packed", "raw"], default="packed",
                     help="scale layout lutgemm_run reads (packed: unit-major, reordered at load time)")
     ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
