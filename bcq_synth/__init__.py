@@ -34,6 +34,7 @@ __all__ = [
     "draw_alpha",
     "draw_uniform",
     "draw_x",
+    "draw_weights",
     "Shape",
     "WORKLOADS",
 ]
@@ -80,6 +81,12 @@ def draw_uniform(gen: torch.Generator, m: int, n: int, g: int, q: int, s_sigma: 
     scale = scale.to(torch.float16).contiguous()
     zero = torch.randint(0, top, (ng, m), generator=gen, dtype=torch.uint8)
     return codes, scale, zero
+
+
+def draw_weights(gen: torch.Generator, m: int, n: int, sigma: float) -> torch.Tensor:
+    """Dense FP16 weights W ~ N(0, sigma) [m][n] (the input of BCQ fitting)."""
+    w = torch.randn((m, n), generator=gen, dtype=torch.float32).mul_(sigma)
+    return w.to(torch.float16).contiguous()
 
 
 def draw_x(gen: torch.Generator, batch: int, n: int, outlier_frac: float = 0.0,

@@ -58,6 +58,7 @@ __all__ = [
     "packed_nbytes", "pack_bcq", "unpack_bcq", "unpack_rows",
     "scales_nbytes", "pack_scales", "unpack_scales",
     "uniform_to_bcq", "uniform_dequant", "bcq_matmul_rows",
+    "fit_bcq", "fit_bcq_trace", "nearest_codes",
 ]
 
 
@@ -342,3 +343,113 @@ def uniform_dequant(codes, scale, zero, g: int) -> np.ndarray:
     s = np.repeat(np.asarray(scale, dtype=np.float16).astype(np.float64), g, axis=0).T
     z = np.repeat(np.asarray(zero, dtype=np.float64), g, axis=0).T
     return s * (c - z)
+
+
+# ---------------------------------------------------------------------------
+# BCQ fitting: FP16 weights -> q sign planes and group scales (the step before
+# the lookup path).  The pages only cite the method (LUT-GEMM card, reference
+# 48: "Alternating multi-bit quantization"; Summary: weights are stored in
+# BCQ).  Reading used here, per (row j, group G of g inputs), in FP64:
+#   1. greedy: r = w; for i = 0..q-1: beta_i = sign(r) (sign(0) = +1),
+#      alpha_i = mean(beta_i * r) = mean|r|, r -= alpha_i * beta_i;
+#   2. `iters` rounds of
+#      a. alpha-step: least squares alpha = argmin |w - B alpha|^2 with the
+#         signs B (g x q) fixed, by Cholesky of B^T B; a pivot <= 1e-6 * g
+#         (planes linearly dependent on the group) keeps the previous alpha;
+#      b. beta-step: each input independently takes the sign combination
+#         whose value sum_i alpha_i s_i is nearest to w (ties: the largest
+#         code c, where bit i of c set means s_i = +1, so w = 0 at q = 1
+#         keeps the greedy sign +1);
+#   3. alpha is rounded to FP16 and a last beta-step uses the rounded alpha, so
+#      the stored signs are the best ones for the stored scales.
+# Each alpha-step and beta-step can only lower |w - B alpha|^2.
+# ---------------------------------------------------------------------------
+PIVOT_REL = 1e-6
+
+
+def _code_signs(q: int) -> np.ndarray:
+    """[2^q][q] sign matrix: row c has s_i = +1 iff bit i of c is set."""
+    c = np.arange(1 << q)[:, None]
+    return np.where((c >> np.arange(q)[None, :]) & 1, 1.0, -1.0)
+
+
+def nearest_codes(w_groups, alpha):
+    """beta-step.  w_groups [..., g], alpha [q, ...] -> signs [q, ..., g] (+-1.0)."""
+    a = np.asarray(alpha, dtype=np.float64)
+    q = a.shape[0]
+    S = _code_signs(q)                                   # [C][q]
+    vals = np.einsum("cq,q...->...c", S, a)              # [..., C]
+    d = np.abs(np.asarray(w_groups, dtype=np.float64)[..., :, None] - vals[..., None, :])
+    C = S.shape[0]
+    best = C - 1 - np.argmin(d[..., ::-1], axis=-1)      # ties: the largest code
+    return np.moveaxis(S[best], -1, 0)                   # [q, ..., g]
+
+
+def _ls_alpha(w_groups, B, a_old, g: int):
+    """alpha-step: Cholesky solve of (B^T B) alpha = B^T w per group."""
+    q = B.shape[0]
+    M = np.einsum("i...k,j...k->...ij", B, B)
+    v = np.einsum("i...k,...k->...i", B, w_groups)
+    L = np.zeros(M.shape)
+    ok = np.ones(M.shape[:-2], dtype=bool)
+    for i in range(q):
+        for j in range(i + 1):
+            acc = M[..., i, j] - np.einsum("...k,...k->...", L[..., i, :j], L[..., j, :j])
+            if i == j:
+                ok &= acc > PIVOT_REL * g
+                L[..., i, i] = np.sqrt(np.maximum(acc, PIVOT_REL * g))
+            else:
+                L[..., i, j] = acc / L[..., j, j]
+    y = np.zeros(v.shape)
+    for i in range(q):                                   # L y = v
+        y[..., i] = (v[..., i] - np.einsum("...k,...k->...", L[..., i, :i], y[..., :i])) / L[..., i, i]
+    a = np.zeros(v.shape)
+    for i in reversed(range(q)):                         # L^T a = y
+        a[..., i] = (y[..., i] - np.einsum("...k,...k->...", L[..., i + 1:, i], a[..., i + 1:])) / L[..., i, i]
+    a = np.moveaxis(a, -1, 0)
+    return np.where(ok[None], a, a_old)
+
+
+def _fit_groups(w, q: int, g: int, iters: int, trace=None):
+    W = np.asarray(w, dtype=np.float64)
+    m, n = W.shape
+    if n % g != 0:
+        raise ValueError("n % g != 0")
+    Wg = W.reshape(m, n // g, g)
+    r = Wg.copy()
+    B = np.empty((q,) + Wg.shape)
+    a = np.empty((q,) + Wg.shape[:-1])
+    for i in range(q):
+        B[i] = np.where(r >= 0, 1.0, -1.0)
+        a[i] = (B[i] * r).sum(-1) / g
+        r -= a[i][..., None] * B[i]
+    if trace is not None:
+        trace.append(((Wg - np.einsum("i...,i...k->...k", a, B)) ** 2).sum(-1))
+    for _ in range(iters):
+        a = _ls_alpha(Wg, B, a, g)
+        if trace is not None:
+            trace.append(((Wg - np.einsum("i...,i...k->...k", a, B)) ** 2).sum(-1))
+        B = nearest_codes(Wg, a)
+        if trace is not None:
+            trace.append(((Wg - np.einsum("i...,i...k->...k", a, B)) ** 2).sum(-1))
+    return Wg, a, B
+
+
+def fit_bcq(w, q: int, g: int, iters: int):
+    """FP16 W [m][n] -> (signs int8 [q][m][n], alpha fp16 [q][n/g][m],
+    squared error per group fp64 [n/g][m] of the stored result)."""
+    Wg, a, _ = _fit_groups(w, q, g, iters)
+    a16 = a.astype(np.float16)
+    B = nearest_codes(Wg, a16.astype(np.float64))
+    err = ((Wg - np.einsum("i...,i...k->...k", a16.astype(np.float64), B)) ** 2).sum(-1)
+    m, ng, _ = Wg.shape
+    signs = B.reshape(q, m, ng * g).astype(np.int8)
+    return signs, np.ascontiguousarray(np.transpose(a16, (0, 2, 1))), np.ascontiguousarray(err.T)
+
+
+def fit_bcq_trace(w, q: int, g: int, iters: int):
+    """Squared error per group after the greedy pass and after every alpha- and
+    beta-step (unrounded alpha), as a list of [m][n/g] arrays."""
+    trace = []
+    _fit_groups(w, q, g, iters, trace)
+    return trace

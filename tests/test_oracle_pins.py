@@ -569,3 +569,192 @@ def test_footprint_matches_printed_ratio():
     assert abs(gold["fp16_gb"] / gold["lutgemm_gb"] - ratio) < 0.01
     # g = 128 would not reproduce it (4.74x): the count is sensitive to the scale term.
     assert round(16.0 / bits_per_weight(3, 128), 2) == 4.74
+
+
+# ---------------------------------------------------------------------------
+# BCQ fitting (greedy + alternating least squares): closed forms, exact
+# recovery of representable weights, brute force on tiny cases, monotone
+# error, and planted mistakes.
+# ---------------------------------------------------------------------------
+def _fp16_weights(rng, m, n, sigma=0.02):
+    return (rng.standard_normal((m, n)) * sigma).astype(np.float16)
+
+
+def pin_fit_q1_closed_form(fit_bcq) -> bool:
+    """q = 1: beta = sign(w) (0 -> +1), alpha = fp16(mean |w|), for any iters."""
+    rng = np.random.default_rng(11)
+    w = _fp16_weights(rng, 6, 256)
+    w[0, :5] = 0
+    for iters in (0, 2):
+        signs, alpha, _ = fit_bcq(w, 1, 64, iters)
+        want_s = np.where(w.astype(np.float64) >= 0, 1, -1)
+        want_a = np.abs(w.astype(np.float64)).reshape(6, 4, 64).mean(-1).astype(np.float16).T
+        if not (np.array_equal(signs[0], want_s) and np.array_equal(alpha[0].view(np.uint16),
+                                                                    want_a.view(np.uint16))):
+            return False
+    return True
+
+
+def _representable(rng, m, ng, g):
+    """w = c * (b1 + b2/2 + b3/4) per group, c a power of two: exact in fp16."""
+    c = 2.0 ** rng.integers(-9, -4, size=(m, ng))
+    b = rng.choice([-1.0, 1.0], size=(3, m, ng, g))
+    w = c[..., None] * (b[0] + b[1] / 2 + b[2] / 4)
+    return w.reshape(m, ng * g).astype(np.float16), b, c
+
+
+def pin_fit_exact_recovery(fit_bcq) -> bool:
+    rng = np.random.default_rng(12)
+    w, b, c = _representable(rng, 5, 3, 128)
+    signs, alpha, err = fit_bcq(w, 3, 128, 3)
+    want_a = np.stack([c, c / 2, c / 4]).transpose(0, 2, 1)
+    return (np.array_equal(signs.reshape(3, 5, 3, 128), b.astype(np.int8))
+            and np.array_equal(alpha.astype(np.float64), want_a) and float(np.abs(err).max()) == 0.0)
+
+
+def pin_fit_q1_global_optimum(fit_bcq) -> bool:
+    """q = 1, g = 8: the fit's error equals the brute-force minimum over all 256 sign vectors."""
+    rng = np.random.default_rng(13)
+    w = _fp16_weights(rng, 3, 8, 1.0)
+    _, alpha, err = fit_bcq(w, 1, 8, 2)
+    for j in range(3):
+        wj = w[j].astype(np.float64)
+        best = min(float(((wj - (s @ wj) / 8 * np.array(s)) ** 2).sum())
+                   for s in itertools.product([-1.0, 1.0], repeat=8))
+        # the fit stores alpha in fp16, so its error may exceed the exact optimum by the rounding
+        a = float(alpha[0, 0, j])
+        if not (best - 1e-12 <= err[0, j] <= best + 8 * abs(a - np.abs(wj).mean()) * np.abs(wj).sum() + 1e-12):
+            return False
+    return True
+
+
+def pin_nearest_codes_bruteforce(nearest_codes) -> bool:
+    rng = np.random.default_rng(14)
+    q, g = 3, 16
+    w = rng.standard_normal((4, g))
+    a = np.abs(rng.standard_normal((q, 4))) + 0.1
+    got = nearest_codes(w, a)
+    for r in range(4):
+        for k in range(g):
+            best, arg = None, None
+            for s in itertools.product([-1.0, 1.0], repeat=q):
+                v = sum(a[i, r] * s[i] for i in range(q))
+                if best is None or abs(w[r, k] - v) < best:
+                    best, arg = abs(w[r, k] - v), s
+            if tuple(got[:, r, k]) != arg:
+                return False
+    return True
+
+
+def pin_fit_stored_signs_are_best(fit_bcq) -> bool:
+    """Every stored sign combination is a nearest one for the stored fp16 scales
+    (brute force over the 2^q combinations), and the returned error is the
+    error of the stored result."""
+    rng = np.random.default_rng(18)
+    q, g, m, n = 3, 128, 24, 512
+    w = _fp16_weights(rng, m, n)
+    signs, alpha, err = fit_bcq(w, q, g, 2)
+    combos = np.array(list(itertools.product([-1.0, 1.0], repeat=q)))      # [8][q]
+    for j in range(m):
+        for G in range(n // g):
+            a = alpha[:, G, j].astype(np.float64)
+            vals = combos @ a
+            wk = w[j, G * g:(G + 1) * g].astype(np.float64)
+            v = np.einsum("i,ik->k", a, signs[:, j, G * g:(G + 1) * g].astype(np.float64))
+            best = np.abs(wk[:, None] - vals[None, :]).min(axis=1)
+            if np.any(np.abs(wk - v) > best + 1e-15):
+                return False
+            e = float(((wk - v) ** 2).sum())
+            if abs(e - err[G, j]) > 1e-12 * max(e, 1e-30):
+                return False
+    return True
+
+
+def test_fit_pins():
+    assert pin_fit_stored_signs_are_best(O.fit_bcq)
+    assert pin_fit_q1_closed_form(O.fit_bcq)
+    assert pin_fit_exact_recovery(O.fit_bcq)
+    assert pin_fit_q1_global_optimum(O.fit_bcq)
+    assert pin_nearest_codes_bruteforce(O.nearest_codes)
+
+
+@pytest.mark.parametrize("q,g", [(2, 64), (3, 128), (4, 128), (3, 8)])
+def test_fit_error_never_rises(q, g):
+    rng = np.random.default_rng(15 + q)
+    w = _fp16_weights(rng, 7, 512)
+    trace = O.fit_bcq_trace(w, q, g, 4)
+    scale = (w.astype(np.float64).reshape(7, -1, g) ** 2).sum(-1)
+    for before, after in zip(trace, trace[1:]):
+        assert np.all(after <= before + 1e-12 * scale)
+    assert np.all(trace[-1] < trace[0] + 1e-12 * scale)
+
+
+def test_alpha_step_matches_least_squares():
+    """The Cholesky alpha-step against numpy's least-squares solver."""
+    rng = np.random.default_rng(16)
+    q, g = 4, 64
+    B = rng.choice([-1.0, 1.0], size=(q, 9, g))
+    w = rng.standard_normal((9, g))
+    a = O._ls_alpha(w, B, np.zeros((q, 9)), g)
+    for r in range(9):
+        ref = np.linalg.lstsq(B[:, r, :].T, w[r], rcond=None)[0]
+        assert np.allclose(a[:, r], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_alpha_step_keeps_alpha_for_dependent_planes():
+    rng = np.random.default_rng(17)
+    B = rng.choice([-1.0, 1.0], size=(2, 1, 32))
+    B[1] = -B[0]                                   # plane 1 = -plane 0: singular normal matrix
+    old = np.array([[0.3], [0.2]])
+    a = O._ls_alpha(rng.standard_normal((1, 32)), B, old, 32)
+    assert np.array_equal(a, old)
+
+
+def _fit_no_residual(w, q, g, iters):
+    """Planted: the greedy pass never subtracts the fitted plane."""
+    W = np.asarray(w, dtype=np.float64)
+    m, n = W.shape
+    Wg = W.reshape(m, n // g, g)
+    B = np.stack([np.where(Wg >= 0, 1.0, -1.0)] * q)
+    a = np.stack([np.abs(Wg).mean(-1)] * q)
+    for _ in range(iters):
+        a = O._ls_alpha(Wg, B, a, g)
+        B = O.nearest_codes(Wg, a)
+    a16 = a.astype(np.float16)
+    B = O.nearest_codes(Wg, a16.astype(np.float64))
+    err = ((Wg - np.einsum("i...,i...k->...k", a16.astype(np.float64), B)) ** 2).sum(-1)
+    return B.reshape(q, m, n).astype(np.int8), np.transpose(a16, (0, 2, 1)), err.T
+
+
+def _fit_alpha_not_rounded_for_signs(w, q, g, iters):
+    """Planted: alpha rounded to fp16 after the signs were chosen with the exact alpha."""
+    Wg, a, B = O._fit_groups(w, q, g, iters)
+    a16 = a.astype(np.float16)
+    err = ((Wg - np.einsum("i...,i...k->...k", a16.astype(np.float64), B)) ** 2).sum(-1)
+    m, ng, _ = Wg.shape
+    return B.reshape(q, m, ng * g).astype(np.int8), np.transpose(a16, (0, 2, 1)), err.T
+
+
+def _nearest_farthest(w_groups, alpha):
+    """Planted: the beta-step takes the farthest code."""
+    a = np.asarray(alpha, dtype=np.float64)
+    S = O._code_signs(a.shape[0])
+    vals = np.einsum("cq,q...->...c", S, a)
+    d = np.abs(np.asarray(w_groups)[..., :, None] - vals[..., None, :])
+    return np.moveaxis(S[np.argmax(d, axis=-1)], -1, 0)
+
+
+def _nearest_bits_reversed(w_groups, alpha):
+    """Planted: code bit i mapped to plane q-1-i."""
+    return O.nearest_codes(w_groups, np.asarray(alpha)[::-1])
+
+
+@pytest.mark.parametrize("mutant", [_fit_no_residual, _fit_alpha_not_rounded_for_signs])
+def test_fit_pins_catch_mistakes(mutant):
+    assert not (pin_fit_q1_closed_form(mutant) and pin_fit_exact_recovery(mutant)
+                and pin_fit_q1_global_optimum(mutant) and pin_fit_stored_signs_are_best(mutant))
+
+
+@pytest.mark.parametrize("mutant", [_nearest_farthest, _nearest_bits_reversed])
+def test_nearest_codes_pin_catches_mistakes(mutant):
+    assert not pin_nearest_codes_bruteforce(mutant)
