@@ -162,6 +162,30 @@ int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
                            uint8_t* packed, uint16_t* alpha, float* offset,
                            int32_t* status_flags, void* stream);
 
+/* Fit q sign planes and group-wise fp16 scales to dense fp16 weights: BCQ
+ * quantisation, the step that produces the weights lutgemm_run consumes
+ * (LUT-GEMM card, Summary: weights stored in BCQ; the pages cite the
+ * alternating multi-bit method, reference 48, without detail).  Per (row,
+ * group of g inputs): greedy signs of the residual with scales mean|r|, then
+ * `iters` rounds of a least-squares scale step (a plane set that is linearly
+ * dependent on the group keeps its scales) and a nearest-code sign step
+ * (ties go to the largest code c, where bit i of c set means beta_i = +1);
+ * scales are rounded to fp16 and the signs refitted to the rounded scales.  Arithmetic is fp32 in a fixed order (results are
+ * reproducible).
+ *   w          dev fp16 [m][n], 16-byte aligned
+ *   q, m, n, g 1 <= q <= 8, m >= 1, n % 8 == 0, g % 8 == 0, n % g == 0,
+ *              g <= 1024
+ *   iters      0..64 alternating rounds (0: greedy only)
+ *   signs      dev int8 [q][m][n], 8-byte aligned (output, each -1 or +1;
+ *              the input of lutgemm_pack_bcq)
+ *   alpha      dev fp16 [q][n/g][m], 2-byte aligned (output)
+ *   err        dev fp32 [n/g][m], 4-byte aligned, or NULL (output: squared
+ *              error of each group with the stored signs and scales)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also for g > 1024), ERR_VALUE
+ * (iters out of range), ERR_ALIGN or ERR_CUDA. */
+int lutgemm_fit_bcq(const uint16_t* w, int q, int m, int n, int g, int iters,
+                    int8_t* signs, uint16_t* alpha, float* err, void* stream);
+
 /* Reorder group-wise plane scales into the unit-major scale layout above
  * (a data movement only: every output is one input value or 0).  The scales
  * are those of the BCQ format (LUT-GEMM card, Summary: q binary planes, each

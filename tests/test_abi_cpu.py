@@ -126,6 +126,28 @@ def test_scales_bytes(L):
     assert L.scales_bytes(9, 64, 1024, 128) == 0
 
 
+def test_fit_validation(L):
+    lib = L.lib()
+    ok = [FAKE, 3, 32, 1024, 128, 3, FAKE, FAKE, None, None]
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[["w", "q", "m", "n", "g", "iters", "signs", "alpha", "err", "stream"].index(k)] = v
+        return lib.lutgemm_fit_bcq(*a)
+    assert call(w=None) == L.ERR_NULL
+    assert call(signs=None) == L.ERR_NULL
+    assert call(alpha=None) == L.ERR_NULL
+    assert call(q=9) == L.ERR_SHAPE
+    assert call(g=96) == L.ERR_SHAPE             # n % g != 0
+    assert call(n=4096, g=2048) == L.ERR_SHAPE   # groups above 1024 inputs
+    assert call(iters=-1) == L.ERR_VALUE
+    assert call(iters=65) == L.ERR_VALUE
+    assert call(w=FAKE + 8) == L.ERR_ALIGN
+    assert call(signs=FAKE + 4) == L.ERR_ALIGN
+    assert call(alpha=FAKE + 1) == L.ERR_ALIGN
+    assert call(err=FAKE + 2) == L.ERR_ALIGN
+
+
 def test_pack_scales_validation(L):
     lib = L.lib()
     assert lib.lutgemm_pack_scales(None, 3, 32, 1024, 128, FAKE, None) == L.ERR_NULL

@@ -16,6 +16,8 @@ cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, con
                                   int32_t* flags, cudaStream_t stream);
 cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
                                cudaStream_t stream);
+cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
+                           float* err, cudaStream_t stream);
 }  // namespace lutgemm
 
 namespace {
@@ -129,6 +131,17 @@ size_t lutgemm_scales_bytes(int q, int m, int n, int g) {
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g % 128 != 0) return 0;
   const size_t sp = q < 4 ? (size_t)q : 4u;
   return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * ceil_div(q, 4) * 512u * sp;
+}
+
+int lutgemm_fit_bcq(const uint16_t* w, int q, int m, int n, int g, int iters, int8_t* signs, uint16_t* alpha,
+                    float* err, void* stream) {
+  if (!w || !signs || !alpha) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g > 1024) return LUTGEMM_ERR_SHAPE;
+  if (iters < 0 || iters > 64) return LUTGEMM_ERR_VALUE;
+  if (!aligned(w, 16) || !aligned(signs, 8) || !aligned(alpha, 2) || !aligned(err, 4)) return LUTGEMM_ERR_ALIGN;
+  const cudaError_t e = launch_fit_bcq(reinterpret_cast<const __half*>(w), q, m, n, g, iters, signs,
+                                       reinterpret_cast<__half*>(alpha), err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 
 int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g, uint16_t* scales, void* stream) {
