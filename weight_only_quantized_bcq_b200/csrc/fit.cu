@@ -13,10 +13,16 @@
 //      a code meaning beta_i = +1);
 //   3. scales rounded to fp16, then a last sign step with the rounded scales.
 //
-// One warp per (row, group); a lane holds up to CPL chunks of 8 consecutive
-// inputs (g <= 256 * CPL).  Signs live in registers as one 64-bit mask per
-// chunk (byte i = plane i).  Sums are taken in a fixed order (per lane in
-// input order, then a butterfly over the warp), so results are reproducible.
+// A group is served by a segment of lpg lanes (the power of two at or above
+// g/8, at most 32), so a warp serves 32/lpg groups at once (two at g = 128);
+// a lane holds up to CPL chunks of 8 consecutive inputs (g <= 256 * CPL).  A chunk's signs are one mask with byte i = plane
+// i (32 bits for q <= 4).  The 2^q code values sit in registers for q <= 4
+// and in shared memory above; a code's mask bits are compile-time constants,
+// so the nearest-code search carries them directly.  Sums are taken in a
+// fixed order (per lane in input order, then a butterfly over the warp), so
+// results are reproducible.
+#include <type_traits>
+
 #include "lutgemm.h"
 #include "lutgemm_common.cuh"
 
@@ -27,60 +33,65 @@ namespace {
 constexpr int kFitWarps = 8;
 constexpr float kPivotRel = 1e-6f;
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+// Sum over an aligned segment of lpg lanes (every lane gets the segment's sum).
+__device__ __forceinline__ float seg_sum(float v, int lpg) {
+  for (int o = lpg >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-__device__ __forceinline__ int warp_sum_i(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+__device__ __forceinline__ int seg_sum_i(int v, int lpg) {
+  for (int o = lpg >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// Nearest code for value w among the 2^q codebook values vals[] (smem).
-__device__ __forceinline__ int nearest(float w, const float* vals, int ncode) {
-  float best = fabsf(w - vals[0]);
-  int arg = 0;
-  for (int c = 1; c < ncode; ++c) {
-    const float d = fabsf(w - vals[c]);
-    if (d <= best) {
-      best = d;
-      arg = c;
-    }
-  }
-  return arg;
+// Code c's sign bits spread to bit 8*i (plane i), element 0.
+__host__ __device__ constexpr uint64_t spread_code(int c, int q) {
+  uint64_t m = 0;
+  for (int i = 0; i < q; ++i) m |= (uint64_t)((c >> i) & 1) << (8 * i);
+  return m;
+}
+
+// Eight 0/1 bits -> eight int8 values +1 / -1 (two 32-bit words).
+__device__ __forceinline__ uint2 bits_to_signs(uint32_t b) {
+  const uint32_t lo = ((b & 0xFu) * 0x00204081u) & 0x01010101u;
+  const uint32_t hi = (((b >> 4) & 0xFu) * 0x00204081u) & 0x01010101u;
+  return make_uint2(0xFFFFFFFFu ^ (lo * 0xFEu), 0xFFFFFFFFu ^ (hi * 0xFEu));
 }
 
 template <int CPL, int Q>
 __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* __restrict__ w, int m, int n, int g,
-                                                               int iters, int8_t* __restrict__ signs,
+                                                               int lpg, int iters, int8_t* __restrict__ signs,
                                                                __half* __restrict__ alpha, float* __restrict__ err) {
-  constexpr int q = Q;
-  __shared__ float codebook[kFitWarps][256];
+  using Mask = std::conditional_t<(Q <= 4), uint32_t, uint64_t>;
+  constexpr int NC = 1 << Q;
+  constexpr bool REG_CODES = Q <= 4;
+  __shared__ float codebook[REG_CODES ? 1 : kFitWarps][REG_CODES ? 1 : NC];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
-  float* vals = codebook[wid];
   const int ng = n / g;
   const int chunks = g / 8;
+  const int gpw = 32 / lpg;                  // groups per warp
+  const int sl = lane & (lpg - 1);           // lane within its segment
   const long long groups = (long long)m * ng;
-  constexpr int ncode = 1 << Q;
   const float inv_g = 1.0f / (float)g;
 
-  for (long long grp = (long long)blockIdx.x * kFitWarps + wid; grp < groups;
-       grp += (long long)gridDim.x * kFitWarps) {
-    const int j = (int)(grp / ng);
-    const int G = (int)(grp - (long long)j * ng);
+  // Warp-uniform loop; a segment whose group is past the end computes on
+  // zeros and stores nothing.
+  for (long long base = ((long long)blockIdx.x * kFitWarps + wid) * gpw; base < groups;
+       base += (long long)gridDim.x * kFitWarps * gpw) {
+    const long long grp = base + lane / lpg;
+    const bool live = grp < groups;
+    const int j = live ? (int)(grp / ng) : 0;
+    const int G = live ? (int)(grp - (long long)j * ng) : 0;
     const __half* src = w + (size_t)j * n + (size_t)G * g;
 
     float x[CPL][8];
-    uint64_t sg[CPL];
+    Mask sg[CPL];
 #pragma unroll
     for (int t = 0; t < CPL; ++t) {
       sg[t] = 0;
-      const int c = lane + 32 * t;
-      if (c < chunks) {
+      const int c = sl + lpg * t;
+      if (live && c < chunks) {
         const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src) + c);
         const __half2* h = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
@@ -96,7 +107,7 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
     }
 
     // 1. Greedy planes on the residual.
-    float a[8];
+    float a[Q];
     {
       float r[CPL][8];
 #pragma unroll
@@ -104,21 +115,20 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
 #pragma unroll
         for (int e = 0; e < 8; ++e) r[t][e] = x[t][e];
 #pragma unroll
-      for (int i = 0; i < q; ++i) {
+      for (int i = 0; i < Q; ++i) {
         float s = 0.f;
 #pragma unroll
         for (int t = 0; t < CPL; ++t) {
-          if (lane + 32 * t >= chunks) continue;
-          uint32_t bits = 0;
+          if (!live || sl + lpg * t >= chunks) continue;
+          Mask bits = 0;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const bool pos = r[t][e] >= 0.f;
-            bits |= (uint32_t)pos << e;
+            bits |= (Mask)(r[t][e] >= 0.f) << e;
             s += fabsf(r[t][e]);
           }
-          sg[t] |= (uint64_t)bits << (8 * i);
+          sg[t] |= bits << (8 * i);
         }
-        const float ai = warp_sum(s) * inv_g;
+        const float ai = seg_sum(s, lpg) * inv_g;
         a[i] = ai;
 #pragma unroll
         for (int t = 0; t < CPL; ++t)
@@ -127,64 +137,101 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
       }
     }
 
-    auto fill_codebook = [&](const float* av) {
-      __syncwarp();
-      for (int c = lane; c < ncode; c += 32) {
-        float v = 0.f;
+    // Nearest-code step for scales av; returns this lane's sum of squared
+    // distances (the group error once the scales are final).
+    auto sign_step = [&](const float (&av)[Q]) -> float {
+      float cb[REG_CODES ? NC : 1];
+      if constexpr (REG_CODES) {
 #pragma unroll
-        for (int i = 0; i < q; ++i) v += ((c >> i) & 1) ? av[i] : -av[i];
-        vals[c] = v;
+        for (int c = 0; c < NC; ++c) {
+          float v = 0.f;
+#pragma unroll
+          for (int i = 0; i < Q; ++i) v += ((c >> i) & 1) ? av[i] : -av[i];
+          cb[c] = v;
+        }
+      } else {
+        __syncwarp();
+        for (int c = lane; c < NC; c += 32) {
+          float v = 0.f;
+#pragma unroll
+          for (int i = 0; i < Q; ++i) v += ((c >> i) & 1) ? av[i] : -av[i];
+          codebook[wid][c] = v;
+        }
+        __syncwarp();
       }
-      __syncwarp();
-    };
-    auto sign_step = [&]() {
+      float e2 = 0.f;
 #pragma unroll
       for (int t = 0; t < CPL; ++t) {
-        if (lane + 32 * t >= chunks) continue;
-        uint64_t m8 = 0;
+        if (!live || sl + lpg * t >= chunks) continue;
+        Mask mk = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint64_t c = (uint64_t)nearest(x[t][e], vals, ncode);
-          // spread code bit i to bit 8*i + e
+          const float xv = x[t][e];
+          float best;
+          Mask arg = 0;
+          if constexpr (REG_CODES) {
+            best = fabsf(xv - cb[0]);
 #pragma unroll
-          for (int i = 0; i < q; ++i) m8 |= ((c >> i) & 1ull) << (8 * i + e);
+            for (int c = 1; c < NC; ++c) {
+              const float d = fabsf(xv - cb[c]);
+              if (d <= best) {
+                best = d;
+                arg = (Mask)spread_code(c, Q);
+              }
+            }
+          } else {
+            best = fabsf(xv - codebook[wid][0]);
+            int ac = 0;
+            for (int c = 1; c < NC; ++c) {
+              const float d = fabsf(xv - codebook[wid][c]);
+              if (d <= best) {
+                best = d;
+                ac = c;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < Q; ++i) arg |= (Mask)((ac >> i) & 1) << (8 * i);
+          }
+          mk |= arg << e;
+          e2 += best * best;
         }
-        sg[t] = m8;
+        sg[t] = mk;
       }
+      return e2;
     };
 
     // 2. Alternating rounds.
     for (int it = 0; it < iters; ++it) {
       // Normal equations: M_ik = g - 2 * #(inputs where planes i and k differ),
       // v_i = sum_k beta_ik * w_k.
-      int diff[36];
-      float v[8];
+      int diff[Q * (Q - 1) / 2 + 1];
+      float v[Q];
 #pragma unroll
-      for (int i = 0; i < q; ++i) {
+      for (int i = 0; i < Q; ++i) {
         float s = 0.f;
 #pragma unroll
         for (int t = 0; t < CPL; ++t) {
-          if (lane + 32 * t >= chunks) continue;
+          if (!live || sl + lpg * t >= chunks) continue;
 #pragma unroll
           for (int e = 0; e < 8; ++e) s += ((sg[t] >> (8 * i + e)) & 1) ? x[t][e] : -x[t][e];
         }
-        v[i] = warp_sum(s);
+        v[i] = seg_sum(s, lpg);
 #pragma unroll
         for (int k = 0; k < i; ++k) {
           int cnt = 0;
 #pragma unroll
           for (int t = 0; t < CPL; ++t) {
-            if (lane + 32 * t >= chunks) continue;
-            cnt += __popc((uint32_t)(((sg[t] >> (8 * i)) ^ (sg[t] >> (8 * k))) & 0xFFull));
+            if (!live || sl + lpg * t >= chunks) continue;
+            cnt += __popc((uint32_t)(((sg[t] >> (8 * i)) ^ (sg[t] >> (8 * k))) & 0xFFu));
           }
-          diff[i * (i - 1) / 2 + k] = warp_sum_i(cnt);
+          diff[i * (i - 1) / 2 + k] = seg_sum_i(cnt, lpg);
         }
       }
       // Cholesky of M (every lane, same arithmetic), then two triangular solves.
-      float L[8][8];
+      float L[Q][Q];
       bool ok = true;
 #pragma unroll
-      for (int i = 0; i < q; ++i) {
+      for (int i = 0; i < Q; ++i) {
 #pragma unroll
         for (int k = 0; k <= i; ++k) {
           float acc = (i == k) ? (float)g : (float)(g - 2 * diff[i * (i - 1) / 2 + k]);
@@ -199,66 +246,45 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
         }
       }
       if (ok) {
-        float y[8];
+        float y[Q];
 #pragma unroll
-        for (int i = 0; i < q; ++i) {
+        for (int i = 0; i < Q; ++i) {
           float acc = v[i];
 #pragma unroll
           for (int l = 0; l < i; ++l) acc -= L[i][l] * y[l];
           y[i] = acc / L[i][i];
         }
 #pragma unroll
-        for (int i = q - 1; i >= 0; --i) {
+        for (int i = Q - 1; i >= 0; --i) {
           float acc = y[i];
 #pragma unroll
-          for (int l = i + 1; l < q; ++l) acc -= L[l][i] * a[l];
+          for (int l = i + 1; l < Q; ++l) acc -= L[l][i] * a[l];
           a[i] = acc / L[i][i];
         }
       }
-      fill_codebook(a);
-      sign_step();
+      (void)sign_step(a);
     }
 
-    // 3. fp16 scales, last sign step with them, outputs.
-    float a16[8];
+    // 3. fp16 scales, last sign step with them (its distances give the error).
+    float a16[Q];
 #pragma unroll
-    for (int i = 0; i < q; ++i) a16[i] = __half2float(__float2half_rn(a[i]));
-    fill_codebook(a16);
-    sign_step();
-    float e2 = 0.f;
+    for (int i = 0; i < Q; ++i) a16[i] = __half2float(__float2half_rn(a[i]));
+    const float e2 = seg_sum(sign_step(a16), lpg);
 #pragma unroll
     for (int t = 0; t < CPL; ++t) {
-      const int c = lane + 32 * t;
-      if (c >= chunks) continue;
+      const int c = sl + lpg * t;
+      if (!live || c >= chunks) continue;
 #pragma unroll
-      for (int i = 0; i < q; ++i) {
-        const uint32_t bits = (uint32_t)((sg[t] >> (8 * i)) & 0xFFull);
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          lo |= (uint32_t)(uint8_t)(((bits >> e) & 1) ? 1 : -1) << (8 * e);
-          hi |= (uint32_t)(uint8_t)(((bits >> (e + 4)) & 1) ? 1 : -1) << (8 * e);
-        }
-        *reinterpret_cast<uint2*>(signs + ((size_t)i * m + j) * n + (size_t)G * g + 8 * c) = make_uint2(lo, hi);
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float vv = 0.f;
-#pragma unroll
-        for (int i = 0; i < q; ++i) vv += ((sg[t] >> (8 * i + e)) & 1) ? a16[i] : -a16[i];
-        const float d = x[t][e] - vv;
-        e2 += d * d;
+      for (int i = 0; i < Q; ++i) {
+        const uint2 sv = bits_to_signs((uint32_t)((sg[t] >> (8 * i)) & 0xFFu));
+        *reinterpret_cast<uint2*>(signs + ((size_t)i * m + j) * n + (size_t)G * g + 8 * c) = sv;
       }
     }
-    e2 = warp_sum(e2);
-    if (lane < q) {
-      float mine = a16[0];
+    // Plane i's scale is written by lane i mod lpg of the segment.
 #pragma unroll
-      for (int i = 1; i < q; ++i)
-        if (lane == i) mine = a16[i];
-      alpha[((size_t)lane * ng + G) * m + j] = __float2half_rn(mine);
-    }
-    if (err && lane == 0) err[(size_t)G * m + j] = e2;
+    for (int i = 0; i < Q; ++i)
+      if (live && (i & (lpg - 1)) == sl) alpha[((size_t)i * ng + G) * m + j] = __float2half_rn(a16[i]);
+    if (live && err && sl == 0) err[(size_t)G * m + j] = e2;
   }
 }
 
@@ -272,7 +298,13 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const long long groups = (long long)m * (n / g);
-  long long blocks = (groups + kFitWarps - 1) / kFitWarps;
+  // Above four planes the codes live in shared memory, one table per warp, so
+  // such a warp serves one group.
+  int lpg = 1;
+  while (lpg < 32 && lpg < g / 8) lpg <<= 1;
+  if (q > 4) lpg = 32;
+  const long long warps = (groups + (32 / lpg) - 1) / (32 / lpg);
+  long long blocks = (warps + kFitWarps - 1) / kFitWarps;
   const long long cap = (long long)sms * 8;
   if (blocks > cap) blocks = cap;
   const int cpl = (g + 255) / 256;
@@ -280,14 +312,14 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
   const unsigned nt = kFitWarps * 32;
 #define LUTGEMM_FIT_Q(CPLv)                                                                        \
   switch (q) {                                                                                     \
-    case 1: fit_bcq_kernel<CPLv, 1><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    case 2: fit_bcq_kernel<CPLv, 2><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    case 3: fit_bcq_kernel<CPLv, 3><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    case 4: fit_bcq_kernel<CPLv, 4><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    case 5: fit_bcq_kernel<CPLv, 5><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    case 6: fit_bcq_kernel<CPLv, 6><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    case 7: fit_bcq_kernel<CPLv, 7><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
-    default: fit_bcq_kernel<CPLv, 8><<<nb, nt, 0, stream>>>(w, m, n, g, iters, signs, alpha, err); break; \
+    case 1: fit_bcq_kernel<CPLv, 1><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    case 2: fit_bcq_kernel<CPLv, 2><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    case 3: fit_bcq_kernel<CPLv, 3><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    case 4: fit_bcq_kernel<CPLv, 4><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    case 5: fit_bcq_kernel<CPLv, 5><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    case 6: fit_bcq_kernel<CPLv, 6><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    case 7: fit_bcq_kernel<CPLv, 7><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+    default: fit_bcq_kernel<CPLv, 8><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
   }
   if (cpl <= 1) {
     LUTGEMM_FIT_Q(1)
