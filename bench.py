@@ -446,6 +446,145 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# BCQ fitting (the step that produces the weights): FP16 W -> signs + scales.
+# ---------------------------------------------------------------------------
+FIT_METRIC = "BCQ fit throughput: FP16 weights fitted per second (greedy + alternating least squares)"
+
+
+def _fit_profile(kernel_hash: str):
+    """Warp instructions per weight of fit_bcq_kernel from the committed ncu summary
+    (null unless it was taken on this kernel source)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "fit_bcq_instructions.json")) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    return d if d.get("kernel_hash") == kernel_hash else None
+
+
+def _fit_hash() -> str:
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc", "fit.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def run_fit(args):
+    from weight_only_quantized_bcq_b200 import lutgemm
+    world, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
+    m, n, q, g, iters = args.fit_m, args.fit_n, args.q, args.fit_g, args.fit_iters
+    w_host = S.draw_weights(S.generator(rank_seed(rank)), m, n, 0.02).pin_memory()
+    w = w_host.to(device)
+    signs = torch.empty((q, m, n), dtype=torch.int8, device=device)
+    alpha = torch.empty((q, n // g, m), dtype=torch.float16, device=device)
+    lib = lutgemm.lib()
+    import ctypes
+
+    def fit_once(src):
+        st = lib.lutgemm_fit_bcq(ctypes.c_void_p(src.data_ptr()), q, m, n, g, iters,
+                                 ctypes.c_void_p(signs.data_ptr()), ctypes.c_void_p(alpha.data_ptr()), None,
+                                 ctypes.c_void_p(stream.cuda_stream))
+        if st != 0:
+            raise RuntimeError(lutgemm.status_string(st))
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        fit_once(w)
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier()
+        t0.record(stream)
+        for _ in range(args.steps):
+            fit_once(w)
+        t1.record(stream)
+        barrier()
+    region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
+    # End to end: W from pinned host memory in, signs and scales back out, per step.
+    s_host = torch.empty(signs.shape, dtype=torch.int8).pin_memory()
+    a_host = torch.empty(alpha.shape, dtype=torch.float16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        w.copy_(w_host, non_blocking=True)
+        fit_once(w)
+        s_host.copy_(signs, non_blocking=True)
+        a_host.copy_(alpha, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1), device)
+    weights = m * n
+    value = weights * args.steps * world / (region_ms * 1e-3) / 1e9
+    e2e = weights * args.steps * world / (e2e_ms * 1e-3) / 1e9
+    if rank == 0:
+        sm = torch.cuda.get_device_properties(device).multi_processor_count
+        clk = clocks.summary()
+        prof = _fit_profile(_fit_hash())
+        # Issue-slot roofline: 4 schedulers per SM, one warp instruction each per clock.
+        peak = 4 * sm * (clk["sm_mhz"] or 1965.0) * 1e6 / 1e9
+        roof = {"bound": "alu", "unit": "G warp-inst/s", "peak": round(peak, 1), "peak_kind":
+                "derived: 4 issue slots x SMs x median SM clock under load", "kernel": "fit_bcq_kernel",
+                "kernel_hash": _fit_hash(), "traffic": None}
+        if prof:
+            ach = prof["warp_inst_per_weight"] * weights * args.steps / (region_ms * 1e-3) / 1e9
+            roof.update({"achieved": round(ach, 1), "frac": round(ach / peak, 4),
+                         "traffic": prof.get("dram_bytes_per_weight", 0) * weights or None})
+        else:
+            roof.update({"achieved": None, "frac": None})
+        out = {
+            "metric": FIT_METRIC, "value": round(value, 2), "unit": "Gweights/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"BCQ fit of FP16 W {m}x{n} ~ N(0, 0.02): q={q}, g={g}, {iters} rounds",
+                       "m": m, "n": n, "q": q, "g": g, "iters": iters,
+                       "l2": f"no flush: W is {2 * m * n / 1e6:.0f} MB (> 126 MB L2)",
+                       "parallelism": "replicas" if world == 1 else f"replicas{world}"},
+            "roofline": roof,
+            "e2e": {"value": round(e2e, 2), "unit": "Gweights/s", "h2d_bytes_per_step": 2 * m * n,
+                    "d2h_bytes_per_step": q * m * n + 2 * q * (n // g) * m},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_fit_baseline(q, g, iters, n, args.fit_cpu_rows)
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def cpu_fit_baseline(q: int, g: int, iters: int, n: int, rows: int):
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    from oracle import bcq_oracle as O
+    w = S.draw_weights(S.generator(77), rows, n, 0.02).numpy()
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        O.fit_bcq(w, q, g, iters)
+        secs = time.perf_counter() - t
+    return {"value": round(rows * n / secs / 1e9, 6), "unit": "Gweights/s", "cores": 1, "kind": "oracle",
+            "seconds": round(secs, 2),
+            "sample": f"{rows} rows x {n} of the same W distribution, oracle fit_bcq (FP64), one thread"}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -463,10 +602,30 @@ def main():
                     help="scale layout lutgemm_run reads (packed: unit-major, reordered at load time)")
     ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
                     help="time one linear of the layer only (profiling)")
+    ap.add_argument("--workload", choices=["layer", "fit"], default="layer",
+                    help="layer: the LUT-GEMM step (default); fit: BCQ fitting of FP16 weights")
+    ap.add_argument("--fit-m", type=int, default=49152)
+    ap.add_argument("--fit-n", type=int, default=12288)
+    ap.add_argument("--fit-g", type=int, default=128)
+    ap.add_argument("--fit-iters", type=int, default=3)
+    ap.add_argument("--fit-cpu-rows", type=int, default=384, help="rows of the CPU baseline fit sample")
     args = ap.parse_args()
     # At least three untimed warm-up steps, whatever the caller asks for.
     args.warmup = max(3, args.warmup)
-    if args.impl == "reference":
+    if args.workload == "fit":
+        if args.impl == "reference":
+            world, rank, _ = _dist_env()
+            if rank == 0:
+                r = cpu_fit_baseline(args.q, args.fit_g, args.fit_iters, args.fit_n, args.fit_cpu_rows)
+                print(json.dumps({"impl": "reference", "metric": FIT_METRIC, "value": r["value"],
+                                  "unit": "Gweights/s", "n_gpus": world, "steps": 1, "warmup": 0,
+                                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                                  "dtype": "f64", "data": "synthetic", "cpu_baseline": r,
+                                  "e2e": {"value": r["value"], "unit": "Gweights/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}), flush=True)
+        else:
+            run_fit(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_lutgemm(args)
