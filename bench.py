@@ -585,6 +585,72 @@ def cpu_fit_baseline(q: int, g: int, iters: int, n: int, rows: int):
             "sample": f"{rows} rows x {n} of the same W distribution, oracle fit_bcq (FP64), one thread"}
 
 
+# ---------------------------------------------------------------------------
+# Config sweep: isolated and back-to-back time of every parity config shape
+# (OPT-175B linears at batch 1..32, LLaMA-70B linears at batch 1..8), one
+# JSON line each, against both rooflines (HBM and shared-memory lookups).
+# ---------------------------------------------------------------------------
+SWEEP = [("opt175b_qkv", 36864, 12288, 3, 128, (1, 2, 4, 8, 16, 32)),
+         ("opt175b_fc1", 49152, 12288, 3, 128, (1, 2, 4, 8, 16, 32)),
+         ("opt175b_fc2", 12288, 49152, 3, 128, (1, 2, 4, 8, 16, 32)),
+         ("llama70b_qkvo", 8192, 8192, 2, 64, (1, 2, 4, 8)),
+         ("llama70b_up", 28672, 8192, 2, 64, (1, 2, 4, 8)),
+         ("llama70b_down", 8192, 28672, 2, 64, (1, 2, 4, 8))]
+
+
+def run_sweep(args):
+    from weight_only_quantized_bcq_b200 import lutgemm
+    torch.cuda.set_device(0)
+    peak, _ = _peaks()
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    sm = torch.cuda.get_device_properties(0).multi_processor_count
+    for name, m, n, q, g, batches in SWEEP:
+        gen = S.generator(3)
+        reps = 3   # distinct weight copies: consecutive launches miss L2
+        bufs = [S.draw_random_bytes(gen, lutgemm.packed_bytes(q, m, n)).cuda() for _ in range(reps)]
+        alpha = S.draw_alpha(gen, q, m, n, g, 0.02).cuda()
+        packed_scales = g % 128 == 0
+        scales = lutgemm.pack_scales(alpha, m, n, g) if packed_scales else alpha
+        for b in batches:
+            x = S.draw_x(gen, b, n).cuda()
+            ws = lutgemm.new_workspace(m, n, b, q, g)
+            y = torch.empty((b, m), device="cuda")
+
+            def run(i):
+                lutgemm.run(bufs[i % reps], scales, x, m, n, q, g, y=y, workspace=ws,
+                            scales_packed=packed_scales, stream=stream)
+            for i in range(max(3, args.warmup)):
+                run(i)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(21)]
+            for i, (a_, b_) in enumerate(ev):
+                a_.record(stream)
+                run(i)
+                b_.record(stream)
+            torch.cuda.synchronize()
+            iso = statistics.median(a_.elapsed_time(b_) for a_, b_ in ev) * 1e3
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(30):
+                run(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            b2b = e0.elapsed_time(e1) * 1e3 / 30
+            nbytes = algorithmic_bytes(m, n, q, g, b)
+            # Lookups: q*m*n/8 table reads per batch column; one conflict-free
+            # wavefront (32 reads) per clock per SM at the measured clock.
+            lookups = q * m * n // 8 * b
+            smem_floor = lookups / 32 / sm / 1.965e3
+            print(json.dumps({"config": name, "m": m, "n": n, "q": q, "g": g, "batch": b,
+                              "us_isolated": round(iso, 1), "us_back_to_back": round(b2b, 1),
+                              "gbs_back_to_back": round(nbytes / (b2b * 1e-6) / 1e9, 1),
+                              "hbm_floor_us": round(nbytes / (peak * 1e3), 1),
+                              "smem_floor_us": round(smem_floor, 1),
+                              "frac_of_binding_floor": round(max(nbytes / (peak * 1e3), smem_floor) / b2b, 3)}),
+                  flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -602,8 +668,9 @@ def main():
                     help="scale layout lutgemm_run reads (packed: unit-major, reordered at load time)")
     ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
                     help="time one linear of the layer only (profiling)")
-    ap.add_argument("--workload", choices=["layer", "fit"], default="layer",
-                    help="layer: the LUT-GEMM step (default); fit: BCQ fitting of FP16 weights")
+    ap.add_argument("--workload", choices=["layer", "fit", "sweep"], default="layer",
+                    help="layer: the LUT-GEMM step (default); fit: BCQ fitting of FP16 weights; "
+                         "sweep: every parity config shape and batch, one line each")
     ap.add_argument("--fit-m", type=int, default=49152)
     ap.add_argument("--fit-n", type=int, default=12288)
     ap.add_argument("--fit-g", type=int, default=128)
@@ -612,7 +679,9 @@ def main():
     args = ap.parse_args()
     # At least three untimed warm-up steps, whatever the caller asks for.
     args.warmup = max(3, args.warmup)
-    if args.workload == "fit":
+    if args.workload == "sweep":
+        run_sweep(args)
+    elif args.workload == "fit":
         if args.impl == "reference":
             world, rank, _ = _dist_env()
             if rank == 0:
