@@ -233,6 +233,25 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
                 unsigned flags, void* workspace, size_t workspace_bytes,
                 void* stream);
 
+/* y = W x for a BCQ weight on the tensor cores: the large-batch path, where
+ * the lookup kernel's per-column table reads dominate (one table per batch
+ * column).  Same operands and result as lutgemm_run (pure BCQ, no offsets).
+ * Each plane enters the tensor cores as its exact fp16 values +-alpha (a
+ * scale times a sign), so no rounded dequantised weight is formed; the planes
+ * accumulate in fp32 (tcgen05.mma, tensor memory).  Tiles: 128 rows x up to
+ * 256 batch columns x 128 inputs.  The pages' kernel is the lookup one; this
+ * path is for prompt-sized batches, where the method is compute-bound (LUT-GEMM
+ * card, Summary and Key points: generation is memory-bound, large batches are
+ * not).
+ *   m, n, batch, q, g  as lutgemm_run, and n % 128 == 0, g % 128 == 0
+ *   packed, alpha, x, y  as lutgemm_run ([q][n/g][m] scales)
+ *   flags      0 or LUTGEMM_Y_F16
+ * Needs no workspace.  Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_VALUE,
+ * ERR_ALIGN or ERR_CUDA. */
+int lutgemm_run_tc(int m, int n, int batch, int q, int g,
+                   const uint8_t* packed, const uint16_t* alpha,
+                   const uint16_t* x, void* y, unsigned flags, void* stream);
+
 /* Bytes of the device scratch array used by lutgemm_run_noalloc (16 MiB). */
 #define LUTGEMM_NOALLOC_SCRATCH_BYTES (16u << 20)
 

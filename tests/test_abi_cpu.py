@@ -126,6 +126,25 @@ def test_scales_bytes(L):
     assert L.scales_bytes(9, 64, 1024, 128) == 0
 
 
+def test_run_tc_validation(L):
+    lib = L.lib()
+    ok = [256, 1024, 16, 3, 128, FAKE, FAKE, FAKE, FAKE, 0, None]
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[["m", "n", "batch", "q", "g", "packed", "alpha", "x", "y", "flags", "stream"].index(k)] = v
+        return lib.lutgemm_run_tc(*a)
+    assert call(packed=None) == L.ERR_NULL
+    assert call(y=None) == L.ERR_NULL
+    assert call(g=64) == L.ERR_SHAPE             # needs g % 128 == 0
+    assert call(n=1032, g=8) == L.ERR_SHAPE      # needs n % 128 == 0
+    assert call(batch=0) == L.ERR_SHAPE
+    assert call(flags=2) == L.ERR_VALUE
+    assert call(x=FAKE + 8) == L.ERR_ALIGN
+    assert call(packed=FAKE + 8) == L.ERR_ALIGN
+    assert call(y=FAKE + 2) == L.ERR_ALIGN
+
+
 def test_fit_validation(L):
     lib = L.lib()
     ok = [FAKE, 3, 32, 1024, 128, 3, FAKE, FAKE, None, None]

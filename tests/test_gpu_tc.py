@@ -1,0 +1,101 @@
+"""GPU parity of the tensor-core large-batch path (lutgemm_run_tc) against the
+FP64 oracle and against the lookup path."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import bcq_synth as S
+from oracle import bcq_oracle as O
+from tests._tol import compare
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def L():
+    from weight_only_quantized_bcq_b200 import lutgemm
+    lutgemm.lib()
+    assert torch.cuda.is_available()
+    return lutgemm
+
+
+def _problem(seed, q, m, n, g, batch):
+    gen = S.generator(seed)
+    signs = S.draw_signs(gen, q, m, n)
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.02)
+    x = S.draw_x(gen, batch, n)
+    return signs, alpha, x
+
+
+CASES = [
+    # q, m, n, g, batch
+    (3, 128, 1024, 128, 16),
+    (3, 300, 2048, 128, 33),
+    (2, 1000, 3072, 128, 64),
+    (4, 129, 1024, 256, 130),
+    (1, 512, 4096, 128, 256),
+    (5, 200, 1024, 128, 300),
+    (8, 64, 1024, 128, 7),
+    (3, 96, 640, 128, 1),
+]
+
+
+@pytest.mark.parametrize("q,m,n,g,batch", CASES)
+def test_tc_matches_oracle_and_lookup_path(L, q, m, n, g, batch):
+    signs, alpha, x = _problem(900 + q * 13 + batch, q, m, n, g, batch)
+    packed = L.pack_bcq(signs.to(DEV))
+    a_d, x_d = alpha.to(DEV), x.to(DEV)
+    y_tc = L.run_tc(packed, a_d, x_d, m, n, q, g)
+    y_lut = L.run(packed, a_d, x_d, m, n, q, g)
+    torch.cuda.synchronize()
+    y_ref = O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), g)
+    ok, st = compare(y_tc.cpu().numpy(), y_ref, alpha.numpy(), x.numpy(), n)
+    assert ok, st
+    ok2, st2 = compare(y_tc.cpu().numpy(), y_lut.cpu().numpy().astype(np.float64), alpha.numpy(), x.numpy(), n)
+    assert ok2, st2
+
+
+def test_tc_fp16_output_is_rounded_fp32(L):
+    signs, alpha, x = _problem(950, 3, 256, 2048, 128, 40)
+    packed = L.pack_bcq(signs.to(DEV))
+    y32 = L.run_tc(packed, alpha.to(DEV), x.to(DEV), 256, 2048, 3, 128)
+    y16 = L.run_tc(packed, alpha.to(DEV), x.to(DEV), 256, 2048, 3, 128, y_f16=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y16, y32.to(torch.float16))
+
+
+def test_tc_is_deterministic(L):
+    signs, alpha, x = _problem(951, 3, 384, 3072, 128, 200)
+    packed = L.pack_bcq(signs.to(DEV))
+    a = L.run_tc(packed, alpha.to(DEV), x.to(DEV), 384, 3072, 3, 128)
+    b = L.run_tc(packed, alpha.to(DEV), x.to(DEV), 384, 3072, 3, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_tc_full_size_fc1_sampled(L):
+    """OPT-175B FC1 (49152 x 12288, q = 3, g = 128) at batch 64: sampled rows."""
+    m, n, q, g, batch = 49152, 12288, 3, 128, 64
+    gen = S.generator(952)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n))
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.02)
+    x = S.draw_x(gen, batch, n)
+    y = L.run_tc(packed.to(DEV), alpha.to(DEV), x.to(DEV), m, n, q, g)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(952).choice(m, 40, replace=False))
+    s_rows = O.unpack_rows(packed.numpy(), q, m, n, rows)
+    a_rows = alpha.numpy()[:, :, rows]
+    y_ref = O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g)
+    ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_rows, x.numpy(), n)
+    assert ok, st
+
+
+def test_tc_rejects_unsupported_shapes(L):
+    signs, alpha, x = _problem(953, 3, 64, 1024, 64, 4)
+    packed = L.pack_bcq(signs.to(DEV))
+    with pytest.raises(L.LutgemmError) as e:
+        L.run_tc(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 64)
+    assert e.value.status == L.ERR_SHAPE

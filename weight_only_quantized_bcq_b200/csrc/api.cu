@@ -16,6 +16,8 @@ cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, con
                                   int32_t* flags, cudaStream_t stream);
 cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
                                cudaStream_t stream);
+cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const __half* x, void* y, int m, int n,
+                           int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
 cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
                            float* err, cudaStream_t stream);
 }  // namespace lutgemm
@@ -131,6 +133,21 @@ size_t lutgemm_scales_bytes(int q, int m, int n, int g) {
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g % 128 != 0) return 0;
   const size_t sp = q < 4 ? (size_t)q : 4u;
   return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * ceil_div(q, 4) * 512u * sp;
+}
+
+int lutgemm_run_tc(int m, int n, int batch, int q, int g, const uint8_t* packed, const uint16_t* alpha,
+                   const uint16_t* x, void* y, unsigned flags, void* stream) {
+  if (!packed || !alpha || !x || !y) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1 || g % 128 != 0 || n % 128 != 0)
+    return LUTGEMM_ERR_SHAPE;
+  if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
+  const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
+  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
+    return LUTGEMM_ERR_ALIGN;
+  const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha),
+                                       reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
+                                       nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 
 int lutgemm_fit_bcq(const uint16_t* w, int q, int m, int n, int g, int iters, int8_t* signs, uint16_t* alpha,

@@ -30,6 +30,7 @@ _SIGNATURES = {
     "lutgemm_scales_bytes": ([_c_int, _c_int, _c_int, _c_int], _c_size),
     "lutgemm_pack_scales": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lutgemm_fit_bcq": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
+    "lutgemm_run_tc": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_uint, _vp], _c_int),
     "lutgemm_pack_bcq": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "lutgemm_uniform_to_bcq": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp],
                                _c_int),
@@ -181,6 +182,22 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
     _check(lib().lutgemm_run(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
                              flags, _ptr(workspace), workspace.numel(), _stream(stream)),
            "lutgemm_run")
+    return y
+
+
+def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
+           y: torch.Tensor = None, y_f16: bool = False, stream=None) -> torch.Tensor:
+    """``run`` on the tensor cores (lutgemm_run_tc), for large batches; pure BCQ,
+    n % 128 == 0 and g % 128 == 0."""
+    _need(packed, torch.uint8, "packed")
+    _need(alpha, torch.float16, "alpha")
+    _need(x, torch.float16, "x")
+    batch = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
+    _check(lib().lutgemm_run_tc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(x), _ptr(y),
+                                Y_F16 if y_f16 else 0, _stream(stream)),
+           "lutgemm_run_tc")
     return y
 
 
