@@ -40,6 +40,10 @@ CASES = [
     (5, 200, 1024, 128, 300),
     (8, 64, 1024, 128, 7),
     (3, 96, 640, 128, 1),
+    # last slice of 2 and of 4 pieces (units of one K block), g spanning two K blocks
+    (3, 256, 1280, 128, 40),
+    (2, 248, 1536, 256, 64),
+    (8, 136, 2048, 128, 129),
 ]
 
 

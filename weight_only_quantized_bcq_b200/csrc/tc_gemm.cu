@@ -10,21 +10,32 @@
 // 128-input piece) and no uniform offsets.
 //
 // CTA tile: 128 rows (MMA M) x BN batch columns (MMA N) over K blocks of 128
-// inputs (one piece of the packed layout).  Warps 0-7 expand a plane's bits
-// for the tile into a 128 x 128 fp16 A tile in shared memory (128-byte
-// swizzled, K-major: the canonical UMMA layout; warps w and w+4 take the two
-// 64-input halves of rows 32(w mod 4)..+31); warp 12 loads the x tile by TMA
-// (same swizzle), issues the 8 tcgen05.mma (K = 16 each) per plane and
-// commits them to mbarriers that free the buffers.  Three A buffers and two
-// x buffers form the pipeline.
+// inputs (one piece of the packed layout).  Warp roles:
+//   warp 21 (producer): streams the operands into a shared-memory ring of
+//     units.  A unit is the K-block pair (P, P ^ 4) of one 1024-input slice:
+//     those two blocks read the same two chunk groups of the packed layout
+//     (lanes 0-15 of a row tile hold piece P in chunk P, lanes 16-31 in
+//     chunk P ^ 4), so one bulk copy per chunk group and row tile serves
+//     both.  Each unit holds the two x tiles (TMA, 128-byte swizzle,
+//     K-major), the 8 chunk groups of the tile's 4 row tiles and the 2 x q
+//     scale rows of the tile.
+//   warps 0-15 (dequant): expand a plane's bits for the tile into a 128 x
+//     128 fp16 A tile in tensor memory (row r in lane r, inputs 2c and 2c+1
+//     in column c: the layout the tensor cores read an A operand from);
+//     warp w takes rows 32(w mod 4)..+31 (the lanes it may access) and the
+//     32-input quarter w / 4.  A never touches shared memory.
+//   warp 20 (MMA): one thread issues the 8 tcgen05.mma (K = 16 each, A from
+//     tensor memory, B from shared memory) per plane and commits them to the
+//     mbarriers that free A stages, units and accumulators.
+//   warps 16-19 (accumulate): see below.
 //
 // Accumulation: the tensor cores add into their fp32 accumulator with
 // truncation, so an error of up to an ulp per MMA step would build up over
 // the q * n / 16 steps of a long row.  Each K block therefore accumulates in
-// a fresh tensor-memory buffer (two, ping-pong), and warps 8-11 add it into
+// a fresh tensor-memory buffer (two, ping-pong), and warps 16-19 add it into
 // fp32 running sums (round to nearest) as soon as its MMAs complete; warp
-// 8+w owns accumulator lanes 32w..32w+31 = tile rows, keeps the running sums
-// in a third tensor-memory buffer and writes them to y.
+// 16+w owns accumulator lanes 32w..32w+31 = tile rows, keeps the running
+// sums in a third tensor-memory buffer and writes them to y.
 // Every mbarrier wait is bounded (1 s); a timeout sets status bit 2, the CTA
 // stops issuing work, waits (bounded) for its tensor-core work in flight and
 // frees its tensor memory before exiting.
@@ -37,13 +48,13 @@ namespace lutgemm {
 
 namespace {
 
-constexpr int kTcDequantThreads = 256;                 // warps 0-7
-constexpr int kTcFlushThreads = 128;                   // warps 8-11
-constexpr int kTcThreads = kTcDequantThreads + kTcFlushThreads + 32;   // + warp 12: TMA and MMA
-constexpr int kTcAStages = 3;
+constexpr int kTcDequantWarps = 16;                    // warps 0-15
+constexpr int kTcFlushWarp0 = kTcDequantWarps;          // warps 16-19
+constexpr int kTcMmaWarp = kTcFlushWarp0 + 4;           // warp 20
+constexpr int kTcProdWarp = kTcMmaWarp + 1;             // warp 21
+constexpr int kTcThreads = (kTcProdWarp + 1) * 32;
 constexpr int kTcBM = 128;
 constexpr int kTcBK = 128;
-constexpr uint32_t kTcATile = kTcBM * kTcBK * 2;      // 32 KB
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -102,6 +113,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t addr, const uint32_t (&v)[32]
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(addr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (start address and offsets in 16-byte units).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
@@ -109,29 +129,64 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// Units of the K loop in processing order: slice s, low piece P (0..3), and
+// whether piece P + 4 exists in the slice.
+struct UnitIter {
+  int n, ns, s, P, np;
+  __device__ __forceinline__ void init(int n_) {
+    n = n_;
+    ns = (n + kSliceInputs - 1) / kSliceInputs;
+    s = 0;
+    P = 0;
+    np = pieces(0);
+  }
+  __device__ __forceinline__ int pieces(int sl) const {
+    const int r = (n - kSliceInputs * sl) / kTcBK;
+    return r < 8 ? r : 8;
+  }
+  __device__ __forceinline__ bool valid() const { return s < ns; }
+  __device__ __forceinline__ int count() const { return P + 4 < np ? 2 : 1; }   // K blocks in the unit
+  __device__ __forceinline__ int kb(int which) const { return 8 * s + P + 4 * which; }
+  __device__ __forceinline__ void next() {
+    if (++P >= 4 || P >= np) {
+      P = 0;
+      if (++s < ns) np = pieces(s);
+    }
+  }
+};
+
+struct TcLayout {
+  uint32_t slot_bytes;     // one unit: x tiles, chunk groups, scale rows (multiple of 1024)
+  uint32_t bits_off;       // 8 chunk groups of q * 512 bytes: (row tile, half) = 2 wq + h
+  uint32_t alpha_off;      // 2 x q scale rows of 128 fp16: (which, plane)
+  int nu;                  // ring depth in units
+  int alpha_bulk;          // scale rows by bulk copy (16-byte aligned rows) or by lane loads
+};
+
 template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed,
                    const __half* __restrict__ alpha, void* y, int m, int n, int batch, int q, int g, int mt,
-                   int y_f16, unsigned* status) {
+                   int y_f16, unsigned* status, TcLayout L) {
   constexpr uint32_t kBTile = (uint32_t)BN * kTcBK * 2;   // x tile: BN rows x 128 inputs
   // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128.
   constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
+  // Tensor memory (all 512 columns): accumulator buffers at columns 0 and BN,
+  // the running sums at 2 BN, then kSA A stages of 64 columns (128 rows x
+  // 128 fp16 inputs, two per column) from column kACol0.
+  constexpr uint32_t kTmemCols = 512;
+  constexpr int kACol0 = (3 * BN + 63) / 64 * 64;
+  constexpr int kSA = (512 - kACol0) / 64 < 6 ? (512 - kACol0) / 64 : 6;
+  static_assert(kSA >= 2, "at least two A stages must fit tensor memory");
 
   extern __shared__ __align__(1024) unsigned char tc_smem_raw[];
   const uint32_t raw = (uint32_t)__cvta_generic_to_shared(tc_smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sA = base;                                  // kTcAStages x 32 KB
-  const uint32_t sB = base + kTcAStages * kTcATile;          // 2 x kBTile
-  const uint32_t bars = sB + 2 * kBTile;                     // 15 mbarriers
-  const uint32_t fullA = bars, emptyA = bars + 24, fullB = bars + 48, emptyB = bars + 64, done = bars + 80;
-  const uint32_t accFull = bars + 88, accFree = bars + 104;
-  const uint32_t tmem_slot = bars + 120;
-  const uint32_t flag_slot = bars + 124;                     // CTA failure flag (shared)
-  // Tensor memory: two accumulator buffers and the running sums, BN columns each.
-  constexpr uint32_t kTmemCols =
-      3 * BN <= 32 ? 32 : (3 * BN <= 64 ? 64 : (3 * BN <= 128 ? 128 : (3 * BN <= 256 ? 256 : 512)));
-  static_assert(3 * BN <= 512, "three BN-column buffers must fit tensor memory");
+  const uint32_t ring = (raw + 1023u) & ~1023u;
+  const uint32_t bars = ring + (uint32_t)L.nu * L.slot_bytes;
+  const uint32_t fullU = bars, emptyU = bars + 64, fullA = bars + 128, emptyA = bars + 176;
+  const uint32_t accFull = bars + 224, accFree = bars + 240, done = bars + 256;
+  const uint32_t tmem_slot = bars + 264;
+  const uint32_t flag_slot = bars + 268;                     // CTA failure flag (shared)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -140,21 +195,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int b0 = blockIdx.y * BN;                            // first batch column
   const int nkb = n / kTcBK;
   const int ng = n / g;
+  const int kb_per_g = g / kTcBK;
 
   if (tid == 0) {
-    for (int s = 0; s < kTcAStages; ++s) {
-      bar_init(fullA + 8 * s, kTcDequantThreads);
+    for (int s = 0; s < L.nu; ++s) {
+      bar_init(fullU + 8 * s, 1);
+      bar_init(emptyU + 8 * s, kTcDequantWarps + 1);       // dequant warps + the MMA commit
+    }
+    for (int s = 0; s < kSA; ++s) {
+      bar_init(fullA + 8 * s, kTcDequantWarps);
       bar_init(emptyA + 8 * s, 1);
     }
     for (int s = 0; s < 2; ++s) {
-      bar_init(fullB + 8 * s, 1);
-      bar_init(emptyB + 8 * s, 1);
+      bar_init(accFull + 8 * s, 1);
+      bar_init(accFree + 8 * s, 128);
     }
     bar_init(done, 1);
-    for (int s = 0; s < 2; ++s) {
-      bar_init(accFull + 8 * s, 1);
-      bar_init(accFree + 8 * s, kTcFlushThreads);
-    }
     asm volatile("st.shared.u32 [%0], 0;" ::"r"(flag_slot) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -180,146 +236,211 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return f != 0;
   };
 
-  if (warp < 8) {
-    // ---- Dequant warps: plane tiles of +-alpha in the swizzled K-major layout.
-    const int wq = warp & 3;                                 // rows 32wq..32wq+31 of the tile
-    const int hsel = warp >> 2;                              // K half: runs 8 hsel .. 8 hsel + 7
-    const int R = rb * 4 + wq;                               // 32-row tile of this warp
-    const int row = R * kTileRows + lane;                    // weight row of this thread
-    const int lrow = wq * 32 + lane;                         // row within the 128-row tile
-    const uint32_t rowoff = (uint32_t)(lrow >> 3) * 1024u + (uint32_t)(lrow & 7) * 128u;
-    const uint32_t sw = (uint32_t)(lrow & 7);
+  if (warp < kTcDequantWarps) {
+    // ---- Dequant warps: plane tiles of +-alpha, written to tensor memory.
+    const int wq = warp & 3;                                 // tile rows (= TMEM lanes) 32wq..32wq+31
+    const int hq = warp >> 2;                                // K quarter: runs 4 hq .. 4 hq + 3
+    const int row = (rb * 4 + wq) * kTileRows + lane;        // weight row of this thread
     const int half_sel = lane >> 4;
-    const int lam = lane & 15;
-    // The plane bits and scale of plane step ai = kb * q + i are loaded kPf
-    // steps ahead, so their global-memory latency overlaps the expansion of
-    // the steps before.
-    constexpr int kPf = 3;
-    const int nsteps = nkb * q;
-    auto load_step = [&](int ai, uint4& bits, uint32_t& ah) {
-      bits = make_uint4(0, 0, 0, 0);
-      ah = 0;
-      if (ai < nsteps && R < mt) {
-        const int kb = ai / q, i = ai - kb * q;
-        const int s = kb >> 3, P = kb & 7;
-        const int U = P ^ (4 * half_sel);
-        const int G = (s * kSliceInputs + 128 * P) / g;
-        bits = __ldg(reinterpret_cast<const uint4*>(packed + ((((size_t)s * mt + R) * 8 + U) * q + i) * 512 +
-                                                    (size_t)lane * 16));
-        if (row < m) ah = __ldg(reinterpret_cast<const unsigned short*>(alpha) + ((size_t)i * ng + G) * m + row);
-      }
-    };
-    uint4 pb[kPf];
-    uint32_t pa[kPf];
+    // The lane's 16-byte piece holds run c in byte c ^ (lane mod 16): runs
+    // 4 hq .. 4 hq + 3 sit in its 32-bit word hq ^ (bits 2-3 of the lane),
+    // byte cc ^ (lane mod 4) for run 4 hq + cc.  One byte permutation per
+    // step puts them in run order.
+    const int wi = hq ^ ((lane >> 2) & 3);
+    uint32_t sel = 0;
 #pragma unroll
-    for (int d = 0; d < kPf; ++d) load_step(d, pb[d], pa[d]);
-    for (int ai = 0; ai < nsteps && !failed(); ++ai) {
-      const int st = ai % kTcAStages;
-      const uint4 bits = pb[0];
-      const uint32_t ah = pa[0];
-#pragma unroll
-      for (int d = 0; d + 1 < kPf; ++d) {
-        pb[d] = pb[d + 1];
-        pa[d] = pa[d + 1];
-      }
-      load_step(ai + kPf, pb[kPf - 1], pa[kPf - 1]);
-      if (ai >= kTcAStages && !bar_wait(emptyA + 8 * st, (uint32_t)(((ai - kTcAStages) / kTcAStages) & 1))) {
-        fail();
+    for (int k = 0; k < 4; ++k) sel |= ((uint32_t)k ^ (uint32_t)(lane & 3)) << (4 * k);
+    const uint32_t row_mask = row < m ? 0xFFFFFFFFu : 0u;   // rows past m get a zero scale
+    const uint32_t a_tm = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)kACol0 + (uint32_t)(16 * hq);
+    const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * 2 * q * 512 + lane * 16 + wi * 4);
+    const uint32_t alpha_lane = L.alpha_off + (uint32_t)((wq * 32 + lane) * 2);
+    UnitIter it;
+    it.init(n);
+    int ai = 0;                                              // plane step (A stage sequence)
+    bool go = true;
+    for (int u = 0; it.valid() && go; it.next(), ++u) {
+      const int sl = u % L.nu;
+      const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
+      if (!__all_sync(0xffffffffu, bar_wait(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)))) {
+        if (lane == 0) fail();
         break;
       }
-      const uint32_t pos = ah, neg = ah ^ 0x8000u;
-      const uint32_t dst = sA + (uint32_t)st * kTcATile + rowoff;
+      go = !__any_sync(0xffffffffu, failed());
+      const int cnt = it.count();
+      for (int w = 0; w < cnt && go; ++w) {
+        const uint32_t bsrc = slot + bits_lane + (uint32_t)((half_sel ^ w) * q * 512);
+        const uint32_t asrc = slot + alpha_lane + (uint32_t)(w * q * 256);
+        for (int i = 0; i < q; ++i, ++ai) {
+          const int st = ai % kSA;
+          uint32_t bits, ah;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits) : "r"(bsrc + (uint32_t)(i * 512)) : "memory");
+          asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc + (uint32_t)(i * 256)) : "memory");
+          const uint32_t wr = __byte_perm(bits, 0u, sel);     // runs 0..3 of the quarter, in order
+          // Element pair (2e, 2e+1) of a run byte b: the product b * (2^(15-2e)
+          // + 2^(30-2e)) puts bit 2e at bit 15 and bit 2e+1 at bit 31 (the two
+          // fp16 sign bits), with no carries between the two copies.  A clear
+          // bit (beta = -1) sets the sign of +alpha.
+          const uint32_t a2 = (ah | (ah << 16)) & row_mask;
+          uint32_t v[16];
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {                      // run c = 8 hsel + cc: inputs 8c..8c+7 of the piece
-        const int c = 8 * hsel + cc;
-        const int j = c ^ lam;                               // byte of the lane's piece holding run c
-        const uint32_t word = j < 4 ? bits.x : (j < 8 ? bits.y : (j < 12 ? bits.z : bits.w));
-        const uint32_t b = (word >> (8 * (j & 3))) & 0xFFu;
-        uint32_t v[4];
+          for (int cc = 0; cc < 4; ++cc) {
+            const uint32_t b = __byte_perm(wr, 0u, 0x4440u | (uint32_t)cc);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t lo = ((b >> (2 * e)) & 1u) ? pos : neg;
-          const uint32_t hi = ((b >> (2 * e + 1)) & 1u) ? pos : neg;
-          v[e] = lo | (hi << 16);
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t t = b * ((1u << (15 - 2 * e)) + (1u << (30 - 2 * e)));
+              v[4 * cc + e] = a2 ^ (~t & 0x80008000u);
+            }
+          }
+          if (ai >= kSA &&
+              !__all_sync(0xffffffffu, bar_wait(emptyA + 8 * st, (uint32_t)(((ai - kSA) / kSA) & 1)))) {
+            if (lane == 0) fail();
+            go = false;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          tmem_st16(a_tm + (uint32_t)(st * 64), v);
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) bar_arrive(fullA + 8 * st);
         }
-        const uint32_t a = dst + (uint32_t)hsel * (kTcATile / 2) + (((uint32_t)cc ^ sw) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[0]), "r"(v[1]), "r"(v[2]),
-                     "r"(v[3])
-                     : "memory");
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      bar_arrive(fullA + 8 * st);
+      // This warp has read all it needs from the unit.
+      __syncwarp();
+      if (lane == 0) bar_arrive(emptyU + 8 * sl);
     }
-  } else if (warp == 12 && lane == 0) {
-    // ---- Control thread: x tiles by TMA, MMAs, commits.
-    auto load_x = [&](int kb) {
-      const int st = kb & 1;
-      const uint32_t bar = fullB + 8 * st;
-      const uint32_t dst = sB + (uint32_t)st * kBTile;
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kBTile) : "memory");
+  } else if (warp == kTcProdWarp) {
+    // ---- Producer: one unit of x tiles, chunk groups and scale rows per ring slot.
+    const int rows_here = m - rb * kTcBM < kTcBM ? m - rb * kTcBM : kTcBM;
+    UnitIter it;
+    it.init(n);
+    for (int u = 0; it.valid(); it.next(), ++u) {
+      const int sl = u % L.nu;
+      const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
+      const uint32_t bar = fullU + 8 * sl;
+      if (u >= L.nu && !__all_sync(0xffffffffu, bar_wait(emptyU + 8 * sl, (uint32_t)(((u / L.nu) - 1) & 1)))) {
+        if (lane == 0) fail();
+        break;
+      }
+      if (__any_sync(0xffffffffu, failed())) break;
+      const int cnt = it.count();
+      if (lane == 0) {
+        uint32_t bytes = (uint32_t)cnt * kBTile;
+        for (int wq = 0; wq < 4; ++wq)
+          if (rb * 4 + wq < mt) bytes += 2u * (uint32_t)q * 512u;
+        if (L.alpha_bulk) bytes += (uint32_t)(cnt * q * rows_here * 2);
+        asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+        for (int w = 0; w < cnt; ++w) {
+          const int kb = it.kb(w);
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-                dst + (uint32_t)h * (kBTile / 2)),
-            "l"(&xmap), "r"(kb * kTcBK + 64 * h), "r"(b0), "r"(bar)
-            : "memory");
-    };
-    load_x(0);
+          for (int h = 0; h < 2; ++h)
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+                "[%4];" ::"r"(slot + (uint32_t)w * kBTile + (uint32_t)h * (kBTile / 2)),
+                "l"(&xmap), "r"(kb * kTcBK + 64 * h), "r"(b0), "r"(bar)
+                : "memory");
+        }
+        for (int wq = 0; wq < 4; ++wq) {
+          const int R = rb * 4 + wq;
+          if (R >= mt) continue;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint8_t* src = packed + (((size_t)it.s * mt + R) * 8 + (size_t)(it.P ^ (4 * h))) * q * 512;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                    slot + L.bits_off + (uint32_t)((wq * 2 + h) * q * 512)),
+                "l"(src), "r"(q * 512), "r"(bar)
+                : "memory");
+          }
+        }
+        if (L.alpha_bulk) {
+          for (int w = 0; w < cnt; ++w) {
+            const int G = it.kb(w) / kb_per_g;
+            for (int i = 0; i < q; ++i)
+              asm volatile(
+                  "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                      slot + L.alpha_off + (uint32_t)((w * q + i) * 256)),
+                  "l"(alpha + ((size_t)i * ng + G) * m + (size_t)rb * kTcBM), "r"(rows_here * 2), "r"(bar)
+                  : "memory");
+          }
+        }
+      }
+      if (!L.alpha_bulk) {
+        // Scale rows by plain loads: lane l covers rows 4l..4l+3 of the tile.
+        for (int w = 0; w < cnt; ++w) {
+          const int G = it.kb(w) / kb_per_g;
+          for (int i = 0; i < q; ++i) {
+            const unsigned short* src = reinterpret_cast<const unsigned short*>(alpha) + ((size_t)i * ng + G) * m;
+            uint32_t v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = rb * kTcBM + 4 * lane + k;
+              v[k] = r < m ? (uint32_t)__ldg(src + r) : 0u;
+            }
+            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(slot + L.alpha_off + (uint32_t)((w * q + i) * 256 +
+                                                                                                  lane * 8)),
+                         "r"(v[0] | (v[1] << 16)), "r"(v[2] | (v[3] << 16))
+                         : "memory");
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) bar_arrive(bar);
+    }
+  } else if (warp == kTcMmaWarp && lane == 0) {
+    // ---- MMA thread: per plane step, 8 MMAs into the K block's accumulator buffer.
+    UnitIter it;
+    it.init(n);
+    int ai = 0, j = 0;                                       // plane step, K block (processing order)
     bool ok = true;
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      const int sb = kb & 1;
-      // Refill the other x buffer (last used by kb - 1) with kb + 1.
-      if (kb + 1 < nkb) {
-        if (kb >= 1 && !bar_wait(emptyB + 8 * ((kb + 1) & 1), (uint32_t)(((kb - 1) >> 1) & 1))) {
-          ok = false;
-          break;
-        }
-        load_x(kb + 1);
-      }
-      if (!bar_wait(fullB + 8 * sb, (uint32_t)((kb >> 1) & 1))) {
+    for (int u = 0; it.valid() && ok; it.next(), ++u) {
+      const int sl = u % L.nu;
+      const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
+      if (!bar_wait(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1))) {
         ok = false;
         break;
       }
-      // The accumulator buffer of this K block is free once warps 4-7 have
-      // added in what it held for K block kb - 2.
-      const uint32_t acc_tm = tmem + (uint32_t)(kb & 1) * BN;
-      if (kb >= 2 && !bar_wait(accFree + 8 * (kb & 1), (uint32_t)(((kb - 2) >> 1) & 1))) {
-        ok = false;
-        break;
-      }
-      for (int i = 0; i < q; ++i) {
-        const int ai = kb * q + i, st = ai % kTcAStages;
-        if (!bar_wait(fullA + 8 * st, (uint32_t)((ai / kTcAStages) & 1))) {
+      const int cnt = it.count();
+      for (int w = 0; w < cnt && ok; ++w, ++j) {
+        // The accumulator buffer of this K block is free once warps 16-19
+        // have added in what it held for K block j - 2.
+        const uint32_t acc_tm = tmem + (uint32_t)(j & 1) * BN;
+        if (j >= 2 && !bar_wait(accFree + 8 * (j & 1), (uint32_t)(((j - 2) >> 1) & 1))) {
           ok = false;
           break;
         }
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t a0 = sA + (uint32_t)st * kTcATile;
-        const uint32_t bb0 = sB + (uint32_t)sb * kBTile;
+        const uint32_t bb0 = slot + (uint32_t)w * kBTile;
+        for (int i = 0; i < q; ++i, ++ai) {
+          const int st = ai % kSA;
+          if (!bar_wait(fullA + 8 * st, (uint32_t)((ai / kSA) & 1))) {
+            ok = false;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint32_t a0 = tmem + (uint32_t)kACol0 + (uint32_t)(st * 64);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = smem_desc(a0 + (uint32_t)(kk >> 2) * (kTcATile / 2) + (uint32_t)(kk & 3) * 32u);
-          const uint64_t db = smem_desc(bb0 + (uint32_t)(kk >> 2) * (kBTile / 2) + (uint32_t)(kk & 3) * 32u);
-          const uint32_t acc = (i | kk) != 0 ? 1u : 0u;     // each K block starts a fresh sum
-          asm volatile(
-              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(acc_tm),
-              "l"(da), "l"(db), "r"(kIdesc), "r"(acc)
-              : "memory");
-        }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                         emptyA + 8 * st)
-                     : "memory");
-        if (i == q - 1) {
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t db = smem_desc(bb0 + (uint32_t)(kk >> 2) * (kBTile / 2) + (uint32_t)(kk & 3) * 32u);
+            const uint32_t acc = (i | kk) != 0 ? 1u : 0u;   // each K block starts a fresh sum
+            asm volatile(
+                "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(acc_tm),
+                "r"(a0 + 8u * (uint32_t)kk), "l"(db), "r"(kIdesc), "r"(acc)
+                : "memory");
+          }
           asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                           emptyB + 8 * sb)
-                       : "memory");
-          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                           accFull + 8 * (kb & 1))
+                           emptyA + 8 * st)
                        : "memory");
         }
+        if (ok)
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           accFull + 8 * (j & 1))
+                       : "memory");
       }
+      // The unit's x tiles are free once its MMAs have completed.
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       emptyU + 8 * sl)
+                   : "memory");
     }
     if (!ok) fail();
     // Completion of everything issued (also after a failure, before tensor memory is freed).
@@ -327,11 +448,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  : "memory");
   }
 
-  // ---- Warps 8-11: add each K block's accumulator into the running sums
+  // ---- Warps 16-19: add each K block's accumulator into the running sums
   // (tensor memory, fp32 adds with round to nearest), then write y.
-  bool wrote = true;
-  if (warp >= 8 && warp < 12) {
-    const int wq = warp - 8;                                 // accumulator lanes 32wq..32wq+31
+  if (warp >= kTcFlushWarp0 && warp < kTcFlushWarp0 + 4) {
+    const int wq = warp - kTcFlushWarp0;                     // accumulator lanes 32wq..32wq+31
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t run_tm = lane_base + 2u * BN;
     bool ok = true;
@@ -355,7 +475,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       bar_arrive(accFree + 8 * (kb & 1));
     }
-    wrote = ok;
     if (!ok && lane == 0) fail();
     const int row = (rb * 4 + wq) * kTileRows + lane;
     if (ok) {
@@ -379,7 +498,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   }
-  (void)wrote;
   // Everything issued has completed before tensor memory is freed.
   const bool all_done = __all_sync(0xffffffffu, bar_wait(done, 0));
   if (!all_done && lane == 0) atomicOr(status, kStatusTimeout);
@@ -397,10 +515,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // Sticky status word of the tensor-core path (bit 2: a wait timed out).
 __device__ unsigned g_tc_status;
 
+// Shared memory: a ring of unit slots (x tiles, chunk groups, scale rows)
+// plus the mbarriers, as deep as fits (2 to 4 units).
 template <int BN>
-size_t tc_smem_bytes() {
-  return 1024 + kTcAStages * (size_t)kTcATile + 2 * (size_t)BN * kTcBK * 2 + 128;
+TcLayout tc_layout(int q, bool alpha_bulk) {
+  TcLayout L;
+  const uint32_t xt = 2u * BN * kTcBK * 2;
+  L.bits_off = xt;
+  L.alpha_off = xt + 8u * (uint32_t)q * 512u;
+  L.slot_bytes = (L.alpha_off + 2u * (uint32_t)q * 256u + 1023u) & ~1023u;
+  const uint32_t budget = 227u * 1024u - 1024u - 512u;
+  const int fit = (int)(budget / L.slot_bytes);
+  L.nu = fit < 4 ? fit : 4;
+  L.alpha_bulk = alpha_bulk ? 1 : 0;
+  return L;
 }
+
+inline size_t tc_smem_bytes(const TcLayout& L) { return 1024 + (size_t)L.nu * L.slot_bytes + 512; }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -432,16 +563,21 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const __half* 
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const size_t smem = tc_smem_bytes<BN>();
+  // Scale rows go by bulk copy when every row segment of a tile starts on a
+  // 16-byte boundary; otherwise the producer warp loads them.
+  const bool alpha_bulk = m % 8 == 0 && (reinterpret_cast<uintptr_t>(alpha) % 16) == 0;
+  const TcLayout L = tc_layout<BN>(q, alpha_bulk);
+  if (L.nu < 2) return cudaErrorInvalidValue;
+  const size_t smem = tc_smem_bytes(L);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static bool attr_done[64] = {false};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
+  static int attr_bytes[64] = {0};
+  if (attr_bytes[dev] < (int)smem) {
     e = cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+    attr_bytes[dev] = (int)smem;
   }
   if (status == nullptr) {
     void* sp = nullptr;
@@ -451,7 +587,8 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const __half* 
   }
   const int mt = (m + kTileRows - 1) / kTileRows;
   dim3 grid((unsigned)((m + kTcBM - 1) / kTcBM), (unsigned)((batch + BN - 1) / BN));
-  tc_gemm_kernel<BN><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, y, m, n, batch, q, g, mt, y_f16, status);
+  tc_gemm_kernel<BN><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, y, m, n, batch, q, g, mt, y_f16, status,
+                                                         L);
   return cudaGetLastError();
 }
 
