@@ -77,6 +77,18 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same, backing off between polls: for warps whose polling would take
+// issue slots from the warps doing the work.
+__device__ __forceinline__ bool bar_wait_sleep(uint32_t bar, uint32_t parity) {
+  if (bar_try(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  while (!bar_try(bar, parity)) {
+    __nanosleep(20);
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
   if (bar_try(bar, parity)) return true;
   const uint64_t t0 = now_ns();
@@ -171,11 +183,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kBTile = (uint32_t)BN * kTcBK * 2;   // x tile: BN rows x 128 inputs
   // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128.
   constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
-  // Tensor memory (all 512 columns): accumulator buffers at columns 0 and BN,
-  // the running sums at 2 BN, then kSA A stages of 64 columns (128 rows x
-  // 128 fp16 inputs, two per column) from column kACol0.
+  // MMAs that add into one accumulator wait on each other; with two
+  // accumulator sets (even and odd K steps of every plane, summed when the K
+  // block is flushed) consecutive MMAs are independent and the tensor pipe
+  // stays full.  At BN = 128 an MMA takes longer than that dependency, and
+  // tensor memory holds one set only.
+  constexpr int kSets = BN <= 64 ? 2 : 1;
+  // Tensor memory (all 512 columns): per K block (two, ping-pong) kSets
+  // accumulators of BN columns, the running sums at 2 kSets BN, then kSA A
+  // stages of 64 columns (128 rows x 128 fp16 inputs, two per column) from
+  // column kACol0.
   constexpr uint32_t kTmemCols = 512;
-  constexpr int kACol0 = (3 * BN + 63) / 64 * 64;
+  constexpr uint32_t kRunCol = 2u * kSets * BN;
+  constexpr int kACol0 = ((2 * kSets + 1) * BN + 63) / 64 * 64;
   constexpr int kSA = (512 - kACol0) / 64 < 6 ? (512 - kACol0) / 64 : 6;
   static_assert(kSA >= 2, "at least two A stages must fit tensor memory");
 
@@ -261,7 +281,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int u = 0; it.valid() && go; it.next(), ++u) {
       const int sl = u % L.nu;
       const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
-      if (!__all_sync(0xffffffffu, bar_wait(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)))) {
+      if (!__all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)))) {
         if (lane == 0) fail();
         break;
       }
@@ -292,7 +312,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
           if (ai >= kSA &&
-              !__all_sync(0xffffffffu, bar_wait(emptyA + 8 * st, (uint32_t)(((ai - kSA) / kSA) & 1)))) {
+              !__all_sync(0xffffffffu, bar_wait_sleep(emptyA + 8 * st, (uint32_t)(((ai - kSA) / kSA) & 1)))) {
             if (lane == 0) fail();
             go = false;
             break;
@@ -318,7 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int sl = u % L.nu;
       const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
       const uint32_t bar = fullU + 8 * sl;
-      if (u >= L.nu && !__all_sync(0xffffffffu, bar_wait(emptyU + 8 * sl, (uint32_t)(((u / L.nu) - 1) & 1)))) {
+      if (u >= L.nu && !__all_sync(0xffffffffu, bar_wait_sleep(emptyU + 8 * sl, (uint32_t)(((u / L.nu) - 1) & 1)))) {
         if (lane == 0) fail();
         break;
       }
@@ -404,7 +424,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int w = 0; w < cnt && ok; ++w, ++j) {
         // The accumulator buffer of this K block is free once warps 16-19
         // have added in what it held for K block j - 2.
-        const uint32_t acc_tm = tmem + (uint32_t)(j & 1) * BN;
+        const uint32_t acc_tm = tmem + (uint32_t)(j & 1) * kSets * BN;
         if (j >= 2 && !bar_wait(accFree + 8 * (j & 1), (uint32_t)(((j - 2) >> 1) & 1))) {
           ok = false;
           break;
@@ -421,10 +441,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t db = smem_desc(bb0 + (uint32_t)(kk >> 2) * (kBTile / 2) + (uint32_t)(kk & 3) * 32u);
-            const uint32_t acc = (i | kk) != 0 ? 1u : 0u;   // each K block starts a fresh sum
+            // Each K block starts fresh sums; K step kk goes to set kk mod kSets.
+            const uint32_t acc = (i | (kk / kSets)) != 0 ? 1u : 0u;
             asm volatile(
                 "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(acc_tm),
+                " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(
+                    acc_tm + (uint32_t)(kk % kSets) * BN),
                 "r"(a0 + 8u * (uint32_t)kk), "l"(db), "r"(kIdesc), "r"(acc)
                 : "memory");
           }
@@ -453,17 +475,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp >= kTcFlushWarp0 && warp < kTcFlushWarp0 + 4) {
     const int wq = warp - kTcFlushWarp0;                     // accumulator lanes 32wq..32wq+31
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-    const uint32_t run_tm = lane_base + 2u * BN;
+    const uint32_t run_tm = lane_base + kRunCol;
     bool ok = true;
     for (int kb = 0; kb < nkb; ++kb) {
-      ok = ok && __all_sync(0xffffffffu, bar_wait(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
+      ok = ok && __all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
       if (!ok) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * BN;
+      const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * kSets * BN;
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t a[32], r[32];
         tmem_ld32(acc_tm + (uint32_t)c0, a);
+        if (kSets == 2) {
+          tmem_ld32(acc_tm + (uint32_t)(BN + c0), r);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) a[jj] = __float_as_uint(__uint_as_float(a[jj]) + __uint_as_float(r[jj]));
+        }
         if (kb > 0) tmem_ld32(run_tm + (uint32_t)c0, r);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
@@ -499,7 +527,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   // Everything issued has completed before tensor memory is freed.
-  const bool all_done = __all_sync(0xffffffffu, bar_wait(done, 0));
+  const bool all_done = __all_sync(0xffffffffu, bar_wait_sleep(done, 0));
   if (!all_done && lane == 0) atomicOr(status, kStatusTimeout);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
