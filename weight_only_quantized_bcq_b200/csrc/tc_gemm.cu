@@ -134,6 +134,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&v)[16]
       : "memory");
 }
 
+// tcgen05.commit from one elected lane of a converged warp: the mbarrier
+// arrives once all tensor-core work this thread issued before has completed.
+__device__ __forceinline__ void commit_one(uint32_t bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}" ::"r"(bar)
+      : "memory");
+}
+
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (start address and offsets in 16-byte units).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
@@ -209,7 +218,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t flag_slot = bars + 268;                     // CTA failure flag (shared)
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5;
+  // Broadcast from lane 0 so that the compiler knows the warp index, and all
+  // that derives from it, is warp-uniform.
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
   const int lane = tid & 31;
   const int rb = blockIdx.x;                                 // 128-row block
   const int b0 = blockIdx.y * BN;                            // first batch column
@@ -344,19 +355,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (__any_sync(0xffffffffu, failed())) break;
       const int cnt = it.count();
-      if (lane == 0) {
+      {
+        // The whole warp computes the copies; one elected lane issues each.
         uint32_t bytes = (uint32_t)cnt * kBTile;
         for (int wq = 0; wq < 4; ++wq)
           if (rb * 4 + wq < mt) bytes += 2u * (uint32_t)q * 512u;
         if (L.alpha_bulk) bytes += (uint32_t)(cnt * q * rows_here * 2);
-        asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+        asm volatile(
+            "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+            " @e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n}" ::"r"(bar),
+            "r"(bytes)
+            : "memory");
         for (int w = 0; w < cnt; ++w) {
           const int kb = it.kb(w);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
             asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-                "[%4];" ::"r"(slot + (uint32_t)w * kBTile + (uint32_t)h * (kBTile / 2)),
+                "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+                " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+                "[%4];\n}" ::"r"(slot + (uint32_t)w * kBTile + (uint32_t)h * (kBTile / 2)),
                 "l"(&xmap), "r"(kb * kTcBK + 64 * h), "r"(b0), "r"(bar)
                 : "memory");
         }
@@ -367,7 +384,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int h = 0; h < 2; ++h) {
             const uint8_t* src = packed + (((size_t)it.s * mt + R) * 8 + (size_t)(it.P ^ (4 * h))) * q * 512;
             asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+                " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
                     slot + L.bits_off + (uint32_t)((wq * 2 + h) * q * 512)),
                 "l"(src), "r"(q * 512), "r"(bar)
                 : "memory");
@@ -378,7 +396,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int G = it.kb(w) / kb_per_g;
             for (int i = 0; i < q; ++i)
               asm volatile(
-                  "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+                  " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
                       slot + L.alpha_off + (uint32_t)((w * q + i) * 256)),
                   "l"(alpha + ((size_t)i * ng + G) * m + (size_t)rb * kTcBM), "r"(rows_here * 2), "r"(bar)
                   : "memory");
@@ -407,8 +426,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) bar_arrive(bar);
     }
-  } else if (warp == kTcMmaWarp && lane == 0) {
-    // ---- MMA thread: per plane step, 8 MMAs into the K block's accumulator buffer.
+  } else if (warp == kTcMmaWarp) {
+    // ---- MMA warp: per plane step, 8 MMAs into the K block's accumulator
+    // buffers.  The whole warp runs the loop (its values stay warp-uniform,
+    // as the MMA operands must be); one elected lane issues each MMA and
+    // commit.
     UnitIter it;
     it.init(n);
     int ai = 0, j = 0;                                       // plane step, K block (processing order)
@@ -416,23 +438,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int u = 0; it.valid() && ok; it.next(), ++u) {
       const int sl = u % L.nu;
       const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
-      if (!bar_wait(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1))) {
+      if (!__all_sync(0xffffffffu, bar_wait(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)))) {
         ok = false;
         break;
       }
       const int cnt = it.count();
       for (int w = 0; w < cnt && ok; ++w, ++j) {
-        // The accumulator buffer of this K block is free once warps 16-19
-        // have added in what it held for K block j - 2.
+        // The accumulator buffers of this K block are free once warps 16-19
+        // have added in what they held for K block j - 2.
         const uint32_t acc_tm = tmem + (uint32_t)(j & 1) * kSets * BN;
-        if (j >= 2 && !bar_wait(accFree + 8 * (j & 1), (uint32_t)(((j - 2) >> 1) & 1))) {
+        if (j >= 2 && !__all_sync(0xffffffffu, bar_wait(accFree + 8 * (j & 1), (uint32_t)(((j - 2) >> 1) & 1)))) {
           ok = false;
           break;
         }
-        const uint32_t bb0 = slot + (uint32_t)w * kBTile;
+        const uint64_t db0 = smem_desc(slot + (uint32_t)w * kBTile);
         for (int i = 0; i < q; ++i, ++ai) {
           const int st = ai % kSA;
-          if (!bar_wait(fullA + 8 * st, (uint32_t)((ai / kSA) & 1))) {
+          if (!__all_sync(0xffffffffu, bar_wait(fullA + 8 * st, (uint32_t)((ai / kSA) & 1)))) {
             ok = false;
             break;
           }
@@ -440,34 +462,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t a0 = tmem + (uint32_t)kACol0 + (uint32_t)(st * 64);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t db = smem_desc(bb0 + (uint32_t)(kk >> 2) * (kBTile / 2) + (uint32_t)(kk & 3) * 32u);
+            // B: K step kk is 32 bytes into the 128-byte swizzle row, in the
+            // first or second 64-input half of the x tile (descriptor start
+            // address in 16-byte units).
+            const uint64_t db = db0 + (uint64_t)(((kk >> 2) * (kBTile / 2) + (kk & 3) * 32) >> 4);
             // Each K block starts fresh sums; K step kk goes to set kk mod kSets.
             const uint32_t acc = (i | (kk / kSets)) != 0 ? 1u : 0u;
             asm volatile(
-                "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(
+                "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+                " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(
                     acc_tm + (uint32_t)(kk % kSets) * BN),
                 "r"(a0 + 8u * (uint32_t)kk), "l"(db), "r"(kIdesc), "r"(acc)
                 : "memory");
           }
-          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                           emptyA + 8 * st)
-                       : "memory");
+          commit_one(emptyA + 8 * st);
         }
-        if (ok)
-          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                           accFull + 8 * (j & 1))
-                       : "memory");
+        if (ok) commit_one(accFull + 8 * (j & 1));
       }
       // The unit's x tiles are free once its MMAs have completed.
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                       emptyU + 8 * sl)
-                   : "memory");
+      commit_one(emptyU + 8 * sl);
     }
-    if (!ok) fail();
+    if (!ok && lane == 0) fail();
     // Completion of everything issued (also after a failure, before tensor memory is freed).
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
-                 : "memory");
+    commit_one(done);
   }
 
   // ---- Warps 16-19: add each K block's accumulator into the running sums
