@@ -586,6 +586,190 @@ def cpu_fit_baseline(q: int, g: int, iters: int, n: int, rows: int):
 
 
 # ---------------------------------------------------------------------------
+# Large-batch path on the tensor cores (lutgemm_run_tc): the layer's linears at
+# a prompt-phase batch.  One plane product per weight and batch column is two
+# flops; the tensor cores execute q of them per weight (one per plane), which
+# is the work this path's roofline counts.
+# ---------------------------------------------------------------------------
+TC_METRIC = ("BCQ tensor-core path (lutgemm_run_tc): plane TFLOP/s (2*q*m*n*batch per matmul) "
+             "over the OPT-175B layer's linears at prompt-phase batch")
+TC_SOURCES = ("tc_gemm.cu",)
+
+
+def _tc_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc")
+    for f in TC_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def _tc_peak():
+    """Dense fp16/bf16 tensor peak: measured (fp16 runs at the bf16 rate), the
+    sustained figure since the timed region is seconds of back-to-back launches."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), float(d["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1400.0, 1590.0, "fallback"
+
+
+def _tc_traffic(kernel_hash: str, names, batch: int):
+    path = os.path.join(ROOT, "profiles", "tc_gemm_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    per = d.get("per_shape_bytes", {})
+    if d.get("kernel_hash") != kernel_hash or d.get("batch") != batch or not all(n in per for n in names):
+        return None
+    return sum(per[n] for n in names) / len(names)
+
+
+def run_tc(args):
+    from weight_only_quantized_bcq_b200 import lutgemm
+    world, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    q, batch = args.q, args.tc_batch
+    w = S.WORKLOADS[WORKLOAD]
+    g = w.g
+    gen = S.generator(rank_seed(rank))
+    mats = []
+    for sh in w.shapes:
+        x_host = S.draw_x(gen, batch, sh.n).pin_memory()
+        mats.append({"name": sh.name, "m": sh.m, "n": sh.n,
+                     "packed": S.draw_random_bytes(gen, lutgemm.packed_bytes(q, sh.m, sh.n)).to(device),
+                     "alpha": S.draw_alpha(gen, q, sh.m, sh.n, g, w.alpha_sigma).to(device),
+                     "x_host": x_host, "x": x_host.to(device),
+                     "y": torch.empty((batch, sh.m), dtype=torch.float32, device=device),
+                     "y_host": torch.empty((batch, sh.m), dtype=torch.float32).pin_memory()})
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
+
+    def step(events=None):
+        for i, mt in enumerate(mats):
+            if events is not None:
+                events[i][0].record(stream)
+            lutgemm.run_tc(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    def e2e_step():
+        for mt in mats:
+            mt["x"].copy_(mt["x_host"], non_blocking=True)
+            lutgemm.run_tc(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], stream=stream)
+            mt["y_host"].copy_(mt["y"], non_blocking=True)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        barrier()
+    region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
+    per_launch = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+                   for _ in mats] for _ in range(args.steps)]
+    for k in range(args.steps):
+        step(per_launch[k])
+    barrier()
+    us_per = {mt["name"]: 1e3 * statistics.median(per_launch[k][i][0].elapsed_time(per_launch[k][i][1])
+                                                  for k in range(args.steps))
+              for i, mt in enumerate(mats)}
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1), device)
+
+    flops = {mt["name"]: 2 * q * mt["m"] * mt["n"] * batch for mt in mats}
+    step_flops = sum(flops.values())
+    value = step_flops * args.steps * world / (region_ms * 1e-3) / 1e12
+    e2e = step_flops * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    # Every launch in the region is tc_gemm_kernel: its achieved rate is the
+    # plane flops of all launches over the region's device time.
+    achieved = step_flops * args.steps / (region_ms * 1e-3) / 1e12
+    peak, peak_burst, peak_kind = _tc_peak()
+    khash = _tc_hash()
+    if rank == 0:
+        clk = clocks.summary()
+        out = {
+            "metric": TC_METRIC, "value": round(value, 1), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {
+                "workload": "OPT-175B decoder-layer linears (QKV 36864x12288, out 12288x12288, "
+                            f"FC1 49152x12288, FC2 12288x49152), BCQ q={q}, g={g}, batch {batch}, tensor cores",
+                "q": q, "g": g, "batch": batch,
+                "l2": "no flush: each step streams 765 MB (> 126 MB L2) of distinct weights",
+                "parallelism": "replicas" if world == 1 else f"replicas{world} (one layer per GPU)",
+            },
+            "us_per_matmul": {k: round(v, 1) for k, v in us_per.items()},
+            "us_per_matmul_note": "median of isolated launches (events around each launch)",
+            "tflops_per_matmul": {k: round(flops[k] / (us_per[k] * 1e-6) / 1e12, 1) for k in us_per},
+            "dense_equivalent_tflops": round(value / q, 1),
+            "dense_equivalent_note": "2*m*n*batch per matmul: the flops of the same product on dequantised weights",
+            "roofline": {
+                "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": _tc_traffic(khash, list(flops), batch),
+                "peak_kind": f"{peak_kind} bf16 sustained (fp16 dense rate = bf16); burst {peak_burst}",
+                "frac_of_burst": round(achieved / peak_burst, 4),
+                "kernel": "tc_gemm_kernel", "kernel_hash": khash,
+            },
+            "e2e": {"value": round(e2e, 1), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
+                    "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
+            "gpu_launches": len(mats) * args.steps,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_tc_baseline(q, batch, args.tc_cpu_rows)
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def cpu_tc_baseline(q: int, batch: int, rows: int):
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        secs, _ = _oracle_sample(q, batch, rows, seed=11)
+    fl = sum(2 * q * (32 * max(1, rows // 32)) * sh.n * batch for sh in S.WORKLOADS[WORKLOAD].shapes)
+    return {"value": round(fl / secs / 1e12, 8), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "seconds": round(secs, 2),
+            "sample": f"{32 * max(1, rows // 32)} rows of each of the 4 layer linears (q={q}, g=128, batch {batch}): "
+                      "oracle unpack + FP64 dequantise + matmul, one thread; plane flops 2*q*rows*n*batch"}
+
+
+# ---------------------------------------------------------------------------
 # Config sweep: isolated and back-to-back time of every parity config shape
 # (OPT-175B linears at batch 1..32, LLaMA-70B linears at batch 1..8), one
 # JSON line each, against both rooflines (HBM and shared-memory lookups).
@@ -668,9 +852,12 @@ def main():
                     help="scale layout lutgemm_run reads (packed: unit-major, reordered at load time)")
     ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
                     help="time one linear of the layer only (profiling)")
-    ap.add_argument("--workload", choices=["layer", "fit", "sweep"], default="layer",
+    ap.add_argument("--workload", choices=["layer", "fit", "sweep", "tc"], default="layer",
                     help="layer: the LUT-GEMM step (default); fit: BCQ fitting of FP16 weights; "
-                         "sweep: every parity config shape and batch, one line each")
+                         "sweep: every parity config shape and batch, one line each; "
+                         "tc: the layer's linears at a large batch on the tensor-core path")
+    ap.add_argument("--tc-batch", type=int, default=256)
+    ap.add_argument("--tc-cpu-rows", type=int, default=128, help="rows per linear in the tc CPU baseline sample")
     ap.add_argument("--fit-m", type=int, default=49152)
     ap.add_argument("--fit-n", type=int, default=12288)
     ap.add_argument("--fit-g", type=int, default=128)
@@ -681,6 +868,19 @@ def main():
     args.warmup = max(3, args.warmup)
     if args.workload == "sweep":
         run_sweep(args)
+    elif args.workload == "tc":
+        if args.impl == "reference":
+            world, rank, _ = _dist_env()
+            if rank == 0:
+                r = cpu_tc_baseline(args.q, args.tc_batch, args.tc_cpu_rows)
+                print(json.dumps({"impl": "reference", "metric": TC_METRIC, "value": r["value"],
+                                  "unit": "TFLOP/s", "n_gpus": world, "steps": 1, "warmup": 0,
+                                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                                  "dtype": "f64", "data": "synthetic", "cpu_baseline": r,
+                                  "e2e": {"value": r["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}), flush=True)
+        else:
+            run_tc(args)
     elif args.workload == "fit":
         if args.impl == "reference":
             world, rank, _ = _dist_env()
