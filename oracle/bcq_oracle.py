@@ -453,3 +453,93 @@ def fit_bcq_trace(w, q: int, g: int, iters: int):
     trace = []
     _fit_groups(w, q, g, iters, trace)
     return trace
+
+
+# ---------------------------------------------------------------------------
+# Variable-grid fitting: the BCQ planes plus one constant per (row, group),
+#   w ~ off + sum_i alpha_i * beta_i,
+# a grid of 2^q points built from bit-planes and scalar coefficients (BPDQ
+# card: "variable quantization grids from bit-planes and scalar
+# coefficients"; the pages give no more than that line).  It is the format
+# lutgemm_run consumes with an offset.  Reading used here, per (row, group):
+#   1. greedy: off = mean(w), r = w - off, then the BCQ greedy planes on r;
+#   2. `iters` rounds of
+#      a. least squares for (alpha_0 .. alpha_{q-1}, off) with the signs
+#         fixed: the columns are the q sign planes and a column of ones, the
+#         unknowns in that order; Cholesky of the (q+1) x (q+1) normal matrix,
+#         the same pivot rule (a dependent column keeps the previous values);
+#      b. each input takes the grid point off + sum_i alpha_i s_i nearest to w
+#         (ties: the largest code);
+#   3. alpha rounded to fp16, off to fp32 (the offset type lutgemm_run reads),
+#      then a last nearest-point step with the stored values.
+# At q = 1 this is Lloyd's algorithm for two levels in one dimension.
+# ---------------------------------------------------------------------------
+def nearest_grid_codes(w_groups, alpha, off):
+    """Nearest grid point off + sum_i alpha_i s_i.  w_groups [..., g],
+    alpha [q, ...], off [...] -> signs [q, ..., g] (+-1.0); ties: the largest code."""
+    a = np.asarray(alpha, dtype=np.float64)
+    S = _code_signs(a.shape[0])                               # [C][q]
+    vals = np.asarray(off, dtype=np.float64)[..., None] + np.einsum("cq,q...->...c", S, a)   # [..., C]
+    d = np.abs(np.asarray(w_groups, dtype=np.float64)[..., :, None] - vals[..., None, :])
+    C = S.shape[0]
+    best = C - 1 - np.argmin(d[..., ::-1], axis=-1)
+    return np.moveaxis(S[best], -1, 0)
+
+
+def _ls_grid(w_groups, B, a_old, off_old, g: int):
+    """Least squares for (alpha, off): the sign planes and a ones column."""
+    ones = np.ones((1,) + B.shape[1:])
+    coef = _ls_alpha(w_groups, np.concatenate([B, ones], axis=0),
+                     np.concatenate([a_old, np.asarray(off_old)[None]], axis=0), g)
+    return coef[:-1], coef[-1]
+
+
+def _grid_value(a, off, B):
+    return off[..., None] + np.einsum("i...,i...k->...k", a, B)
+
+
+def _fit_groups_grid(w, q: int, g: int, iters: int, trace=None):
+    W = np.asarray(w, dtype=np.float64)
+    m, n = W.shape
+    if n % g != 0:
+        raise ValueError("n % g != 0")
+    Wg = W.reshape(m, n // g, g)
+    off = Wg.mean(-1)
+    r = Wg - off[..., None]
+    B = np.empty((q,) + Wg.shape)
+    a = np.empty((q,) + Wg.shape[:-1])
+    for i in range(q):
+        B[i] = np.where(r >= 0, 1.0, -1.0)
+        a[i] = (B[i] * r).sum(-1) / g
+        r -= a[i][..., None] * B[i]
+    if trace is not None:
+        trace.append(((Wg - _grid_value(a, off, B)) ** 2).sum(-1))
+    for _ in range(iters):
+        a, off = _ls_grid(Wg, B, a, off, g)
+        if trace is not None:
+            trace.append(((Wg - _grid_value(a, off, B)) ** 2).sum(-1))
+        B = nearest_grid_codes(Wg, a, off)
+        if trace is not None:
+            trace.append(((Wg - _grid_value(a, off, B)) ** 2).sum(-1))
+    return Wg, a, off, B
+
+
+def fit_bcq_grid(w, q: int, g: int, iters: int):
+    """FP16 W [m][n] -> (signs int8 [q][m][n], alpha fp16 [q][n/g][m],
+    offset fp32 [n/g][m], squared error per group fp64 [n/g][m] of the stored result)."""
+    Wg, a, off, _ = _fit_groups_grid(w, q, g, iters)
+    a16 = a.astype(np.float16)
+    off32 = off.astype(np.float32)
+    B = nearest_grid_codes(Wg, a16.astype(np.float64), off32.astype(np.float64))
+    err = ((Wg - _grid_value(a16.astype(np.float64), off32.astype(np.float64), B)) ** 2).sum(-1)
+    m, ng, _ = Wg.shape
+    signs = B.reshape(q, m, ng * g).astype(np.int8)
+    return (signs, np.ascontiguousarray(np.transpose(a16, (0, 2, 1))), np.ascontiguousarray(off32.T),
+            np.ascontiguousarray(err.T))
+
+
+def fit_bcq_grid_trace(w, q: int, g: int, iters: int):
+    """Squared error per group after the greedy pass and after every step (unrounded values)."""
+    trace = []
+    _fit_groups_grid(w, q, g, iters, trace)
+    return trace

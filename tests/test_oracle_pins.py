@@ -758,3 +758,147 @@ def test_fit_pins_catch_mistakes(mutant):
 @pytest.mark.parametrize("mutant", [_nearest_farthest, _nearest_bits_reversed])
 def test_nearest_codes_pin_catches_mistakes(mutant):
     assert not pin_nearest_codes_bruteforce(mutant)
+
+
+# ---------------------------------------------------------------------------
+# Variable-grid fitting (planes + one constant per group): at q = 1 it is
+# Lloyd's two-level algorithm (checked against scikit-learn's k-means),
+# representable grids are recovered exactly, stored points are the nearest
+# grid points by brute force, the error never rises, and planted mistakes fail.
+# ---------------------------------------------------------------------------
+def pin_grid_q1_is_lloyd(fit_groups) -> bool:
+    """q = 1: the two grid points off -/+ alpha after k rounds are the centres
+    k-means (Lloyd, two clusters) reaches in k iterations from the greedy start."""
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(21)
+    w = (rng.standard_normal((3, 128)) * 0.02 + rng.standard_normal((3, 1)) * 0.01).astype(np.float16)
+    g = 64
+    for iters in (1, 3):
+        _, a0, off0, _ = fit_groups(w, 1, g, 0)
+        _, a, off, _ = fit_groups(w, 1, g, iters)
+        for j in range(3):
+            for G in range(2):
+                x = w[j, G * g:(G + 1) * g].astype(np.float64)[:, None]
+                init = np.array([[off0[j, G] - a0[0, j, G]], [off0[j, G] + a0[0, j, G]]])
+                km = KMeans(n_clusters=2, init=init, n_init=1, max_iter=iters, tol=0.0, algorithm="lloyd").fit(x)
+                want = np.sort(km.cluster_centers_[:, 0])
+                got = np.sort([off[j, G] - a[0, j, G], off[j, G] + a[0, j, G]])
+                if not np.allclose(got, want, rtol=0, atol=1e-12):
+                    return False
+    return True
+
+
+def pin_grid_exact_recovery(fit) -> bool:
+    """w = off + c (b1 + b2 / 2): signs, scales, offset recovered, error 0."""
+    rng = np.random.default_rng(22)
+    m, ng, g = 4, 3, 128
+    c = 2.0 ** rng.integers(-9, -5, size=(m, ng))
+    off = rng.integers(-64, 64, size=(m, ng)) * 2.0 ** -12
+    b = rng.choice([-1.0, 1.0], size=(2, m, ng, g))
+    w = (off[..., None] + c[..., None] * (b[0] + b[1] / 2)).reshape(m, ng * g).astype(np.float16)
+    signs, alpha, offset, err = fit(w, 2, g, 3)
+    return (np.array_equal(signs.reshape(2, m, ng, g), b.astype(np.int8))
+            and np.array_equal(alpha.astype(np.float64), np.stack([c, c / 2]).transpose(0, 2, 1))
+            and np.array_equal(offset.astype(np.float64), off.T) and float(np.abs(err).max()) == 0.0)
+
+
+def pin_grid_stored_points_are_nearest(fit) -> bool:
+    rng = np.random.default_rng(23)
+    q, g, m, n = 3, 64, 10, 256
+    w = (rng.standard_normal((m, n)) * 0.02 + 0.015).astype(np.float16)
+    signs, alpha, offset, err = fit(w, q, g, 2)
+    combos = np.array(list(itertools.product([-1.0, 1.0], repeat=q)))
+    for j in range(m):
+        for G in range(n // g):
+            a = alpha[:, G, j].astype(np.float64)
+            o = float(offset[G, j])
+            vals = o + combos @ a
+            wk = w[j, G * g:(G + 1) * g].astype(np.float64)
+            v = o + np.einsum("i,ik->k", a, signs[:, j, G * g:(G + 1) * g].astype(np.float64))
+            best = np.abs(wk[:, None] - vals[None, :]).min(axis=1)
+            if np.any(np.abs(wk - v) > best + 1e-15):
+                return False
+            e = float(((wk - v) ** 2).sum())
+            if abs(e - err[G, j]) > 1e-12 * max(e, 1e-30):
+                return False
+    return True
+
+
+def test_grid_pins():
+    assert pin_grid_q1_is_lloyd(O._fit_groups_grid)
+    assert pin_grid_exact_recovery(O.fit_bcq_grid)
+    assert pin_grid_stored_points_are_nearest(O.fit_bcq_grid)
+
+
+@pytest.mark.parametrize("q,g", [(1, 64), (2, 64), (3, 128), (4, 128)])
+def test_grid_error_never_rises_and_beats_plain_bcq_on_shifted_weights(q, g):
+    rng = np.random.default_rng(24 + q)
+    w = (rng.standard_normal((6, 512)) * 0.02 + 0.02).astype(np.float16)
+    trace = O.fit_bcq_grid_trace(w, q, g, 4)
+    scale = (w.astype(np.float64).reshape(6, -1, g) ** 2).sum(-1)
+    for before, after in zip(trace, trace[1:]):
+        assert np.all(after <= before + 1e-12 * scale)
+    # The plain BCQ grid is symmetric about 0; a constant per group can only help.
+    assert O.fit_bcq_grid(w, q, g, 4)[3].sum() < O.fit_bcq(w, q, g, 4)[2].sum()
+
+
+def test_grid_step_matches_least_squares():
+    rng = np.random.default_rng(25)
+    q, g = 3, 64
+    B = rng.choice([-1.0, 1.0], size=(q, 7, g))
+    w = rng.standard_normal((7, g)) + 0.5
+    a, off = O._ls_grid(w, B, np.zeros((q, 7)), np.zeros(7), g)
+    for r in range(7):
+        X = np.concatenate([B[:, r, :].T, np.ones((g, 1))], axis=1)
+        ref = np.linalg.lstsq(X, w[r], rcond=None)[0]
+        assert np.allclose(np.append(a[:, r], off[r]), ref, rtol=1e-10, atol=1e-12)
+
+
+def test_grid_step_keeps_values_when_a_plane_is_constant():
+    rng = np.random.default_rng(26)
+    B = rng.choice([-1.0, 1.0], size=(2, 1, 32))
+    B[1] = 1.0                                      # plane 1 = the ones column: singular
+    a_old, off_old = np.array([[0.3], [0.2]]), np.array([0.05])
+    a, off = O._ls_grid(rng.standard_normal((1, 32)), B, a_old, off_old, 32)
+    assert np.array_equal(a, a_old) and np.array_equal(off, off_old)
+
+
+def _grid_groups_offset_frozen(w, q, g, iters, trace=None):
+    """Planted: the offset stays at the group mean (only the scales are refit)."""
+    W = np.asarray(w, dtype=np.float64)
+    m, n = W.shape
+    Wg = W.reshape(m, n // g, g)
+    off = Wg.mean(-1)
+    r = Wg - off[..., None]
+    B = np.empty((q,) + Wg.shape)
+    a = np.empty((q,) + Wg.shape[:-1])
+    for i in range(q):
+        B[i] = np.where(r >= 0, 1.0, -1.0)
+        a[i] = (B[i] * r).sum(-1) / g
+        r -= a[i][..., None] * B[i]
+    for _ in range(iters):
+        a = O._ls_alpha(Wg - off[..., None], B, a, g)
+        B = O.nearest_grid_codes(Wg, a, off)
+    return Wg, a, off, B
+
+
+def _grid_fit_offset_ignored_in_codes(w, q, g, iters):
+    """Planted: the last nearest-point step forgets the offset."""
+    Wg, a, off, _ = O._fit_groups_grid(w, q, g, iters)
+    a16, off32 = a.astype(np.float16), off.astype(np.float32)
+    B = O.nearest_codes(Wg, a16.astype(np.float64))
+    err = ((Wg - O._grid_value(a16.astype(np.float64), off32.astype(np.float64), B)) ** 2).sum(-1)
+    m, ng, _ = Wg.shape
+    return B.reshape(q, m, ng * g).astype(np.int8), np.transpose(a16, (0, 2, 1)), off32.T, err.T
+
+
+def _grid_fit_offset_negated(w, q, g, iters):
+    """Planted: the stored offset has the wrong sign."""
+    s, a, off, err = O.fit_bcq_grid(w, q, g, iters)
+    return s, a, -off, err
+
+
+def test_grid_pins_catch_mistakes():
+    assert not pin_grid_q1_is_lloyd(_grid_groups_offset_frozen)
+    for mutant in (_grid_fit_offset_ignored_in_codes, _grid_fit_offset_negated):
+        assert not (pin_grid_exact_recovery(mutant) and pin_grid_stored_points_are_nearest(mutant))
