@@ -452,15 +452,15 @@ def run_reference(args):
 FIT_METRIC = "BCQ fit throughput: FP16 weights fitted per second (greedy + alternating least squares)"
 
 
-def _fit_profile(kernel_hash: str):
-    """Warp instructions per weight of fit_bcq_kernel from the committed ncu summary
-    (null unless it was taken on this kernel source)."""
+def _fit_profile(kernel_hash: str, variant: str):
+    """Warp instructions (and DRAM bytes) per weight of fit_bcq_kernel, plain or
+    grid, from the committed ncu summary (null unless taken on this kernel source)."""
     try:
         with open(os.path.join(ROOT, "profiles", "fit_bcq_instructions.json")) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
-    return d if d.get("kernel_hash") == kernel_hash else None
+    return d.get(variant) if d.get("kernel_hash") == kernel_hash else None
 
 
 def _fit_hash() -> str:
@@ -488,13 +488,20 @@ def run_fit(args):
     w = w_host.to(device)
     signs = torch.empty((q, m, n), dtype=torch.int8, device=device)
     alpha = torch.empty((q, n // g, m), dtype=torch.float16, device=device)
+    offset = torch.empty((n // g, m), dtype=torch.float32, device=device)
     lib = lutgemm.lib()
     import ctypes
 
     def fit_once(src):
-        st = lib.lutgemm_fit_bcq(ctypes.c_void_p(src.data_ptr()), q, m, n, g, iters,
-                                 ctypes.c_void_p(signs.data_ptr()), ctypes.c_void_p(alpha.data_ptr()), None,
-                                 ctypes.c_void_p(stream.cuda_stream))
+        if args.fit_grid:
+            st = lib.lutgemm_fit_bcq_grid(ctypes.c_void_p(src.data_ptr()), q, m, n, g, iters,
+                                          ctypes.c_void_p(signs.data_ptr()), ctypes.c_void_p(alpha.data_ptr()),
+                                          ctypes.c_void_p(offset.data_ptr()), None,
+                                          ctypes.c_void_p(stream.cuda_stream))
+        else:
+            st = lib.lutgemm_fit_bcq(ctypes.c_void_p(src.data_ptr()), q, m, n, g, iters,
+                                     ctypes.c_void_p(signs.data_ptr()), ctypes.c_void_p(alpha.data_ptr()), None,
+                                     ctypes.c_void_p(stream.cuda_stream))
         if st != 0:
             raise RuntimeError(lutgemm.status_string(st))
 
@@ -519,6 +526,7 @@ def run_fit(args):
     # End to end: W from pinned host memory in, signs and scales back out, per step.
     s_host = torch.empty(signs.shape, dtype=torch.int8).pin_memory()
     a_host = torch.empty(alpha.shape, dtype=torch.float16).pin_memory()
+    o_host = torch.empty(offset.shape, dtype=torch.float32).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     e0.record(stream)
@@ -527,6 +535,8 @@ def run_fit(args):
         fit_once(w)
         s_host.copy_(signs, non_blocking=True)
         a_host.copy_(alpha, non_blocking=True)
+        if args.fit_grid:
+            o_host.copy_(offset, non_blocking=True)
     e1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1), device)
@@ -536,7 +546,8 @@ def run_fit(args):
     if rank == 0:
         sm = torch.cuda.get_device_properties(device).multi_processor_count
         clk = clocks.summary()
-        prof = _fit_profile(_fit_hash())
+        variant = "grid" if args.fit_grid else "plain"
+        prof = _fit_profile(_fit_hash(), variant)
         # Issue-slot roofline: 4 schedulers per SM, one warp instruction each per clock.
         peak = 4 * sm * (clk["sm_mhz"] or 1965.0) * 1e6 / 1e9
         roof = {"bound": "alu", "unit": "G warp-inst/s", "peak": round(peak, 1), "peak_kind":
@@ -553,36 +564,39 @@ def run_fit(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": f"BCQ fit of FP16 W {m}x{n} ~ N(0, 0.02): q={q}, g={g}, {iters} rounds",
-                       "m": m, "n": n, "q": q, "g": g, "iters": iters,
+            "config": {"workload": (f"BCQ fit of FP16 W {m}x{n} ~ N(0, 0.02): q={q}, g={g}, {iters} rounds"
+                                    + (", variable grid (planes + one constant per group)" if args.fit_grid
+                                       else "")),
+                       "m": m, "n": n, "q": q, "g": g, "iters": iters, "grid": bool(args.fit_grid),
                        "l2": f"no flush: W is {2 * m * n / 1e6:.0f} MB (> 126 MB L2)",
                        "parallelism": "replicas" if world == 1 else f"replicas{world}"},
             "roofline": roof,
             "e2e": {"value": round(e2e, 2), "unit": "Gweights/s", "h2d_bytes_per_step": 2 * m * n,
-                    "d2h_bytes_per_step": q * m * n + 2 * q * (n // g) * m},
+                    "d2h_bytes_per_step": q * m * n + 2 * q * (n // g) * m
+                    + (4 * (n // g) * m if args.fit_grid else 0)},
             "gpu_launches": args.steps,
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_fit_baseline(q, g, iters, n, args.fit_cpu_rows)
+            out["cpu_baseline"] = cpu_fit_baseline(q, g, iters, n, args.fit_cpu_rows, args.fit_grid)
         print(json.dumps(out), flush=True)
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
 
 
-def cpu_fit_baseline(q: int, g: int, iters: int, n: int, rows: int):
-    import numpy as np
+def cpu_fit_baseline(q: int, g: int, iters: int, n: int, rows: int, grid: bool = False):
     from threadpoolctl import threadpool_limits
     from oracle import bcq_oracle as O
     w = S.draw_weights(S.generator(77), rows, n, 0.02).numpy()
+    fit = O.fit_bcq_grid if grid else O.fit_bcq
     with threadpool_limits(limits=1):
         t = time.perf_counter()
-        O.fit_bcq(w, q, g, iters)
+        fit(w, q, g, iters)
         secs = time.perf_counter() - t
     return {"value": round(rows * n / secs / 1e9, 6), "unit": "Gweights/s", "cores": 1, "kind": "oracle",
             "seconds": round(secs, 2),
-            "sample": f"{rows} rows x {n} of the same W distribution, oracle fit_bcq (FP64), one thread"}
+            "sample": f"{rows} rows x {n} of the same W distribution, oracle {fit.__name__} (FP64), one thread"}
 
 
 # ---------------------------------------------------------------------------
@@ -863,6 +877,8 @@ def main():
     ap.add_argument("--fit-g", type=int, default=128)
     ap.add_argument("--fit-iters", type=int, default=3)
     ap.add_argument("--fit-cpu-rows", type=int, default=384, help="rows of the CPU baseline fit sample")
+    ap.add_argument("--fit-grid", action="store_true",
+                    help="fit the variable grid (planes + one constant per group) instead of plain BCQ")
     args = ap.parse_args()
     # At least three untimed warm-up steps, whatever the caller asks for.
     args.warmup = max(3, args.warmup)
@@ -885,7 +901,7 @@ def main():
         if args.impl == "reference":
             world, rank, _ = _dist_env()
             if rank == 0:
-                r = cpu_fit_baseline(args.q, args.fit_g, args.fit_iters, args.fit_n, args.fit_cpu_rows)
+                r = cpu_fit_baseline(args.q, args.fit_g, args.fit_iters, args.fit_n, args.fit_cpu_rows, args.fit_grid)
                 print(json.dumps({"impl": "reference", "metric": FIT_METRIC, "value": r["value"],
                                   "unit": "Gweights/s", "n_gpus": world, "steps": 1, "warmup": 0,
                                   "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -186,6 +186,23 @@ int lutgemm_uniform_to_bcq(const uint8_t* codes, const uint16_t* scale,
 int lutgemm_fit_bcq(const uint16_t* w, int q, int m, int n, int g, int iters,
                     int8_t* signs, uint16_t* alpha, float* err, void* stream);
 
+/* The same fit on a variable grid: the planes plus one constant per (row,
+ * group), w ~ offset + sum_i alpha_i beta_i, a grid of 2^q points built from
+ * bit-planes and scalar coefficients (BPDQ card; the pages give no more than
+ * that line).  The greedy pass starts from the group mean; the least-squares
+ * step solves for the scales and the constant together (a plane set that is
+ * linearly dependent on the group and the constant keeps its values); the
+ * sign step takes the nearest grid point.  The result is the format
+ * lutgemm_run consumes with an offset: pack the signs with lutgemm_pack_bcq
+ * and pass alpha and offset.
+ *   w, q, m, n, g, iters, signs, alpha, err   as lutgemm_fit_bcq
+ *   offset     dev fp32 [n/g][m], 4-byte aligned (output; not rounded to fp16)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also for g > 1024), ERR_VALUE
+ * (iters out of range), ERR_ALIGN or ERR_CUDA. */
+int lutgemm_fit_bcq_grid(const uint16_t* w, int q, int m, int n, int g, int iters,
+                         int8_t* signs, uint16_t* alpha, float* offset, float* err,
+                         void* stream);
+
 /* Reorder group-wise plane scales into the unit-major scale layout above
  * (a data movement only: every output is one input value or 0).  The scales
  * are those of the BCQ format (LUT-GEMM card, Summary: q binary planes, each

@@ -167,6 +167,27 @@ def test_fit_validation(L):
     assert call(err=FAKE + 2) == L.ERR_ALIGN
 
 
+def test_fit_grid_validation(L):
+    lib = L.lib()
+    names = ["w", "q", "m", "n", "g", "iters", "signs", "alpha", "offset", "err", "stream"]
+    ok = [FAKE, 3, 32, 1024, 128, 3, FAKE, FAKE, FAKE, None, None]
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.lutgemm_fit_bcq_grid(*a)
+    assert call(w=None) == L.ERR_NULL
+    assert call(offset=None) == L.ERR_NULL       # the grid's constant is an output
+    assert call(signs=None) == L.ERR_NULL
+    assert call(q=0) == L.ERR_SHAPE
+    assert call(g=96) == L.ERR_SHAPE
+    assert call(n=4096, g=2048) == L.ERR_SHAPE
+    assert call(iters=65) == L.ERR_VALUE
+    assert call(w=FAKE + 8) == L.ERR_ALIGN
+    assert call(offset=FAKE + 2) == L.ERR_ALIGN
+    assert call(err=FAKE + 2) == L.ERR_ALIGN
+
+
 def test_pack_scales_validation(L):
     lib = L.lib()
     assert lib.lutgemm_pack_scales(None, 3, 32, 1024, 128, FAKE, None) == L.ERR_NULL

@@ -142,3 +142,91 @@ def test_fit_full_size_sampled_rows(L):
     e_exact = _check_signs_optimal(wr, s_np, a_np, g)
     assert np.allclose(err[:, torch.from_numpy(rows)].cpu().numpy(), e_exact, rtol=1e-4, atol=1e-12)
     assert abs(e_exact.sum() - o_err.sum()) <= 2e-3 * o_err.sum()
+
+
+# ---------------------------------------------------------------------------
+# Variable grid (lutgemm_fit_bcq_grid): planes plus one constant per group.
+# ---------------------------------------------------------------------------
+def _shifted_weights(seed, m, n, sigma=0.02):
+    """N(0, sigma) weights plus a per-row shift (what a constant per group can absorb)."""
+    gen = S.generator(seed)
+    w = S.draw_weights(gen, m, n, sigma).to(torch.float32)
+    shift = torch.randn((m, 1), generator=gen) * sigma
+    return (w + shift).to(torch.float16)
+
+
+def _check_grid_points_nearest(w, signs, alpha, offset, g):
+    q, m, n = signs.shape
+    W = w.astype(np.float64).reshape(m, n // g, g)
+    A = alpha.astype(np.float64).transpose(2, 1, 0)                      # [m][ng][q]
+    off = offset.astype(np.float64).T                                    # [m][ng]
+    B = signs.astype(np.float64).reshape(q, m, n // g, g)
+    v = off[..., None] + np.einsum("mgq,qmgk->mgk", A, B)
+    vals = off[..., None] + np.einsum("cq,mgq->mgc", O._code_signs(q), A)
+    best = np.abs(W[..., None] - vals[..., None, :]).min(-1)
+    slack = 2e-6 * (np.abs(W) + np.abs(off)[..., None] + np.abs(A).sum(-1, keepdims=True))
+    assert np.all(np.abs(W - v) <= best + slack)
+    return ((W - v) ** 2).sum(-1).T
+
+
+def test_grid_recovers_representable_grids_exactly(L):
+    rng = np.random.default_rng(520)
+    m, ng, g = 40, 5, 128
+    c = 2.0 ** rng.integers(-9, -5, size=(m, ng))
+    off = rng.integers(-64, 64, size=(m, ng)) * 2.0 ** -12
+    b = rng.choice([-1.0, 1.0], size=(2, m, ng, g))
+    w = (off[..., None] + c[..., None] * (b[0] + b[1] / 2)).reshape(m, ng * g).astype(np.float16)
+    signs, alpha, offset, err = L.fit_bcq_grid(torch.from_numpy(w).to(DEV), 2, g, iters=3, with_error=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(signs.cpu().numpy().reshape(2, m, ng, g), b.astype(np.int8))
+    assert np.array_equal(alpha.cpu().numpy().astype(np.float64), np.stack([c, c / 2]).transpose(0, 2, 1))
+    # The constant comes out of an fp32 solve: exact up to fp32 rounding of the
+    # group's magnitude (the FP64 oracle recovers it exactly).
+    tol = 8 * np.spacing((np.abs(off) + 1.5 * c).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(offset.cpu().numpy().astype(np.float64) - off.T) <= tol.T)
+    assert np.all(err.cpu().numpy() <= g * (tol.T ** 2))
+
+
+@pytest.mark.parametrize("q,g,iters,m,n", [(1, 64, 3, 64, 1024), (2, 64, 3, 96, 2048), (3, 128, 3, 80, 3072),
+                                           (4, 128, 2, 40, 2048), (6, 256, 2, 16, 1024)])
+def test_grid_matches_oracle(L, q, g, iters, m, n):
+    w = _shifted_weights(620 + q * 10 + g, m, n)
+    signs, alpha, offset, err = L.fit_bcq_grid(w.to(DEV), q, g, iters=iters, with_error=True)
+    torch.cuda.synchronize()
+    s_np, a_np, o_np = signs.cpu().numpy(), alpha.cpu().numpy(), offset.cpu().numpy()
+    e_exact = _check_grid_points_nearest(w.numpy(), s_np, a_np, o_np, g)
+    assert np.allclose(err.cpu().numpy().astype(np.float64), e_exact, rtol=1e-4, atol=1e-12)
+    o_signs, o_alpha, o_off, o_err = O.fit_bcq_grid(w.numpy(), q, g, iters)
+    same = np.all(s_np.reshape(q, m, n // g, g) == o_signs.reshape(q, m, n // g, g), axis=(0, 3)).T
+    assert same.mean() >= 0.97, same.mean()
+    assert abs(e_exact.sum() - o_err.sum()) <= 2e-3 * o_err.sum()
+    ulp = np.spacing(np.abs(o_alpha).astype(np.float16)).astype(np.float64)
+    assert (np.abs(a_np.astype(np.float64) - o_alpha.astype(np.float64)) <= 2 * ulp)[:, same].all()
+    # The constant comes out of the same fp32 solve: within fp32 rounding of the group's scale.
+    tol = 1e-5 * (np.abs(o_off) + np.abs(o_alpha.astype(np.float64)).sum(0))
+    assert (np.abs(o_np.astype(np.float64) - o_off.astype(np.float64)) <= tol)[same].all()
+    # On shifted weights the grid beats the plain (zero-centred) BCQ fit.
+    _, _, e_plain = L.fit_bcq(w.to(DEV), q, g, iters=iters, with_error=True)
+    assert e_exact.sum() < e_plain.cpu().numpy().sum()
+
+
+def test_grid_then_lutgemm_with_offset_matches_oracle_product(L):
+    """Fit a grid -> pack -> lutgemm_run with the offset: the lookup kernel
+    consumes the variable-grid format unchanged."""
+    m, n, q, g = 260, 2048, 3, 128
+    w = _shifted_weights(720, m, n)
+    x = S.draw_x(S.generator(721), 3, n)
+    signs, alpha, offset = L.fit_bcq_grid(w.to(DEV), q, g, iters=3)
+    y = L.run(L.pack_bcq(signs), alpha, x.to(DEV), m, n, q, g, offset=offset)
+    torch.cuda.synchronize()
+    y_ref = O.bcq_matmul(x.numpy(), signs.cpu().numpy(), alpha.cpu().numpy(), g, offset.cpu().numpy())
+    ok, st = compare(y.cpu().numpy(), y_ref, alpha.cpu().numpy(), x.numpy(), n)
+    assert ok, st
+
+
+def test_grid_is_deterministic(L):
+    w = _shifted_weights(722, 64, 2048).to(DEV)
+    a = L.fit_bcq_grid(w, 3, 128, iters=3)
+    b = L.fit_bcq_grid(w, 3, 128, iters=3)
+    torch.cuda.synchronize()
+    assert all(torch.equal(u, v) for u, v in zip(a, b))

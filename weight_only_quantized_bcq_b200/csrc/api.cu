@@ -19,6 +19,7 @@ cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, 
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const __half* x, void* y, int m, int n,
                            int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
 cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
+                           float* offset,
                            float* err, cudaStream_t stream);
 }  // namespace lutgemm
 
@@ -157,7 +158,21 @@ int lutgemm_fit_bcq(const uint16_t* w, int q, int m, int n, int g, int iters, in
   if (iters < 0 || iters > 64) return LUTGEMM_ERR_VALUE;
   if (!aligned(w, 16) || !aligned(signs, 8) || !aligned(alpha, 2) || !aligned(err, 4)) return LUTGEMM_ERR_ALIGN;
   const cudaError_t e = launch_fit_bcq(reinterpret_cast<const __half*>(w), q, m, n, g, iters, signs,
-                                       reinterpret_cast<__half*>(alpha), err, reinterpret_cast<cudaStream_t>(stream));
+                                       reinterpret_cast<__half*>(alpha), nullptr, err,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
+int lutgemm_fit_bcq_grid(const uint16_t* w, int q, int m, int n, int g, int iters, int8_t* signs, uint16_t* alpha,
+                         float* offset, float* err, void* stream) {
+  if (!w || !signs || !alpha || !offset) return LUTGEMM_ERR_NULL;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g > 1024) return LUTGEMM_ERR_SHAPE;
+  if (iters < 0 || iters > 64) return LUTGEMM_ERR_VALUE;
+  if (!aligned(w, 16) || !aligned(signs, 8) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(err, 4))
+    return LUTGEMM_ERR_ALIGN;
+  const cudaError_t e = launch_fit_bcq(reinterpret_cast<const __half*>(w), q, m, n, g, iters, signs,
+                                       reinterpret_cast<__half*>(alpha), offset, err,
+                                       reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 

@@ -13,6 +13,14 @@
 //      a code meaning beta_i = +1);
 //   3. scales rounded to fp16, then a last sign step with the rounded scales.
 //
+// With GRID (the variable grid: the planes plus one constant per group,
+// w ~ off + sum_i alpha_i beta_i; BPDQ card: grids from bit-planes and scalar
+// coefficients) the greedy pass starts from the group mean, the least-squares
+// step adds a column of ones (its normal-matrix entries are again exact
+// integer counts: sum_k beta_ik = 2 #(+1) - g, and g), the codes are
+// off + sum_i +-alpha_i, and the constant is stored in fp32 (the offset type
+// of lutgemm_run).
+//
 // A group is served by a segment of lpg lanes (the power of two at or above
 // g/8, at most 32), so a warp serves 32/lpg groups at once (two at g = 128);
 // a lane holds up to CPL chunks of 8 consecutive inputs (g <= 256 * CPL).  A chunk's signs are one mask with byte i = plane
@@ -58,10 +66,12 @@ __device__ __forceinline__ uint2 bits_to_signs(uint32_t b) {
   return make_uint2(0xFFFFFFFFu ^ (lo * 0xFEu), 0xFFFFFFFFu ^ (hi * 0xFEu));
 }
 
-template <int CPL, int Q>
+template <int CPL, int Q, bool GRID>
 __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* __restrict__ w, int m, int n, int g,
                                                                int lpg, int iters, int8_t* __restrict__ signs,
-                                                               __half* __restrict__ alpha, float* __restrict__ err) {
+                                                               __half* __restrict__ alpha, float* __restrict__ offset,
+                                                               float* __restrict__ err) {
+  constexpr int D = Q + (GRID ? 1 : 0);   // least-squares unknowns: the planes' scales (+ the constant)
   using Mask = std::conditional_t<(Q <= 4), uint32_t, uint64_t>;
   constexpr int NC = 1 << Q;
   constexpr bool REG_CODES = Q <= 4;
@@ -106,14 +116,23 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
       }
     }
 
-    // 1. Greedy planes on the residual.
+    // 1. Greedy planes on the residual (from the group mean on a grid).
     float a[Q];
+    float off = 0.f;
+    if constexpr (GRID) {
+      float s = 0.f;
+#pragma unroll
+      for (int t = 0; t < CPL; ++t)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += x[t][e];
+      off = seg_sum(s, lpg) * inv_g;
+    }
     {
       float r[CPL][8];
 #pragma unroll
       for (int t = 0; t < CPL; ++t)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) r[t][e] = x[t][e];
+        for (int e = 0; e < 8; ++e) r[t][e] = x[t][e] - off;
 #pragma unroll
       for (int i = 0; i < Q; ++i) {
         float s = 0.f;
@@ -139,12 +158,12 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
 
     // Nearest-code step for scales av; returns this lane's sum of squared
     // distances (the group error once the scales are final).
-    auto sign_step = [&](const float (&av)[Q]) -> float {
+    auto sign_step = [&](const float (&av)[Q], float ov) -> float {
       float cb[REG_CODES ? NC : 1];
       if constexpr (REG_CODES) {
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-          float v = 0.f;
+          float v = ov;
 #pragma unroll
           for (int i = 0; i < Q; ++i) v += ((c >> i) & 1) ? av[i] : -av[i];
           cb[c] = v;
@@ -152,7 +171,7 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
       } else {
         __syncwarp();
         for (int c = lane; c < NC; c += 32) {
-          float v = 0.f;
+          float v = ov;
 #pragma unroll
           for (int i = 0; i < Q; ++i) v += ((c >> i) & 1) ? av[i] : -av[i];
           codebook[wid][c] = v;
@@ -203,9 +222,11 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
     // 2. Alternating rounds.
     for (int it = 0; it < iters; ++it) {
       // Normal equations: M_ik = g - 2 * #(inputs where planes i and k differ),
-      // v_i = sum_k beta_ik * w_k.
+      // v_i = sum_k beta_ik * w_k; on a grid also M_iq = 2 #(beta_i = +1) - g,
+      // M_qq = g and v_q = sum_k w_k.
       int diff[Q * (Q - 1) / 2 + 1];
-      float v[Q];
+      int plus[Q];
+      float v[D];
 #pragma unroll
       for (int i = 0; i < Q; ++i) {
         float s = 0.f;
@@ -226,15 +247,38 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
           }
           diff[i * (i - 1) / 2 + k] = seg_sum_i(cnt, lpg);
         }
+        if constexpr (GRID) {
+          int cnt = 0;
+#pragma unroll
+          for (int t = 0; t < CPL; ++t) {
+            if (!live || sl + lpg * t >= chunks) continue;
+            cnt += __popc((uint32_t)((sg[t] >> (8 * i)) & 0xFFu));
+          }
+          plus[i] = seg_sum_i(cnt, lpg);
+        }
       }
+      if constexpr (GRID) {
+        float s = 0.f;
+#pragma unroll
+        for (int t = 0; t < CPL; ++t)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s += x[t][e];
+        v[Q] = seg_sum(s, lpg);
+      }
+      // Entry (i, k) of the normal matrix, i >= k.
+      auto mij = [&](int i, int k) -> float {
+        if (i < Q) return (i == k) ? (float)g : (float)(g - 2 * diff[i * (i - 1) / 2 + k]);
+        return (k < Q) ? (float)(2 * plus[k] - g) : (float)g;
+      };
+      (void)plus;
       // Cholesky of M (every lane, same arithmetic), then two triangular solves.
-      float L[Q][Q];
+      float L[D][D];
       bool ok = true;
 #pragma unroll
-      for (int i = 0; i < Q; ++i) {
+      for (int i = 0; i < D; ++i) {
 #pragma unroll
         for (int k = 0; k <= i; ++k) {
-          float acc = (i == k) ? (float)g : (float)(g - 2 * diff[i * (i - 1) / 2 + k]);
+          float acc = mij(i, k);
 #pragma unroll
           for (int l = 0; l < k; ++l) acc -= L[i][l] * L[k][l];
           if (i == k) {
@@ -246,30 +290,33 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
         }
       }
       if (ok) {
-        float y[Q];
+        float y[D], sol[D];
 #pragma unroll
-        for (int i = 0; i < Q; ++i) {
+        for (int i = 0; i < D; ++i) {
           float acc = v[i];
 #pragma unroll
           for (int l = 0; l < i; ++l) acc -= L[i][l] * y[l];
           y[i] = acc / L[i][i];
         }
 #pragma unroll
-        for (int i = Q - 1; i >= 0; --i) {
+        for (int i = D - 1; i >= 0; --i) {
           float acc = y[i];
 #pragma unroll
-          for (int l = i + 1; l < Q; ++l) acc -= L[l][i] * a[l];
-          a[i] = acc / L[i][i];
+          for (int l = i + 1; l < D; ++l) acc -= L[l][i] * sol[l];
+          sol[i] = acc / L[i][i];
         }
+#pragma unroll
+        for (int i = 0; i < Q; ++i) a[i] = sol[i];
+        if constexpr (GRID) off = sol[Q];
       }
-      (void)sign_step(a);
+      (void)sign_step(a, off);
     }
 
     // 3. fp16 scales, last sign step with them (its distances give the error).
     float a16[Q];
 #pragma unroll
     for (int i = 0; i < Q; ++i) a16[i] = __half2float(__float2half_rn(a[i]));
-    const float e2 = seg_sum(sign_step(a16), lpg);
+    const float e2 = seg_sum(sign_step(a16, off), lpg);
 #pragma unroll
     for (int t = 0; t < CPL; ++t) {
       const int c = sl + lpg * t;
@@ -285,13 +332,15 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
     for (int i = 0; i < Q; ++i)
       if (live && (i & (lpg - 1)) == sl) alpha[((size_t)i * ng + G) * m + j] = __float2half_rn(a16[i]);
     if (live && err && sl == 0) err[(size_t)G * m + j] = e2;
+    if constexpr (GRID)
+      if (live && sl == 0) offset[(size_t)G * m + j] = off;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
-                           float* err, cudaStream_t stream) {
+                           float* offset, float* err, cudaStream_t stream) {
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -310,16 +359,21 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
   const int cpl = (g + 255) / 256;
   const unsigned nb = (unsigned)blocks;
   const unsigned nt = kFitWarps * 32;
-#define LUTGEMM_FIT_Q(CPLv)                                                                        \
-  switch (q) {                                                                                     \
-    case 1: fit_bcq_kernel<CPLv, 1><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    case 2: fit_bcq_kernel<CPLv, 2><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    case 3: fit_bcq_kernel<CPLv, 3><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    case 4: fit_bcq_kernel<CPLv, 4><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    case 5: fit_bcq_kernel<CPLv, 5><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    case 6: fit_bcq_kernel<CPLv, 6><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    case 7: fit_bcq_kernel<CPLv, 7><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
-    default: fit_bcq_kernel<CPLv, 8><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, err); break; \
+#define LUTGEMM_FIT_QG(CPLv, Qv)                                                                        \
+  if (offset)                                                                                           \
+    fit_bcq_kernel<CPLv, Qv, true><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, offset, err); \
+  else                                                                                                  \
+    fit_bcq_kernel<CPLv, Qv, false><<<nb, nt, 0, stream>>>(w, m, n, g, lpg, iters, signs, alpha, offset, err);
+#define LUTGEMM_FIT_Q(CPLv)                \
+  switch (q) {                             \
+    case 1: LUTGEMM_FIT_QG(CPLv, 1) break; \
+    case 2: LUTGEMM_FIT_QG(CPLv, 2) break; \
+    case 3: LUTGEMM_FIT_QG(CPLv, 3) break; \
+    case 4: LUTGEMM_FIT_QG(CPLv, 4) break; \
+    case 5: LUTGEMM_FIT_QG(CPLv, 5) break; \
+    case 6: LUTGEMM_FIT_QG(CPLv, 6) break; \
+    case 7: LUTGEMM_FIT_QG(CPLv, 7) break; \
+    default: LUTGEMM_FIT_QG(CPLv, 8) break; \
   }
   if (cpl <= 1) {
     LUTGEMM_FIT_Q(1)
@@ -328,6 +382,7 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
   } else {
     LUTGEMM_FIT_Q(4)
   }
+#undef LUTGEMM_FIT_QG
 #undef LUTGEMM_FIT_Q
   return cudaGetLastError();
 }

@@ -30,6 +30,7 @@ _SIGNATURES = {
     "lutgemm_scales_bytes": ([_c_int, _c_int, _c_int, _c_int], _c_size),
     "lutgemm_pack_scales": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lutgemm_fit_bcq": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
+    "lutgemm_fit_bcq_grid": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
     "lutgemm_run_tc": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_uint, _vp], _c_int),
     "lutgemm_pack_bcq": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "lutgemm_uniform_to_bcq": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp],
@@ -132,6 +133,23 @@ def fit_bcq(w: torch.Tensor, q: int, g: int, iters: int = 3, with_error: bool = 
     _check(lib().lutgemm_fit_bcq(_ptr(w), q, m, n, g, iters, _ptr(signs), _ptr(alpha), _ptr(err), _stream(stream)),
            "lutgemm_fit_bcq")
     return (signs, alpha, err) if with_error else (signs, alpha)
+
+
+def fit_bcq_grid(w: torch.Tensor, q: int, g: int, iters: int = 3, with_error: bool = False, stream=None):
+    """fp16 weights [m][n] on the GPU -> (int8 signs [q][m][n], fp16 alpha [q][n/g][m],
+    fp32 offset [n/g][m] [, fp32 squared error per group [n/g][m]]) by lutgemm_fit_bcq_grid:
+    the variable grid offset + sum_i alpha_i beta_i, run with ``run(..., offset=offset)``."""
+    _need(w, torch.float16, "w")
+    m, n = w.shape
+    ng = n // g if g > 0 else 0
+    signs = torch.empty((q, m, n), dtype=torch.int8, device=w.device)
+    alpha = torch.empty((q, ng, m), dtype=torch.float16, device=w.device)
+    offset = torch.empty((ng, m), dtype=torch.float32, device=w.device)
+    err = torch.empty((ng, m), dtype=torch.float32, device=w.device) if with_error else None
+    _check(lib().lutgemm_fit_bcq_grid(_ptr(w), q, m, n, g, iters, _ptr(signs), _ptr(alpha), _ptr(offset), _ptr(err),
+                                      _stream(stream)),
+           "lutgemm_fit_bcq_grid")
+    return (signs, alpha, offset, err) if with_error else (signs, alpha, offset)
 
 
 def pack_bcq(signs: torch.Tensor, packed: torch.Tensor = None, status_flags: torch.Tensor = None,
