@@ -97,6 +97,25 @@ def test_tc_full_size_fc1_sampled(L):
     assert ok, st
 
 
+@pytest.mark.parametrize("name,m,n", [("fc2", 12288, 49152), ("qkv", 36864, 12288)])
+def test_tc_full_size_bench_configuration_sampled(L, name, m, n):
+    """The launch configuration bench.py --workload tc times: OPT-175B linears at
+    q = 3, g = 128, batch 256 (the 128-column batch blocks): sampled rows."""
+    q, g, batch = 3, 128, 256
+    gen = S.generator(954 + m % 7)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n))
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.02)
+    x = S.draw_x(gen, batch, n)
+    y = L.run_tc(packed.to(DEV), alpha.to(DEV), x.to(DEV), m, n, q, g)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(955).choice(m, 24, replace=False))
+    s_rows = O.unpack_rows(packed.numpy(), q, m, n, rows)
+    a_rows = alpha.numpy()[:, :, rows]
+    y_ref = O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g)
+    ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_rows, x.numpy(), n)
+    assert ok, st
+
+
 def test_tc_rejects_unsupported_shapes(L):
     signs, alpha, x = _problem(953, 3, 64, 1024, 64, 4)
     packed = L.pack_bcq(signs.to(DEV))

@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bar_init(emptyU + 8 * s, kTcDequantWarps + 1);       // dequant warps + the MMA commit
     }
     for (int s = 0; s < kSA; ++s) {
-      bar_init(fullA + 8 * s, kTcDequantWarps);
+      bar_init(fullA + 8 * s, kTcDequantWarps / 2);       // one group of dequant warps per step
       bar_init(emptyA + 8 * s, 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -269,21 +269,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp < kTcDequantWarps) {
     // ---- Dequant warps: plane tiles of +-alpha, written to tensor memory.
+    // Two groups of 8 warps take alternate plane steps, so each warp has two
+    // step periods for its part of a step and consecutive A stages are filled
+    // by different warps.
+    const int grp = warp >> 3;                               // plane steps ai with ai mod 2 == grp
     const int wq = warp & 3;                                 // tile rows (= TMEM lanes) 32wq..32wq+31
-    const int hq = warp >> 2;                                // K quarter: runs 4 hq .. 4 hq + 3
+    const int hsel = (warp >> 2) & 1;                        // K half: runs 8 hsel .. 8 hsel + 7
     const int row = (rb * 4 + wq) * kTileRows + lane;        // weight row of this thread
     const int half_sel = lane >> 4;
     // The lane's 16-byte piece holds run c in byte c ^ (lane mod 16): runs
-    // 4 hq .. 4 hq + 3 sit in its 32-bit word hq ^ (bits 2-3 of the lane),
-    // byte cc ^ (lane mod 4) for run 4 hq + cc.  One byte permutation per
-    // step puts them in run order.
-    const int wi = hq ^ ((lane >> 2) & 3);
-    uint32_t sel = 0;
+    // 8 hsel .. 8 hsel + 7 sit in its 8-byte half hsel ^ (bit 3 of the lane),
+    // byte cc ^ (lane mod 8) for run 8 hsel + cc.  Two byte permutations per
+    // step put them in run order.
+    const int h8 = hsel ^ ((lane >> 3) & 1);
+    uint32_t sel0 = 0, sel1 = 0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) sel |= ((uint32_t)k ^ (uint32_t)(lane & 3)) << (4 * k);
+    for (int k = 0; k < 4; ++k) {
+      sel0 |= ((uint32_t)k ^ (uint32_t)(lane & 7)) << (4 * k);
+      sel1 |= ((uint32_t)(k + 4) ^ (uint32_t)(lane & 7)) << (4 * k);
+    }
     const uint32_t row_mask = row < m ? 0xFFFFFFFFu : 0u;   // rows past m get a zero scale
-    const uint32_t a_tm = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)kACol0 + (uint32_t)(16 * hq);
-    const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * 2 * q * 512 + lane * 16 + wi * 4);
+    const uint32_t a_tm = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)kACol0 + (uint32_t)(32 * hsel);
+    const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * 2 * q * 512 + lane * 16 + h8 * 8);
     const uint32_t alpha_lane = L.alpha_off + (uint32_t)((wq * 32 + lane) * 2);
     UnitIter it;
     it.init(n);
@@ -302,20 +309,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t bsrc = slot + bits_lane + (uint32_t)((half_sel ^ w) * q * 512);
         const uint32_t asrc = slot + alpha_lane + (uint32_t)(w * q * 256);
         for (int i = 0; i < q; ++i, ++ai) {
+          if ((ai & 1) != grp) continue;
           const int st = ai % kSA;
-          uint32_t bits, ah;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits) : "r"(bsrc + (uint32_t)(i * 512)) : "memory");
+          uint32_t b0w, b1w, ah;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0w), "=r"(b1w) : "r"(bsrc + (uint32_t)(i * 512))
+                       : "memory");
           asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc + (uint32_t)(i * 256)) : "memory");
-          const uint32_t wr = __byte_perm(bits, 0u, sel);     // runs 0..3 of the quarter, in order
+          const uint32_t w0 = __byte_perm(b0w, b1w, sel0);   // runs 0..3 of the half, in order
+          const uint32_t w1 = __byte_perm(b0w, b1w, sel1);   // runs 4..7
           // Element pair (2e, 2e+1) of a run byte b: the product b * (2^(15-2e)
           // + 2^(30-2e)) puts bit 2e at bit 15 and bit 2e+1 at bit 31 (the two
           // fp16 sign bits), with no carries between the two copies.  A clear
           // bit (beta = -1) sets the sign of +alpha.
           const uint32_t a2 = (ah | (ah << 16)) & row_mask;
-          uint32_t v[16];
+          uint32_t v[32];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const uint32_t b = __byte_perm(wr, 0u, 0x4440u | (uint32_t)cc);
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint32_t b = __byte_perm(cc < 4 ? w0 : w1, 0u, 0x4440u | (uint32_t)(cc & 3));
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const uint32_t t = b * ((1u << (15 - 2 * e)) + (1u << (30 - 2 * e)));
@@ -329,7 +339,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          tmem_st16(a_tm + (uint32_t)(st * 64), v);
+          tmem_st32(a_tm + (uint32_t)(st * 64), v);
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
           __syncwarp();
