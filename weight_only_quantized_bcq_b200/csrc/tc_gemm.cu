@@ -101,6 +101,17 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// 16 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(addr)
+      : "memory");
+}
+
 // 32 consecutive fp32 columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&v)[32]) {
   asm volatile(
@@ -198,13 +209,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // stays full.  At BN = 128 an MMA takes longer than that dependency, and
   // tensor memory holds one set only.
   constexpr int kSets = BN <= 64 ? 2 : 1;
+  // At BN = 32 the accumulate warps keep the running sums in registers (32
+  // per thread); wider tiles keep them in tensor memory.
+  constexpr bool kRunRegs = BN <= 32;
   // Tensor memory (all 512 columns): per K block (two, ping-pong) kSets
   // accumulators of BN columns, the running sums at 2 kSets BN, then kSA A
   // stages of 64 columns (128 rows x 128 fp16 inputs, two per column) from
   // column kACol0.
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kRunCol = 2u * kSets * BN;
-  constexpr int kACol0 = ((2 * kSets + 1) * BN + 63) / 64 * 64;
+  constexpr int kACol0 = ((2 * kSets + (kRunRegs ? 0 : 1)) * BN + 63) / 64 * 64;
   constexpr int kSA = (512 - kACol0) / 64 < 6 ? (512 - kACol0) / 64 : 6;
   static_assert(kSA >= 2, "at least two A stages must fit tensor memory");
 
@@ -498,60 +512,90 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // ---- Warps 16-19: add each K block's accumulator into the running sums
-  // (tensor memory, fp32 adds with round to nearest), then write y.
+  // (fp32 adds with round to nearest; registers at BN = 32, tensor memory
+  // above), then write y.
   if (warp >= kTcFlushWarp0 && warp < kTcFlushWarp0 + 4) {
     const int wq = warp - kTcFlushWarp0;                     // accumulator lanes 32wq..32wq+31
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t run_tm = lane_base + kRunCol;
-    bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      ok = ok && __all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
-      if (!ok) break;
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * kSets * BN;
+    const int row = (rb * 4 + wq) * kTileRows + lane;
+    auto store_y = [&](int c0, const uint32_t (&r)[32]) {
+      if (row >= m) return;
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t a[32], r[32];
-        tmem_ld32(acc_tm + (uint32_t)c0, a);
-        if (kSets == 2) {
-          tmem_ld32(acc_tm + (uint32_t)(BN + c0), r);
+      for (int jj = 0; jj < 32; ++jj) {
+        const int b = b0 + c0 + jj;
+        if (b < batch) {
+          const size_t o = (size_t)b * m + row;
+          const float f = __uint_as_float(r[jj]);
+          if (y_f16) reinterpret_cast<__half*>(y)[o] = __float2half_rn(f);
+          else reinterpret_cast<float*>(y)[o] = f;
+        }
+      }
+    };
+    bool ok = true;
+    if constexpr (kRunRegs) {
+      uint32_t run[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) run[jj] = 0u;
+      for (int kb = 0; kb < nkb; ++kb) {
+        ok = ok && __all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
+        if (!ok) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * kSets * BN;
+#pragma unroll
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+          uint32_t a[16], b[16];
+          tmem_ld16(acc_tm + (uint32_t)c0, a);
+          tmem_ld16(acc_tm + (uint32_t)(BN + c0), b);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) a[jj] = __float_as_uint(__uint_as_float(a[jj]) + __uint_as_float(r[jj]));
-        }
-        if (kb > 0) tmem_ld32(run_tm + (uint32_t)c0, r);
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj)
-          r[jj] = kb > 0 ? __float_as_uint(__uint_as_float(r[jj]) + __uint_as_float(a[jj])) : a[jj];
-        tmem_st32(run_tm + (uint32_t)c0, r);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      bar_arrive(accFree + 8 * (kb & 1));
-    }
-    if (!ok && lane == 0) fail();
-    const int row = (rb * 4 + wq) * kTileRows + lane;
-    if (ok) {
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(run_tm + (uint32_t)c0, r);
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (row < m) {
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const int b = b0 + c0 + jj;
-            if (b < batch) {
-              const size_t o = (size_t)b * m + row;
-              const float f = __uint_as_float(r[jj]);
-              if (y_f16) reinterpret_cast<__half*>(y)[o] = __float2half_rn(f);
-              else reinterpret_cast<float*>(y)[o] = f;
-            }
+          for (int jj = 0; jj < 16; ++jj) {
+            const float f = __uint_as_float(a[jj]) + __uint_as_float(b[jj]);
+            run[c0 + jj] = kb > 0 ? __float_as_uint(__uint_as_float(run[c0 + jj]) + f) : __float_as_uint(f);
           }
         }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        bar_arrive(accFree + 8 * (kb & 1));
+      }
+      if (ok) store_y(0, run);
+    } else {
+      for (int kb = 0; kb < nkb; ++kb) {
+        ok = ok && __all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
+        if (!ok) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * kSets * BN;
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t a[32], r[32];
+          tmem_ld32(acc_tm + (uint32_t)c0, a);
+          if (kSets == 2) {
+            tmem_ld32(acc_tm + (uint32_t)(BN + c0), r);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) a[jj] = __float_as_uint(__uint_as_float(a[jj]) + __uint_as_float(r[jj]));
+          }
+          if (kb > 0) tmem_ld32(run_tm + (uint32_t)c0, r);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            r[jj] = kb > 0 ? __float_as_uint(__uint_as_float(r[jj]) + __uint_as_float(a[jj])) : a[jj];
+          tmem_st32(run_tm + (uint32_t)c0, r);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        bar_arrive(accFree + 8 * (kb & 1));
+      }
+      if (ok) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(run_tm + (uint32_t)c0, r);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          store_y(c0, r);
+        }
       }
     }
+    if (!ok && lane == 0) fail();
   }
   // Everything issued has completed before tensor memory is freed.
   const bool all_done = __all_sync(0xffffffffu, bar_wait_sleep(done, 0));
