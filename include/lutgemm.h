@@ -255,8 +255,9 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
  * column).  Same operands and result as lutgemm_run (pure BCQ, no offsets).
  * Each plane enters the tensor cores as its exact fp16 values +-alpha (a
  * scale times a sign), so no rounded dequantised weight is formed; the planes
- * accumulate in fp32 (tcgen05.mma, tensor memory).  Tiles: 128 rows x up to
- * 256 batch columns x 128 inputs.  The pages' kernel is the lookup one; this
+ * accumulate in fp32 (tcgen05.mma, tensor memory; each 128-input block's sum
+ * is added into round-to-nearest fp32 running sums).  Tiles: 128 rows x 32,
+ * 64 or 128 batch columns x 128 inputs.  The pages' kernel is the lookup one; this
  * path is for prompt-sized batches, where the method is compute-bound (LUT-GEMM
  * card, Summary and Key points: generation is memory-bound, large batches are
  * not).

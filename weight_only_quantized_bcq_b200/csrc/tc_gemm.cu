@@ -19,23 +19,27 @@
 //     both.  Each unit holds the two x tiles (TMA, 128-byte swizzle,
 //     K-major), the 8 chunk groups of the tile's 4 row tiles and the 2 x q
 //     scale rows of the tile.
-//   warps 0-15 (dequant): expand a plane's bits for the tile into a 128 x
-//     128 fp16 A tile in tensor memory (row r in lane r, inputs 2c and 2c+1
-//     in column c: the layout the tensor cores read an A operand from);
-//     warp w takes rows 32(w mod 4)..+31 (the lanes it may access) and the
-//     32-input quarter w / 4.  A never touches shared memory.
-//   warp 20 (MMA): one thread issues the 8 tcgen05.mma (K = 16 each, A from
-//     tensor memory, B from shared memory) per plane and commits them to the
-//     mbarriers that free A stages, units and accumulators.
+//   warps 0-15 (dequant, two groups of 8 taking alternate plane steps):
+//     expand a plane's bits for the tile into a 128 x 128 fp16 A tile in
+//     tensor memory (row r in lane r, inputs 2c and 2c+1 in column c: the
+//     layout the tensor cores read an A operand from); in a group, warp w
+//     takes rows 32(w mod 4)..+31 (the lanes it may access) and the
+//     64-input half (w / 4) mod 2.  A never touches shared memory.
+//   warp 20 (MMA): the converged warp runs the loop and one elected lane
+//     issues the 8 tcgen05.mma (K = 16 each, A from tensor memory, B from
+//     shared memory) per plane and the commits that free A stages, units
+//     and accumulators.
 //   warps 16-19 (accumulate): see below.
 //
 // Accumulation: the tensor cores add into their fp32 accumulator with
 // truncation, so an error of up to an ulp per MMA step would build up over
 // the q * n / 16 steps of a long row.  Each K block therefore accumulates in
-// a fresh tensor-memory buffer (two, ping-pong), and warps 16-19 add it into
-// fp32 running sums (round to nearest) as soon as its MMAs complete; warp
-// 16+w owns accumulator lanes 32w..32w+31 = tile rows, keeps the running
-// sums in a third tensor-memory buffer and writes them to y.
+// fresh tensor-memory buffers (two per K block at BN <= 64, even and odd K
+// steps, so consecutive MMAs are independent; ping-pong between K blocks),
+// and warps 16-19 add them into fp32 running sums (round to nearest) as soon
+// as the block's MMAs complete; warp 16+w owns accumulator lanes
+// 32w..32w+31 = tile rows, keeps the running sums (in registers at BN = 32,
+// in tensor memory above) and writes them to y.
 // Every mbarrier wait is bounded (1 s); a timeout sets status bit 2, the CTA
 // stops issuing work, waits (bounded) for its tensor-core work in flight and
 // frees its tensor memory before exiting.
