@@ -53,14 +53,25 @@ def _peaks():
 KERNEL_SOURCES = ("lutgemm_common.cuh", "lutgemm_run.cuh")
 
 
-def _kernel_hash() -> str:
-    """Hash of the sources that define lut_gemm_kernel (ncu counters are tied to it)."""
+def _code_hash(files) -> str:
+    """Hash of CUDA sources with their comments removed: the ncu counters in
+    profiles/ are tied to the code, and an edit of comments alone keeps them."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc")
-    for f in KERNEL_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+    for f in files:
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        text = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(f.encode() + text.encode())
     return h.hexdigest()[:16]
+
+
+def _kernel_hash() -> str:
+    """Hash of the code that defines lut_gemm_kernel (ncu counters are tied to it)."""
+    return _code_hash(KERNEL_SOURCES)
 
 
 def _traffic(kernel_hash: str, names):
@@ -464,10 +475,7 @@ def _fit_profile(kernel_hash: str, variant: str):
 
 
 def _fit_hash() -> str:
-    h = hashlib.sha256()
-    with open(os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc", "fit.cu"), "rb") as f:
-        h.update(f.read())
-    return h.hexdigest()[:16]
+    return _code_hash(("fit.cu",))
 
 
 def run_fit(args):
@@ -611,12 +619,7 @@ TC_SOURCES = ("tc_gemm.cu",)
 
 
 def _tc_hash() -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "weight_only_quantized_bcq_b200", "csrc")
-    for f in TC_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
-    return h.hexdigest()[:16]
+    return _code_hash(TC_SOURCES)
 
 
 def _tc_peak():
