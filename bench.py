@@ -170,30 +170,44 @@ def make_layer(q: int, batch: int, seed: int, device, only=None, scales="packed"
 
     With scales="packed" the [q][n/g][m] scales are reordered once, at load
     time, into the unit-major layout that lutgemm_run reads with
-    LUTGEMM_SCALES_PACKED (same bytes for g = 128)."""
+    LUTGEMM_SCALES_PACKED (same bytes for g = 128).
+
+    The step's inputs x and outputs y of all linears sit in one buffer each
+    (host: pinned; device), each linear's x and y a view into it, so the end
+    to end step moves them with one copy each way."""
     from weight_only_quantized_bcq_b200 import lutgemm
     w = S.WORKLOADS[WORKLOAD]
     gen = S.generator(seed)
+    shapes = [sh for sh in w.shapes if not only or sh.name == only]
+    xs = sum(batch * sh.n for sh in shapes)
+    ys = sum(batch * sh.m for sh in shapes)
+    io = {"x_host": torch.empty(xs, dtype=torch.float16).pin_memory(),
+          "x": torch.empty(xs, dtype=torch.float16, device=device),
+          "y_host": torch.empty(ys, dtype=torch.float32).pin_memory(),
+          "y": torch.empty(ys, dtype=torch.float32, device=device)}
     mats = []
-    for sh in w.shapes:
-        if only and sh.name != only:
-            continue
+    xo = yo = 0
+    for sh in shapes:
         nbytes = lutgemm.packed_bytes(q, sh.m, sh.n)
         packed = S.draw_random_bytes(gen, nbytes).to(device)
         alpha = S.draw_alpha(gen, q, sh.m, sh.n, w.g, w.alpha_sigma).to(device)
         if scales == "packed":
             alpha = lutgemm.pack_scales(alpha, sh.m, sh.n, w.g)
-        x_host = S.draw_x(gen, batch, sh.n).pin_memory()
+        x_host = io["x_host"][xo: xo + batch * sh.n].view(batch, sh.n)
+        x_host.copy_(S.draw_x(gen, batch, sh.n))
         mats.append({
             "name": sh.name, "m": sh.m, "n": sh.n, "packed": packed, "alpha": alpha,
             "scales_packed": scales == "packed", "launches": 1 + (sh.n > 1024),
-            "x_host": x_host, "x": x_host.to(device),
-            "y": torch.empty((batch, sh.m), dtype=torch.float32, device=device),
-            "y_host": torch.empty((batch, sh.m), dtype=torch.float32).pin_memory(),
+            "x_host": x_host, "x": io["x"][xo: xo + batch * sh.n].view(batch, sh.n),
+            "y": io["y"][yo: yo + batch * sh.m].view(batch, sh.m),
+            "y_host": io["y_host"][yo: yo + batch * sh.m].view(batch, sh.m),
             "ws": lutgemm.new_workspace(sh.m, sh.n, batch, q, w.g, device=device),
             "bytes": algorithmic_bytes(sh.m, sh.n, q, w.g, batch),
         })
-    return mats, w.g
+        xo += batch * sh.n
+        yo += batch * sh.m
+    io["x"].copy_(io["x_host"])
+    return mats, w.g, io
 
 
 def max_over_ranks(dist, v: float, device) -> float:
@@ -236,7 +250,7 @@ def run_lutgemm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
         pg = dist
     q, batch = args.q, args.batch
-    mats, g = make_layer(q, batch, seed=rank_seed(rank), device=device, only=args.only, scales=args.scales)
+    mats, g, io = make_layer(q, batch, seed=rank_seed(rank), device=device, only=args.only, scales=args.scales)
     # All work goes on one non-default stream (a CUDA graph cannot be captured
     # on the legacy default stream); it is made current so torch's copies use it.
     stream = torch.cuda.Stream(device=device)
@@ -252,11 +266,11 @@ def run_lutgemm(args):
                 events[i][1].record(stream)
 
     def e2e_step():
+        io["x"].copy_(io["x_host"], non_blocking=True)
         for mt in mats:
-            mt["x"].copy_(mt["x_host"], non_blocking=True)
             lutgemm.run(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"],
                         workspace=mt["ws"], scales_packed=mt["scales_packed"], stream=stream)
-            mt["y_host"].copy_(mt["y"], non_blocking=True)
+        io["y_host"].copy_(io["y"], non_blocking=True)
 
     def barrier():
         torch.cuda.synchronize()
@@ -371,8 +385,9 @@ def run_lutgemm(args):
                 "peak_kind": peak_kind, "kernel": "lut_gemm_kernel", "kernel_hash": khash,
             },
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
-                    "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
-                    "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
+                    "h2d_bytes_per_step": io["x_host"].numel() * 2,
+                    "d2h_bytes_per_step": io["y_host"].numel() * 4,
+                    "copies_per_step": "one H2D of all x, one D2H of all y (pinned host buffers)"},
             # Per lutgemm_run: the lookup kernel, plus the split-K reduce when n > 1024.
             "gpu_launches": sum(mt["launches"] for mt in mats) * args.steps,
             "clocks": clocks.summary(),
@@ -663,15 +678,26 @@ def run_tc(args):
     w = S.WORKLOADS[WORKLOAD]
     g = w.g
     gen = S.generator(rank_seed(rank))
+    # All linears' x and y in one buffer each (views per linear): one copy each way per e2e step.
+    xs, ys = sum(batch * sh.n for sh in w.shapes), sum(batch * sh.m for sh in w.shapes)
+    io = {"x_host": torch.empty(xs, dtype=torch.float16).pin_memory(),
+          "x": torch.empty(xs, dtype=torch.float16, device=device),
+          "y_host": torch.empty(ys, dtype=torch.float32).pin_memory(),
+          "y": torch.empty(ys, dtype=torch.float32, device=device)}
     mats = []
+    xo = yo = 0
     for sh in w.shapes:
-        x_host = S.draw_x(gen, batch, sh.n).pin_memory()
+        x_host = io["x_host"][xo: xo + batch * sh.n].view(batch, sh.n)
+        x_host.copy_(S.draw_x(gen, batch, sh.n))
         mats.append({"name": sh.name, "m": sh.m, "n": sh.n,
                      "packed": S.draw_random_bytes(gen, lutgemm.packed_bytes(q, sh.m, sh.n)).to(device),
                      "alpha": S.draw_alpha(gen, q, sh.m, sh.n, g, w.alpha_sigma).to(device),
-                     "x_host": x_host, "x": x_host.to(device),
-                     "y": torch.empty((batch, sh.m), dtype=torch.float32, device=device),
-                     "y_host": torch.empty((batch, sh.m), dtype=torch.float32).pin_memory()})
+                     "x_host": x_host, "x": io["x"][xo: xo + batch * sh.n].view(batch, sh.n),
+                     "y": io["y"][yo: yo + batch * sh.m].view(batch, sh.m),
+                     "y_host": io["y_host"][yo: yo + batch * sh.m].view(batch, sh.m)})
+        xo += batch * sh.n
+        yo += batch * sh.m
+    io["x"].copy_(io["x_host"])
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)
 
@@ -684,10 +710,10 @@ def run_tc(args):
                 events[i][1].record(stream)
 
     def e2e_step():
+        io["x"].copy_(io["x_host"], non_blocking=True)
         for mt in mats:
-            mt["x"].copy_(mt["x_host"], non_blocking=True)
             lutgemm.run_tc(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], stream=stream)
-            mt["y_host"].copy_(mt["y"], non_blocking=True)
+        io["y_host"].copy_(io["y"], non_blocking=True)
 
     def barrier():
         torch.cuda.synchronize()
@@ -762,8 +788,9 @@ def run_tc(args):
                 "kernel": "tc_gemm_kernel", "kernel_hash": khash,
             },
             "e2e": {"value": round(e2e, 1), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
-                    "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
+                    "h2d_bytes_per_step": io["x_host"].numel() * 2,
+                    "d2h_bytes_per_step": io["y_host"].numel() * 4,
+                    "copies_per_step": "one H2D of all x, one D2H of all y (pinned host buffers)"},
             "gpu_launches": len(mats) * args.steps,
             "clocks": clk,
         }
