@@ -101,6 +101,7 @@ extern "C" {
 /* Flags of lutgemm_run. */
 #define LUTGEMM_Y_F16          1u /* write y as fp16 (round to nearest even of the fp32 sum) */
 #define LUTGEMM_SCALES_PACKED  2u /* alpha is in the unit-major scale layout (g % 128 == 0) */
+#define LUTGEMM_ALLOW_TENSOR_CORES 4u /* lutgemm_run may compute on the tensor cores (see there) */
 
 /* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
 int lutgemm_version(void);
@@ -236,8 +237,15 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *              fp16 (2-byte aligned); fully overwritten.  For n > 1024 the
  *   call enqueues two kernels: the lookup kernel writes per-slice partial
  *   sums to the workspace and a reduce kernel adds them in slice order.
- *   flags      OR of LUTGEMM_Y_F16 and LUTGEMM_SCALES_PACKED; other bits,
- *              or LUTGEMM_SCALES_PACKED with g % 128 != 0, give ERR_VALUE
+ *   flags      OR of LUTGEMM_Y_F16, LUTGEMM_SCALES_PACKED and
+ *              LUTGEMM_ALLOW_TENSOR_CORES; other bits, or
+ *              LUTGEMM_SCALES_PACKED with g % 128 != 0, give ERR_VALUE.
+ *              With LUTGEMM_ALLOW_TENSOR_CORES the call computes the product
+ *              as lutgemm_run_tc does (same result within the same
+ *              tolerance, not the same bits) when that path is the faster
+ *              one and takes the operands: batch >= 8, no offset, scales in
+ *              [q][n/g][m], n % 128 == 0 and g % 128 == 0; the workspace is
+ *              then left untouched.  Otherwise the flag changes nothing.
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
  *              16-byte aligned, zero-filled before its first use; left
  *              zero-filled by every successful call.  Calls that share a
@@ -287,7 +295,8 @@ int lutgemm_run_tc(int m, int n, int batch, int q, int g,
  *   workspace.  Returns LUTGEMM_ERR_WORKSPACE when the problem needs more
  *   scratch than the array holds: more than 16 MiB - 4 KiB - 256 B of
  *   split-K partial sums (batch * ceil(n/1024) * ceil(m/32) * 128 bytes when
- *   n > 1024).  Other statuses as for lutgemm_run.
+ *   n > 1024); a call that LUTGEMM_ALLOW_TENSOR_CORES sends to the tensor
+ *   cores needs no scratch.  Other statuses as for lutgemm_run.
  *   The first call on a device does a one-time set-up on that device (looks
  *   up the array's device address and zeroes its counters on `stream`); make
  *   that first call before any stream capture.  Every call shares the one

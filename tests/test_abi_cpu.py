@@ -109,8 +109,9 @@ def test_run_rejects_misaligned(L):
 
 
 def test_run_rejects_bad_flags_and_small_workspace(L):
-    assert _run(L, flags=4) == L.ERR_VALUE
-    assert _run(L, flags=8 | L.Y_F16) == L.ERR_VALUE
+    assert _run(L, flags=8) == L.ERR_VALUE
+    assert _run(L, flags=16 | L.Y_F16) == L.ERR_VALUE
+    assert _run(L, flags=8 | L.ALLOW_TENSOR_CORES) == L.ERR_VALUE
     # Unit-major scales need g % 128 == 0 and a 16-byte aligned scale buffer.
     assert _run(L, n=1024, g=64, flags=L.SCALES_PACKED) == L.ERR_VALUE
     assert _run(L, alpha=FAKE + 2, flags=L.SCALES_PACKED) == L.ERR_ALIGN

@@ -122,3 +122,45 @@ def test_tc_rejects_unsupported_shapes(L):
     with pytest.raises(L.LutgemmError) as e:
         L.run_tc(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 64)
     assert e.value.status == L.ERR_SHAPE
+
+
+def test_run_with_tensor_cores_allowed_takes_the_faster_path(L):
+    """lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: from batch 8 (pure BCQ,
+    g % 128 == 0, [q][n/g][m] scales) the result is bit for bit that of
+    lutgemm_run_tc; below batch 8, or with an offset, that of the lookup path."""
+    q, m, n, g = 3, 384, 2048, 128
+    for batch, want_tc in ((8, True), (40, True), (4, False)):
+        signs, alpha, x = _problem(960 + batch, q, m, n, g, batch)
+        packed, a_d, x_d = L.pack_bcq(signs.to(DEV)), alpha.to(DEV), x.to(DEV)
+        y = L.run(packed, a_d, x_d, m, n, q, g, allow_tensor_cores=True)
+        ref = L.run_tc(packed, a_d, x_d, m, n, q, g) if want_tc else L.run(packed, a_d, x_d, m, n, q, g)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), batch
+        ok, st = compare(y.cpu().numpy(), O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), g),
+                         alpha.numpy(), x.numpy(), n)
+        assert ok, st
+    # With an offset the lookup path runs, whatever the batch.
+    signs, alpha, x = _problem(970, q, m, n, g, 16)
+    off = torch.randn((n // g, m), generator=S.generator(971)) * 0.01
+    packed, a_d, x_d, o_d = L.pack_bcq(signs.to(DEV)), alpha.to(DEV), x.to(DEV), off.to(DEV)
+    y = L.run(packed, a_d, x_d, m, n, q, g, offset=o_d, allow_tensor_cores=True)
+    ref = L.run(packed, a_d, x_d, m, n, q, g, offset=o_d)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+
+
+def test_noalloc_with_tensor_cores_allowed_needs_no_scratch(L):
+    """FC1 at batch 64 needs more split-K scratch than the no-alloc array holds;
+    with the tensor cores allowed it takes that path and needs none."""
+    m, n, q, g, batch = 49152, 12288, 3, 128, 64
+    gen = S.generator(972)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n)).to(DEV)
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.02).to(DEV)
+    x = S.draw_x(gen, batch, n).to(DEV)
+    with pytest.raises(L.LutgemmError) as e:
+        L.run_noalloc(packed, alpha, x, m, n, q, g)
+    assert e.value.status == L.ERR_WORKSPACE
+    y = L.run_noalloc(packed, alpha, x, m, n, q, g, allow_tensor_cores=True)
+    ref = L.run_tc(packed, alpha, x, m, n, q, g)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)

@@ -220,7 +220,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   if (!packed || !alpha || !x || !y || !workspace) return LUTGEMM_ERR_NULL;
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED)) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_ALLOW_TENSOR_CORES)) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
   if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
@@ -228,6 +228,15 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
     return LUTGEMM_ERR_ALIGN;
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
+  // From batch 8 the tensor-core path is the faster one (FC1-sized layers:
+  // 275 against 300 us at batch 8, 320 against 2360 us at 64).
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && offset == nullptr && !scales_packed &&
+      n % 128 == 0 && g % 128 == 0) {
+    const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha),
+                                         reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
+                                         nullptr, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+  }
 
   RunParams p;
   p.packed = packed;

@@ -25,6 +25,11 @@
 #include "lutgemm.h"
 #include "lutgemm_common.cuh"
 
+namespace lutgemm {
+cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const __half* x, void* y, int m, int n,
+                           int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
+}  // namespace lutgemm
+
 namespace {
 
 using namespace lutgemm;
@@ -47,6 +52,7 @@ DeviceScratch g_dev[64];
 std::set<std::pair<const void*, int>> g_smem_done;
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
+const __half* alpha_ptr_h(const uint16_t* a) { return reinterpret_cast<const __half*>(a); }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 RunKernel pick_kernel(int q, int g, bool has_offset, bool packed) {
@@ -113,13 +119,20 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   if (q < 1 || q > 8 || m < 1 || n < 8 || n % 8 != 0 || g < 8 || g % 8 != 0 || n % g != 0 || batch < 1)
     return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED)) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_ALLOW_TENSOR_CORES)) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
   if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
   if (!aligned(packed, 16) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(offset, 4) ||
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
+  // The tensor-core path needs no scratch at all (same rule as lutgemm_run).
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && offset == nullptr && !scales_packed &&
+      n % 128 == 0 && g % 128 == 0) {
+    const cudaError_t e = launch_tc_gemm(packed, alpha_ptr_h(alpha), reinterpret_cast<const __half*>(x), y, m, n,
+                                         batch, q, g, y_f16 ? 1 : 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+  }
   const int ns = ceil_div(n, kSliceInputs);
   const int mt = ceil_div(m, kTileRows);
   const size_t partials = (size_t)batch * ns * mt * kTileRows * sizeof(float);

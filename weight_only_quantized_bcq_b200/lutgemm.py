@@ -18,6 +18,7 @@ OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_VALUE, ERR_CUDA = range(7
 FLAG_BAD_SIGN, FLAG_BAD_CODE, FLAG_BAD_ZERO = 1, 2, 4
 Y_F16 = 1
 SCALES_PACKED = 2
+ALLOW_TENSOR_CORES = 4
 
 _lib = None
 
@@ -183,9 +184,11 @@ def uniform_to_bcq(codes: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
 
 def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
         offset: torch.Tensor = None, y: torch.Tensor = None, workspace: torch.Tensor = None,
-        y_f16: bool = False, scales_packed: bool = False, stream=None) -> torch.Tensor:
+        y_f16: bool = False, scales_packed: bool = False, allow_tensor_cores: bool = False,
+        stream=None) -> torch.Tensor:
     """y[b] = W x[b] for a packed BCQ weight W (m x n), computed by lutgemm_run.
-    With ``scales_packed`` alpha is the output of ``pack_scales``."""
+    With ``scales_packed`` alpha is the output of ``pack_scales``; with
+    ``allow_tensor_cores`` the library may take the tensor-core path (batch >= 8)."""
     _need(packed, torch.uint8, "packed")
     _need(alpha, torch.float16, "alpha")
     _need(x, torch.float16, "x")
@@ -196,7 +199,8 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     if workspace is None:
         workspace = new_workspace(m, n, batch, q, g, device=x.device)
-    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0)
+    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0) | \
+        (ALLOW_TENSOR_CORES if allow_tensor_cores else 0)
     _check(lib().lutgemm_run(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
                              flags, _ptr(workspace), workspace.numel(), _stream(stream)),
            "lutgemm_run")
@@ -221,7 +225,7 @@ def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n
 
 def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
                 offset: torch.Tensor = None, y: torch.Tensor = None, y_f16: bool = False,
-                scales_packed: bool = False, stream=None) -> torch.Tensor:
+                scales_packed: bool = False, allow_tensor_cores: bool = False, stream=None) -> torch.Tensor:
     """``run`` through lutgemm_run_noalloc, for callers that cannot allocate a
     workspace: the library uses its own fixed 16 MiB device scratch instead.
     Only ``y`` is allocated here, and only when the caller passes none.  Calls
@@ -234,7 +238,8 @@ def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: i
     batch = x.shape[0] if x.dim() == 2 else 1
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
-    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0)
+    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0) | \
+        (ALLOW_TENSOR_CORES if allow_tensor_cores else 0)
     _check(lib().lutgemm_run_noalloc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x),
                                      _ptr(y), flags, _stream(stream)),
            "lutgemm_run_noalloc")
