@@ -243,7 +243,7 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *              With LUTGEMM_ALLOW_TENSOR_CORES the call computes the product
  *              as lutgemm_run_tc does (same result within the same
  *              tolerance, not the same bits) when that path is the faster
- *              one and takes the operands: batch >= 8, no offset, scales in
+ *              one and takes the operands: batch >= 8, scales in
  *              [q][n/g][m], n % 128 == 0 and g % 128 == 0; the workspace is
  *              then left untouched.  Otherwise the flag changes nothing.
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
@@ -260,7 +260,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
 
 /* y = W x for a BCQ weight on the tensor cores: the large-batch path, where
  * the lookup kernel's per-column table reads dominate (one table per batch
- * column).  Same operands and result as lutgemm_run (pure BCQ, no offsets).
+ * column).  Same operands and result as lutgemm_run.
  * Each plane enters the tensor cores as its exact fp16 values +-alpha (a
  * scale times a sign), so no rounded dequantised weight is formed; the planes
  * accumulate in fp32 (tcgen05.mma, tensor memory; each 128-input block's sum
@@ -270,13 +270,16 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
  * card, Summary and Key points: generation is memory-bound, large batches are
  * not).
  *   m, n, batch, q, g  as lutgemm_run, and n % 128 == 0, g % 128 == 0
- *   packed, alpha, x, y  as lutgemm_run ([q][n/g][m] scales)
+ *   packed, alpha, offset, x, y  as lutgemm_run ([q][n/g][m] scales; offset
+ *              NULL for pure BCQ, else fp32 [n/g][m], 4-byte aligned: each
+ *              128-input block adds offset * (the block's input sum) in fp32)
  *   flags      0 or LUTGEMM_Y_F16
  * Needs no workspace.  Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_VALUE,
  * ERR_ALIGN or ERR_CUDA. */
 int lutgemm_run_tc(int m, int n, int batch, int q, int g,
                    const uint8_t* packed, const uint16_t* alpha,
-                   const uint16_t* x, void* y, unsigned flags, void* stream);
+                   const float* offset, const uint16_t* x, void* y,
+                   unsigned flags, void* stream);
 
 /* Bytes of the device scratch array used by lutgemm_run_noalloc (16 MiB). */
 #define LUTGEMM_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -129,11 +129,11 @@ def test_scales_bytes(L):
 
 def test_run_tc_validation(L):
     lib = L.lib()
-    ok = [256, 1024, 16, 3, 128, FAKE, FAKE, FAKE, FAKE, 0, None]
+    ok = [256, 1024, 16, 3, 128, FAKE, FAKE, None, FAKE, FAKE, 0, None]
     def call(**kw):
         a = list(ok)
         for k, v in kw.items():
-            a[["m", "n", "batch", "q", "g", "packed", "alpha", "x", "y", "flags", "stream"].index(k)] = v
+            a[["m", "n", "batch", "q", "g", "packed", "alpha", "offset", "x", "y", "flags", "stream"].index(k)] = v
         return lib.lutgemm_run_tc(*a)
     assert call(packed=None) == L.ERR_NULL
     assert call(y=None) == L.ERR_NULL
@@ -144,6 +144,7 @@ def test_run_tc_validation(L):
     assert call(x=FAKE + 8) == L.ERR_ALIGN
     assert call(packed=FAKE + 8) == L.ERR_ALIGN
     assert call(y=FAKE + 2) == L.ERR_ALIGN
+    assert call(offset=FAKE + 2) == L.ERR_ALIGN  # offsets are fp32
 
 
 def test_fit_validation(L):

@@ -127,7 +127,7 @@ def test_tc_rejects_unsupported_shapes(L):
 def test_run_with_tensor_cores_allowed_takes_the_faster_path(L):
     """lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: from batch 8 (pure BCQ,
     g % 128 == 0, [q][n/g][m] scales) the result is bit for bit that of
-    lutgemm_run_tc; below batch 8, or with an offset, that of the lookup path."""
+    lutgemm_run_tc; below batch 8 that of the lookup path."""
     q, m, n, g = 3, 384, 2048, 128
     for batch, want_tc in ((8, True), (40, True), (4, False)):
         signs, alpha, x = _problem(960 + batch, q, m, n, g, batch)
@@ -139,12 +139,12 @@ def test_run_with_tensor_cores_allowed_takes_the_faster_path(L):
         ok, st = compare(y.cpu().numpy(), O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), g),
                          alpha.numpy(), x.numpy(), n)
         assert ok, st
-    # With an offset the lookup path runs, whatever the batch.
+    # With an offset the tensor-core path takes it too.
     signs, alpha, x = _problem(970, q, m, n, g, 16)
     off = torch.randn((n // g, m), generator=S.generator(971)) * 0.01
     packed, a_d, x_d, o_d = L.pack_bcq(signs.to(DEV)), alpha.to(DEV), x.to(DEV), off.to(DEV)
     y = L.run(packed, a_d, x_d, m, n, q, g, offset=o_d, allow_tensor_cores=True)
-    ref = L.run(packed, a_d, x_d, m, n, q, g, offset=o_d)
+    ref = L.run_tc(packed, a_d, x_d, m, n, q, g, offset=o_d)
     torch.cuda.synchronize()
     assert torch.equal(y, ref)
 
@@ -164,3 +164,29 @@ def test_noalloc_with_tensor_cores_allowed_needs_no_scratch(L):
     ref = L.run_tc(packed, alpha, x, m, n, q, g)
     torch.cuda.synchronize()
     assert torch.equal(y, ref)
+
+
+
+@pytest.mark.parametrize("q,m,n,g,batch", [(4, 256, 2048, 128, 40), (3, 300, 2560, 256, 100), (2, 128, 1024, 128, 7),
+                                           (4, 136, 1280, 128, 129)])
+def test_tc_uniform_weights_with_offsets(L, q, m, n, g, batch):
+    """Uniform q-bit weights rewritten as BCQ plus group offsets (the lookup
+    path's config of converted weights) on the tensor cores, against the
+    oracle's dequantised product."""
+    gen = S.generator(980 + q + batch)
+    codes = torch.randint(0, 1 << q, (m, n), generator=gen, dtype=torch.uint8)
+    scale = (torch.randn((n // g, m), generator=gen).abs() * 0.01).to(torch.float16)
+    zero = torch.randint(0, 1 << q, (n // g, m), generator=gen, dtype=torch.uint8)
+    x = S.draw_x(gen, batch, n)
+    packed, alpha, offset = L.uniform_to_bcq(codes.to(DEV), scale.to(DEV), zero.to(DEV), q, g)
+    y = L.run_tc(packed, alpha, x.to(DEV), m, n, q, g, offset=offset)
+    torch.cuda.synchronize()
+    w = O.uniform_dequant(codes.numpy(), scale.numpy(), zero.numpy(), g)
+    y_ref = x.numpy().astype(np.float64) @ w.T
+    ok, st = compare(y.cpu().numpy(), y_ref, alpha.cpu().numpy(), x.numpy(), n)
+    assert ok, st
+    # The lookup path on the same operands meets the same bound.
+    y_lut = L.run(packed, alpha, x.to(DEV), m, n, q, g, offset=offset)
+    torch.cuda.synchronize()
+    ok, st = compare(y_lut.cpu().numpy(), y_ref, alpha.cpu().numpy(), x.numpy(), n)
+    assert ok, st

@@ -16,8 +16,8 @@ cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, con
                                   int32_t* flags, cudaStream_t stream);
 cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
                                cudaStream_t stream);
-cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const __half* x, void* y, int m, int n,
-                           int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
+cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
+                           int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
 cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
                            float* offset,
                            float* err, cudaStream_t stream);
@@ -137,15 +137,16 @@ size_t lutgemm_scales_bytes(int q, int m, int n, int g) {
 }
 
 int lutgemm_run_tc(int m, int n, int batch, int q, int g, const uint8_t* packed, const uint16_t* alpha,
-                   const uint16_t* x, void* y, unsigned flags, void* stream) {
+                   const float* offset, const uint16_t* x, void* y, unsigned flags, void* stream) {
   if (!packed || !alpha || !x || !y) return LUTGEMM_ERR_NULL;
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1 || g % 128 != 0 || n % 128 != 0)
     return LUTGEMM_ERR_SHAPE;
   if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
-  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
+  if (!aligned(packed, 16) || !aligned(alpha, 2) || !aligned(offset, 4) || !aligned(x, 16) ||
+      !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
-  const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha),
+  const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
                                        reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
                                        nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
@@ -230,9 +231,8 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
   // From batch 8 the tensor-core path is the faster one (FC1-sized layers:
   // 275 against 300 us at batch 8, 320 against 2360 us at 64).
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && offset == nullptr && !scales_packed &&
-      n % 128 == 0 && g % 128 == 0) {
-    const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha),
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 128 == 0) {
+    const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
                                          reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
                                          nullptr, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;

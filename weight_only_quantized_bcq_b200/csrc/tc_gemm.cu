@@ -7,7 +7,8 @@
 // its exact fp16 values +-alpha_i (an fp16 times a sign is exact), so no
 // dequantised weight is ever rounded; the planes accumulate into one fp32
 // tensor-memory accumulator.  Needs g % 128 == 0 (one scale per plane and
-// 128-input piece) and no uniform offsets.
+// 128-input piece); group offsets (uniform weights rewritten as BCQ) are
+// added per K block in fp32 by the accumulate warps.
 //
 // CTA tile: 128 rows (MMA M) x BN batch columns (MMA N) over K blocks of 128
 // inputs (one piece of the packed layout).  Warp roles:
@@ -105,6 +106,14 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// 8 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(addr)
+               : "memory");
+}
+
 // 16 consecutive fp32 columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&v)[16]) {
   asm volatile(
@@ -199,11 +208,11 @@ struct TcLayout {
   int alpha_bulk;          // scale rows by bulk copy (16-byte aligned rows) or by lane loads
 };
 
-template <int BN>
+template <int BN, bool HAS_OFF>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed,
-                   const __half* __restrict__ alpha, void* y, int m, int n, int batch, int q, int g, int mt,
-                   int y_f16, unsigned* status, TcLayout L) {
+                   const __half* __restrict__ alpha, const float* __restrict__ offset, void* y, int m, int n,
+                   int batch, int q, int g, int mt, int y_f16, unsigned* status, TcLayout L) {
   constexpr uint32_t kBTile = (uint32_t)BN * kTcBK * 2;   // x tile: BN rows x 128 inputs
   // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128.
   constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
@@ -249,7 +258,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < L.nu; ++s) {
       bar_init(fullU + 8 * s, 1);
-      bar_init(emptyU + 8 * s, kTcDequantWarps + 1);       // dequant warps + the MMA commit
+      // dequant warps + the MMA commit (+ the accumulate warps, which read the
+      // x tiles for the offset term)
+      bar_init(emptyU + 8 * s, kTcDequantWarps + 1 + (HAS_OFF ? 4 : 0));
     }
     for (int s = 0; s < kSA; ++s) {
       bar_init(fullA + 8 * s, kTcDequantWarps / 2);       // one group of dequant warps per step
@@ -517,12 +528,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ---- Warps 16-19: add each K block's accumulator into the running sums
   // (fp32 adds with round to nearest; registers at BN = 32, tensor memory
-  // above), then write y.
+  // above), then write y.  With offsets (uniform weights rewritten as BCQ)
+  // each K block also adds off[G][r] * S_b, where S_b is the sum of the
+  // block's 128 inputs of batch column b, summed in fp32 by every accumulate
+  // warp from the x tile in shared memory (lane l holds the columns l, l + 32,
+  // ...; a row of the 128-byte swizzled tile is one 128-byte line whose
+  // 16-byte pieces are only permuted, so their sum is the row's sum).
   if (warp >= kTcFlushWarp0 && warp < kTcFlushWarp0 + 4) {
     const int wq = warp - kTcFlushWarp0;                     // accumulator lanes 32wq..32wq+31
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t run_tm = lane_base + kRunCol;
     const int row = (rb * 4 + wq) * kTileRows + lane;
+    constexpr int kCols = BN / 32;                           // x columns summed by each lane
     auto store_y = [&](int c0, const uint32_t (&r)[32]) {
       if (row >= m) return;
 #pragma unroll
@@ -536,39 +553,69 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     };
-    bool ok = true;
-    if constexpr (kRunRegs) {
-      uint32_t run[32];
+    // Sums of this K block's inputs for the lane's x columns, and the row's offset.
+    auto offset_terms = [&](uint32_t xtile, int kb, float (&sx)[kCols], float& offr) {
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) run[jj] = 0u;
-      for (int kb = 0; kb < nkb; ++kb) {
-        ok = ok && __all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
-        if (!ok) break;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * kSets * BN;
+      for (int k = 0; k < kCols; ++k) {
+        float acc = 0.f;
 #pragma unroll
-        for (int c0 = 0; c0 < 32; c0 += 16) {
-          uint32_t a[16], b[16];
-          tmem_ld16(acc_tm + (uint32_t)c0, a);
-          tmem_ld16(acc_tm + (uint32_t)(BN + c0), b);
-          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t line = xtile + (uint32_t)h * (kBTile / 2) + (uint32_t)(lane + 32 * k) * 128u;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const float f = __uint_as_float(a[jj]) + __uint_as_float(b[jj]);
-            run[c0 + jj] = kb > 0 ? __float_as_uint(__uint_as_float(run[c0 + jj]) + f) : __float_as_uint(f);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w0, w1, w2, w3;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                         : "r"(line + 16u * c)
+                         : "memory");
+            const uint32_t wv[4] = {w0, w1, w2, w3};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
+              acc += f.x;
+              acc += f.y;
+            }
           }
         }
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        bar_arrive(accFree + 8 * (kb & 1));
+        sx[k] = acc;
       }
-      if (ok) store_y(0, run);
-    } else {
-      for (int kb = 0; kb < nkb; ++kb) {
-        ok = ok && __all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (kb & 1), (uint32_t)((kb >> 1) & 1)));
-        if (!ok) break;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t acc_tm = lane_base + (uint32_t)(kb & 1) * kSets * BN;
+      offr = row < m ? __ldg(offset + (size_t)(kb / kb_per_g) * m + row) : 0.f;
+    };
+    bool ok = true;
+    uint32_t run[kRunRegs ? 32 : 1];
 #pragma unroll
+    for (int jj = 0; jj < (kRunRegs ? 32 : 1); ++jj) run[jj] = 0u;
+    // K block j (processing order): wait for its MMAs, add its accumulators
+    // (and the offset term) into the running sums, free the buffers.
+    auto add_block = [&](int j, const float (&sx)[kCols], float offr) -> bool {
+      if (!__all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (j & 1), (uint32_t)((j >> 1) & 1)))) return false;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t acc_tm = lane_base + (uint32_t)(j & 1) * kSets * BN;
+      if constexpr (kRunRegs) {
+        // 16-column pieces (two round trips per block); 8 with the offset
+        // term, whose values need the registers.
+        constexpr int kPiece = HAS_OFF ? 8 : 16;
+#pragma unroll
+        for (int c0 = 0; c0 < 32; c0 += kPiece) {
+          uint32_t a[kPiece], b[kPiece];
+          if constexpr (kPiece == 16) {
+            tmem_ld16(acc_tm + (uint32_t)c0, a);
+            tmem_ld16(acc_tm + (uint32_t)(BN + c0), b);
+          } else {
+            tmem_ld8(acc_tm + (uint32_t)c0, a);
+            tmem_ld8(acc_tm + (uint32_t)(BN + c0), b);
+          }
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+          for (int jj = 0; jj < kPiece; ++jj) {
+            const float f = __uint_as_float(a[jj]) + __uint_as_float(b[jj]);
+            float r = j > 0 ? __uint_as_float(run[c0 + jj]) + f : f;
+            if constexpr (HAS_OFF) r = fmaf(offr, __shfl_sync(0xffffffffu, sx[0], c0 + jj), r);
+            run[c0 + jj] = __float_as_uint(r);
+          }
+        }
+      } else {
+#pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t a[32], r[32];
           tmem_ld32(acc_tm + (uint32_t)c0, a);
@@ -578,18 +625,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) a[jj] = __float_as_uint(__uint_as_float(a[jj]) + __uint_as_float(r[jj]));
           }
-          if (kb > 0) tmem_ld32(run_tm + (uint32_t)c0, r);
+          if (j > 0) tmem_ld32(run_tm + (uint32_t)c0, r);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj)
-            r[jj] = kb > 0 ? __float_as_uint(__uint_as_float(r[jj]) + __uint_as_float(a[jj])) : a[jj];
+          for (int jj = 0; jj < 32; ++jj) {
+            float v = j > 0 ? __uint_as_float(r[jj]) + __uint_as_float(a[jj]) : __uint_as_float(a[jj]);
+            if constexpr (HAS_OFF) v = fmaf(offr, __shfl_sync(0xffffffffu, sx[c0 / 32], jj), v);
+            r[jj] = __float_as_uint(v);
+          }
           tmem_st32(run_tm + (uint32_t)c0, r);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        bar_arrive(accFree + 8 * (kb & 1));
       }
-      if (ok) {
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      bar_arrive(accFree + 8 * (j & 1));
+      return true;
+    };
+    if constexpr (HAS_OFF) {
+      UnitIter it;
+      it.init(n);
+      int j = 0;
+      for (int u = 0; it.valid() && ok; it.next(), ++u) {
+        const int sl = u % L.nu;
+        const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
+        ok = __all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)));
+        if (!ok) break;
+        const int cnt = it.count();
+        for (int w = 0; w < cnt && ok; ++w, ++j) {
+          float sx[kCols];
+          float offr;
+          offset_terms(slot + (uint32_t)w * kBTile, it.kb(w), sx, offr);
+          ok = add_block(j, sx, offr);
+        }
+        // This warp has read the unit's x tiles.
+        __syncwarp();
+        if (lane == 0) bar_arrive(emptyU + 8 * sl);
+      }
+    } else {
+      const float none[kCols] = {};
+      for (int j = 0; j < nkb && ok; ++j) ok = add_block(j, none, 0.f);
+    }
+    if (ok) {
+      if constexpr (kRunRegs) {
+        store_y(0, run);
+      } else {
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t r[32];
@@ -652,9 +731,9 @@ EncodeTiled encode_fn() {
   return fn;
 }
 
-template <int BN>
-cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const __half* x, void* y, int m, int n,
-                      int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream) {
+template <int BN, bool HAS_OFF>
+cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
+                      int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream) {
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
@@ -678,7 +757,7 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const __half* 
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   static int attr_bytes[64] = {0};
   if (attr_bytes[dev] < (int)smem) {
-    e = cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(tc_gemm_kernel<BN, HAS_OFF>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_bytes[dev] = (int)smem;
   }
@@ -690,18 +769,23 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const __half* 
   }
   const int mt = (m + kTileRows - 1) / kTileRows;
   dim3 grid((unsigned)((m + kTcBM - 1) / kTcBM), (unsigned)((batch + BN - 1) / BN));
-  tc_gemm_kernel<BN><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, y, m, n, batch, q, g, mt, y_f16, status,
-                                                         L);
+  tc_gemm_kernel<BN, HAS_OFF><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, offset, y, m, n, batch, q, g,
+                                                                   mt, y_f16, status, L);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const __half* x, void* y, int m, int n,
-                           int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream) {
-  if (batch <= 32) return launch_bn<32>(packed, alpha, x, y, m, n, batch, q, g, y_f16, status, stream);
-  if (batch <= 64) return launch_bn<64>(packed, alpha, x, y, m, n, batch, q, g, y_f16, status, stream);
-  return launch_bn<128>(packed, alpha, x, y, m, n, batch, q, g, y_f16, status, stream);
+cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
+                           int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream) {
+  if (offset != nullptr) {
+    if (batch <= 32) return launch_bn<32, true>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+    if (batch <= 64) return launch_bn<64, true>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+    return launch_bn<128, true>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+  }
+  if (batch <= 32) return launch_bn<32, false>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+  if (batch <= 64) return launch_bn<64, false>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+  return launch_bn<128, false>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
 }
 
 }  // namespace lutgemm

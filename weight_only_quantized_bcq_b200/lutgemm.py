@@ -32,7 +32,7 @@ _SIGNATURES = {
     "lutgemm_pack_scales": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lutgemm_fit_bcq": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
     "lutgemm_fit_bcq_grid": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
-    "lutgemm_run_tc": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_uint, _vp], _c_int),
+    "lutgemm_run_tc": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_uint, _vp], _c_int),
     "lutgemm_pack_bcq": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "lutgemm_uniform_to_bcq": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp],
                                _c_int),
@@ -208,16 +208,18 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
 
 
 def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
-           y: torch.Tensor = None, y_f16: bool = False, stream=None) -> torch.Tensor:
-    """``run`` on the tensor cores (lutgemm_run_tc), for large batches; pure BCQ,
-    n % 128 == 0 and g % 128 == 0."""
+           y: torch.Tensor = None, y_f16: bool = False, offset: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """``run`` on the tensor cores (lutgemm_run_tc), for large batches;
+    n % 128 == 0 and g % 128 == 0, [q][n/g][m] scales, optional fp32 offsets."""
     _need(packed, torch.uint8, "packed")
     _need(alpha, torch.float16, "alpha")
     _need(x, torch.float16, "x")
+    if offset is not None:
+        _need(offset, torch.float32, "offset")
     batch = x.shape[0] if x.dim() == 2 else 1
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
-    _check(lib().lutgemm_run_tc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(x), _ptr(y),
+    _check(lib().lutgemm_run_tc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
                                 Y_F16 if y_f16 else 0, _stream(stream)),
            "lutgemm_run_tc")
     return y
