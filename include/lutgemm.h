@@ -244,7 +244,7 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *              as lutgemm_run_tc does (same result within the same
  *              tolerance, not the same bits) when that path is the faster
  *              one and takes the operands: batch >= 8, scales in
- *              [q][n/g][m], n % 128 == 0 and g % 128 == 0; the workspace is
+ *              [q][n/g][m], n % 128 == 0 and g % 64 == 0; the workspace is
  *              then left untouched.  Otherwise the flag changes nothing.
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
  *              16-byte aligned, zero-filled before its first use; left
@@ -269,7 +269,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
  * path is for prompt-sized batches, where the method is compute-bound (LUT-GEMM
  * card, Summary and Key points: generation is memory-bound, large batches are
  * not).
- *   m, n, batch, q, g  as lutgemm_run, and n % 128 == 0, g % 128 == 0
+ *   m, n, batch, q, g  as lutgemm_run, and n % 128 == 0, g % 64 == 0
  *   packed, alpha, offset, x, y  as lutgemm_run ([q][n/g][m] scales; offset
  *              NULL for pure BCQ, else fp32 [n/g][m], 4-byte aligned: each
  *              128-input block adds offset * (the block's input sum) in fp32)

@@ -137,7 +137,7 @@ def test_run_tc_validation(L):
         return lib.lutgemm_run_tc(*a)
     assert call(packed=None) == L.ERR_NULL
     assert call(y=None) == L.ERR_NULL
-    assert call(g=64) == L.ERR_SHAPE             # needs g % 128 == 0
+    assert call(g=32) == L.ERR_SHAPE             # needs g % 64 == 0
     assert call(n=1032, g=8) == L.ERR_SHAPE      # needs n % 128 == 0
     assert call(batch=0) == L.ERR_SHAPE
     assert call(flags=2) == L.ERR_VALUE

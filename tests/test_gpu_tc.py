@@ -44,6 +44,11 @@ CASES = [
     (3, 256, 1280, 128, 40),
     (2, 248, 1536, 256, 64),
     (8, 136, 2048, 128, 129),
+    # g = 64: two scale groups per 128-input block (the LLaMA configs)
+    (2, 256, 2048, 64, 8),
+    (2, 300, 1536, 64, 40),
+    (3, 128, 1024, 64, 130),
+    (2, 200, 1920, 192, 33),
 ]
 
 
@@ -117,16 +122,16 @@ def test_tc_full_size_bench_configuration_sampled(L, name, m, n):
 
 
 def test_tc_rejects_unsupported_shapes(L):
-    signs, alpha, x = _problem(953, 3, 64, 1024, 64, 4)
+    signs, alpha, x = _problem(953, 3, 64, 1024, 32, 4)
     packed = L.pack_bcq(signs.to(DEV))
-    with pytest.raises(L.LutgemmError) as e:
-        L.run_tc(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 64)
+    with pytest.raises(L.LutgemmError) as e:            # g % 64 != 0
+        L.run_tc(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 32)
     assert e.value.status == L.ERR_SHAPE
 
 
 def test_run_with_tensor_cores_allowed_takes_the_faster_path(L):
-    """lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: from batch 8 (pure BCQ,
-    g % 128 == 0, [q][n/g][m] scales) the result is bit for bit that of
+    """lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: from batch 8 (g % 64 == 0,
+    [q][n/g][m] scales) the result is bit for bit that of
     lutgemm_run_tc; below batch 8 that of the lookup path."""
     q, m, n, g = 3, 384, 2048, 128
     for batch, want_tc in ((8, True), (40, True), (4, False)):
@@ -168,7 +173,7 @@ def test_noalloc_with_tensor_cores_allowed_needs_no_scratch(L):
 
 
 @pytest.mark.parametrize("q,m,n,g,batch", [(4, 256, 2048, 128, 40), (3, 300, 2560, 256, 100), (2, 128, 1024, 128, 7),
-                                           (4, 136, 1280, 128, 129)])
+                                           (4, 136, 1280, 128, 129), (4, 256, 2048, 64, 20), (3, 96, 1536, 192, 64)])
 def test_tc_uniform_weights_with_offsets(L, q, m, n, g, batch):
     """Uniform q-bit weights rewritten as BCQ plus group offsets (the lookup
     path's config of converted weights) on the tensor cores, against the
@@ -189,4 +194,25 @@ def test_tc_uniform_weights_with_offsets(L, q, m, n, g, batch):
     y_lut = L.run(packed, alpha, x.to(DEV), m, n, q, g, offset=offset)
     torch.cuda.synchronize()
     ok, st = compare(y_lut.cpu().numpy(), y_ref, alpha.cpu().numpy(), x.numpy(), n)
+    assert ok, st
+
+
+
+@pytest.mark.parametrize("name,m,n", [("up", 28672, 8192), ("down", 8192, 28672)])
+def test_tc_full_size_llama70b_sampled(L, name, m, n):
+    """LLaMA-70B linears, q = 2, g = 64, batch 8 (the config's largest batch),
+    x with 0.1 % outlier columns scaled x20: sampled rows against the oracle."""
+    q, g, batch = 2, 64, 8
+    w = S.WORKLOADS["llama70b"]
+    gen = S.generator(990 + m % 11)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n))
+    alpha = S.draw_alpha(gen, q, m, n, g, w.alpha_sigma)
+    x = S.draw_x(gen, batch, n, outlier_frac=w.outlier_frac)
+    y = L.run_tc(packed.to(DEV), alpha.to(DEV), x.to(DEV), m, n, q, g)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(991).choice(m, 24, replace=False))
+    s_rows = O.unpack_rows(packed.numpy(), q, m, n, rows)
+    a_rows = alpha.numpy()[:, :, rows]
+    y_ref = O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g)
+    ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_rows, x.numpy(), n)
     assert ok, st

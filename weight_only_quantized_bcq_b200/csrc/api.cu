@@ -139,7 +139,7 @@ size_t lutgemm_scales_bytes(int q, int m, int n, int g) {
 int lutgemm_run_tc(int m, int n, int batch, int q, int g, const uint8_t* packed, const uint16_t* alpha,
                    const float* offset, const uint16_t* x, void* y, unsigned flags, void* stream) {
   if (!packed || !alpha || !x || !y) return LUTGEMM_ERR_NULL;
-  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1 || g % 128 != 0 || n % 128 != 0)
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1 || g % 64 != 0 || n % 128 != 0)
     return LUTGEMM_ERR_SHAPE;
   if ((flags & ~LUTGEMM_Y_F16) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
@@ -231,7 +231,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
   // From batch 8 the tensor-core path is the faster one (FC1-sized layers:
   // 275 against 300 us at batch 8, 320 against 2360 us at 64).
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 128 == 0) {
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0) {
     const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
                                          reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
                                          nullptr, reinterpret_cast<cudaStream_t>(stream));

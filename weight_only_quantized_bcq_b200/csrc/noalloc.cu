@@ -127,7 +127,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
   // The tensor-core path needs no scratch at all (same rule as lutgemm_run).
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 128 == 0) {
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0) {
     const cudaError_t e = launch_tc_gemm(packed, alpha_ptr_h(alpha), offset, reinterpret_cast<const __half*>(x), y,
                                          m, n, batch, q, g, y_f16 ? 1 : 0, nullptr,
                                          reinterpret_cast<cudaStream_t>(stream));

@@ -6,8 +6,8 @@
 // planes with group-wise scales).  Each plane is fed to the tensor cores as
 // its exact fp16 values +-alpha_i (an fp16 times a sign is exact), so no
 // dequantised weight is ever rounded; the planes accumulate into one fp32
-// tensor-memory accumulator.  Needs g % 128 == 0 (one scale per plane and
-// 128-input piece); group offsets (uniform weights rewritten as BCQ) are
+// tensor-memory accumulator.  Needs g % 64 == 0: a 64-input half of a
+// 128-input K block then lies in one scale group; group offsets (uniform weights rewritten as BCQ) are
 // added per K block in fp32 by the accumulate warps.
 //
 // CTA tile: 128 rows (MMA M) x BN batch columns (MMA N) over K blocks of 128
@@ -203,7 +203,7 @@ struct UnitIter {
 struct TcLayout {
   uint32_t slot_bytes;     // one unit: x tiles, chunk groups, scale rows (multiple of 1024)
   uint32_t bits_off;       // 8 chunk groups of q * 512 bytes: (row tile, half) = 2 wq + h
-  uint32_t alpha_off;      // 2 x q scale rows of 128 fp16: (which, plane)
+  uint32_t alpha_off;      // 2 x q x 2 scale rows of 128 fp16: (which, plane, K half)
   int nu;                  // ring depth in units
   int alpha_bulk;          // scale rows by bulk copy (16-byte aligned rows) or by lane loads
 };
@@ -253,7 +253,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int b0 = blockIdx.y * BN;                            // first batch column
   const int nkb = n / kTcBK;
   const int ng = n / g;
-  const int kb_per_g = g / kTcBK;
+  // Scale group of K half h of K block kb (one per block when g % 128 == 0).
+  const int halves_per_g = g / 64;
+  const int apb = g % kTcBK == 0 ? 1 : 2;                   // distinct scale rows per K block and plane
 
   if (tid == 0) {
     for (int s = 0; s < L.nu; ++s) {
@@ -336,14 +338,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int cnt = it.count();
       for (int w = 0; w < cnt && go; ++w) {
         const uint32_t bsrc = slot + bits_lane + (uint32_t)((half_sel ^ w) * q * 512);
-        const uint32_t asrc = slot + alpha_lane + (uint32_t)(w * q * 256);
+        const uint32_t asrc = slot + alpha_lane + (uint32_t)((w * q * 2 + (apb == 2 ? hsel : 0)) * 256);
         for (int i = 0; i < q; ++i, ++ai) {
           if ((ai & 1) != grp) continue;
           const int st = ai % kSA;
           uint32_t b0w, b1w, ah;
           asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0w), "=r"(b1w) : "r"(bsrc + (uint32_t)(i * 512))
                        : "memory");
-          asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc + (uint32_t)(i * 256)) : "memory");
+          asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc + (uint32_t)(i * 512)) : "memory");
           const uint32_t w0 = __byte_perm(b0w, b1w, sel0);   // runs 0..3 of the half, in order
           const uint32_t w1 = __byte_perm(b0w, b1w, sel1);   // runs 4..7
           // Element pair (2e, 2e+1) of a run byte b: the product b * (2^(15-2e)
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t bytes = (uint32_t)cnt * kBTile;
         for (int wq = 0; wq < 4; ++wq)
           if (rb * 4 + wq < mt) bytes += 2u * (uint32_t)q * 512u;
-        if (L.alpha_bulk) bytes += (uint32_t)(cnt * q * rows_here * 2);
+        if (L.alpha_bulk) bytes += (uint32_t)(cnt * q * apb * rows_here * 2);
         asm volatile(
             "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
             " @e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n}" ::"r"(bar),
@@ -431,36 +433,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         if (L.alpha_bulk) {
-          for (int w = 0; w < cnt; ++w) {
-            const int G = it.kb(w) / kb_per_g;
-            for (int i = 0; i < q; ++i)
-              asm volatile(
-                  "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-                  " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
-                      slot + L.alpha_off + (uint32_t)((w * q + i) * 256)),
-                  "l"(alpha + ((size_t)i * ng + G) * m + (size_t)rb * kTcBM), "r"(rows_here * 2), "r"(bar)
-                  : "memory");
-          }
+          for (int w = 0; w < cnt; ++w)
+            for (int h = 0; h < apb; ++h) {
+              const int G = (2 * it.kb(w) + h) / halves_per_g;
+              for (int i = 0; i < q; ++i)
+                asm volatile(
+                    "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+                    " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
+                        slot + L.alpha_off + (uint32_t)(((w * q + i) * 2 + h) * 256)),
+                    "l"(alpha + ((size_t)i * ng + G) * m + (size_t)rb * kTcBM), "r"(rows_here * 2), "r"(bar)
+                    : "memory");
+            }
         }
       }
       if (!L.alpha_bulk) {
         // Scale rows by plain loads: lane l covers rows 4l..4l+3 of the tile.
-        for (int w = 0; w < cnt; ++w) {
-          const int G = it.kb(w) / kb_per_g;
-          for (int i = 0; i < q; ++i) {
-            const unsigned short* src = reinterpret_cast<const unsigned short*>(alpha) + ((size_t)i * ng + G) * m;
-            uint32_t v[4];
+        for (int w = 0; w < cnt; ++w)
+          for (int h = 0; h < apb; ++h) {
+            const int G = (2 * it.kb(w) + h) / halves_per_g;
+            for (int i = 0; i < q; ++i) {
+              const unsigned short* src = reinterpret_cast<const unsigned short*>(alpha) + ((size_t)i * ng + G) * m;
+              uint32_t v[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int r = rb * kTcBM + 4 * lane + k;
-              v[k] = r < m ? (uint32_t)__ldg(src + r) : 0u;
+              for (int k = 0; k < 4; ++k) {
+                const int r = rb * kTcBM + 4 * lane + k;
+                v[k] = r < m ? (uint32_t)__ldg(src + r) : 0u;
+              }
+              asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(
+                               slot + L.alpha_off + (uint32_t)(((w * q + i) * 2 + h) * 256 + lane * 8)),
+                           "r"(v[0] | (v[1] << 16)), "r"(v[2] | (v[3] << 16))
+                           : "memory");
             }
-            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(slot + L.alpha_off + (uint32_t)((w * q + i) * 256 +
-                                                                                                  lane * 8)),
-                         "r"(v[0] | (v[1] << 16)), "r"(v[2] | (v[3] << 16))
-                         : "memory");
           }
-        }
       }
       __syncwarp();
       if (lane == 0) bar_arrive(bar);
@@ -553,13 +557,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     };
-    // Sums of this K block's inputs for the lane's x columns, and the row's offset.
-    auto offset_terms = [&](uint32_t xtile, int kb, float (&sx)[kCols], float& offr) {
+    // Sums of each 64-input half of this K block for the lane's x columns,
+    // and the row's offsets of the halves' groups.
+    auto offset_terms = [&](uint32_t xtile, int kb, float (&sx)[2][kCols], float (&offr)[2]) {
 #pragma unroll
       for (int k = 0; k < kCols; ++k) {
-        float acc = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          float acc = 0.f;
           const uint32_t line = xtile + (uint32_t)h * (kBTile / 2) + (uint32_t)(lane + 32 * k) * 128u;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -576,10 +581,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               acc += f.y;
             }
           }
+          sx[h][k] = acc;
         }
-        sx[k] = acc;
       }
-      offr = row < m ? __ldg(offset + (size_t)(kb / kb_per_g) * m + row) : 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        offr[h] = row < m ? __ldg(offset + (size_t)((2 * kb + h) / halves_per_g) * m + row) : 0.f;
     };
     bool ok = true;
     uint32_t run[kRunRegs ? 32 : 1];
@@ -587,7 +594,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int jj = 0; jj < (kRunRegs ? 32 : 1); ++jj) run[jj] = 0u;
     // K block j (processing order): wait for its MMAs, add its accumulators
     // (and the offset term) into the running sums, free the buffers.
-    auto add_block = [&](int j, const float (&sx)[kCols], float offr) -> bool {
+    auto add_block = [&](int j, const float (&sx)[2][kCols], const float (&offr)[2]) -> bool {
       if (!__all_sync(0xffffffffu, bar_wait_sleep(accFull + 8 * (j & 1), (uint32_t)((j >> 1) & 1)))) return false;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t acc_tm = lane_base + (uint32_t)(j & 1) * kSets * BN;
@@ -610,7 +617,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int jj = 0; jj < kPiece; ++jj) {
             const float f = __uint_as_float(a[jj]) + __uint_as_float(b[jj]);
             float r = j > 0 ? __uint_as_float(run[c0 + jj]) + f : f;
-            if constexpr (HAS_OFF) r = fmaf(offr, __shfl_sync(0xffffffffu, sx[0], c0 + jj), r);
+            if constexpr (HAS_OFF) {
+              r = fmaf(offr[0], __shfl_sync(0xffffffffu, sx[0][0], c0 + jj), r);
+              r = fmaf(offr[1], __shfl_sync(0xffffffffu, sx[1][0], c0 + jj), r);
+            }
             run[c0 + jj] = __float_as_uint(r);
           }
         }
@@ -630,7 +640,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
             float v = j > 0 ? __uint_as_float(r[jj]) + __uint_as_float(a[jj]) : __uint_as_float(a[jj]);
-            if constexpr (HAS_OFF) v = fmaf(offr, __shfl_sync(0xffffffffu, sx[c0 / 32], jj), v);
+            if constexpr (HAS_OFF) {
+              v = fmaf(offr[0], __shfl_sync(0xffffffffu, sx[0][c0 / 32], jj), v);
+              v = fmaf(offr[1], __shfl_sync(0xffffffffu, sx[1][c0 / 32], jj), v);
+            }
             r[jj] = __float_as_uint(v);
           }
           tmem_st32(run_tm + (uint32_t)c0, r);
@@ -652,8 +665,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
         const int cnt = it.count();
         for (int w = 0; w < cnt && ok; ++w, ++j) {
-          float sx[kCols];
-          float offr;
+          float sx[2][kCols];
+          float offr[2];
           offset_terms(slot + (uint32_t)w * kBTile, it.kb(w), sx, offr);
           ok = add_block(j, sx, offr);
         }
@@ -662,8 +675,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) bar_arrive(emptyU + 8 * sl);
       }
     } else {
-      const float none[kCols] = {};
-      for (int j = 0; j < nkb && ok; ++j) ok = add_block(j, none, 0.f);
+      const float none[2][kCols] = {};
+      const float zero2[2] = {0.f, 0.f};
+      for (int j = 0; j < nkb && ok; ++j) ok = add_block(j, none, zero2);
     }
     if (ok) {
       if constexpr (kRunRegs) {
@@ -705,7 +719,7 @@ TcLayout tc_layout(int q, bool alpha_bulk) {
   const uint32_t xt = 2u * BN * kTcBK * 2;
   L.bits_off = xt;
   L.alpha_off = xt + 8u * (uint32_t)q * 512u;
-  L.slot_bytes = (L.alpha_off + 2u * (uint32_t)q * 256u + 1023u) & ~1023u;
+  L.slot_bytes = (L.alpha_off + 4u * (uint32_t)q * 256u + 1023u) & ~1023u;
   const uint32_t budget = 227u * 1024u - 1024u - 512u;
   const int fit = (int)(budget / L.slot_bytes);
   L.nu = fit < 4 ? fit : 4;

@@ -210,7 +210,7 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
 def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
            y: torch.Tensor = None, y_f16: bool = False, offset: torch.Tensor = None, stream=None) -> torch.Tensor:
     """``run`` on the tensor cores (lutgemm_run_tc), for large batches;
-    n % 128 == 0 and g % 128 == 0, [q][n/g][m] scales, optional fp32 offsets."""
+    n % 128 == 0 and g % 64 == 0, [q][n/g][m] scales, optional fp32 offsets."""
     _need(packed, torch.uint8, "packed")
     _need(alpha, torch.float16, "alpha")
     _need(x, torch.float16, "x")
