@@ -870,13 +870,26 @@ def run_sweep(args):
             # wavefront (32 reads) per clock per SM at the measured clock.
             lookups = q * m * n // 8 * b
             smem_floor = lookups / 32 / sm / 1.965e3
-            print(json.dumps({"config": name, "m": m, "n": n, "q": q, "g": g, "batch": b,
-                              "us_isolated": round(iso, 1), "us_back_to_back": round(b2b, 1),
-                              "gbs_back_to_back": round(nbytes / (b2b * 1e-6) / 1e9, 1),
-                              "hbm_floor_us": round(nbytes / (peak * 1e3), 1),
-                              "smem_floor_us": round(smem_floor, 1),
-                              "frac_of_binding_floor": round(max(nbytes / (peak * 1e3), smem_floor) / b2b, 3)}),
-                  flush=True)
+            line = {"config": name, "m": m, "n": n, "q": q, "g": g, "batch": b,
+                    "us_isolated": round(iso, 1), "us_back_to_back": round(b2b, 1),
+                    "gbs_back_to_back": round(nbytes / (b2b * 1e-6) / 1e9, 1),
+                    "hbm_floor_us": round(nbytes / (peak * 1e3), 1),
+                    "smem_floor_us": round(smem_floor, 1),
+                    "frac_of_binding_floor": round(max(nbytes / (peak * 1e3), smem_floor) / b2b, 3)}
+            if b >= 8 and n % 128 == 0 and g % 64 == 0:
+                # The same product on the tensor cores (lutgemm_run_tc), back to back.
+                def run_tc(i):
+                    lutgemm.run_tc(bufs[i % reps], alpha, x, m, n, q, g, y=y, stream=stream)
+                for i in range(3):
+                    run_tc(i)
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                t0.record(stream)
+                for i in range(30):
+                    run_tc(i)
+                t1.record(stream)
+                torch.cuda.synchronize()
+                line["us_tensor_cores_back_to_back"] = round(t0.elapsed_time(t1) * 1e3 / 30, 1)
+            print(json.dumps(line), flush=True)
 
 
 def main():

@@ -242,10 +242,12 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *              LUTGEMM_SCALES_PACKED with g % 128 != 0, give ERR_VALUE.
  *              With LUTGEMM_ALLOW_TENSOR_CORES the call computes the product
  *              as lutgemm_run_tc does (same result within the same
- *              tolerance, not the same bits) when that path is the faster
- *              one and takes the operands: batch >= 8, scales in
- *              [q][n/g][m], n % 128 == 0 and g % 64 == 0; the workspace is
- *              then left untouched.  Otherwise the flag changes nothing.
+ *              tolerance, not the same bits) when that path takes the
+ *              operands (batch >= 8, scales in [q][n/g][m], n % 128 == 0,
+ *              g % 64 == 0) and a cost model of both paths on B200 expects
+ *              it to be faster (tall matrices: many 128-row blocks to spread
+ *              over the SMs, or large batches); the workspace is then left
+ *              untouched.  Otherwise the flag changes nothing.
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
  *              16-byte aligned, zero-filled before its first use; left
  *              zero-filled by every successful call.  Calls that share a

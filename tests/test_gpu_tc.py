@@ -130,28 +130,42 @@ def test_tc_rejects_unsupported_shapes(L):
 
 
 def test_run_with_tensor_cores_allowed_takes_the_faster_path(L):
-    """lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: from batch 8 (g % 64 == 0,
-    [q][n/g][m] scales) the result is bit for bit that of
-    lutgemm_run_tc; below batch 8 that of the lookup path."""
-    q, m, n, g = 3, 384, 2048, 128
-    for batch, want_tc in ((8, True), (40, True), (4, False)):
-        signs, alpha, x = _problem(960 + batch, q, m, n, g, batch)
-        packed, a_d, x_d = L.pack_bcq(signs.to(DEV)), alpha.to(DEV), x.to(DEV)
-        y = L.run(packed, a_d, x_d, m, n, q, g, allow_tensor_cores=True)
-        ref = L.run_tc(packed, a_d, x_d, m, n, q, g) if want_tc else L.run(packed, a_d, x_d, m, n, q, g)
-        torch.cuda.synchronize()
-        assert torch.equal(y, ref), batch
-        ok, st = compare(y.cpu().numpy(), O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), g),
-                         alpha.numpy(), x.numpy(), n)
-        assert ok, st
-    # With an offset the tensor-core path takes it too.
-    signs, alpha, x = _problem(970, q, m, n, g, 16)
-    off = torch.randn((n // g, m), generator=S.generator(971)) * 0.01
-    packed, a_d, x_d, o_d = L.pack_bcq(signs.to(DEV)), alpha.to(DEV), x.to(DEV), off.to(DEV)
-    y = L.run(packed, a_d, x_d, m, n, q, g, offset=o_d, allow_tensor_cores=True)
-    ref = L.run_tc(packed, a_d, x_d, m, n, q, g, offset=o_d)
+    """lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES runs the tensor-core kernel
+    (bit for bit lutgemm_run_tc's result) where its cost model expects it to
+    win -- a tall matrix, many 128-row blocks per SM -- and the lookup kernel
+    otherwise: a short matrix even at batch 40, any matrix below batch 8."""
+    q, g = 3, 128
+    # Tall: 49152 rows (384 row blocks), batch 40 and 16 (with offsets).
+    m, n = 49152, 1024
+    gen = S.generator(960)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n)).to(DEV)
+    a_d = S.draw_alpha(gen, q, m, n, g, 0.02).to(DEV)
+    x_d = S.draw_x(gen, 40, n).to(DEV)
+    y = L.run(packed, a_d, x_d, m, n, q, g, allow_tensor_cores=True)
+    ref = L.run_tc(packed, a_d, x_d, m, n, q, g)
     torch.cuda.synchronize()
     assert torch.equal(y, ref)
+    off = (torch.randn((n // g, m), generator=S.generator(961)) * 0.01).to(DEV)
+    y = L.run(packed, a_d, x_d[:16], m, n, q, g, offset=off, allow_tensor_cores=True)
+    ref = L.run_tc(packed, a_d, x_d[:16], m, n, q, g, offset=off)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    # Below batch 8: the lookup kernel.
+    y = L.run(packed, a_d, x_d[:4], m, n, q, g, allow_tensor_cores=True)
+    ref = L.run(packed, a_d, x_d[:4], m, n, q, g)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    # Short: 384 rows (3 row blocks) at batch 40 -- the lookup kernel.
+    m, n = 384, 2048
+    signs, alpha, x = _problem(962, q, m, n, g, 40)
+    packed, a_d, x_d = L.pack_bcq(signs.to(DEV)), alpha.to(DEV), x.to(DEV)
+    y = L.run(packed, a_d, x_d, m, n, q, g, allow_tensor_cores=True)
+    ref = L.run(packed, a_d, x_d, m, n, q, g)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    ok, st = compare(y.cpu().numpy(), O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), g),
+                     alpha.numpy(), x.numpy(), n)
+    assert ok, st
 
 
 def test_noalloc_with_tensor_cores_allowed_needs_no_scratch(L):

@@ -1,6 +1,7 @@
 // C ABI of the LUT-GEMM library: argument validation, workspace sizing and
 // kernel launches on the caller's stream.  Declarations and the contract of
 // every call are in include/lutgemm.h.
+#include <cmath>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -18,9 +19,40 @@ cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, 
                                cudaStream_t stream);
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
                            int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
+bool tc_preferred(int m, int n, int batch, int q);
 cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
                            float* offset,
                            float* err, cudaStream_t stream);
+
+// Whether the tensor-core path is expected to beat the lookup kernel, from a
+// cost model fitted to B200 measurements of both (OPT-175B and LLaMA-70B
+// linears, batch 8-32, isolated back-to-back launches):
+//   tensor cores: waves x K blocks x c(BN) + 15k cycles, with waves =
+//     ceil(ceil(m/128) * ceil(batch/BN) / SMs) and c = 1900 / 2170 / 2700
+//     cycles per 128-input block at BN = 32 / 64 / 128 (nearly independent of
+//     q: the per-block hand-offs dominate);
+//   lookups: q m n batch / 8 table reads at 0.62 of one 32-read wavefront per
+//     clock per SM, + 15k cycles.
+// It picks the faster path for all 12 measured (shape, batch >= 8) cases.
+bool tc_preferred(int m, int n, int batch, int q) {
+  static int sms_cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (sms_cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return false;
+    sms_cache[dev] = v;
+  }
+  const double sms = sms_cache[dev];
+  const int bn = batch <= 32 ? 32 : (batch <= 64 ? 64 : 128);
+  const double block_cycles = bn == 32 ? 1900.0 : (bn == 64 ? 2170.0 : 2700.0);
+  const double ctas = (double)((m + 127) / 128) * (double)((batch + bn - 1) / bn);
+  const double waves = std::ceil(ctas / sms);
+  const double t_tc = waves * ((double)n / 128.0) * block_cycles + 15000.0;
+  const double t_lut = (double)q * m * n * batch / 8.0 / (sms * 32.0) / 0.62 + 15000.0;
+  return t_tc < t_lut;
+}
+
 }  // namespace lutgemm
 
 namespace {
@@ -229,9 +261,10 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
     return LUTGEMM_ERR_ALIGN;
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
-  // From batch 8 the tensor-core path is the faster one (FC1-sized layers:
-  // 275 against 300 us at batch 8, 320 against 2360 us at 64).
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0) {
+  // The tensor-core path, where it takes the operands and its cost model
+  // says it is the faster one (never below batch 8).
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0 &&
+      tc_preferred(m, n, batch, q)) {
     const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
                                          reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
                                          nullptr, reinterpret_cast<cudaStream_t>(stream));

@@ -28,6 +28,7 @@
 namespace lutgemm {
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
                            int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
+bool tc_preferred(int m, int n, int batch, int q);
 }  // namespace lutgemm
 
 namespace {
@@ -127,7 +128,8 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
   // The tensor-core path needs no scratch at all (same rule as lutgemm_run).
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0) {
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0 &&
+      tc_preferred(m, n, batch, q)) {
     const cudaError_t e = launch_tc_gemm(packed, alpha_ptr_h(alpha), offset, reinterpret_cast<const __half*>(x), y,
                                          m, n, batch, q, g, y_f16 ? 1 : 0, nullptr,
                                          reinterpret_cast<cudaStream_t>(stream));
