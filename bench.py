@@ -628,8 +628,8 @@ def cpu_fit_baseline(q: int, g: int, iters: int, n: int, rows: int, grid: bool =
 # flops; the tensor cores execute q of them per weight (one per plane), which
 # is the work this path's roofline counts.
 # ---------------------------------------------------------------------------
-TC_METRIC = ("BCQ tensor-core path (lutgemm_run_tc): plane TFLOP/s (2*q*m*n*batch per matmul) "
-             "over the OPT-175B layer's linears at prompt-phase batch")
+TC_METRIC = ("BCQ tensor-core path (lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES): plane TFLOP/s "
+             "(2*q*m*n*batch per matmul) over the OPT-175B layer's linears at prompt-phase batch")
 TC_SOURCES = ("tc_gemm.cu",)
 
 
@@ -694,25 +694,36 @@ def run_tc(args):
                      "alpha": S.draw_alpha(gen, q, sh.m, sh.n, g, w.alpha_sigma).to(device),
                      "x_host": x_host, "x": io["x"][xo: xo + batch * sh.n].view(batch, sh.n),
                      "y": io["y"][yo: yo + batch * sh.m].view(batch, sh.m),
-                     "y_host": io["y_host"][yo: yo + batch * sh.m].view(batch, sh.m)})
+                     "y_host": io["y_host"][yo: yo + batch * sh.m].view(batch, sh.m),
+                     "ws": None if args.tc_direct else lutgemm.new_workspace(sh.m, sh.n, batch, q, g, device=device)})
         xo += batch * sh.n
         yo += batch * sh.m
     io["x"].copy_(io["x_host"])
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)
 
+    def one(mt):
+        # The library's tensor-core path as a caller gets it: lutgemm_run with
+        # the tensor cores allowed (its cost model picks K splits for short
+        # matrices); --tc-direct calls lutgemm_run_tc (one split) instead.
+        if args.tc_direct:
+            lutgemm.run_tc(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], stream=stream)
+        else:
+            lutgemm.run(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], workspace=mt["ws"],
+                        allow_tensor_cores=True, stream=stream)
+
     def step(events=None):
         for i, mt in enumerate(mats):
             if events is not None:
                 events[i][0].record(stream)
-            lutgemm.run_tc(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], stream=stream)
+            one(mt)
             if events is not None:
                 events[i][1].record(stream)
 
     def e2e_step():
         io["x"].copy_(io["x_host"], non_blocking=True)
         for mt in mats:
-            lutgemm.run_tc(mt["packed"], mt["alpha"], mt["x"], mt["m"], mt["n"], q, g, y=mt["y"], stream=stream)
+            one(mt)
         io["y_host"].copy_(io["y"], non_blocking=True)
 
     def barrier():
@@ -791,15 +802,41 @@ def run_tc(args):
                     "h2d_bytes_per_step": io["x_host"].numel() * 2,
                     "d2h_bytes_per_step": io["y_host"].numel() * 4,
                     "copies_per_step": "one H2D of all x, one D2H of all y (pinned host buffers)"},
-            "gpu_launches": len(mats) * args.steps,
+            "gpu_launches": args.steps * sum(1 + (0 if args.tc_direct else int(tc_splits(mt["m"], mt["n"], batch, q) > 1))
+                                             for mt in mats),
+            "gpu_launches_note": "tc_gemm_kernel per matmul, plus the split-K reduce where the library splits K",
             "clocks": clk,
         }
+        out["config"]["call"] = "lutgemm_run_tc" if args.tc_direct else "lutgemm_run + LUTGEMM_ALLOW_TENSOR_CORES"
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_tc_baseline(q, batch, args.tc_cpu_rows)
         print(json.dumps(out), flush=True)
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
+
+
+def tc_splits(m: int, n: int, batch: int, q: int, sms: int = 148) -> int:
+    """The K-split count lutgemm_run's tensor-core cost model picks (1 when it
+    does not split; the same arithmetic as the library), for launch counting."""
+    import math
+    bn = 32 if batch <= 32 else (64 if batch <= 64 else 128)
+    c = {32: 1900.0, 64: 2170.0, 128: 2700.0}[bn]
+    ctas = math.ceil(m / 128) * math.ceil(batch / bn)
+    s_all, nkb, mt32 = math.ceil(n / 1024), n // 128, math.ceil(m / 32) * 32
+    best, best_s, unsplit = None, 1, None
+    for sp in range(1, min(s_all, 8) + 1):
+        spz = math.ceil(s_all / sp)
+        if math.ceil(s_all / spz) != sp:
+            continue
+        t = math.ceil(ctas * sp / sms) * (min(8 * spz, nkb) * c + 12000.0) + 15000.0
+        if sp > 1:
+            t += 4000.0 + (batch * mt32 * sp * 4.0 + batch * m * 4.0) / 6.4e12 * 1.965e9
+        if sp == 1:
+            unsplit = t
+        if best is None or t < best:
+            best, best_s = t, sp
+    return 1 if best_s > 1 and best > 0.95 * unsplit else best_s
 
 
 def cpu_tc_baseline(q: int, batch: int, rows: int):
@@ -889,6 +926,19 @@ def run_sweep(args):
                 t1.record(stream)
                 torch.cuda.synchronize()
                 line["us_tensor_cores_back_to_back"] = round(t0.elapsed_time(t1) * 1e3 / 30, 1)
+                # lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: the library's own choice
+                # (lookups, or tensor cores with K splits and the reduce).
+                def run_auto(i):
+                    lutgemm.run(bufs[i % reps], alpha, x, m, n, q, g, y=y, workspace=ws, allow_tensor_cores=True,
+                                stream=stream)
+                for i in range(3):
+                    run_auto(i)
+                t0.record(stream)
+                for i in range(30):
+                    run_auto(i)
+                t1.record(stream)
+                torch.cuda.synchronize()
+                line["us_auto_back_to_back"] = round(t0.elapsed_time(t1) * 1e3 / 30, 1)
             print(json.dumps(line), flush=True)
 
 
@@ -914,6 +964,8 @@ def main():
                          "sweep: every parity config shape and batch, one line each; "
                          "tc: the layer's linears at a large batch on the tensor-core path")
     ap.add_argument("--tc-batch", type=int, default=256)
+    ap.add_argument("--tc-direct", action="store_true",
+                    help="tc workload: call lutgemm_run_tc (one K split) instead of lutgemm_run with the tensor cores allowed")
     ap.add_argument("--tc-cpu-rows", type=int, default=128, help="rows per linear in the tc CPU baseline sample")
     ap.add_argument("--fit-m", type=int, default=49152)
     ap.add_argument("--fit-n", type=int, default=12288)

@@ -230,3 +230,30 @@ def test_tc_full_size_llama70b_sampled(L, name, m, n):
     y_ref = O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g)
     ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_rows, x.numpy(), n)
     assert ok, st
+
+
+@pytest.mark.parametrize("name,m,n,batch", [("fc2", 12288, 49152, 32), ("out", 12288, 12288, 16)])
+def test_run_with_tensor_cores_split_k_matches_oracle(L, name, m, n, batch):
+    """Short matrices: the cost model splits K over CTAs (fp32 partials in the
+    workspace, the split-K reduce adds them): sampled rows against the oracle,
+    and within the same bound as the single-split tensor-core result."""
+    q, g = 3, 128
+    gen = S.generator(995 + m % 13 + batch)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n))
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.02)
+    x = S.draw_x(gen, batch, n)
+    p_d, a_d, x_d = packed.to(DEV), alpha.to(DEV), x.to(DEV)
+    y = L.run(p_d, a_d, x_d, m, n, q, g, allow_tensor_cores=True)
+    y_lut = L.run(p_d, a_d, x_d, m, n, q, g)
+    torch.cuda.synchronize()
+    assert not torch.equal(y, y_lut)          # not the lookup path's bits: the tensor cores ran
+    rows = np.sort(np.random.default_rng(996).choice(m, 32, replace=False))
+    s_rows = O.unpack_rows(packed.numpy(), q, m, n, rows)
+    a_rows = alpha.numpy()[:, :, rows]
+    y_ref = O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g)
+    ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_rows, x.numpy(), n)
+    assert ok, st
+    # Deterministic: the partials are added in split order.
+    y2 = L.run(p_d, a_d, x_d, m, n, q, g, allow_tensor_cores=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)

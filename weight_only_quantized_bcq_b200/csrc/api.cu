@@ -18,39 +18,65 @@ cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, con
 cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
                                cudaStream_t stream);
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
-                           int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
-bool tc_preferred(int m, int n, int batch, int q);
+                           float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
+                           cudaStream_t stream);
 cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iters, int8_t* signs, __half* alpha,
                            float* offset,
                            float* err, cudaStream_t stream);
 
-// Whether the tensor-core path is expected to beat the lookup kernel, from a
-// cost model fitted to B200 measurements of both (OPT-175B and LLaMA-70B
-// linears, batch 8-32, isolated back-to-back launches):
-//   tensor cores: waves x K blocks x c(BN) + 15k cycles, with waves =
-//     ceil(ceil(m/128) * ceil(batch/BN) / SMs) and c = 1900 / 2170 / 2700
-//     cycles per 128-input block at BN = 32 / 64 / 128 (nearly independent of
-//     q: the per-block hand-offs dominate);
+// The tensor-core plan: how many K splits to run it with, or 0 when the
+// lookup kernel is expected to be faster.  A cost model fitted to B200
+// measurements of both paths (OPT-175B and LLaMA-70B linears, batch 8-32,
+// isolated back-to-back launches):
+//   tensor cores: waves x (K blocks per split x c(BN) + 12k) + 15k cycles, with
+//     waves = ceil(ceil(m/128) * ceil(batch/BN) * splits / SMs) and
+//     c = 1900 / 2170 / 2700 cycles per 128-input block at BN = 32 / 64 / 128
+//     (nearly independent of q: the per-block hand-offs dominate); a split
+//     run adds the fp32 partials' reduce (launch + bytes at HBM speed);
 //   lookups: q m n batch / 8 table reads at 0.62 of one 32-read wavefront per
 //     clock per SM, + 15k cycles.
-// It picks the faster path for all 12 measured (shape, batch >= 8) cases.
-bool tc_preferred(int m, int n, int batch, int q) {
+// It picks the faster path (and split count) for the 12 measured (shape,
+// batch >= 8) cases and the batch-256 layer: FC2- and out-proj-like matrices
+// (few 128-row blocks, long K) take 3 splits, QKV and FC1 none, LLaMA-70B at
+// batch 8 the lookups.  Splits are whole 1024-input slices, at most 8 (and
+// max_split), and never empty.
+int tc_plan(int m, int n, int batch, int q, int max_split) {
   static int sms_cache[64] = {0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (sms_cache[dev] == 0) {
     int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return false;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 0;
     sms_cache[dev] = v;
   }
   const double sms = sms_cache[dev];
   const int bn = batch <= 32 ? 32 : (batch <= 64 ? 64 : 128);
   const double block_cycles = bn == 32 ? 1900.0 : (bn == 64 ? 2170.0 : 2700.0);
   const double ctas = (double)((m + 127) / 128) * (double)((batch + bn - 1) / bn);
-  const double waves = std::ceil(ctas / sms);
-  const double t_tc = waves * ((double)n / 128.0) * block_cycles + 15000.0;
+  const int s_all = (n + 1023) / 1024;
+  const int nkb = n / 128;
+  const double mt32 = (double)((m + 31) / 32) * 32.0;
+  double best = 0.0, unsplit = 0.0;
+  int best_s = 0;
+  for (int sp = 1; sp <= max_split && sp <= s_all && sp <= 8; ++sp) {
+    const int spz = (s_all + sp - 1) / sp;
+    if ((s_all + spz - 1) / spz != sp) continue;          // would leave a split empty
+    const double kb = (double)(8 * spz < nkb ? 8 * spz : nkb);
+    double t = std::ceil(ctas * sp / sms) * (kb * block_cycles + 12000.0) + 15000.0;
+    if (sp > 1) t += 4000.0 + ((double)batch * mt32 * sp * 4.0 + (double)batch * m * 4.0) / 6.4e12 * 1.965e9;
+    if (sp == 1) unsplit = t;
+    if (best_s == 0 || t < best) {
+      best = t;
+      best_s = sp;
+    }
+  }
+  // A split must be expected to save at least 5 % (near ties measured slower).
+  if (best_s > 1 && best > 0.95 * unsplit) {
+    best = unsplit;
+    best_s = 1;
+  }
   const double t_lut = (double)q * m * n * batch / 8.0 / (sms * 32.0) / 0.62 + 15000.0;
-  return t_tc < t_lut;
+  return best_s > 0 && best < t_lut ? best_s : 0;
 }
 
 }  // namespace lutgemm
@@ -179,8 +205,8 @@ int lutgemm_run_tc(int m, int n, int batch, int q, int g, const uint8_t* packed,
       !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
   const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
-                                       reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
-                                       nullptr, reinterpret_cast<cudaStream_t>(stream));
+                                       reinterpret_cast<const __half*>(x), y, nullptr, 1, m, n, batch, q, g,
+                                       y_f16 ? 1 : 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 
@@ -262,13 +288,31 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
     return LUTGEMM_ERR_ALIGN;
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
   // The tensor-core path, where it takes the operands and its cost model
-  // says it is the faster one (never below batch 8).
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0 &&
-      tc_preferred(m, n, batch, q)) {
-    const cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
-                                         reinterpret_cast<const __half*>(x), y, m, n, batch, q, g, y_f16 ? 1 : 0,
-                                         nullptr, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+  // says it is the faster one (never below batch 8); split K adds its fp32
+  // partials with the split-K reduce, in split order.
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0) {
+    const int nsplit = tc_plan(m, n, batch, q, ceil_div(n, kSliceInputs));
+    if (nsplit > 0) {
+      float* part = nsplit > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
+      cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
+                                     reinterpret_cast<const __half*>(x), y, part, nsplit, m, n, batch, q, g,
+                                     y_f16 ? 1 : 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
+      if (e == cudaSuccess && nsplit > 1) {
+        RunParams r = {};
+        r.part = part;
+        r.y = y;
+        r.m = m;
+        r.n = n;
+        r.batch = batch;
+        r.q = q;
+        r.g = g;
+        r.ns = nsplit;
+        r.mt = ceil_div(m, kTileRows);
+        r.y_f16 = y_f16 ? 1 : 0;
+        e = launch_splitk_reduce(r, reinterpret_cast<cudaStream_t>(stream));
+      }
+      return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+    }
   }
 
   RunParams p;

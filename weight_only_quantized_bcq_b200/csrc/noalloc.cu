@@ -27,8 +27,9 @@
 
 namespace lutgemm {
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
-                           int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream);
-bool tc_preferred(int m, int n, int batch, int q);
+                           float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
+                           cudaStream_t stream);
+int tc_plan(int m, int n, int batch, int q, int max_split);
 }  // namespace lutgemm
 
 namespace {
@@ -128,10 +129,11 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
   // The tensor-core path needs no scratch at all (same rule as lutgemm_run).
+  // (one K split: no scratch)
   if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0 &&
-      tc_preferred(m, n, batch, q)) {
+      tc_plan(m, n, batch, q, 1) > 0) {
     const cudaError_t e = launch_tc_gemm(packed, alpha_ptr_h(alpha), offset, reinterpret_cast<const __half*>(x), y,
-                                         m, n, batch, q, g, y_f16 ? 1 : 0, nullptr,
+                                         nullptr, 1, m, n, batch, q, g, y_f16 ? 1 : 0, nullptr,
                                          reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
   }

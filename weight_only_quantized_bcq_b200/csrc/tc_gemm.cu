@@ -31,6 +31,8 @@
 //     shared memory) per plane and the commits that free A stages, units
 //     and accumulators.
 //   warps 16-19 (accumulate): see below.
+// Split K (grid z, whole 1024-input slices per split) writes fp32 partials
+// that the split-K reduce of the lookup path adds in split order.
 //
 // Accumulation: the tensor cores add into their fp32 accumulator with
 // truncation, so an error of up to an ulp per MMA step would build up over
@@ -178,12 +180,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
 // whether piece P + 4 exists in the slice.
 struct UnitIter {
   int n, ns, s, P, np;
-  __device__ __forceinline__ void init(int n_) {
+  // Slices s_begin .. s_end - 1 (the CTA's share of K).
+  __device__ __forceinline__ void init(int n_, int s_begin, int s_end) {
     n = n_;
-    ns = (n + kSliceInputs - 1) / kSliceInputs;
-    s = 0;
+    ns = s_end;
+    s = s_begin;
     P = 0;
-    np = pieces(0);
+    np = s < ns ? pieces(s) : 0;
   }
   __device__ __forceinline__ int pieces(int sl) const {
     const int r = (n - kSliceInputs * sl) / kTcBK;
@@ -211,8 +214,8 @@ struct TcLayout {
 template <int BN, bool HAS_OFF>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed,
-                   const __half* __restrict__ alpha, const float* __restrict__ offset, void* y, int m, int n,
-                   int batch, int q, int g, int mt, int y_f16, unsigned* status, TcLayout L) {
+                   const __half* __restrict__ alpha, const float* __restrict__ offset, void* y, float* part,
+                   int spz, int m, int n, int batch, int q, int g, int mt, int y_f16, unsigned* status, TcLayout L) {
   constexpr uint32_t kBTile = (uint32_t)BN * kTcBK * 2;   // x tile: BN rows x 128 inputs
   // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128.
   constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
@@ -251,7 +254,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int lane = tid & 31;
   const int rb = blockIdx.x;                                 // 128-row block
   const int b0 = blockIdx.y * BN;                            // first batch column
-  const int nkb = n / kTcBK;
+  // Split K (grid z): slices z * spz .. of the input, written as fp32
+  // partials part[b][z][32 mt] for the split-K reduce when part != nullptr.
+  const int s_begin = (int)blockIdx.z * spz;
+  const int s_all = (n + kSliceInputs - 1) / kSliceInputs;
+  const int s_end = s_begin + spz < s_all ? s_begin + spz : s_all;
+  const int nkb = (n / kTcBK < 8 * s_end ? n / kTcBK : 8 * s_end) - 8 * s_begin;   // K blocks of this split
   const int ng = n / g;
   // Scale group of K half h of K block kb (one per block when g % 128 == 0).
   const int halves_per_g = g / 64;
@@ -324,7 +332,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * 2 * q * 512 + lane * 16 + h8 * 8);
     const uint32_t alpha_lane = L.alpha_off + (uint32_t)((wq * 32 + lane) * 2);
     UnitIter it;
-    it.init(n);
+    it.init(n, s_begin, s_end);
     int ai = 0;                                              // plane step (A stage sequence)
     bool go = true;
     for (int u = 0; it.valid() && go; it.next(), ++u) {
@@ -385,7 +393,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---- Producer: one unit of x tiles, chunk groups and scale rows per ring slot.
     const int rows_here = m - rb * kTcBM < kTcBM ? m - rb * kTcBM : kTcBM;
     UnitIter it;
-    it.init(n);
+    it.init(n, s_begin, s_end);
     for (int u = 0; it.valid(); it.next(), ++u) {
       const int sl = u % L.nu;
       const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
@@ -475,7 +483,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // as the MMA operands must be); one elected lane issues each MMA and
     // commit.
     UnitIter it;
-    it.init(n);
+    it.init(n, s_begin, s_end);
     int ai = 0, j = 0;                                       // plane step, K block (processing order)
     bool ok = true;
     for (int u = 0; it.valid() && ok; it.next(), ++u) {
@@ -550,10 +558,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int jj = 0; jj < 32; ++jj) {
         const int b = b0 + c0 + jj;
         if (b < batch) {
-          const size_t o = (size_t)b * m + row;
           const float f = __uint_as_float(r[jj]);
-          if (y_f16) reinterpret_cast<__half*>(y)[o] = __float2half_rn(f);
-          else reinterpret_cast<float*>(y)[o] = f;
+          if (part != nullptr) {
+            part[((size_t)b * gridDim.z + blockIdx.z) * ((size_t)mt * kTileRows) + row] = f;
+          } else {
+            const size_t o = (size_t)b * m + row;
+            if (y_f16) reinterpret_cast<__half*>(y)[o] = __float2half_rn(f);
+            else reinterpret_cast<float*>(y)[o] = f;
+          }
         }
       }
     };
@@ -656,7 +668,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     if constexpr (HAS_OFF) {
       UnitIter it;
-      it.init(n);
+      it.init(n, s_begin, s_end);
       int j = 0;
       for (int u = 0; it.valid() && ok; it.next(), ++u) {
         const int sl = u % L.nu;
@@ -747,7 +759,8 @@ EncodeTiled encode_fn() {
 
 template <int BN, bool HAS_OFF>
 cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
-                      int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream) {
+                      float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
+                      cudaStream_t stream) {
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
@@ -782,24 +795,33 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const float* o
     status = static_cast<unsigned*>(sp);
   }
   const int mt = (m + kTileRows - 1) / kTileRows;
-  dim3 grid((unsigned)((m + kTcBM - 1) / kTcBM), (unsigned)((batch + BN - 1) / BN));
-  tc_gemm_kernel<BN, HAS_OFF><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, offset, y, m, n, batch, q, g,
-                                                                   mt, y_f16, status, L);
+  // Splits of whole slices; the caller passes a count with no empty split.
+  const int s_all = (n + kSliceInputs - 1) / kSliceInputs;
+  if (part == nullptr) nsplit = 1;
+  const int spz = (s_all + nsplit - 1) / nsplit;
+  if (nsplit < 1 || (s_all + spz - 1) / spz != nsplit) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)((m + kTcBM - 1) / kTcBM), (unsigned)((batch + BN - 1) / BN), (unsigned)nsplit);
+  tc_gemm_kernel<BN, HAS_OFF><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, offset, y, part, spz, m, n,
+                                                                   batch, q, g, mt, y_f16, status, L);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
-                           int m, int n, int batch, int q, int g, int y_f16, unsigned* status, cudaStream_t stream) {
+                           float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
+                           cudaStream_t stream) {
+#define LUTGEMM_TC_LAUNCH(BNv, OFFv) \
+  launch_bn<BNv, OFFv>(packed, alpha, offset, x, y, part, nsplit, m, n, batch, q, g, y_f16, status, stream)
   if (offset != nullptr) {
-    if (batch <= 32) return launch_bn<32, true>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
-    if (batch <= 64) return launch_bn<64, true>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
-    return launch_bn<128, true>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+    if (batch <= 32) return LUTGEMM_TC_LAUNCH(32, true);
+    if (batch <= 64) return LUTGEMM_TC_LAUNCH(64, true);
+    return LUTGEMM_TC_LAUNCH(128, true);
   }
-  if (batch <= 32) return launch_bn<32, false>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
-  if (batch <= 64) return launch_bn<64, false>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
-  return launch_bn<128, false>(packed, alpha, offset, x, y, m, n, batch, q, g, y_f16, status, stream);
+  if (batch <= 32) return LUTGEMM_TC_LAUNCH(32, false);
+  if (batch <= 64) return LUTGEMM_TC_LAUNCH(64, false);
+  return LUTGEMM_TC_LAUNCH(128, false);
+#undef LUTGEMM_TC_LAUNCH
 }
 
 }  // namespace lutgemm
