@@ -816,27 +816,11 @@ def run_tc(args):
         pg.destroy_process_group()
 
 
-def tc_splits(m: int, n: int, batch: int, q: int, sms: int = 148) -> int:
-    """The K-split count lutgemm_run's tensor-core cost model picks (1 when it
-    does not split; the same arithmetic as the library), for launch counting."""
-    import math
-    bn = 32 if batch <= 32 else (64 if batch <= 64 else 128)
-    c = {32: 1900.0, 64: 2170.0, 128: 2700.0}[bn]
-    ctas = math.ceil(m / 128) * math.ceil(batch / bn)
-    s_all, nkb, mt32 = math.ceil(n / 1024), n // 128, math.ceil(m / 32) * 32
-    best, best_s, unsplit = None, 1, None
-    for sp in range(1, min(s_all, 8) + 1):
-        spz = math.ceil(s_all / sp)
-        if math.ceil(s_all / spz) != sp:
-            continue
-        t = math.ceil(ctas * sp / sms) * (min(8 * spz, nkb) * c + 12000.0) + 15000.0
-        if sp > 1:
-            t += 4000.0 + (batch * mt32 * sp * 4.0 + batch * m * 4.0) / 6.4e12 * 1.965e9
-        if sp == 1:
-            unsplit = t
-        if best is None or t < best:
-            best, best_s = t, sp
-    return 1 if best_s > 1 and best > 0.95 * unsplit else best_s
+def tc_splits(m: int, n: int, batch: int, q: int) -> int:
+    """K splits of lutgemm_run's tensor-core plan on this device (for launch counting)."""
+    from weight_only_quantized_bcq_b200 import lutgemm
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return lutgemm.tc_plan(m, n, batch, q, sms)
 
 
 def cpu_tc_baseline(q: int, batch: int, rows: int):

@@ -124,6 +124,19 @@ size_t lutgemm_scales_bytes(int q, int m, int n, int g);
  * function. */
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g);
 
+/* The tensor-core plan lutgemm_run uses with LUTGEMM_ALLOW_TENSOR_CORES: the
+ * number of K splits it runs tc_gemm with (whole 1024-input slices, at most
+ * 8 and max_split), or 0 when its cost model expects the lookup kernel to
+ * be faster (always 0 below batch 8).  The model is fitted to B200
+ * measurements of both paths: tensor cores ~ waves x (K blocks per split x
+ * 1900 / 2170 / 2700 cycles at 32 / 64 / 128 batch columns per tile + 12k)
+ * + 15k (+ the reduce when split); lookups ~ q m n batch / 8 table reads at
+ * 0.62 of a 32-read wavefront per clock per SM + 15k.  lutgemm_run passes
+ * ceil(n / 1024) and the device's SM count.  A pure host function (whether
+ * the operands suit the tensor-core path -- n % 128, g % 64, scale layout --
+ * is checked by lutgemm_run, not here). */
+int lutgemm_tc_plan(int m, int n, int batch, int q, int max_split, int sm_count);
+
 /* Pack q planes of +-1 signs into the packed bit-plane layout above.
  * Defines the BCQ binary planes of the LUT-GEMM card (Summary; Interesting
  * ideas: weights are binary +-1 vectors with scales).

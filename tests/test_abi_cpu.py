@@ -231,3 +231,29 @@ def test_product_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
                 assert "bcq_oracle" not in text, f
+
+
+def test_tensor_core_plan_matches_the_measured_choices(L):
+    """lutgemm_tc_plan on 148 SMs picks, for each measured (shape, batch), the
+    path and split count that measured fastest on a B200 (OPT-175B and
+    LLaMA-70B linears; see the config sweep): QKV and FC1 one split, out-proj
+    and FC2 three, the LLaMA-70B linears at batch 8 the lookup kernel."""
+    sms = 148
+    want = {  # (m, n, q): {batch: splits}
+        (36864, 12288, 3): {8: 1, 16: 1, 32: 1, 256: 1},
+        (49152, 12288, 3): {8: 1, 16: 1, 32: 1, 256: 1},
+        (12288, 49152, 3): {8: 3, 16: 3, 32: 3, 256: 3},
+        (12288, 12288, 3): {256: 3},
+        (8192, 8192, 2): {8: 0},
+        (28672, 8192, 2): {8: 0},
+        (8192, 28672, 2): {8: 0},
+    }
+    for (m, n, q), cases in want.items():
+        for batch, splits in cases.items():
+            assert L.tc_plan(m, n, batch, q, sms) == splits, (m, n, q, batch)
+    # Below batch 8, and with splitting disallowed, the plan never splits.
+    assert L.tc_plan(49152, 12288, 7, 3, sms) == 0
+    assert L.tc_plan(12288, 49152, 32, 3, sms, max_split=1) == 1
+    # Splits are whole 1024-input slices: never more splits than slices.
+    for batch in (8, 64, 256):
+        assert 0 <= L.tc_plan(12288, 3072, batch, 3, sms) <= 3

@@ -40,16 +40,9 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
 // (few 128-row blocks, long K) take 3 splits, QKV and FC1 none, LLaMA-70B at
 // batch 8 the lookups.  Splits are whole 1024-input slices, at most 8 (and
 // max_split), and never empty.
-int tc_plan(int m, int n, int batch, int q, int max_split) {
-  static int sms_cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (sms_cache[dev] == 0) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 0;
-    sms_cache[dev] = v;
-  }
-  const double sms = sms_cache[dev];
+int tc_plan_for(int m, int n, int batch, int q, int max_split, int sm_count) {
+  if (m < 1 || n < 128 || batch < 8 || q < 1 || max_split < 1 || sm_count < 1) return 0;
+  const double sms = sm_count;
   const int bn = batch <= 32 ? 32 : (batch <= 64 ? 64 : 128);
   const double block_cycles = bn == 32 ? 1900.0 : (bn == 64 ? 2170.0 : 2700.0);
   const double ctas = (double)((m + 127) / 128) * (double)((batch + bn - 1) / bn);
@@ -77,6 +70,19 @@ int tc_plan(int m, int n, int batch, int q, int max_split) {
   }
   const double t_lut = (double)q * m * n * batch / 8.0 / (sms * 32.0) / 0.62 + 15000.0;
   return best_s > 0 && best < t_lut ? best_s : 0;
+}
+
+// The plan on the current device (its SM count read once per device).
+int tc_plan(int m, int n, int batch, int q, int max_split) {
+  static int sms_cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (sms_cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 0;
+    sms_cache[dev] = v;
+  }
+  return tc_plan_for(m, n, batch, q, max_split, sms_cache[dev]);
 }
 
 }  // namespace lutgemm
@@ -242,6 +248,10 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g, uint1
   const cudaError_t err = launch_pack_scales(reinterpret_cast<const __half*>(alpha), q, m, n, g, scales,
                                              reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
+int lutgemm_tc_plan(int m, int n, int batch, int q, int max_split, int sm_count) {
+  return lutgemm::tc_plan_for(m, n, batch, q, max_split, sm_count);
 }
 
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g) {

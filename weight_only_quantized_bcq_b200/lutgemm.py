@@ -29,6 +29,7 @@ _SIGNATURES = {
     "lutgemm_packed_bytes": ([_c_int, _c_int, _c_int], _c_size),
     "lutgemm_workspace_size": ([_c_int, _c_int, _c_int, _c_int, _c_int], _c_size),
     "lutgemm_scales_bytes": ([_c_int, _c_int, _c_int, _c_int], _c_size),
+    "lutgemm_tc_plan": ([_c_int, _c_int, _c_int, _c_int, _c_int, _c_int], _c_int),
     "lutgemm_pack_scales": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lutgemm_fit_bcq": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
     "lutgemm_fit_bcq_grid": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp], _c_int),
@@ -94,6 +95,14 @@ def packed_bytes(q: int, m: int, n: int) -> int:
 
 def workspace_size(m: int, n: int, batch: int, q: int, g: int) -> int:
     return int(lib().lutgemm_workspace_size(m, n, batch, q, g))
+
+
+def tc_plan(m: int, n: int, batch: int, q: int, sm_count: int, max_split: int = None) -> int:
+    """K splits lutgemm_run would run the tensor cores with under
+    LUTGEMM_ALLOW_TENSOR_CORES (0: the lookup kernel), by lutgemm_tc_plan."""
+    if max_split is None:
+        max_split = -(-n // 1024)
+    return int(lib().lutgemm_tc_plan(m, n, batch, q, max_split, sm_count))
 
 
 def new_workspace(m: int, n: int, batch: int, q: int, g: int, device=None) -> torch.Tensor:
