@@ -14,6 +14,15 @@ no data-path collective: weak scaling); the timed region is bracketed by a
 barrier and device synchronisation and its length is the max over ranks.
 "--impl reference" times the FP64 CPU oracle on a bounded sample of the same
 workload instead (rank 0 only).
+
+Other workloads (one JSON line each, same timing rules):
+    --workload tc     the same linears at batch 256 (--tc-batch) through
+                      lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES (tensor-core
+                      path, K splits where the library's model picks them);
+                      --tc-direct calls lutgemm_run_tc instead
+    --workload fit    BCQ fitting of FP16 weights (--fit-grid: variable grid)
+    --workload sweep  every configured shape and batch: lookup kernel, tensor
+                      cores and the library's choice, against both floors
 """
 from __future__ import annotations
 
