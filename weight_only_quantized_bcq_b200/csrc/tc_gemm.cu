@@ -7,8 +7,9 @@
 // its exact fp16 values +-alpha_i (an fp16 times a sign is exact), so no
 // dequantised weight is ever rounded; the planes accumulate into one fp32
 // tensor-memory accumulator.  Needs g % 64 == 0: a 64-input half of a
-// 128-input K block then lies in one scale group; group offsets (uniform weights rewritten as BCQ) are
-// added per K block in fp32 by the accumulate warps.
+// 128-input K block then lies in one scale group.  Group offsets (uniform
+// weights rewritten as BCQ) are added per K block in fp32 by the accumulate
+// warps.
 //
 // CTA tile: 128 rows (MMA M) x BN batch columns (MMA N) over K blocks of 128
 // inputs (one piece of the packed layout).  Warp roles:
@@ -18,8 +19,9 @@
 //     (lanes 0-15 of a row tile hold piece P in chunk P, lanes 16-31 in
 //     chunk P ^ 4), so one bulk copy per chunk group and row tile serves
 //     both.  Each unit holds the two x tiles (TMA, 128-byte swizzle,
-//     K-major), the 8 chunk groups of the tile's 4 row tiles and the 2 x q
-//     scale rows of the tile.
+//     K-major), the 8 chunk groups of the tile's 4 row tiles and the scale
+//     rows of the tile (per K block and plane one row, or one per 64-input
+//     half when g = 64).
 //   warps 0-15 (dequant, two groups of 8 taking alternate plane steps):
 //     expand a plane's bits for the tile into a 128 x 128 fp16 A tile in
 //     tensor memory (row r in lane r, inputs 2c and 2c+1 in column c: the
