@@ -254,13 +254,17 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *              LUTGEMM_ALLOW_TENSOR_CORES; other bits, or
  *              LUTGEMM_SCALES_PACKED with g % 128 != 0, give ERR_VALUE.
  *              With LUTGEMM_ALLOW_TENSOR_CORES the call computes the product
- *              as lutgemm_run_tc does (same result within the same
- *              tolerance, not the same bits) when that path takes the
- *              operands (batch >= 8, scales in [q][n/g][m], n % 128 == 0,
- *              g % 64 == 0) and a cost model of both paths on B200 expects
- *              it to be faster (tall matrices: many 128-row blocks to spread
- *              over the SMs, or large batches); the workspace is then left
- *              untouched.  Otherwise the flag changes nothing.
+ *              on the tensor cores as lutgemm_run_tc does (same result within
+ *              the same tolerance, not the same bits) when that path takes
+ *              the operands (batch >= 8, scales in [q][n/g][m],
+ *              n % 128 == 0, g % 64 == 0) and the cost model of
+ *              lutgemm_tc_plan expects it to be faster (tall matrices: many
+ *              128-row blocks to spread over the SMs, or large batches).
+ *              When that model splits K, each split writes fp32 partial sums
+ *              to the workspace's partial-sum area and the split-K reduce
+ *              adds them in split order (deterministic); the workspace's
+ *              counters are not touched.  Otherwise the flag changes
+ *              nothing.
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
  *              16-byte aligned, zero-filled before its first use; left
  *              zero-filled by every successful call.  Calls that share a
@@ -280,10 +284,11 @@ int lutgemm_run(int m, int n, int batch, int q, int g,
  * scale times a sign), so no rounded dequantised weight is formed; the planes
  * accumulate in fp32 (tcgen05.mma, tensor memory; each 128-input block's sum
  * is added into round-to-nearest fp32 running sums).  Tiles: 128 rows x 32,
- * 64 or 128 batch columns x 128 inputs.  The pages' kernel is the lookup one; this
- * path is for prompt-sized batches, where the method is compute-bound (LUT-GEMM
- * card, Summary and Key points: generation is memory-bound, large batches are
- * not).
+ * 64 or 128 batch columns x 128 inputs; one K split (lutgemm_run with
+ * LUTGEMM_ALLOW_TENSOR_CORES may split K).  The pages' kernel is the lookup
+ * one; this path is for prompt-sized batches, where the method is
+ * compute-bound (LUT-GEMM card, Summary and Key points: generation is
+ * memory-bound, large batches are not).
  *   m, n, batch, q, g  as lutgemm_run, and n % 128 == 0, g % 64 == 0
  *   packed, alpha, offset, x, y  as lutgemm_run ([q][n/g][m] scales; offset
  *              NULL for pure BCQ, else fp32 [n/g][m], 4-byte aligned: each
