@@ -257,3 +257,23 @@ def test_tensor_core_plan_matches_the_measured_choices(L):
     # Splits are whole 1024-input slices: never more splits than slices.
     for batch in (8, 64, 256):
         assert 0 <= L.tc_plan(12288, 3072, batch, 3, sms) <= 3
+
+
+def test_binding_signatures_match_the_header(L):
+    """Every function the binding declares has the header's argument count and
+    a return type of the same kind (int status, size_t size, const char*)."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = {}
+    for ret, name, args in re.findall(r"(\w[\w\s\*]*?)\s*\b(lutgemm_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S):
+        args = args.strip()
+        n = 0 if args in ("", "void") else len([a for a in args.split(",") if a.strip()])
+        decls[name] = (ret.split()[-1] if ret.split() else ret, n)
+    import ctypes
+    kinds = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "char*": ctypes.c_char_p}
+    for name, (argtypes, restype) in L._SIGNATURES.items():
+        assert name in decls, name
+        ret, n = decls[name]
+        assert len(argtypes) == n, (name, len(argtypes), n)
+        want = kinds.get(ret.replace("const", "").strip())
+        if want is not None:
+            assert restype is want, (name, ret, restype)
