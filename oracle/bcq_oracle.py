@@ -59,6 +59,7 @@ __all__ = [
     "scales_nbytes", "pack_scales", "unpack_scales",
     "uniform_to_bcq", "uniform_dequant", "bcq_matmul_rows",
     "fit_bcq", "fit_bcq_trace", "nearest_codes",
+    "fit_bcq_grid", "fit_bcq_grid_trace", "nearest_grid_codes",
 ]
 
 
