@@ -7,6 +7,7 @@ CUDA kernels.  If the library is missing the calls raise: there is no fallback.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -84,15 +85,57 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need(t, dtype, name):
-    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+def _need(t, dtype, name, numel=None):
+    """Host checks of one tensor argument: dtype, contiguity and size.
+
+    ``numel`` is the element count the call reads or writes through the
+    pointer; the library sees only the pointer, so a smaller tensor would be
+    accessed past its end on the GPU.  Devices are checked by ``_one_device``
+    once every argument has passed these checks."""
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call needs {numel}")
 
 
+def _one_device(stream, **named):
+    """Every tensor argument (None: absent) on one CUDA device, which is the
+    current device (the library launches there) and, when given, the stream's."""
+    dev = None
+    for name, t in named.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, other arguments on {dev}: all must be on one device")
+    cur = torch.cuda.current_device()
+    if dev.index != cur:
+        raise ValueError(f"arguments on {dev} but the current device is cuda:{cur}: "
+                         f"call under torch.cuda.device({dev.index})")
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream on {stream.device}, arguments on {dev}")
+
+
+def _groups(n: int, g: int) -> int:
+    return n // g if g > 0 else 0
+
+
+def _batch_of(x, n: int) -> int:
+    """x is [n] (batch 1) or [batch][n]."""
+    if x.dim() not in (1, 2) or x.shape[-1] != n:
+        raise ValueError(f"x must be [n] or [batch][n] with n = {n}; got {tuple(x.shape)}")
+    return x.shape[0] if x.dim() == 2 else 1
+
+
+@functools.lru_cache(maxsize=256)
 def packed_bytes(q: int, m: int, n: int) -> int:
     return int(lib().lutgemm_packed_bytes(q, m, n))
 
 
+@functools.lru_cache(maxsize=256)
 def workspace_size(m: int, n: int, batch: int, q: int, g: int) -> int:
     return int(lib().lutgemm_workspace_size(m, n, batch, q, g))
 
@@ -113,6 +156,7 @@ def new_workspace(m: int, n: int, batch: int, q: int, g: int, device=None) -> to
     return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
 
 
+@functools.lru_cache(maxsize=256)
 def scales_bytes(q: int, m: int, n: int, g: int) -> int:
     """Bytes of the unit-major scale buffer (0 when g % 128 != 0 or the shape is invalid)."""
     return lib().lutgemm_scales_bytes(q, m, n, g)
@@ -121,8 +165,9 @@ def scales_bytes(q: int, m: int, n: int, g: int) -> int:
 def pack_scales(alpha: torch.Tensor, m: int, n: int, g: int, stream=None) -> torch.Tensor:
     """fp16 alpha [q][n/g][m] on the GPU -> unit-major scales (fp16, 1-D), for
     ``run(..., scales_packed=True)``; needs g % 128 == 0."""
-    _need(alpha, torch.float16, "alpha")
-    q = alpha.shape[0]
+    q = alpha.shape[0] if alpha.dim() else 0
+    _need(alpha, torch.float16, "alpha", q * _groups(n, g) * m)
+    _one_device(stream, alpha=alpha)
     nbytes = scales_bytes(q, m, n, g)
     if nbytes == 0:
         raise LutgemmError(ERR_SHAPE, "lutgemm_scales_bytes")
@@ -136,6 +181,7 @@ def fit_bcq(w: torch.Tensor, q: int, g: int, iters: int = 3, with_error: bool = 
     """fp16 weights [m][n] on the GPU -> (int8 signs [q][m][n], fp16 alpha [q][n/g][m]
     [, fp32 squared error per group [n/g][m]]) by lutgemm_fit_bcq."""
     _need(w, torch.float16, "w")
+    _one_device(stream, w=w)
     m, n = w.shape
     signs = torch.empty((q, m, n), dtype=torch.int8, device=w.device)
     alpha = torch.empty((q, n // g if g > 0 else 0, m), dtype=torch.float16, device=w.device)
@@ -150,6 +196,7 @@ def fit_bcq_grid(w: torch.Tensor, q: int, g: int, iters: int = 3, with_error: bo
     fp32 offset [n/g][m] [, fp32 squared error per group [n/g][m]]) by lutgemm_fit_bcq_grid:
     the variable grid offset + sum_i alpha_i beta_i, run with ``run(..., offset=offset)``."""
     _need(w, torch.float16, "w")
+    _one_device(stream, w=w)
     m, n = w.shape
     ng = n // g if g > 0 else 0
     signs = torch.empty((q, m, n), dtype=torch.int8, device=w.device)
@@ -167,6 +214,11 @@ def pack_bcq(signs: torch.Tensor, packed: torch.Tensor = None, status_flags: tor
     """int8 signs [q][m][n] (+-1) on the GPU -> packed uint8 planes."""
     _need(signs, torch.int8, "signs")
     q, m, n = signs.shape
+    if packed is not None:
+        _need(packed, torch.uint8, "packed", packed_bytes(q, m, n))
+    if status_flags is not None:
+        _need(status_flags, torch.int32, "status_flags", 1)
+    _one_device(stream, signs=signs, packed=packed, status_flags=status_flags)
     if packed is None:
         packed = torch.empty(max(packed_bytes(q, m, n), 16), dtype=torch.uint8, device=signs.device)
     _check(lib().lutgemm_pack_bcq(_ptr(signs), q, m, n, _ptr(packed), _ptr(status_flags), _stream(stream)),
@@ -178,9 +230,12 @@ def uniform_to_bcq(codes: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
                    status_flags: torch.Tensor = None, stream=None):
     """Uniform codes [m][n], scale fp16 [n/g][m], zero uint8 [n/g][m] -> (packed, alpha, offset)."""
     _need(codes, torch.uint8, "codes")
-    _need(scale, torch.float16, "scale")
-    _need(zero, torch.uint8, "zero")
     m, n = codes.shape
+    _need(scale, torch.float16, "scale", _groups(n, g) * m)
+    _need(zero, torch.uint8, "zero", _groups(n, g) * m)
+    if status_flags is not None:
+        _need(status_flags, torch.int32, "status_flags", 1)
+    _one_device(stream, codes=codes, scale=scale, zero=zero, status_flags=status_flags)
     dev = codes.device
     packed = torch.empty(max(packed_bytes(q, m, n), 16), dtype=torch.uint8, device=dev)
     alpha = torch.empty((q, n // g, m), dtype=torch.float16, device=dev)
@@ -191,6 +246,23 @@ def uniform_to_bcq(codes: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
     return packed, alpha, offset
 
 
+def _check_product_args(packed, alpha, x, offset, y, workspace, m, n, q, g, y_f16, scales_packed, stream) -> int:
+    """The checks shared by the product calls; returns the batch."""
+    batch = _batch_of(x, n)
+    _need(packed, torch.uint8, "packed", packed_bytes(q, m, n))
+    a_need = scales_bytes(q, m, n, g) // 2 if scales_packed else q * _groups(n, g) * m
+    _need(alpha, torch.float16, "alpha", a_need)
+    _need(x, torch.float16, "x")
+    if offset is not None:
+        _need(offset, torch.float32, "offset", _groups(n, g) * m)
+    if y is not None:
+        _need(y, torch.float16 if y_f16 else torch.float32, "y", batch * m)
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+    _one_device(stream, x=x, packed=packed, alpha=alpha, offset=offset, y=y, workspace=workspace)
+    return batch
+
+
 def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
         offset: torch.Tensor = None, y: torch.Tensor = None, workspace: torch.Tensor = None,
         y_f16: bool = False, scales_packed: bool = False, allow_tensor_cores: bool = False,
@@ -198,12 +270,7 @@ def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: i
     """y[b] = W x[b] for a packed BCQ weight W (m x n), computed by lutgemm_run.
     With ``scales_packed`` alpha is the output of ``pack_scales``; with
     ``allow_tensor_cores`` the library may take the tensor-core path (batch >= 8)."""
-    _need(packed, torch.uint8, "packed")
-    _need(alpha, torch.float16, "alpha")
-    _need(x, torch.float16, "x")
-    if offset is not None:
-        _need(offset, torch.float32, "offset")
-    batch = x.shape[0] if x.dim() == 2 else 1
+    batch = _check_product_args(packed, alpha, x, offset, y, workspace, m, n, q, g, y_f16, scales_packed, stream)
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     if workspace is None:
@@ -220,12 +287,7 @@ def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n
            y: torch.Tensor = None, y_f16: bool = False, offset: torch.Tensor = None, stream=None) -> torch.Tensor:
     """``run`` on the tensor cores (lutgemm_run_tc), for large batches;
     n % 128 == 0 and g % 64 == 0, [q][n/g][m] scales, optional fp32 offsets."""
-    _need(packed, torch.uint8, "packed")
-    _need(alpha, torch.float16, "alpha")
-    _need(x, torch.float16, "x")
-    if offset is not None:
-        _need(offset, torch.float32, "offset")
-    batch = x.shape[0] if x.dim() == 2 else 1
+    batch = _check_product_args(packed, alpha, x, offset, y, None, m, n, q, g, y_f16, False, stream)
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     _check(lib().lutgemm_run_tc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
@@ -241,12 +303,7 @@ def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: i
     workspace: the library uses its own fixed 16 MiB device scratch instead.
     Only ``y`` is allocated here, and only when the caller passes none.  Calls
     that overlap on the GPU share that scratch and race."""
-    _need(packed, torch.uint8, "packed")
-    _need(alpha, torch.float16, "alpha")
-    _need(x, torch.float16, "x")
-    if offset is not None:
-        _need(offset, torch.float32, "offset")
-    batch = x.shape[0] if x.dim() == 2 else 1
+    batch = _check_product_args(packed, alpha, x, offset, y, None, m, n, q, g, y_f16, scales_packed, stream)
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0) | \
