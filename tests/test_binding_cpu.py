@@ -108,3 +108,30 @@ def test_set_up_calls_check_their_buffers(L):
         L.pack_scales(torch.zeros(Q, N // G, M - 1, dtype=torch.float16), M, N, G)
     with pytest.raises(ValueError, match="w must be a CUDA tensor"):
         L.fit_bcq(torch.zeros(M, N, dtype=torch.float16), Q, G)
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor (only what the device check reads)."""
+
+    def __init__(self, index):
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+
+
+class _FakeStream:
+    def __init__(self, index):
+        self.device = torch.device("cuda", index)
+
+
+def test_device_check_wants_one_device_the_current_one(L, monkeypatch):
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    L._one_device(None, x=_FakeCuda(1), y=_FakeCuda(1), offset=None)
+    L._one_device(_FakeStream(1), x=_FakeCuda(1))
+    with pytest.raises(ValueError, match="y is on cuda:0, other arguments on cuda:1"):
+        L._one_device(None, x=_FakeCuda(1), y=_FakeCuda(0))
+    with pytest.raises(ValueError, match="current device is cuda:1"):
+        L._one_device(None, x=_FakeCuda(0), y=_FakeCuda(0))
+    with pytest.raises(ValueError, match="stream on cuda:0"):
+        L._one_device(_FakeStream(0), x=_FakeCuda(1))
+    with pytest.raises(ValueError, match="packed must be a CUDA tensor"):
+        L._one_device(None, x=_FakeCuda(1), packed=torch.zeros(1))
