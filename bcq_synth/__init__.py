@@ -35,6 +35,8 @@ __all__ = [
     "draw_uniform",
     "draw_x",
     "draw_weights",
+    "draw_block_planes",
+    "draw_outliers",
     "Shape",
     "WORKLOADS",
 ]
@@ -98,6 +100,28 @@ def draw_x(gen: torch.Generator, batch: int, n: int, outlier_frac: float = 0.0,
         idx = torch.randperm(n, generator=gen)[:k]
         x[:, idx] *= outlier_scale
     return x.to(torch.float16).contiguous()
+
+
+def draw_block_planes(gen: torch.Generator, m: int, n: int, frac_hi: float, lo: int = 2,
+                      hi: int = 4) -> torch.Tensor:
+    """Plane count of every (1024-input slice, 32-row tile) block, uint8
+    [ceil(n/1024)][ceil(m/32)]: `hi` with probability frac_hi, else `lo`."""
+    ns, mt = -(-n // 1024), -(-m // 32)
+    u = torch.rand((ns, mt), generator=gen)
+    return torch.where(u < frac_hi, hi, lo).to(torch.uint8).contiguous()
+
+
+def draw_outliers(gen: torch.Generator, m: int, n: int, density: float, sigma: float = 0.1):
+    """Sparse fp16 outlier weights ~ N(0, sigma) at round(density*m*n)
+    positions drawn without replacement, as row CSR: (row_ptr int32 [m+1],
+    col int32 [nnz] increasing within a row, val fp16 [nnz])."""
+    nnz = int(round(density * m * n))
+    flat = torch.randperm(m * n, generator=gen)[:nnz].sort().values
+    rows, cols = flat // n, flat % n
+    val = (torch.randn(nnz, generator=gen) * sigma).to(torch.float16)
+    row_ptr = torch.zeros(m + 1, dtype=torch.int64)
+    row_ptr[1:] = torch.bincount(rows, minlength=m).cumsum(0)
+    return row_ptr.to(torch.int32), cols.to(torch.int32), val
 
 
 @dataclass(frozen=True)

@@ -55,11 +55,13 @@ BLOCK_BYTES = 4096  # bytes of one (slice, row tile, plane): 8 chunks of 512
 
 __all__ = [
     "lut_table", "dequantize_bcq", "bcq_matmul", "lut_matmul",
-    "packed_nbytes", "pack_bcq", "unpack_bcq", "unpack_rows",
+    "packed_nbytes", "pack_bcq", "unpack_bcq", "unpack_rows", "unpack_bcq_vec", "packed_row_tiles",
     "scales_nbytes", "pack_scales", "unpack_scales",
     "uniform_to_bcq", "uniform_dequant", "bcq_matmul_rows",
     "fit_bcq", "fit_bcq_trace", "nearest_codes",
     "fit_bcq_grid", "fit_bcq_grid_trace", "nearest_grid_codes",
+    "mixed_block_offsets", "mixed_packed_nbytes", "pack_mixed", "unpack_mixed",
+    "mixed_weights", "mixed_matmul", "pack_outliers", "unpack_outliers", "outlier_dense",
 ]
 
 
@@ -220,6 +222,41 @@ def unpack_rows(packed, q: int, m: int, n: int, rows) -> np.ndarray:
                     out_bits[:, ri, np.arange(ns) * SLICE + k0 + t] = bit.T
     bits = out_bits[:, :, :n]
     return (bits.astype(np.int8) * 2 - 1)
+
+
+def unpack_bcq_vec(packed, q: int, m: int, n: int) -> np.ndarray:
+    """``unpack_bcq`` with the layout's index map applied to whole arrays at
+    once, for checking every output of full-size problems in seconds.
+
+    Every byte is split into its 8 bits (bit t = input 8c + t, LSB first);
+    then for each lane l the pieces and runs are put back in input order:
+    piece P sits at step U = P xor 4*(l // 16) and run c at byte
+    j = c xor (l % 16), the same map as ``unpack_rows``."""
+    pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    assert pk.size == packed_nbytes(q, m, n)
+    ns, mt = math.ceil(n / SLICE), math.ceil(m / TILE_ROWS)
+    chunks = pk.reshape(ns, mt, 8, q, TILE_ROWS, 16)
+    bits = np.unpackbits(chunks[..., None], axis=-1, bitorder="little")   # [ns][mt][U][q][l][j][t]
+    out = np.empty((q, mt, TILE_ROWS, ns, SLICE), dtype=np.uint8)
+    for l in range(TILE_ROWS):
+        U_of_P = np.arange(8) ^ (4 * (l // 16))
+        j_of_c = np.arange(16) ^ (l % 16)
+        lane = bits[:, :, :, :, l][:, :, U_of_P][:, :, :, :, j_of_c]       # [ns][mt][P][q][c][t]
+        out[:, :, l] = lane.transpose(3, 1, 0, 2, 4, 5).reshape(q, mt, ns, SLICE)
+    out = out.reshape(q, mt * TILE_ROWS, ns * SLICE)
+    return out[:, :m, :n].astype(np.int8) * 2 - 1
+
+
+def packed_row_tiles(packed, q: int, m: int, n: int, R0: int, R1: int):
+    """The bytes of row tiles [R0, R1) of a packed buffer, which are the packed
+    buffer of the sub-matrix of rows 32*R0 .. min(m, 32*R1) - 1 (blocks are
+    ordered slice-major, row tile minor).  Returns (buffer, rows of the sub-matrix)."""
+    pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    assert pk.size == packed_nbytes(q, m, n)
+    ns, mt = math.ceil(n / SLICE), math.ceil(m / TILE_ROWS)
+    assert 0 <= R0 < R1 <= mt
+    blocks = pk.reshape(ns, mt, q * BLOCK_BYTES)
+    return np.ascontiguousarray(blocks[:, R0:R1]).reshape(-1), min(m, TILE_ROWS * R1) - TILE_ROWS * R0
 
 
 # ---------------------------------------------------------------------------
@@ -544,3 +581,161 @@ def fit_bcq_grid_trace(w, q: int, g: int, iters: int):
     trace = []
     _fit_groups_grid(w, q, g, iters, trace)
     return trace
+
+
+# ---------------------------------------------------------------------------
+# Mixed storage: 2-, 4- and 16-bit weights in one matrix (OpenAlex record
+# "Fast and Efficient 2-bit LLM Inference on GPU: 2/4/16-bit in a Weight
+# Matrix with Asynchronous Dequantization", abstract: weights are quantised
+# by groups, some groups hold a large range, and sparse outliers are kept at
+# higher precision).  The record gives the idea only (its abstract stops at
+# the problem statement).  Reading used here, in BCQ form:
+#   * a precision block (s, R) is rows 32R .. 32R+31 by inputs 1024s ..
+#     1024s+1023, the unit the lookup kernel streams; it carries q_b planes,
+#     1 <= q_b <= q_max (2 planes for most blocks, 4 for wide-range ones);
+#   * W[j,k] = sum_{i < q_b(j // 32, k // 1024)} alpha[i, k // g, j] * beta[i, j, k]
+#              + S[j, k],
+#     where S is a sparse fp16 matrix, the 16-bit outliers, ADDED to the
+#     BCQ value (a sign plane has no zero, so the BCQ part cannot leave a
+#     position out; a fitter stores the outlier's residual);
+#   * packed planes: blocks in (s, R) order, block (s, R) holds q_b * 4096
+#     bytes from byte 4096 * off[s * m_t + R], off the exclusive prefix sum
+#     of q_b in that order; inside a block, chunk (U, i) sits at
+#     (U * q_b + i) * 512 with the byte map of the uniform layout (so with
+#     q_b = q everywhere the buffer equals pack_bcq's);
+#   * outliers for the kernel: slice-major CSR, the entries of (slice s,
+#     row r) at [optr[s * m + r], optr[s * m + r + 1]), sorted by input, each
+#     a uint32 (k - 1024 s) | (fp16 bits << 16).
+# block_planes is uint8 [n_s][m_t]; outliers are given as row CSR
+# (row_ptr [m + 1], col [nnz] increasing within a row, val fp16 [nnz]).
+# ---------------------------------------------------------------------------
+def _check_blocks(block_planes, m: int, n: int):
+    bp = np.asarray(block_planes, dtype=np.int64)
+    ns, mt = math.ceil(n / SLICE), math.ceil(m / TILE_ROWS)
+    if bp.shape != (ns, mt):
+        raise ValueError(f"block_planes must be [{ns}][{mt}]")
+    if bp.min(initial=1) < 1:
+        raise ValueError("every block needs at least one plane")
+    return bp
+
+
+def mixed_block_offsets(block_planes) -> np.ndarray:
+    """Exclusive prefix sum of the plane counts in (s, R) order, in 4096-byte
+    blocks: uint32 [n_s * m_t + 1]; the last entry is the total."""
+    bp = np.asarray(block_planes, dtype=np.int64).reshape(-1)
+    return np.concatenate([[0], np.cumsum(bp)]).astype(np.uint32)
+
+
+def mixed_packed_nbytes(block_planes) -> int:
+    return int(np.asarray(block_planes, dtype=np.int64).sum()) * BLOCK_BYTES
+
+
+def pack_mixed(signs, block_planes) -> np.ndarray:
+    """int8 signs [q_max][m][n] -> the mixed packed buffer.  Block (s, R)
+    stores planes 0 .. q_b - 1 of its rows and inputs, packed as a one-tile,
+    one-slice matrix by ``pack_bcq``; planes from q_b on are not stored."""
+    sg = np.asarray(signs)
+    q_max, m, n = sg.shape
+    bp = _check_blocks(block_planes, m, n)
+    if bp.max(initial=1) > q_max:
+        raise ValueError("a block has more planes than signs were given")
+    ns, mt = bp.shape
+    parts = []
+    for s_ in range(ns):
+        for R in range(mt):
+            qb = int(bp[s_, R])
+            blk = sg[:qb, TILE_ROWS * R: TILE_ROWS * (R + 1), SLICE * s_: SLICE * (s_ + 1)]
+            parts.append(pack_bcq(blk))
+    return np.concatenate(parts)
+
+
+def unpack_mixed(packed, block_planes, q_max: int, m: int, n: int) -> np.ndarray:
+    """Inverse of ``pack_mixed``: signs int8 [q_max][m][n], with 0 where a
+    block stores no plane."""
+    pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    bp = _check_blocks(block_planes, m, n)
+    assert pk.size == mixed_packed_nbytes(bp)
+    off = mixed_block_offsets(bp)
+    ns, mt = bp.shape
+    out = np.zeros((q_max, m, n), dtype=np.int8)
+    for s_ in range(ns):
+        for R in range(mt):
+            u = s_ * mt + R
+            qb = int(bp[s_, R])
+            r0, k0 = TILE_ROWS * R, SLICE * s_
+            mr, nk = min(m, r0 + TILE_ROWS) - r0, min(n, k0 + SLICE) - k0
+            blk = pk[int(off[u]) * BLOCK_BYTES: int(off[u + 1]) * BLOCK_BYTES]
+            out[:qb, r0: r0 + mr, k0: k0 + nk] = unpack_bcq(blk, qb, mr, nk)
+    return out
+
+
+def outlier_dense(row_ptr, col, val, m: int, n: int) -> np.ndarray:
+    """The sparse outlier matrix S as a dense FP64 [m][n] array."""
+    rp = np.asarray(row_ptr, dtype=np.int64)
+    c = np.asarray(col, dtype=np.int64)
+    v = np.asarray(val, dtype=np.float16).astype(np.float64)
+    S_ = np.zeros((m, n), dtype=np.float64)
+    for r in range(m):
+        ks = c[rp[r]: rp[r + 1]]
+        if np.any(np.diff(ks) <= 0) or (ks.size and (ks.min() < 0 or ks.max() >= n)):
+            raise ValueError("outlier columns must increase within a row and lie in [0, n)")
+        S_[r, ks] = v[rp[r]: rp[r + 1]]
+    return S_
+
+
+def mixed_weights(signs, alpha, block_planes, g: int, outliers=None) -> np.ndarray:
+    """The plain FP64 W of the mixed format (definition above).
+
+    signs [q_max][m][n] (planes a block does not store are ignored);
+    alpha [q_max][n/g][m]; outliers None or (row_ptr, col, val)."""
+    sg = np.asarray(signs)
+    q_max, m, n = sg.shape
+    bp = _check_blocks(block_planes, m, n)
+    a = np.asarray(alpha, dtype=np.float64)
+    assert a.shape == (q_max, n // g, m)
+    qb = np.repeat(np.repeat(bp.T, TILE_ROWS, axis=0)[:m], SLICE, axis=1)[:, :n]   # [m][n]
+    W = np.zeros((m, n), dtype=np.float64)
+    for i in range(q_max):
+        a_rows = np.repeat(a[i], g, axis=0).T
+        W += np.where(i < qb, a_rows * sg[i].astype(np.float64), 0.0)
+    if outliers is not None:
+        W += outlier_dense(*outliers, m, n)
+    return W
+
+
+def mixed_matmul(x, signs, alpha, block_planes, g: int, outliers=None) -> np.ndarray:
+    """y[b, j] = sum_k W[j, k] x[b, k] with W from ``mixed_weights``; FP64 [batch][m]."""
+    return np.asarray(x, dtype=np.float64) @ mixed_weights(signs, alpha, block_planes, g, outliers).T
+
+
+def pack_outliers(row_ptr, col, val, m: int, n: int):
+    """Row CSR outliers -> (optr uint32 [n_s * m + 1], oent uint32 [nnz]): the
+    slice-major layout above."""
+    rp = np.asarray(row_ptr, dtype=np.int64)
+    c = np.asarray(col, dtype=np.int64)
+    bits = np.asarray(val, dtype=np.float16).view(np.uint16).astype(np.uint32)
+    ns = math.ceil(n / SLICE)
+    outlier_dense(rp, c, np.asarray(val, dtype=np.float16), m, n)     # validates the CSR
+    optr = np.zeros(ns * m + 1, dtype=np.uint32)
+    ent = []
+    for s_ in range(ns):
+        for r in range(m):
+            e = np.arange(rp[r], rp[r + 1])
+            e = e[(c[e] >= SLICE * s_) & (c[e] < SLICE * (s_ + 1))]
+            ent.extend(((c[e] - SLICE * s_) | (bits[e] << 16)).tolist())
+            optr[s_ * m + r + 1] = len(ent)
+    return optr, np.asarray(ent, dtype=np.uint32)
+
+
+def unpack_outliers(optr, oent, m: int, n: int) -> np.ndarray:
+    """Inverse of ``pack_outliers``, as a dense FP64 [m][n] array."""
+    optr = np.asarray(optr, dtype=np.int64)
+    oent = np.asarray(oent, dtype=np.uint32)
+    ns = math.ceil(n / SLICE)
+    S_ = np.zeros((m, n), dtype=np.float64)
+    for s_ in range(ns):
+        for r in range(m):
+            for e in range(optr[s_ * m + r], optr[s_ * m + r + 1]):
+                k = SLICE * s_ + int(oent[e] & 0xFFFF)
+                S_[r, k] = float(np.uint16(oent[e] >> 16).view(np.float16))
+    return S_

@@ -336,6 +336,52 @@ def test_pack_roundtrip(q, m, n):
     assert np.array_equal(O.unpack_rows(pk, q, m, n, rows), s[:, rows, :])
 
 
+def test_vectorised_unpack_pins():
+    assert pin_unpack_golden(O.unpack_bcq_vec)
+
+
+@pytest.mark.parametrize("q,m,n", [(1, 32, 1024), (3, 45, 2056), (2, 70, 3000), (4, 1, 8), (8, 33, 1032)])
+def test_vectorised_unpack_equals_loop_unpack(q, m, n):
+    rng = np.random.default_rng(q * 77 + m)
+    s = _signs(rng, q, m, n)
+    pk = O.pack_bcq(s)
+    assert np.array_equal(O.unpack_bcq_vec(pk, q, m, n), s)
+    assert np.array_equal(O.unpack_bcq_vec(pk, q, m, n), O.unpack_bcq(pk, q, m, n))
+
+
+@pytest.mark.parametrize("q,m,n,R0,R1", [(3, 100, 2056, 1, 3), (2, 100, 2056, 2, 4), (1, 64, 1024, 0, 2),
+                                          (4, 33, 8, 1, 2)])
+def test_packed_row_tiles_is_the_packed_sub_matrix(q, m, n, R0, R1):
+    rng = np.random.default_rng(q + m + R0)
+    s = _signs(rng, q, m, n)
+    sub, m_sub = O.packed_row_tiles(O.pack_bcq(s), q, m, n, R0, R1)
+    rows = s[:, 32 * R0: 32 * R0 + m_sub]
+    assert m_sub == rows.shape[1]
+    assert np.array_equal(sub, O.pack_bcq(rows))
+    assert np.array_equal(O.unpack_bcq_vec(sub, q, m_sub, n), rows)
+
+
+def _unpack_vec_msb_first(packed, q, m, n):
+    # Bit order reversed inside each byte: must fail the golden single bits.
+    pk = np.asarray(packed, dtype=np.uint8)
+    rev = np.unpackbits(pk[:, None], axis=1, bitorder="little")
+    return O.unpack_bcq_vec(np.packbits(rev, axis=1, bitorder="big").reshape(-1), q, m, n)
+
+
+def _unpack_vec_no_half_swap(packed, q, m, n):
+    # Lanes 16..31 read the same piece as lanes 0..15.
+    pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    ns, mt = math.ceil(n / 1024), math.ceil(m / 32)
+    ch = pk.reshape(ns, mt, 8, q, 32, 16).copy()
+    ch[:, :, :, :, 16:, :] = ch[:, :, [4, 5, 6, 7, 0, 1, 2, 3], :, 16:, :]
+    return O.unpack_bcq_vec(ch.reshape(-1), q, m, n)
+
+
+@pytest.mark.parametrize("mutant", [_unpack_vec_msb_first, _unpack_vec_no_half_swap])
+def test_vectorised_unpack_pins_catch_mistakes(mutant):
+    assert not pin_unpack_golden(mutant)
+
+
 def test_pack_rejects_non_sign_values():
     s = np.ones((1, 4, 8), dtype=np.int8)
     s[0, 1, 3] = 0
