@@ -12,6 +12,8 @@ drawn by bcq_synth; the step's working set (765 MB) is far larger than the
 N > 1 runs under torchrun: every rank runs its own layer (independent weights,
 no data-path collective: weak scaling); the timed region is bracketed by a
 barrier and device synchronisation and its length is the max over ranks.
+"--parallel rows|inputs|paired" instead splits one matrix (OPT-175B FC1, FC2,
+or the FC1 -> FC2 block) over the ranks with an NCCL exchange (strong scaling).
 "--impl reference" times the FP64 CPU oracle on a bounded sample of the same
 workload instead (rank 0 only).
 
@@ -23,6 +25,9 @@ Other workloads (one JSON line each, same timing rules):
     --workload fit    BCQ fitting of FP16 weights (--fit-grid: variable grid)
     --workload sweep  every configured shape and batch: lookup kernel, tensor
                       cores and the library's choice, against both floors
+    --workload mixed  mixed 2/4/16-bit storage (lutgemm_run_mixed) on the
+                      LLaMA-70B-shaped linears: 2-plane blocks, --mixed-hi of
+                      them at 4 planes, --mixed-outliers fp16 outliers
 """
 from __future__ import annotations
 
@@ -39,10 +44,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-import torch  # noqa: E402
+if __name__ != "__mp_main__":
+    # A process the CPU baseline spawns re-imports this file under that name
+    # and only runs _oracle_job: it needs neither torch nor the library.
+    import torch  # noqa: E402
 
-import bcq_synth as S  # noqa: E402
-from weight_only_quantized_bcq_b200.roofline import algorithmic_bytes  # noqa: E402
+    import bcq_synth as S  # noqa: E402
+    from weight_only_quantized_bcq_b200.roofline import algorithmic_bytes  # noqa: E402
 
 METRIC = "LUT-GEMM µs/matmul and achieved HBM GB/s (fraction of B200 peak) at batch 1"
 WORKLOAD = "opt175b_layer"
@@ -198,14 +206,17 @@ def make_layer(q: int, batch: int, seed: int, device, only=None, scales="packed"
     xo = yo = 0
     for sh in shapes:
         nbytes = lutgemm.packed_bytes(q, sh.m, sh.n)
-        packed = S.draw_random_bytes(gen, nbytes).to(device)
-        alpha = S.draw_alpha(gen, q, sh.m, sh.n, w.g, w.alpha_sigma).to(device)
+        packed_host = S.draw_random_bytes(gen, nbytes)
+        alpha_host = S.draw_alpha(gen, q, sh.m, sh.n, w.g, w.alpha_sigma)
+        packed = packed_host.to(device)
+        alpha = alpha_host.to(device)
         if scales == "packed":
             alpha = lutgemm.pack_scales(alpha, sh.m, sh.n, w.g)
         x_host = io["x_host"][xo: xo + batch * sh.n].view(batch, sh.n)
         x_host.copy_(S.draw_x(gen, batch, sh.n))
         mats.append({
             "name": sh.name, "m": sh.m, "n": sh.n, "packed": packed, "alpha": alpha,
+            "packed_host": packed_host, "alpha_host": alpha_host,
             "scales_packed": scales == "packed", "launches": 1 + (sh.n > 1024),
             "x_host": x_host, "x": io["x"][xo: xo + batch * sh.n].view(batch, sh.n),
             "y": io["y"][yo: yo + batch * sh.m].view(batch, sh.m),
@@ -321,6 +332,9 @@ def run_lutgemm(args):
     region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
     if graph is not None:
         del graph
+    # The outputs of the last timed step, kept for the parity check against
+    # the oracle (outside the timed region).
+    y_timed = io["y"].cpu().clone()
 
     # Per-linear times: a separate pass with events around every launch (the
     # events serialise the launches, so these are isolated kernel times).
@@ -404,7 +418,8 @@ def run_lutgemm(args):
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline(q, batch, args.cpu_rows)
+            out["cpu_baseline"], out["parity"] = cpu_baseline_and_parity(mats, q, g, batch, args.cpu_rows,
+                                                                         y_timed, io)
         print(json.dumps(out), flush=True)
     if pg is not None:
         pg.barrier()
@@ -414,6 +429,133 @@ def run_lutgemm(args):
 # ---------------------------------------------------------------------------
 # The FP64 oracle on the host cores, on a bounded sample of the same workload.
 # ---------------------------------------------------------------------------
+def _oracle_job(args):
+    """One piece of CPU-baseline work: the oracle's product (unpack the signs,
+    dequantise in FP64, matmul) on the row tiles of one packed sub-buffer.
+    Runs in the bench process or in a spawned one (which has no torch)."""
+    from oracle import bcq_oracle as O
+    sub, q, m_sub, n, alpha_rows, x, g = args
+    t = time.perf_counter()
+    y = O.bcq_matmul(x, O.unpack_bcq(sub, q, m_sub, n), alpha_rows, g)
+    return y, time.perf_counter() - t
+
+
+def _host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+class OraclePool:
+    """A pool of `cores` spawned processes running _oracle_job (spawned, not
+    forked: a child forked from a process that has used CUDA can hang).  One
+    trivial job per worker starts them all before any timing."""
+
+    def __init__(self, cores: int):
+        import multiprocessing as mp
+        from concurrent.futures import ProcessPoolExecutor
+        import numpy as np
+        self.cores = cores
+        self.ex = ProcessPoolExecutor(max_workers=cores, mp_context=mp.get_context("spawn"))
+        tiny = (np.zeros(4096, dtype=np.uint8), 1, 32, 1024, np.zeros((1, 8, 32), dtype=np.float16),
+                np.zeros((1, 1024), dtype=np.float16), 128)
+        list(self.ex.map(_oracle_job, [tiny] * cores))
+
+    def run(self, jobs):
+        """Wall seconds for all jobs on the pool, and their outputs."""
+        t = time.perf_counter()
+        res = list(self.ex.map(_oracle_job, jobs))
+        return time.perf_counter() - t, [r[0] for r in res]
+
+    def close(self):
+        self.ex.shutdown()
+
+
+def _tile_job(packed_host, alpha_host, x, q, m, n, g, tiles):
+    """Job arguments for the row tiles `tiles` of one linear, and the rows they cover."""
+    import numpy as np
+    ns, mt = -(-n // 1024), -(-m // 32)
+    blocks = packed_host.numpy().reshape(ns, mt, q * 4096)
+    sub = np.ascontiguousarray(blocks[:, tiles]).reshape(-1)
+    rows = (32 * np.asarray(tiles)[:, None] + np.arange(32)[None, :]).reshape(-1)
+    rows = rows[rows < m]
+    return (sub, q, rows.size, n, np.ascontiguousarray(alpha_host.numpy()[:, :, rows]), x, g), rows
+
+
+def cpu_baseline_and_parity(mats, q: int, g: int, batch: int, rows: int, y_timed, io):
+    """The oracle on sampled row tiles of the bench's own weights and inputs.
+
+    1 thread: `rows` rows (whole 32-row tiles, the first and last tile
+    included) of each linear, timed, and the outputs compared with the
+    timed region's last y (the parity field).  All host cores: a pool of
+    spawned processes, one tile per job, about four tiles per core."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    from tests._tol import compare
+    rng = np.random.default_rng(7)
+    k = max(2, rows // 32)
+    jobs, picks = [], []
+    for mt_ in mats:
+        mtiles = -(-mt_["m"] // 32)
+        inner = rng.choice(np.arange(1, mtiles - 1), size=min(k - 2, mtiles - 2), replace=False)
+        tiles = np.unique(np.r_[0, mtiles - 1, inner])
+        job, r = _tile_job(mt_["packed_host"], mt_["alpha_host"], mt_["x_host"].numpy(), q, mt_["m"], mt_["n"],
+                           g, tiles)
+        jobs.append(job)
+        picks.append(r)
+    with threadpool_limits(limits=1):
+        res = [_oracle_job(j) for j in jobs]
+    secs1 = sum(t for _, t in res)
+    bytes1 = sum(algorithmic_bytes(j[2], j[3], q, g, batch) for j in jobs)
+    # Parity of the timed step's outputs on the sampled rows.
+    per, ok_all, yo = {}, True, 0
+    y_all = y_timed.numpy()
+    for mt_, (y_ref, _), r, job in zip(mats, res, picks, jobs):
+        got = y_all[yo: yo + batch * mt_["m"]].reshape(batch, mt_["m"])[:, r]
+        ok, st = compare(got, y_ref, job[4], job[5], mt_["n"])
+        per[mt_["name"]] = {"rows": int(r.size), "rel_l2": st["rel_l2"],
+                            "max_abs_over_bound": round(st["max_abs_over_bound"], 5)}
+        ok_all = ok_all and ok
+        yo += batch * mt_["m"]
+    parity = {"ok": bool(ok_all), "per_linear": per,
+              "what": "the last graph-replayed step's y against the FP64 oracle on the sampled rows "
+                      "(rel-L2 <= 1e-3 and per-output max-abs bound)"}
+    # All host cores: one tile per job, about four per core, spread over the linears.
+    cores = min(_host_cores(), 64)
+    pool = OraclePool(cores)
+    try:
+        per_lin = max(1, -(-4 * cores // len(mats)))
+        jobs_all = []
+        for mt_ in mats:
+            mtiles = -(-mt_["m"] // 32)
+            for t in rng.choice(mtiles, size=min(per_lin, mtiles), replace=False):
+                jobs_all.append(_tile_job(mt_["packed_host"], mt_["alpha_host"], mt_["x_host"].numpy(), q, mt_["m"],
+                                          mt_["n"], g, [int(t)])[0])
+        wall, _ = pool.run(jobs_all)
+    finally:
+        pool.close()
+    bytes_all = sum(algorithmic_bytes(j[2], j[3], q, g, batch) for j in jobs_all)
+    base = {"value": round(bytes_all / wall / 1e9, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "seconds": round(wall, 2), "host_cores": _host_cores(), "cpu_model": _cpu_model(),
+            "sample": f"{len(jobs_all)} row tiles (32 rows each) of the 4 layer linears of this run's weights "
+                      f"and x (q={q}, g={g}, batch {batch}), one tile per job on {cores} spawned processes: "
+                      "oracle unpack + FP64 dequantise + matmul",
+            "single_thread": {"value": round(bytes1 / secs1 / 1e9, 6), "cores": 1, "seconds": round(secs1, 2),
+                              "sample": f"{sum(r.size for r in picks)} rows ({k} tiles of each linear, first "
+                                        "and last included), one thread"}}
+    return base, parity
 def _oracle_sample(q: int, batch: int, rows_per_matrix: int, seed: int):
     """Timed oracle work on `rows_per_matrix` sampled rows of each of the four linears.
 
@@ -441,43 +583,64 @@ def _oracle_sample(q: int, batch: int, rows_per_matrix: int, seed: int):
     return secs, nbytes
 
 
-def cpu_baseline(q: int, batch: int, rows: int):
-    from threadpoolctl import threadpool_limits
-    with threadpool_limits(limits=1):
-        secs, nbytes = _oracle_sample(q, batch, rows, seed=7)
-    return {"value": round(nbytes / secs / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seconds": round(secs, 2),
-            "sample": f"{rows} rows of each of the 4 layer linears (q={q}, g=128, batch {batch}): "
-                      "oracle unpack + FP64 dequantise + matmul, one thread"}
+def _random_tile_jobs(q: int, batch: int, n_tiles: int, seed: int):
+    """Oracle jobs of one random 32-row tile each, spread over the 4 layer
+    linears, drawn on the CPU with the workload's distributions."""
+    w = S.WORKLOADS[WORKLOAD]
+    jobs = []
+    for t in range(n_tiles):
+        sh = w.shapes[t % len(w.shapes)]
+        gen = S.generator(seed * 7919 + t)
+        packed = S.draw_random_bytes(gen, -(-sh.n // 1024) * q * 4096).numpy()   # one row tile, every slice
+        alpha = S.draw_alpha(gen, q, 32, sh.n, w.g, w.alpha_sigma).numpy()
+        x = S.draw_x(gen, batch, sh.n).numpy()
+        jobs.append((packed, q, 32, sh.n, alpha, x, w.g))
+    return jobs
 
 
 def run_reference(args):
+    """The reference arm: the FP64 oracle as it stands on the host cores (a
+    pool of spawned processes, one 32-row tile per job, one job per core and
+    step), on random tiles of the same four linears."""
     world, rank, _ = _dist_env()
     if rank != 0:
         return
     q, batch = args.q, args.batch
+    g = S.WORKLOADS[WORKLOAD].g
     from threadpoolctl import threadpool_limits
-    threadpool_limits(limits=1)
-    for k in range(args.warmup):
-        _oracle_sample(q, batch, args.ref_rows, seed=100 + k)
-    secs, nbytes = 0.0, 0
-    for k in range(args.steps):
-        s, b = _oracle_sample(q, batch, args.ref_rows, seed=200 + k)
-        secs += s
-        nbytes += b
+    cores = min(_host_cores(), 64)
+    nb = lambda jobs: sum(algorithmic_bytes(j[2], j[3], q, g, batch) for j in jobs)
+    pool = OraclePool(cores)
+    try:
+        for k in range(args.warmup):
+            pool.run(_random_tile_jobs(q, batch, cores, seed=100 + k))
+        secs, nbytes = 0.0, 0
+        for k in range(args.steps):
+            jobs = _random_tile_jobs(q, batch, cores, seed=200 + k)
+            wall, _ = pool.run(jobs)
+            secs += wall
+            nbytes += nb(jobs)
+    finally:
+        pool.close()
+    one = _random_tile_jobs(q, batch, 4, seed=999)
+    with threadpool_limits(limits=1):
+        secs1 = sum(_oracle_job(j)[1] for j in one)
     value = nbytes / secs / 1e9
-    sample = (f"{args.ref_rows} rows of each of the 4 layer linears per step (q={q}, g=128, batch {batch}): "
-              "oracle unpack + FP64 dequantise + matmul, one thread")
+    sample = (f"{cores} random 32-row tiles of the 4 layer linears per step (q={q}, g={g}, batch {batch}), one "
+              f"tile per job on {cores} spawned processes: oracle unpack + FP64 dequantise + matmul")
     out = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "OPT-175B decoder-layer linears (QKV 36864x12288, out 12288x12288, "
-                               f"FC1 49152x12288, FC2 12288x49152), BCQ q={q}, g=128, batch {batch}",
-                   "q": q, "g": 128, "batch": batch, "parallelism": "host cores"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                               f"FC1 49152x12288, FC2 12288x49152), BCQ q={q}, g={g}, batch {batch}",
+                   "q": q, "g": g, "batch": batch, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample, "host_cores": _host_cores(), "cpu_model": _cpu_model(),
+                         "single_thread": {"value": round(nb(one) / secs1 / 1e9, 6), "cores": 1,
+                                           "seconds": round(secs1, 2),
+                                           "sample": "one random tile of each linear, one thread"}},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
@@ -938,6 +1101,332 @@ def run_sweep(args):
             print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# One matrix split over the ranks (--parallel): OPT-175B FC1 by rows with an
+# all-gather, FC2 by inputs with an all-reduce, or the FC1 -> FC2 block with
+# FC1 by rows and FC2 by inputs and one all-reduce.  Total work is fixed as N
+# grows (strong scaling).  The exchange is NCCL (torch.distributed); every
+# kernel reads only its own GPU's memory.
+# ---------------------------------------------------------------------------
+PARALLEL_SHAPES = {"fc1": (49152, 12288), "fc2": (12288, 49152)}
+
+
+def parallel_plans(mode: str, q: int, g: int, world: int, rank: int, shapes=None):
+    """The shard plans of this rank for a --parallel mode: rows (FC1), inputs
+    (FC2) or paired (FC1 by rows, then FC2 by inputs over the same range)."""
+    from weight_only_quantized_bcq_b200 import sharded as T
+    shp = shapes or PARALLEL_SHAPES
+    (m1, n1), (m2, n2) = shp["fc1"], shp["fc2"]
+    if mode == "rows":
+        return [T.plan_rows(m1, n1, q, g, world, rank)]
+    if mode == "inputs":
+        return [T.plan_inputs(m2, n2, q, g, world, rank)]
+    if mode == "paired":
+        assert n2 == m1
+        return list(T.plan_paired(m1, n1, m2, q, g, world, rank))
+    raise ValueError(mode)
+
+
+def parallel_bytes(plans, batch: int):
+    """(algorithmic bytes of the whole matrices, of this rank's shards) per step."""
+    whole = sum(algorithmic_bytes(p.m, p.n, p.q, p.g, batch) for p in plans)
+    mine = sum(algorithmic_bytes(p.local_m, p.local_n, p.q, p.g, batch) for p in plans)
+    return whole, mine
+
+
+def parallel_step(mode: str, lins, x):
+    """One step of a --parallel mode: the shard products and their exchange."""
+    from weight_only_quantized_bcq_b200 import sharded as T
+    if mode == "paired":
+        return T.paired_block(lins[0], lins[1], x)
+    return lins[0](x)
+
+
+def run_parallel(args):
+    import datetime
+    import torch.distributed as dist
+    from weight_only_quantized_bcq_b200 import lutgemm
+    from weight_only_quantized_bcq_b200 import sharded as T
+    world, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if "MASTER_ADDR" not in os.environ:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT="29533")
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120),
+                            device_id=device)
+    q, batch, g = args.q, args.batch, S.WORKLOADS[WORKLOAD].g
+    plans = parallel_plans(args.parallel, q, g, world, rank)
+    gen = S.generator(rank_seed(rank))
+    lins = []
+    for p in plans:
+        packed = S.draw_random_bytes(gen, lutgemm.packed_bytes(q, p.local_m, p.local_n)).to(device)
+        alpha = S.draw_alpha(gen, q, p.local_m, p.local_n, g, 0.02).to(device)
+        lins.append(T.ShardedLinear.from_packed(p, packed, alpha, batch=batch))
+    # Every rank draws the same x (same seed): the input the matrix multiplies.
+    n_in = plans[0].n
+    x_host = S.draw_x(S.generator(77), batch, n_in).pin_memory()
+    x = x_host.to(device)
+    x_in = T.take_input_slice(plans[0], x) if args.parallel == "inputs" else x
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, steps):
+        barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            fn()
+        t1.record(stream)
+        barrier()
+        return max_over_ranks(dist, t0.elapsed_time(t1), device)
+
+    for _ in range(args.warmup):
+        parallel_step(args.parallel, lins, x_in)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        region_ms = timed(lambda: parallel_step(args.parallel, lins, x_in), args.steps)
+    y = parallel_step(args.parallel, lins, x_in)
+
+    # The products alone (no exchange), to give the collective's share.
+    def products_only():
+        if args.parallel == "paired":
+            h = lins[0].local_product(x_in)
+            lins[1].local_product(h.to(torch.float16))
+        else:
+            lins[0].local_product(x_in if args.parallel == "rows" else x_in)
+    prod_ms = timed(products_only, args.steps)
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        xi = T.take_input_slice(plans[0], x) if args.parallel == "inputs" else x
+        y_host.copy_(parallel_step(args.parallel, lins, xi), non_blocking=True)
+    e2e_ms = timed(e2e_step, args.steps)
+
+    whole, mine = parallel_bytes(plans, batch)
+    value = whole * args.steps / (region_ms * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    if rank == 0:
+        names = {"rows": "OPT-175B FC1 (49152x12288) split by rows, all-gather of y",
+                 "inputs": "OPT-175B FC2 (12288x49152) split by inputs, all-reduce of y",
+                 "paired": "OPT-175B FC1 -> FC2 block, FC1 by rows and FC2 by inputs, one all-reduce"}
+        out = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": names[args.parallel] + f", BCQ q={q}, g={g}, batch {batch}", "q": q, "g": g,
+                       "batch": batch, "parallelism": f"tp{world} ({args.parallel})",
+                       "bytes_per_step_whole": whole, "bytes_per_step_rank0": mine,
+                       "l2": "no flush: every step streams each shard's weights once; a shard below 126 MB "
+                             "may stay in L2 at large N",
+                       "launch": "eager launches; collectives by torch.distributed (NCCL)"},
+            "products_ms_per_step": round(prod_ms / args.steps, 5),
+            "collective_share": round(max(0.0, 1.0 - prod_ms / region_ms), 4),
+            "roofline": {"bound": "hbm", "achieved": round(mine * args.steps / (region_ms * 1e-3) / 1e9, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(mine * args.steps / (region_ms * 1e-3) / 1e9 / peak, 4), "traffic": None,
+                         "peak_kind": peak_kind, "kernel": "lut_gemm_kernel (one rank's shards, exchange included)"},
+            "e2e": {"value": round(whole * args.steps / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host.numel() * 4},
+            "gpu_launches": args.steps * sum(1 + (p.local_n > 1024) for p in plans),
+            "gpu_launches_note": "lookup kernel and split-K reduce per shard product; NCCL kernels not counted",
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(out), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# Mixed storage (2/4/16-bit in one matrix): the LLaMA-70B-shaped linears with
+# 2-plane blocks, a fraction of 4-plane blocks and sparse fp16 outliers,
+# through lutgemm_run_mixed.
+# ---------------------------------------------------------------------------
+MIXED_METRIC = "Mixed 2/4/16-bit LUT-GEMM (lutgemm_run_mixed): achieved HBM GB/s at batch 1"
+MIXED_SHAPES = (("llama70b_qkvo", 8192, 8192), ("llama70b_up", 28672, 8192), ("llama70b_down", 8192, 28672))
+
+
+def _mixed_layer(q_max, g, batch, frac_hi, density, seed, device, reps):
+    from weight_only_quantized_bcq_b200 import lutgemm
+    from weight_only_quantized_bcq_b200.roofline import mixed_algorithmic_bytes
+    gen = S.generator(seed)
+    mats = []
+    for name, m, n in MIXED_SHAPES:
+        bp = S.draw_block_planes(gen, m, n, frac_hi, lo=2, hi=q_max)
+        boff_h = lutgemm.mixed_offsets(bp, q_max, m, n)
+        nbytes = int(boff_h[-1]) * 4096
+        copies_h = [S.draw_random_bytes(gen, nbytes) for _ in range(reps)]
+        alpha_h = S.draw_alpha(gen, q_max, m, n, g, 0.03)
+        x_h = S.draw_x(gen, batch, n, outlier_frac=0.001).pin_memory()
+        rp, col, val = S.draw_outliers(gen, m, n, density)
+        optr, oent = lutgemm.pack_outliers(rp, col, val, m, n)
+        mats.append({"name": name, "m": m, "n": n, "bp": bp, "boff": boff_h.to(device),
+                     "copies": [c.to(device) for c in copies_h], "packed_host": copies_h[-1],
+                     "alpha": alpha_h.to(device), "alpha_host": alpha_h, "x_host": x_h, "x": x_h.to(device),
+                     "outliers_host": (rp, col, val), "optr": optr.to(device), "oent": oent.to(device),
+                     "y": torch.empty((batch, m), dtype=torch.float32, device=device),
+                     "y_host": torch.empty((batch, m), dtype=torch.float32).pin_memory(),
+                     "ws": lutgemm.new_workspace(m, n, batch, q_max, g, device=device),
+                     "bytes": mixed_algorithmic_bytes(bp.numpy(), m, n, g, batch, col.numel()),
+                     "nnz": col.numel(), "avg_planes": float(bp.float().mean())})
+    return mats
+
+
+def run_mixed_workload(args):
+    from weight_only_quantized_bcq_b200 import lutgemm
+    world, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    q_max, g, batch = 4, 64, args.batch
+    reps = 2      # weight copies used in turn: consecutive steps miss L2
+    mats = _mixed_layer(q_max, g, batch, args.mixed_hi, args.mixed_outliers, rank_seed(rank), device, reps)
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
+
+    def one(mt, k):
+        lutgemm.run_mixed(mt["copies"][k % reps], mt["boff"], mt["alpha"], mt["x"], mt["m"], mt["n"], q_max, g,
+                          optr=mt["optr"], oent=mt["oent"], y=mt["y"], workspace=mt["ws"], stream=stream)
+
+    def step(k, events=None):
+        for i, mt in enumerate(mats):
+            if events is not None:
+                events[i][0].record(stream)
+            one(mt, k)
+            if events is not None:
+                events[i][1].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    for k in range(args.warmup):
+        step(k)
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier()
+        t0.record(stream)
+        for k in range(args.steps):
+            step(k)
+        t1.record(stream)
+        barrier()
+    region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
+    k_last = args.steps - 1
+    y_timed = [mt["y"].cpu().clone() for mt in mats]
+    status = [lutgemm.workspace_status(mt["ws"]) for mt in mats]
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in mats]
+          for _ in range(args.steps)]
+    for k in range(args.steps):
+        step(k, ev[k])
+    barrier()
+    us_per = {mt["name"]: 1e3 * statistics.median(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps))
+              for i, mt in enumerate(mats)}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for k in range(args.steps):
+        for mt in mats:
+            mt["x"].copy_(mt["x_host"], non_blocking=True)
+        step(k)
+        for mt in mats:
+            mt["y_host"].copy_(mt["y"], non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1), device)
+    step_bytes = sum(mt["bytes"] for mt in mats)
+    value = step_bytes * args.steps * world / (region_ms * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    if rank == 0:
+        out = {
+            "metric": MIXED_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "LLaMA-70B-shaped linears (8192x8192, 28672x8192, 8192x28672), mixed storage: "
+                                   f"2-plane blocks, {args.mixed_hi:.3f} of blocks at 4 planes, "
+                                   f"{100 * args.mixed_outliers:.2f}% fp16 outliers, g={g}, batch {batch}",
+                       "q_max": q_max, "g": g, "batch": batch, "frac_4plane_blocks": args.mixed_hi,
+                       "outlier_density": args.mixed_outliers, "bytes_per_step": step_bytes,
+                       "avg_planes": {mt["name"]: round(mt["avg_planes"], 3) for mt in mats},
+                       "l2": f"two weight copies used in turn: {2 * step_bytes / 1e6:.0f} MB between reuses "
+                             "(> 126 MB L2)",
+                       "parallelism": "replicas" if world == 1 else f"replicas{world}"},
+            "us_per_matmul": {k: round(v, 2) for k, v in us_per.items()},
+            "us_per_matmul_note": "median of isolated launches (events around each launch)",
+            "gbs_per_matmul": {mt["name"]: round(mt["bytes"] / (us_per[mt["name"]] * 1e-6) / 1e9, 1) for mt in mats},
+            "hbm_floor_us": {mt["name"]: round(mt["bytes"] / (peak * 1e3), 2) for mt in mats},
+            "roofline": {"bound": "hbm", "achieved": round(step_bytes * args.steps / (region_ms * 1e-3) / 1e9, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(step_bytes * args.steps / (region_ms * 1e-3) / 1e9 / peak, 4),
+                         "traffic": None, "peak_kind": peak_kind, "kernel": "lut_gemm_kernel (mixed)"},
+            "e2e": {"value": round(step_bytes * args.steps * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
+                    "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
+            "gpu_launches": args.steps * len(mats) * 2,
+            "device_status": status,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"], out["parity"] = cpu_mixed_baseline(mats, q_max, g, batch, y_timed, k_last % reps)
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def cpu_mixed_baseline(mats, q_max, g, batch, y_timed, copy_index):
+    """The oracle on 8 row tiles of each linear (first and last included) of
+    the copy the last timed step used, one thread: its rate, and the timed
+    outputs compared with it on those rows."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    from oracle import bcq_oracle as O
+    from tests._tol import compare
+    rng = np.random.default_rng(3)
+    secs, nbytes, per, ok_all = 0.0, 0, {}, True
+    for mt_, y in zip(mats, y_timed):
+        mtiles = -(-mt_["m"] // 32)
+        tiles = np.unique(np.r_[0, mtiles - 1, rng.choice(mtiles, 6, replace=False)])
+        packed = mt_["copies"][copy_index].cpu().numpy()
+        outl = tuple(t.numpy() for t in mt_["outliers_host"])
+        with threadpool_limits(limits=1):
+            t = time.perf_counter()
+            y_ref, rows = O.mixed_matmul_tiles(mt_["x_host"].numpy(), packed, mt_["bp"].numpy(),
+                                               mt_["alpha_host"].numpy(), g, mt_["m"], mt_["n"], tiles, outl)
+            secs += time.perf_counter() - t
+        a = mt_["alpha_host"].numpy().astype(np.float64)[:, :, rows].copy()
+        bp = mt_["bp"].numpy()
+        for G in range(mt_["n"] // g):
+            for ti, R in enumerate(tiles):
+                a[bp[(G * g) // 1024, R]:, G, 32 * ti: 32 * ti + 32] = 0.0
+        ok, st = compare(y.numpy()[:, rows], y_ref, a, mt_["x_host"].numpy(), mt_["n"])
+        per[mt_["name"]] = {"rows": int(rows.size), "rel_l2": st["rel_l2"],
+                            "max_abs_over_bound": round(st["max_abs_over_bound"], 5)}
+        ok_all = ok_all and ok
+        frac = rows.size / mt_["m"]
+        nbytes += int(mt_["bytes"] * frac)
+    base = {"value": round(nbytes / secs / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(secs, 2), "cpu_model": _cpu_model(),
+            "sample": "8 row tiles of each linear of this run's weights: oracle unpack of each block, FP64 "
+                      "mixed dequantise + outliers + matmul, one thread"}
+    return base, {"ok": bool(ok_all), "per_linear": per,
+                  "what": "the last timed step's y against the FP64 oracle on the sampled rows"}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -947,7 +1436,6 @@ def main():
     ap.add_argument("--q", type=int, default=3)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-rows", type=int, default=512, help="rows per linear in the CPU baseline sample")
-    ap.add_argument("--ref-rows", type=int, default=64, help="rows per linear per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph-steps", type=int, default=10,
                     help="steps per captured CUDA graph in the timed region (0: eager launches)")
@@ -955,7 +1443,11 @@ def main():
                     help="scale layout lutgemm_run reads (packed: unit-major, reordered at load time)")
     ap.add_argument("--only", choices=[sh.name for sh in S.WORKLOADS[WORKLOAD].shapes], default=None,
                     help="time one linear of the layer only (profiling)")
-    ap.add_argument("--workload", choices=["layer", "fit", "sweep", "tc"], default="layer",
+    ap.add_argument("--parallel", choices=["rows", "inputs", "paired"], default=None,
+                    help="split one matrix over the --gpus ranks (strong scaling, NCCL exchange)")
+    ap.add_argument("--mixed-hi", type=float, default=0.125, help="mixed workload: fraction of 4-plane blocks")
+    ap.add_argument("--mixed-outliers", type=float, default=0.005, help="mixed workload: fp16 outlier density")
+    ap.add_argument("--workload", choices=["layer", "fit", "sweep", "tc", "mixed"], default="layer",
                     help="layer: the LUT-GEMM step (default); fit: BCQ fitting of FP16 weights; "
                          "sweep: every parity config shape and batch, one line each; "
                          "tc: the layer's linears at a large batch on the tensor-core path")
@@ -973,8 +1465,12 @@ def main():
     args = ap.parse_args()
     # At least three untimed warm-up steps, whatever the caller asks for.
     args.warmup = max(3, args.warmup)
-    if args.workload == "sweep":
+    if args.parallel is not None and args.impl == "lutgemm":
+        run_parallel(args)
+    elif args.workload == "sweep":
         run_sweep(args)
+    elif args.workload == "mixed":
+        run_mixed_workload(args)
     elif args.workload == "tc":
         if args.impl == "reference":
             world, rank, _ = _dist_env()

@@ -20,8 +20,9 @@
  * Conventions shared by every call
  *   - Every buffer is caller-owned and caller-allocated.  The library
  *     allocates nothing and keeps no state between calls, except that the
- *     workspace of lutgemm_run must be zero-filled once before its first use
- *     and is left zero-filled again by every call that returns LUTGEMM_OK.
+ *     workspace of lutgemm_run must be zero-filled once before its first use;
+ *     its tile counters are left zero by every call, and its status word
+ *     keeps its bits until lutgemm_workspace_status clears them.
  *   - "dev" pointers are CUDA device pointers on the current device; fp16
  *     values are passed as their raw 16-bit patterns (uint16_t).
  *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
@@ -29,6 +30,16 @@
  *   - Arguments are validated before anything is enqueued: a status other
  *     than LUTGEMM_OK means no work was enqueued (LUTGEMM_ERR_CUDA: the launch
  *     itself failed, as reported by cudaGetLastError).
+ *   - A status returned by a call describes the enqueueing only: the kernels
+ *     run later.  A kernel that fails while it runs (a bounded wait inside
+ *     it ran out, or its shared-memory window is not where its tables are
+ *     placed) does not hang or fault: it ORs a LUTGEMM_STATUS_* bit into a
+ *     sticky status word and its outputs are not valid.  The word of a
+ *     lutgemm_run call is the first 4 bytes of its workspace
+ *     (lutgemm_workspace_status reads it); lutgemm_run_tc and
+ *     lutgemm_run_noalloc use words held by the library
+ *     (lutgemm_library_status reads them).  A caller that must know that
+ *     y is valid reads the word after the calls it covers.
  *   - Values that can only be checked on the device (a sign that is not +-1,
  *     a code or zero-point >= 2^q) are reported through an optional
  *     device int32 *status_flags: the kernel ORs LUTGEMM_FLAG_* bits into it.
@@ -97,11 +108,29 @@ extern "C" {
 #define LUTGEMM_FLAG_BAD_SIGN  1  /* lutgemm_pack_bcq: a sign was neither -1 nor +1 */
 #define LUTGEMM_FLAG_BAD_CODE  2  /* lutgemm_uniform_to_bcq: a code >= 2^q */
 #define LUTGEMM_FLAG_BAD_ZERO  4  /* lutgemm_uniform_to_bcq: a zero-point >= 2^q */
+#define LUTGEMM_FLAG_BAD_BLOCK 8  /* lutgemm_pack_bcq_mixed: a block-table entry out of range (block not written) */
+
+/* Bits of the sticky status word a kernel sets when it fails while it runs
+ * (read with lutgemm_workspace_status / lutgemm_library_status).  Any bit
+ * set means the outputs of the calls since the word was last cleared are
+ * not valid. */
+#define LUTGEMM_STATUS_WINDOW  1u /* the lookup kernel's shared-memory window does not start where its
+                                     tables are placed: nothing was computed */
+#define LUTGEMM_STATUS_TIMEOUT 2u /* a bounded wait on a copy or an MMA ran out (1 s): the kernel stopped */
+#define LUTGEMM_STATUS_FORMAT  4u /* lutgemm_run_mixed: a block-table entry or an outlier entry was out of
+                                     range; the rows it touches are not valid */
 
 /* Flags of lutgemm_run. */
 #define LUTGEMM_Y_F16          1u /* write y as fp16 (round to nearest even of the fp32 sum) */
 #define LUTGEMM_SCALES_PACKED  2u /* alpha is in the unit-major scale layout (g % 128 == 0) */
 #define LUTGEMM_ALLOW_TENSOR_CORES 4u /* lutgemm_run may compute on the tensor cores (see there) */
+/* Test hook of lutgemm_run and lutgemm_run_noalloc, for checking error
+ * reporting: every warp of the lookup kernel makes its first weight wait on
+ * a barrier that nothing signals, gives up after 1 ms, lets its copies in
+ * flight land and stops, so the call sets LUTGEMM_STATUS_TIMEOUT and y is
+ * not valid.  The tensor-core path is not taken with this flag.  Not for
+ * production use. */
+#define LUTGEMM_TEST_STALL     0x80000000u
 
 /* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
 int lutgemm_version(void);
@@ -119,10 +148,43 @@ size_t lutgemm_packed_bytes(int q, int m, int n);
  * invalid shapes and when g % 128 != 0.  Pure host function. */
 size_t lutgemm_scales_bytes(int q, int m, int n, int g);
 
-/* Bytes of the lutgemm_run workspace (split-K partial sums, per-slice tile
- * counters and a status word).  Returns 0 for invalid shapes.  Pure host
- * function. */
+/* Bytes of the lutgemm_run workspace: [status word, 256 B | per-segment tile
+ * counters, 4 KB | split-K partial sums, batch * ceil(n/1024) *
+ * ceil(m/32) * 128 B rounded up to 256 B].  Returns 0 for invalid shapes.
+ * Pure host function. */
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g);
+
+/* Read the sticky status word of a lutgemm_run workspace: waits for the work
+ * enqueued on `stream` so far (cudaStreamSynchronize), stores the word's
+ * LUTGEMM_STATUS_* bits in *status (host) and, when clear != 0 and a bit is
+ * set, enqueues its reset to 0 on `stream`.  0 means every lutgemm_run on
+ * this workspace since the last clear ran to the end.  Synchronous: not for
+ * use inside a stream capture.
+ *   workspace        dev, 16-byte aligned, as given to lutgemm_run
+ *   workspace_bytes  at least 256 + 4096
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_ALIGN, ERR_WORKSPACE or ERR_CUDA. */
+int lutgemm_workspace_status(void* workspace, size_t workspace_bytes, uint32_t* status, int clear, void* stream);
+
+/* The same for the status words the library holds on the current device,
+ * OR-ed together: the one of lutgemm_run_noalloc (in its scratch array) and
+ * the one lutgemm_run_tc uses.  The first call on a device does the set-up
+ * lutgemm_run_noalloc describes.  Synchronous, like lutgemm_workspace_status.
+ * Returns LUTGEMM_OK, ERR_NULL or ERR_CUDA. */
+int lutgemm_library_status(uint32_t* status, int clear, void* stream);
+
+/* How lutgemm_run spreads the lookup kernel over `sm_count` SMs: the same
+ * choice the call makes (pure host function).  Outputs (host):
+ *   *grid           CTAs launched (one persistent 512-thread CTA per SM)
+ *   *seg_aligned    1 when every (batch column, slice) segment gets its own
+ *                   group of CTAs, whose warps take two row tiles each and
+ *                   the rest of the segment's tiles from a per-segment tile
+ *                   counter; 0 when the list of (batch column, slice, row
+ *                   tile) units is cut into one contiguous range per CTA
+ *   *dynamic_tiles  row tiles taken through the counters, summed over the
+ *                   segments (0 when *seg_aligned is 0)
+ * m, batch, sm_count >= 1, n >= 8, n % 8 == 0.
+ * Returns LUTGEMM_OK, ERR_NULL or ERR_SHAPE. */
+int lutgemm_launch_plan(int m, int n, int batch, int sm_count, int* grid, int* seg_aligned, int* dynamic_tiles);
 
 /* The tensor-core plan lutgemm_run uses with LUTGEMM_ALLOW_TENSOR_CORES: the
  * number of K splits it runs tc_gemm with (whole 1024-input slices, at most
@@ -300,6 +362,83 @@ int lutgemm_run_tc(int m, int n, int batch, int q, int g,
                    const uint8_t* packed, const uint16_t* alpha,
                    const float* offset, const uint16_t* x, void* y,
                    unsigned flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Mixed storage: 2-, 4- and 16-bit weights in one matrix (OpenAlex record
+ * "Fast and Efficient 2-bit LLM Inference on GPU: 2/4/16-bit in a Weight
+ * Matrix with Asynchronous Dequantization", abstract: weights are quantised
+ * by groups, wide-range groups need more bits, and sparse outliers are kept
+ * in 16 bits; the record gives no format).  This library's format:
+ *   - a precision block is 32 rows x 1024 inputs (row tile R, slice s, the
+ *     unit the lookup kernel streams); block (s, R) stores q_b planes,
+ *     1 <= q_b <= q_max <= 4 (for example 2 for most blocks, 4 for blocks
+ *     with a wide range);
+ *   - W[j,k] = sum_{i < q_b} alpha[i][k/g][j] * beta[i][j][k] + S[j,k],
+ *     S a sparse fp16 matrix (the outliers), added to the BCQ value;
+ *   - block_planes  uint8 [n_s][m_t]: q_b of block (s, R);
+ *   - block table   uint32 [n_s*m_t + 1]: the exclusive prefix sum of q_b
+ *     in (s, R) order, in 4096-byte units (lutgemm_mixed_offsets); the last
+ *     entry is the total, and the packed buffer holds 4096 * total bytes;
+ *   - packed planes: block (s, R) occupies q_b * 4096 bytes from byte
+ *     4096 * table[s*m_t + R]; inside it chunk (U, i) (U < 8, i < q_b)
+ *     sits at (U * q_b + i) * 512, with the byte map of the uniform layout
+ *     (so all q_b = q gives lutgemm_pack_bcq's buffer);
+ *   - alpha fp16 [q_max][n/g][m]: entries of planes a block does not store
+ *     are never read;
+ *   - outliers, as the caller gives them: row CSR, row_ptr int32 [m+1],
+ *     col int32 [nnz] strictly increasing within a row, val fp16 [nnz];
+ *     as the kernel reads them (lutgemm_pack_outliers): slice-major CSR,
+ *     optr uint32 [n_s*m + 1] with the entries of (slice s, row r) at
+ *     [optr[s*m + r], optr[s*m + r + 1]) sorted by input, each entry a
+ *     uint32 (k - 1024 s) | (fp16 bits << 16).
+ * ------------------------------------------------------------------------- */
+
+/* The block table of a mixed matrix, on the host (pure host function).
+ *   block_planes  host uint8 [ceil(n/1024)][ceil(m/32)], each in [1, q_max]
+ *   q_max         1..4;  m >= 1, n >= 8, n % 8 == 0
+ *   offsets       host uint32 [ceil(n/1024)*ceil(m/32) + 1] (output)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also when the total exceeds
+ * 2^32 - 1 blocks) or ERR_VALUE (a plane count out of range). */
+int lutgemm_mixed_offsets(const uint8_t* block_planes, int q_max, int m, int n, uint32_t* offsets);
+
+/* Pack the planes of a mixed matrix: block (s, R) stores planes 0..q_b-1.
+ *   signs         dev int8 [q_max][m][n], 8-byte aligned; the signs of planes
+ *                 a block does not store are not read
+ *   block_off     dev uint32 block table (lutgemm_mixed_offsets), 4-byte aligned
+ *   packed        dev, packed_bytes = 4096 * (the table's last entry),
+ *                 16-byte aligned; every stored byte is written
+ *   status_flags  dev int32 or NULL: LUTGEMM_FLAG_BAD_SIGN as for
+ *                 lutgemm_pack_bcq; LUTGEMM_FLAG_BAD_BLOCK for a table entry
+ *                 with no plane, more than q_max planes or past packed_bytes
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_VALUE (packed_bytes
+ * not a multiple of 4096 or below one plane per block) or ERR_CUDA. */
+int lutgemm_pack_bcq_mixed(const int8_t* signs, const uint32_t* block_off, int q_max, int m, int n,
+                           uint8_t* packed, size_t packed_bytes, int32_t* status_flags, void* stream);
+
+/* Row-CSR outliers -> the slice-major layout the kernel reads (pure host
+ * function; all pointers host).  optr: uint32 [ceil(n/1024)*m + 1];
+ * oent: uint32 [nnz].  Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE or ERR_VALUE
+ * (row_ptr not from 0 to nnz and non-decreasing, a column outside [0, n), or
+ * columns not strictly increasing within a row). */
+int lutgemm_pack_outliers(const int32_t* row_ptr, const int32_t* col, const uint16_t* val, int m, int n, int nnz,
+                          uint32_t* optr, uint32_t* oent);
+
+/* y = W x for a mixed matrix, by the lookup kernel: the same tables, with
+ * each block's own plane count, and each row's outliers added after its
+ * planes (w * x in fp32, in entry order), so repeated calls give identical
+ * bits.  Operands as described above; x, y, flags (LUTGEMM_Y_F16, or the
+ * test hook LUTGEMM_TEST_STALL) and workspace (lutgemm_workspace_size with
+ * q = q_max) as lutgemm_run.  optr and oent may be NULL when nnz == 0.
+ * The kernel checks every block-table and outlier entry it uses against
+ * packed_bytes, q_max, nnz and n; one out of range sets
+ * LUTGEMM_STATUS_FORMAT in the workspace's status word instead of reading
+ * outside the buffers.
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also q_max outside 1..4),
+ * ERR_VALUE, ERR_ALIGN, ERR_WORKSPACE or ERR_CUDA. */
+int lutgemm_run_mixed(int m, int n, int batch, int q_max, int g, const uint8_t* packed, size_t packed_bytes,
+                      const uint32_t* block_off, const uint16_t* alpha, const uint32_t* optr, const uint32_t* oent,
+                      int nnz, const uint16_t* x, void* y, unsigned flags, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 /* Bytes of the device scratch array used by lutgemm_run_noalloc (16 MiB). */
 #define LUTGEMM_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -62,6 +62,7 @@ __all__ = [
     "fit_bcq_grid", "fit_bcq_grid_trace", "nearest_grid_codes",
     "mixed_block_offsets", "mixed_packed_nbytes", "pack_mixed", "unpack_mixed",
     "mixed_weights", "mixed_matmul", "pack_outliers", "unpack_outliers", "outlier_dense",
+    "mixed_matmul_tiles",
 ]
 
 
@@ -665,7 +666,7 @@ def unpack_mixed(packed, block_planes, q_max: int, m: int, n: int) -> np.ndarray
             r0, k0 = TILE_ROWS * R, SLICE * s_
             mr, nk = min(m, r0 + TILE_ROWS) - r0, min(n, k0 + SLICE) - k0
             blk = pk[int(off[u]) * BLOCK_BYTES: int(off[u + 1]) * BLOCK_BYTES]
-            out[:qb, r0: r0 + mr, k0: k0 + nk] = unpack_bcq(blk, qb, mr, nk)
+            out[:qb, r0: r0 + mr, k0: k0 + nk] = unpack_bcq_vec(blk, qb, mr, nk)
     return out
 
 
@@ -739,3 +740,44 @@ def unpack_outliers(optr, oent, m: int, n: int) -> np.ndarray:
                 k = SLICE * s_ + int(oent[e] & 0xFFFF)
                 S_[r, k] = float(np.uint16(oent[e] >> 16).view(np.float16))
     return S_
+
+
+def mixed_matmul_tiles(x, packed, block_planes, alpha, g: int, m: int, n: int, tiles, outliers=None):
+    """``mixed_matmul`` restricted to the rows of the given row tiles, read
+    straight from a mixed packed buffer: each block of those tiles is
+    unpacked, the rows' scales and outliers are taken, and the product is the
+    plain definition on that sub-matrix.  Returns (y [batch][rows], rows)."""
+    pk = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    bp = _check_blocks(block_planes, m, n)
+    off = mixed_block_offsets(bp)
+    a = np.asarray(alpha)
+    q_max = a.shape[0]
+    ns, mt = bp.shape
+    tiles = np.asarray(tiles, dtype=np.int64)
+    rows = (TILE_ROWS * tiles[:, None] + np.arange(TILE_ROWS)[None, :]).reshape(-1)
+    rows = rows[rows < m]
+    signs = np.zeros((q_max, rows.size, n), dtype=np.int8)
+    r0 = 0
+    for R in tiles:
+        mr = min(m, TILE_ROWS * (int(R) + 1)) - TILE_ROWS * int(R)
+        for s_ in range(ns):
+            u = s_ * mt + int(R)
+            qb = int(bp[s_, R])
+            k0 = SLICE * s_
+            nk = min(n, k0 + SLICE) - k0
+            blk = pk[int(off[u]) * BLOCK_BYTES: int(off[u + 1]) * BLOCK_BYTES]
+            signs[:qb, r0: r0 + mr, k0: k0 + nk] = unpack_bcq_vec(blk, qb, mr, nk)
+        r0 += mr
+    sub = None
+    if outliers is not None:
+        rp, col, val = (np.asarray(t) for t in outliers)
+        sub_rp, sub_col, sub_val = [0], [], []
+        for r in rows:
+            sub_col.extend(col[rp[r]: rp[r + 1]].tolist())
+            sub_val.extend(val[rp[r]: rp[r + 1]].tolist())
+            sub_rp.append(len(sub_col))
+        sub = (np.asarray(sub_rp), np.asarray(sub_col, dtype=np.int64), np.asarray(sub_val, dtype=np.float16))
+    # The sub-matrix's row tiles are the chosen tiles in order, so its block
+    # plane counts are those columns of block_planes.
+    y = mixed_matmul(x, signs, a[:, :, rows], bp[:, tiles], g, sub)
+    return y, rows

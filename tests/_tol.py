@@ -35,3 +35,19 @@ def compare(y, y_ref, alpha, x, n: int):
     ok = finite and rel <= REL_L2 and ratio <= 1.0
     return ok, {"rel_l2": rel, "max_abs_over_bound": ratio, "max_abs": float(err.max(initial=0.0)),
                 "finite": finite}
+
+
+def compare_f16(y16, y_ref, alpha, x, n: int):
+    """fp16 output against the FP64 oracle: the fp16 mode is RNE of the fp32
+    sum, so |y16 - y_ref| <= half an fp16 ulp (taken at the larger of |y16|,
+    |y_ref|, which covers rounding up into the next binade) plus the fp32
+    per-output bound.  Returns (ok, stats)."""
+    y16 = np.asarray(y16, dtype=np.float16)
+    y = y16.astype(np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    half_ulp = 0.5 * np.spacing(np.maximum(np.abs(y), np.abs(y_ref)).astype(np.float16)).astype(np.float64)
+    bound = half_ulp + abs_bound(alpha, x, n)
+    err = np.abs(y - y_ref)
+    ratio = float((err / bound).max()) if err.size else 0.0
+    finite = bool(np.all(np.isfinite(y)))
+    return finite and ratio <= 1.0, {"max_err_over_bound": ratio, "finite": finite}

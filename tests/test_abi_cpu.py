@@ -66,7 +66,7 @@ def test_workspace_size(L):
     ns, mt = math.ceil(n / 1024), math.ceil(m / 32)
     part = b * ns * mt * 32 * 4
     rup = lambda v: (v + 255) // 256 * 256
-    assert L.workspace_size(m, n, b, 3, 128) == rup(part) + 4096 + 256   # + tile counters, status word
+    assert L.workspace_size(m, n, b, 3, 128) == 256 + 4096 + rup(part)   # status word, tile counters, partials
     assert L.workspace_size(m, n, 0, 3, 128) == 0
     assert L.workspace_size(m, n, 1, 3, 100) == 0          # g % 8 != 0
     assert L.workspace_size(m, 12288, 1, 3, 5000) == 0     # n % g != 0
@@ -277,3 +277,63 @@ def test_binding_signatures_match_the_header(L):
         want = kinds.get(ret.replace("const", "").strip())
         if want is not None:
             assert restype is want, (name, ret, restype)
+
+
+# ---------------------------------------------------------------------------
+# The launch plan query and the status-word calls' host-side validation.
+# ---------------------------------------------------------------------------
+def _plan(L, m, n, batch, sms=148):
+    return L.launch_plan(m, n, batch, sms)
+
+
+def test_launch_plan_matches_the_kernels_grouping(L):
+    # 37 batch columns x 4 slices = 148 segments, one CTA each: 64 row tiles
+    # per segment, 32 of them static, so 32 per segment come from the counters.
+    assert _plan(L, 2048, 4096, 37) == (148, 1, 148 * 32)
+    # OPT-175B FC1 at batch 1: 12 segments of 12 CTAs (144 launched), 384
+    # static tiles and 1152 dynamic ones per segment.
+    assert _plan(L, 49152, 12288, 1) == (144, 1, 12 * 1152)
+    # Two tiles: one CTA per tile, no counters needed.
+    assert _plan(L, 64, 1024, 1) == (2, 1, 0)
+    # More segments than SMs: the unit list is cut into contiguous ranges.
+    assert _plan(L, 64, 1024, 200) == (148, 0, 0)
+
+
+def test_launch_plan_group_sizes_are_the_kernels():
+    """The dynamic count is the sum over segments of mt - 32 * (CTAs of the
+    segment), with the kernel's own rule for a segment's CTA count."""
+    from weight_only_quantized_bcq_b200 import lutgemm as L
+    L.lib()
+    for (m, n, b) in [(2048, 4096, 37), (12600, 12288, 1), (40000, 2048, 3)]:
+        grid, aligned, dyn = _plan(L, m, n, b)
+        segs = b * math.ceil(n / 1024)
+        mt = math.ceil(m / 32)
+        if aligned:
+            want = sum(max(0, mt - 32 * ((grid - z + segs - 1) // segs)) for z in range(segs))
+            assert dyn == want
+
+
+def test_launch_plan_rejects_bad_arguments(L):
+    lib = L.lib()
+    import ctypes
+    a = ctypes.c_int(0)
+    assert lib.lutgemm_launch_plan(64, 1024, 1, 148, None, ctypes.byref(a), ctypes.byref(a)) == L.ERR_NULL
+    for args in [(0, 1024, 1, 148), (64, 12, 1, 148), (64, 1024, 0, 148), (64, 1024, 1, 0)]:
+        assert lib.lutgemm_launch_plan(*args, ctypes.byref(a), ctypes.byref(a), ctypes.byref(a)) == L.ERR_SHAPE
+
+
+def test_status_calls_validate_before_touching_the_device(L):
+    lib = L.lib()
+    import ctypes
+    v = ctypes.c_uint32(0)
+    assert lib.lutgemm_workspace_status(None, 1 << 20, ctypes.byref(v), 1, None) == L.ERR_NULL
+    assert lib.lutgemm_workspace_status(FAKE, 1 << 20, None, 1, None) == L.ERR_NULL
+    assert lib.lutgemm_workspace_status(FAKE + 4, 1 << 20, ctypes.byref(v), 1, None) == L.ERR_ALIGN
+    assert lib.lutgemm_workspace_status(FAKE, 256 + 4095, ctypes.byref(v), 1, None) == L.ERR_WORKSPACE
+    assert lib.lutgemm_library_status(None, 1, None) == L.ERR_NULL
+
+
+def test_test_stall_flag_is_accepted_by_validation_only_with_valid_arguments(L):
+    # The flag passes flag validation (the call then fails on the null pointer).
+    assert _run(L, flags=L.TEST_STALL, packed=None) == L.ERR_NULL
+    assert _run(L, flags=L.TEST_STALL | 8) == L.ERR_VALUE

@@ -15,7 +15,7 @@ import torch
 
 import bcq_synth as S
 from oracle import bcq_oracle as O
-from tests._tol import compare
+from tests._tol import compare, compare_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -307,8 +307,8 @@ def test_y_f16_is_rounded_fp32(L):
     assert y16.dtype == torch.float16
     assert torch.equal(y16, y32.to(torch.float16))
     y_ref = O.bcq_matmul(x.numpy(), signs.numpy(), alpha.numpy(), 128)
-    ulp = np.spacing(np.abs(y_ref).astype(np.float16)).astype(np.float64)
-    assert np.all(np.abs(y16.float().cpu().numpy() - y_ref) <= ulp)
+    ok, st = compare_f16(y16.cpu().numpy(), y_ref, alpha.numpy(), x.numpy(), 3072)
+    assert ok, st
 
 
 def test_deterministic_and_workspace_reuse(L):
@@ -326,12 +326,11 @@ def test_deterministic_and_workspace_reuse(L):
     y3_ref = O.bcq_matmul(x2.cpu().numpy(), signs.numpy(), alpha.numpy(), g)
     ok, st = compare(y3.cpu().numpy(), y3_ref, alpha.numpy(), x2.cpu().numpy(), n)
     assert ok, st
-    # The tile counters and the status word follow the 256-aligned partial
-    # sums and are zero again after the calls.
+    # The status word (256 B) and the tile counters (4 KB) come first, then
+    # the 256-aligned partial sums; status and counters are zero after the calls.
     ns, mt = math.ceil(n / 1024), math.ceil(m / 32)
-    tiles_off = (b * ns * mt * 32 * 4 + 255) // 256 * 256
-    assert ws.numel() == tiles_off + 4096 + 256
-    assert not ws[tiles_off:].cpu().numpy().any()
+    assert ws.numel() == 256 + 4096 + (b * ns * mt * 32 * 4 + 255) // 256 * 256
+    assert not ws[: 256 + 4096].cpu().numpy().any()
 
 
 def test_small_workspace_is_rejected(L):

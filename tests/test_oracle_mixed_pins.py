@@ -184,6 +184,16 @@ def test_mixed_roundtrips(q, m, n):
     assert np.array_equal(O.unpack_outliers(optr, oent, m, n), O.outlier_dense(rp, col, val, m, n))
 
 
+@pytest.mark.parametrize("tiles", [[0], [1, 3], [0, 2, 3]])
+def test_tile_rows_equal_the_whole_product(tiles):
+    signs, alpha, bp, outl, x = _random_mixed(21, 4, 100, 2100, 84)
+    pk = O.pack_mixed(signs, bp)
+    y, rows = O.mixed_matmul_tiles(x, pk, bp, alpha, 84, 100, 2100, tiles, outl)
+    full = O.mixed_matmul(x, signs, alpha, bp, 84, outl)
+    assert np.array_equal(rows, np.concatenate([np.arange(32 * t, min(100, 32 * t + 32)) for t in tiles]))
+    assert np.allclose(y, full[:, rows], rtol=1e-13, atol=1e-13)
+
+
 def test_mixed_rejects_bad_inputs():
     signs, alpha, bp, outl, _ = _random_mixed(3, 2, 40, 2048, 64)
     with pytest.raises(ValueError):

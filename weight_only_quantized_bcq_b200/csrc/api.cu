@@ -17,6 +17,8 @@ cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, con
                                   int32_t* flags, cudaStream_t stream);
 cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, uint16_t* scales,
                                cudaStream_t stream);
+cudaError_t launch_pack_signs_mixed(const int8_t* signs, const uint32_t* block_off, int q_max, int m, int n,
+                                    uint8_t* packed, size_t packed_bytes, int32_t* flags, cudaStream_t stream);
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
                            float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
                            cudaStream_t stream);
@@ -161,14 +163,48 @@ RunKernel select_kernel(int q, int mode, bool has_offset, bool packed) {
   }
 }
 
-// Workspace: [split-K partials | tile counters | status word], each part
-// 256-byte aligned.
+// Workspace: [status word (256 B) | tile counters (4 KB) | split-K partials].
+// The status word sits at the start whatever the shape, so that
+// lutgemm_workspace_status can find it from the pointer alone.
 size_t part_bytes(int m, int n, int batch) {
   return (size_t)batch * ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * kTileRows * sizeof(float);
 }
 
 constexpr size_t kStatusBytes = 256;
 constexpr size_t kTileCounterBytes = kMaxTileCounters * sizeof(unsigned);
+constexpr size_t kPartOffset = kStatusBytes + kTileCounterBytes;
+
+// Fill the workspace pointers and geometry of `p` and enqueue the lookup
+// kernel (and the split-K reduce when there are several slices).
+int launch_lookup(RunParams& p, RunKernel kernel, void* workspace, cudaStream_t stream) {
+  char* ws = reinterpret_cast<char*>(workspace);
+  p.ns = ceil_div(p.n, kSliceInputs);
+  p.mt = ceil_div(p.m, kTileRows);
+  p.ng = p.n / p.g;
+  p.total_units = (long long)p.batch * p.ns * p.mt;
+  p.part = reinterpret_cast<float*>(ws + kPartOffset);
+  p.tile_cnt = reinterpret_cast<unsigned*>(ws + kStatusBytes);
+  p.status = reinterpret_cast<unsigned*>(ws);
+  if (kernel == nullptr) return LUTGEMM_ERR_VALUE;
+  int sm_count = 0;
+  if (device_setup(kernel, &sm_count) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  long long grid = 0;
+  choose_launch(sm_count, (long long)p.batch * p.ns, p.mt, &grid, &p.seg_aligned);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  if (p.ns > 1 && launch_splitk_reduce(p, stream) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  return LUTGEMM_OK;
+}
 
 }  // namespace
 
@@ -254,9 +290,46 @@ int lutgemm_tc_plan(int m, int n, int batch, int q, int max_split, int sm_count)
   return lutgemm::tc_plan_for(m, n, batch, q, max_split, sm_count);
 }
 
+int lutgemm_launch_plan(int m, int n, int batch, int sm_count, int* grid, int* seg_aligned, int* dynamic_tiles) {
+  if (!grid || !seg_aligned || !dynamic_tiles) return LUTGEMM_ERR_NULL;
+  if (m < 1 || n < 8 || n % 8 != 0 || batch < 1 || sm_count < 1) return LUTGEMM_ERR_SHAPE;
+  if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
+  const long long segments = (long long)batch * ceil_div(n, kSliceInputs);
+  const long long mt = ceil_div(m, kTileRows);
+  long long g = 0;
+  int aligned_mode = 0;
+  choose_launch(sm_count, segments, mt, &g, &aligned_mode);
+  *grid = (int)g;
+  *seg_aligned = aligned_mode;
+  long long dyn = 0;
+  if (aligned_mode) {
+    // Segment z has (grid - z + segments - 1) / segments CTAs (the kernel's
+    // group_size); their warps take two static tiles each, 32 per CTA.
+    for (long long z = 0; z < segments; ++z) {
+      const long long cz = (g - z + segments - 1) / segments;
+      dyn += mt > 32 * cz ? mt - 32 * cz : 0;
+    }
+  }
+  *dynamic_tiles = dyn > 0x7fffffffLL ? 0x7fffffff : (int)dyn;
+  return LUTGEMM_OK;
+}
+
+int lutgemm_workspace_status(void* workspace, size_t workspace_bytes, uint32_t* status, int clear, void* stream) {
+  if (!workspace || !status) return LUTGEMM_ERR_NULL;
+  if (!aligned(workspace, 16)) return LUTGEMM_ERR_ALIGN;
+  if (workspace_bytes < kPartOffset) return LUTGEMM_ERR_WORKSPACE;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  *status = v;
+  if (clear && v != 0u && cudaMemsetAsync(workspace, 0, sizeof(v), st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  return LUTGEMM_OK;
+}
+
 size_t lutgemm_workspace_size(int m, int n, int batch, int q, int g) {
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return 0;
-  return round_up(part_bytes(m, n, batch), 256) + kTileCounterBytes + kStatusBytes;
+  return kPartOffset + round_up(part_bytes(m, n, batch), 256);
 }
 
 int lutgemm_pack_bcq(const int8_t* signs, int q, int m, int n, uint8_t* packed, int32_t* status_flags,
@@ -289,7 +362,9 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   if (!packed || !alpha || !x || !y || !workspace) return LUTGEMM_ERR_NULL;
   if (!valid_matrix(q, m, n) || !valid_groups(n, g) || batch < 1) return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_ALLOW_TENSOR_CORES)) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_ALLOW_TENSOR_CORES | LUTGEMM_TEST_STALL)) != 0u)
+    return LUTGEMM_ERR_VALUE;
+  const bool stall = (flags & LUTGEMM_TEST_STALL) != 0u;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
   if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
@@ -297,16 +372,19 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
     return LUTGEMM_ERR_ALIGN;
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q, g)) return LUTGEMM_ERR_WORKSPACE;
+  char* ws = reinterpret_cast<char*>(workspace);
+  unsigned* const status = reinterpret_cast<unsigned*>(ws);
   // The tensor-core path, where it takes the operands and its cost model
   // says it is the faster one (never below batch 8); split K adds its fp32
   // partials with the split-K reduce, in split order.
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0) {
+  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && !stall && batch >= 8 && !scales_packed && n % 128 == 0 &&
+      g % 64 == 0) {
     const int nsplit = tc_plan(m, n, batch, q, ceil_div(n, kSliceInputs));
     if (nsplit > 0) {
-      float* part = nsplit > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
+      float* part = nsplit > 1 ? reinterpret_cast<float*>(ws + kPartOffset) : nullptr;
       cudaError_t e = launch_tc_gemm(packed, reinterpret_cast<const __half*>(alpha), offset,
                                      reinterpret_cast<const __half*>(x), y, part, nsplit, m, n, batch, q, g,
-                                     y_f16 ? 1 : 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
+                                     y_f16 ? 1 : 0, status, reinterpret_cast<cudaStream_t>(stream));
       if (e == cudaSuccess && nsplit > 1) {
         RunParams r = {};
         r.part = part;
@@ -325,7 +403,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
     }
   }
 
-  RunParams p;
+  RunParams p = {};
   p.packed = packed;
   p.alpha = reinterpret_cast<const __half*>(alpha);
   p.offset = offset;
@@ -336,38 +414,104 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   p.batch = batch;
   p.q = q;
   p.g = g;
-  p.ns = ceil_div(n, kSliceInputs);
-  p.mt = ceil_div(m, kTileRows);
-  p.ng = n / g;
   p.y_f16 = y_f16 ? 1 : 0;
-  p.total_units = (long long)batch * p.ns * p.mt;
-  char* ws = reinterpret_cast<char*>(workspace);
-  const size_t tile_off = round_up(part_bytes(m, n, batch), 256);
-  p.part = reinterpret_cast<float*>(ws);
-  p.tile_cnt = reinterpret_cast<unsigned*>(ws + tile_off);
-  p.status = reinterpret_cast<unsigned*>(ws + tile_off + kTileCounterBytes);
+  p.stall_test = stall ? 1 : 0;
+  return launch_lookup(p, select_kernel(q, group_mode(g), offset != nullptr, scales_packed), workspace,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
 
-  const RunKernel kernel = select_kernel(q, group_mode(g), offset != nullptr, scales_packed);
-  if (kernel == nullptr) return LUTGEMM_ERR_VALUE;
-  int sm_count = 0;
-  if (device_setup(kernel, &sm_count) != cudaSuccess) return LUTGEMM_ERR_CUDA;
-  long long grid = 0;
-  choose_launch(sm_count, (long long)batch * p.ns, p.mt, &grid, &p.seg_aligned);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
-  if (cudaGetLastError() != cudaSuccess) return LUTGEMM_ERR_CUDA;
-  if (p.ns > 1 && launch_splitk_reduce(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return LUTGEMM_ERR_CUDA;
+int lutgemm_mixed_offsets(const uint8_t* block_planes, int q_max, int m, int n, uint32_t* offsets) {
+  if (!block_planes || !offsets) return LUTGEMM_ERR_NULL;
+  if (q_max < 1 || q_max > 4 || m < 1 || n < 8 || n % 8 != 0) return LUTGEMM_ERR_SHAPE;
+  const long long blocks = (long long)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows);
+  unsigned long long acc = 0;
+  for (long long u = 0; u < blocks; ++u)
+    if (block_planes[u] < 1 || block_planes[u] > q_max) return LUTGEMM_ERR_VALUE;
+  for (long long u = 0; u < blocks; ++u) {
+    offsets[u] = (uint32_t)acc;
+    acc += block_planes[u];
+  }
+  if (acc > 0xFFFFFFFFull) return LUTGEMM_ERR_SHAPE;
+  offsets[blocks] = (uint32_t)acc;
   return LUTGEMM_OK;
+}
+
+int lutgemm_pack_outliers(const int32_t* row_ptr, const int32_t* col, const uint16_t* val, int m, int n, int nnz,
+                          uint32_t* optr, uint32_t* oent) {
+  if (!row_ptr || !optr || (nnz > 0 && (!col || !val || !oent))) return LUTGEMM_ERR_NULL;
+  if (m < 1 || n < 8 || n % 8 != 0 || nnz < 0) return LUTGEMM_ERR_SHAPE;
+  if (row_ptr[0] != 0 || row_ptr[m] != nnz) return LUTGEMM_ERR_VALUE;
+  for (int r = 0; r < m; ++r) {
+    if (row_ptr[r + 1] < row_ptr[r]) return LUTGEMM_ERR_VALUE;
+    for (int e = row_ptr[r]; e < row_ptr[r + 1]; ++e)
+      if (col[e] < 0 || col[e] >= n || (e > row_ptr[r] && col[e] <= col[e - 1])) return LUTGEMM_ERR_VALUE;
+  }
+  const int ns = ceil_div(n, kSliceInputs);
+  // Within a row the entries are sorted by input, so each row's entries of
+  // slice s are one run; a cursor per row walks them slice by slice.
+  uint32_t out = 0;
+  optr[0] = 0;
+  for (int s_ = 0; s_ < ns; ++s_) {
+    for (int r = 0; r < m; ++r) {
+      int e = row_ptr[r];
+      while (e < row_ptr[r + 1] && col[e] < s_ * kSliceInputs) ++e;
+      for (; e < row_ptr[r + 1] && col[e] < (s_ + 1) * kSliceInputs; ++e)
+        oent[out++] = (uint32_t)(col[e] - s_ * kSliceInputs) | ((uint32_t)val[e] << 16);
+      optr[(size_t)s_ * m + r + 1] = out;
+    }
+  }
+  return LUTGEMM_OK;
+}
+
+int lutgemm_pack_bcq_mixed(const int8_t* signs, const uint32_t* block_off, int q_max, int m, int n,
+                           uint8_t* packed, size_t packed_bytes, int32_t* status_flags, void* stream) {
+  if (!signs || !block_off || !packed) return LUTGEMM_ERR_NULL;
+  if (q_max < 1 || q_max > 4 || !valid_matrix(q_max, m, n)) return LUTGEMM_ERR_SHAPE;
+  if (!aligned(signs, 8) || !aligned(block_off, 4) || !aligned(packed, 16) || !aligned(status_flags, 4))
+    return LUTGEMM_ERR_ALIGN;
+  if (packed_bytes % kBlockBytes != 0 ||
+      packed_bytes < (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * kBlockBytes)
+    return LUTGEMM_ERR_VALUE;
+  const cudaError_t err = launch_pack_signs_mixed(signs, block_off, q_max, m, n, packed, packed_bytes, status_flags,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
+int lutgemm_run_mixed(int m, int n, int batch, int q_max, int g, const uint8_t* packed, size_t packed_bytes,
+                      const uint32_t* block_off, const uint16_t* alpha, const uint32_t* optr, const uint32_t* oent,
+                      int nnz, const uint16_t* x, void* y, unsigned flags, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  if (!packed || !block_off || !alpha || !x || !y || !workspace) return LUTGEMM_ERR_NULL;
+  if (nnz > 0 && (optr == nullptr || oent == nullptr)) return LUTGEMM_ERR_NULL;
+  if (q_max < 1 || q_max > 4 || !valid_matrix(q_max, m, n) || !valid_groups(n, g) || batch < 1 || nnz < 0)
+    return LUTGEMM_ERR_SHAPE;
+  if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_TEST_STALL)) != 0u) return LUTGEMM_ERR_VALUE;
+  const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
+  if (packed_bytes % kBlockBytes != 0 || packed_bytes / kBlockBytes > 0xFFFFFFFFull) return LUTGEMM_ERR_VALUE;
+  if (!aligned(packed, 16) || !aligned(block_off, 4) || !aligned(alpha, 2) || !aligned(optr, 4) ||
+      !aligned(oent, 4) || !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
+    return LUTGEMM_ERR_ALIGN;
+  if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q_max, g)) return LUTGEMM_ERR_WORKSPACE;
+  RunParams p = {};
+  p.packed = packed;
+  p.alpha = reinterpret_cast<const __half*>(alpha);
+  p.offset = nullptr;
+  p.x = reinterpret_cast<const __half*>(x);
+  p.y = y;
+  p.m = m;
+  p.n = n;
+  p.batch = batch;
+  p.q = q_max;
+  p.g = g;
+  p.y_f16 = y_f16 ? 1 : 0;
+  p.stall_test = (flags & LUTGEMM_TEST_STALL) != 0u ? 1 : 0;
+  p.block_off = block_off;
+  p.packed_blocks = (uint32_t)(packed_bytes / kBlockBytes);
+  p.optr = nnz > 0 ? optr : nullptr;
+  p.oent = nnz > 0 ? oent : nullptr;
+  p.nnz = (uint32_t)nnz;
+  return launch_lookup(p, run_kernel_mixed(group_mode(g)), workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

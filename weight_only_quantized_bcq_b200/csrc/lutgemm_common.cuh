@@ -78,7 +78,14 @@ struct RunParams {
   int ns, mt, ng;
   int y_f16;
   int seg_aligned;         // 1: CTAs grouped per segment; 0: unit list cut evenly
+  int stall_test;          // test hook: each warp's first ring wait runs out (see LUTGEMM_TEST_STALL)
   long long total_units;   // batch * ns * mt
+  // Mixed storage (lutgemm_run_mixed): per-block plane counts and sparse outliers.
+  const uint32_t* block_off;  // [ns*mt + 1] exclusive prefix sums of the plane counts (4096-byte blocks)
+  uint32_t packed_blocks;     // 4096-byte blocks in the packed buffer (bounds of block_off's values)
+  const uint32_t* optr;       // [ns*m + 1] slice-major outlier pointers, or nullptr
+  const uint32_t* oent;       // [nnz] outlier entries: (k - 1024 s) | fp16 << 16
+  uint32_t nnz;
 };
 
 // Range [begin, end) of units of CTA c out of G: either a share of one
@@ -143,6 +150,7 @@ cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream);
 
 constexpr unsigned kStatusWindow = 1u;
 constexpr unsigned kStatusTimeout = 2u;
+constexpr unsigned kStatusFormat = 4u;   // a mixed-storage block or outlier entry out of range
 
 // Kernel for q planes, group mode, offsets on/off and unit-major scales on/off
 // (nullptr for unit-major scales with a mode that has several per piece).
@@ -151,5 +159,6 @@ RunKernel run_kernel_q2(int mode, bool has_offset, bool packed);
 RunKernel run_kernel_q3(int mode, bool has_offset, bool packed);
 RunKernel run_kernel_q4(int mode, bool has_offset, bool packed);
 RunKernel run_kernel_q8(int mode, bool has_offset, bool packed);   // 5 <= q <= 8, planes in groups of four
+RunKernel run_kernel_mixed(int mode);   // mixed storage: 1..4 planes per block, sparse outliers
 
 }  // namespace lutgemm

@@ -108,12 +108,13 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier; give up after about one second.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for phase `parity` of an mbarrier; give up after `limit_ns`
+// nanoseconds (one second unless told otherwise).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = 1000000000ull) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (!mbar_try(bar, parity)) {
-    if (global_ns() - t0 > 1000000000ull) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
   return true;
 }
@@ -231,7 +232,10 @@ __device__ __forceinline__ void static_for(std::integer_sequence<int, Is...>, F&
 
 }  // namespace detail
 
-template <int Q, int MODE, bool MULTI, bool HAS_OFF, bool PK>
+// MIXED: mixed storage (lutgemm_run_mixed).  Every (slice, row tile) block
+// holds its own number of planes, 1..Q, at the offset p.block_off gives, and
+// sparse fp16 outliers (slice-major CSR) are added to each row's sum.
+template <int Q, int MODE, bool MULTI, bool HAS_OFF, bool PK, bool MIXED = false>
 __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p) {
   using namespace detail;
   constexpr int SP = step_planes(MULTI ? 8 : Q);       // planes in one step (<= 4)
@@ -240,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr uint32_t STEP_BYTES = 512u * SP;
   constexpr uint32_t STAGE_BYTES = STEP_BYTES * CH;
   static_assert(!MULTI || CH == 1, "plane groups are fetched one step at a time");
-  static_assert(S >= 2 && S <= 8, "weight ring of 2..8 stages");
+  static_assert(!MIXED || (Q <= 4 && !MULTI && !HAS_OFF && !PK), "mixed storage: up to 4 planes, [q][n/g][m] scales");
+  static_assert(S >= 2 && S <= 7, "weight ring of 2..7 stages (barrier slot 7 is the test hook's)");
   constexpr int NPG = MULTI ? 2 : 1;                   // plane groups of a unit
 
   extern __shared__ __align__(16) unsigned char smem[];
@@ -266,7 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   // Register stages of prefetched scales: step j's are loaded NA-1 steps
   // ahead (7 with one scale per piece, 3 with two, to bound registers); the
   // scales come from HBM and their latency under full load is microseconds.
-  constexpr int NA = APP == 1 ? 8 : 4;
+  // Mixed storage: 3 steps ahead, so that the next tile's block entry (read
+  // when the tile becomes known, a tile ahead) has arrived first.
+  constexpr int NA = (APP == 1 && !MIXED) ? 8 : 4;
   static_assert((8 * NPG) % NA == 0, "scale stages must tile the unit");
   // Step of a unit at which the next tile is first needed: the scale
   // prefetch reaches it NA-1 steps before the end, the ring refill S stages
@@ -276,7 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr int NEED_P = PK ? 8 * (NPG - 1) : 8 * NPG;   // next tile's scales: start of its last pass
   constexpr int NEED_AR = NEED_A < NEED_R ? NEED_A : NEED_R;
   constexpr int NEED = NEED_AR < NEED_P ? NEED_AR : NEED_P;
-  constexpr bool AHEAD1 = NEED >= 3;
+  // Mixed storage grabs two tiles ahead: a tile's block entry is read as soon
+  // as the tile is known, a whole tile before its copies are issued.
+  constexpr bool AHEAD1 = NEED >= 3 && !MIXED;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -305,9 +314,14 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   // consumed.
   const uint32_t ring = kRingBase + (uint32_t)warp * kRingBytesPerWarp;
   const uint32_t bars = kBarBase + (uint32_t)warp * 64u;
+  // Slot 7 of the warp's barriers is never signalled: with the test hook
+  // (p.stall_test) the warp's first ring wait is on it, runs out after 1 ms
+  // and takes the timeout path.
+  const uint32_t dead_bar = bars + 56u;
   if (lane == 0) {
 #pragma unroll
     for (int st0 = 0; st0 < S; ++st0) mbar_init(bars + 8u * st0);
+    if (p.stall_test) mbar_init(dead_bar);
   }
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncwarp();
@@ -393,17 +407,47 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     constexpr int CPT = 8 / CH;                      // ring chunks per unit and plane group
     const int chunks_per_unit = CPT * npg;
 
-    // TMA copy of chunk c (steps c*CH .. c*CH+CH-1) of row tile R into ring
-    // stage `stage` (lane 0 only).  The CH steps are contiguous.
-    auto issue = [&](int R_, int c, int stage) {
-      const int pg_ = c / CPT, U_ = (c - pg_ * CPT) * CH;
-      const int planes = MULTI ? min(4, p.q - 4 * pg_) : Q;
-      const uint8_t* src = slice_base + (size_t)R_ * unit_bytes + ((size_t)U_ * p.q + 4 * pg_) * 512;
-      tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * planes * CH, bars + 8u * stage, wpol);
+    // Mixed storage: (first 4096-byte block, planes) of row tile R_ of this
+    // slice, from the block table.  An entry outside the packed buffer or
+    // with no plane or more than Q planes is reported and its tile skipped
+    // (planes = 0).  Uniform storage: (unused, Q).
+    auto tile_info = [&](int R_) -> uint2 {
+      if constexpr (MIXED) {
+        const uint32_t* bo = p.block_off + (size_t)s * p.mt + R_;
+        const uint32_t b0 = __ldg(bo), b1 = __ldg(bo + 1);
+        const uint32_t qb = b1 - b0;
+        if (b1 < b0 || qb < 1u || qb > (uint32_t)Q || b1 > p.packed_blocks) {
+          if (lane == 0) atomicOr(p.status, kStatusFormat);
+          return make_uint2(0u, 0u);
+        }
+        return make_uint2(b0, qb);
+      } else {
+        return make_uint2(0u, (uint32_t)Q);
+      }
     };
 
-    // Per-piece scales (and offsets) of step j of row tile R into register stage SLOT.
-    auto load_alpha = [&]<int SLOT>(int R_, int j) {
+    // TMA copy of chunk c (steps c*CH .. c*CH+CH-1) of row tile R into ring
+    // stage `stage` (lane 0 only).  The CH steps are contiguous.  A mixed
+    // tile with no valid entry fetches nothing and completes its stage.
+    auto issue = [&](int R_, uint2 ti, int c, int stage) {
+      const int pg_ = c / CPT, U_ = (c - pg_ * CPT) * CH;
+      if constexpr (MIXED) {
+        if (ti.y == 0u) {
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bars + 8u * stage) : "memory");
+          return;
+        }
+        const uint8_t* src = p.packed + (size_t)ti.x * kBlockBytes + (size_t)U_ * ti.y * 512;
+        tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * ti.y * CH, bars + 8u * stage, wpol);
+      } else {
+        const int planes = MULTI ? min(4, p.q - 4 * pg_) : Q;
+        const uint8_t* src = slice_base + (size_t)R_ * unit_bytes + ((size_t)U_ * p.q + 4 * pg_) * 512;
+        tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * planes * CH, bars + 8u * stage, wpol);
+      }
+    };
+
+    // Per-piece scales (and offsets) of step j of row tile R into register
+    // stage SLOT; `planes` of them (the tile's plane count in mixed storage).
+    auto load_alpha = [&]<int SLOT>(int R_, int j, uint32_t planes) {
       if constexpr (PRE_ALPHA) {
         const int pg_ = j >> 3, U_ = j & 7;
         const int row = R_ * kTileRows + lane;
@@ -419,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           if constexpr (!PK) {
 #pragma unroll
             for (int i = 0; i < Q; ++i) {
-              const bool live = !MULTI || (pg_ * 4 + i < p.q);
+              const bool live = (!MULTI || (pg_ * 4 + i < p.q)) && (!MIXED || (uint32_t)i < planes);
               ab[SLOT][i][r] = (ok && live) ? ld_u16(ap + (size_t)(pg_ * 4 + i) * plane_stride) : (uint16_t)0;
             }
           }
@@ -428,11 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
       }
     };
 
+    uint2 ti_cur = busy ? tile_info(t_cur) : make_uint2(0u, 0u);
+    uint2 ti_nxt = t_nxt >= 0 ? tile_info(t_nxt) : make_uint2(0u, 0u);
     // The first S copies of the first tile go out before the tables are built.
     if (busy && lane == 0) {
       int st2 = st;
       for (int c = 0; c < S; ++c) {
-        issue(t_cur, c, st2);
+        issue(t_cur, ti_cur, c, st2);
         st2 = st2 + 1 == S ? 0 : st2 + 1;
       }
     }
@@ -457,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     if (busy) {
       load_scales(t_cur, 0, sc_cur);
       static_for(std::make_integer_sequence<int, NA - 1>{}, [&]<int D>() {
-        load_alpha.template operator()<D>(t_cur, D);
+        load_alpha.template operator()<D>(t_cur, D, ti_cur.y);
       });
       const int steps_per_unit_ = steps_per_unit;
       bool more = dyn;        // grabs may still succeed
@@ -482,6 +528,16 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         const int R = t_cur;
         const int row = R * kTileRows + lane;
         float yacc = 0.f;
+        // Mixed storage: this row's outliers in this slice, [o0, o1) of the
+        // entries; the first two are fetched mid-unit.
+        uint32_t o0 = 0u, o1 = 0u, oe[2] = {0u, 0u};
+        if constexpr (MIXED) {
+          if (p.optr != nullptr && row < p.m) {
+            const uint32_t* op = p.optr + (size_t)s * p.m + row;
+            o0 = __ldg(op);
+            o1 = __ldg(op + 1);
+          }
+        }
         for (int pg = 0; pg < npg && !failed; ++pg) {
           static_for(std::make_integer_sequence<int, 8>{}, [&]<int U>() {
             if (failed) return;
@@ -506,15 +562,23 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
             }
             {
               const int ja = j + NA - 1;       // scales NA-1 steps ahead
-              if (ja < steps_per_unit_) load_alpha.template operator()<(U + NA - 1) % NA>(t_cur, ja);
-              else if (t_nxt >= 0) load_alpha.template operator()<(U + NA - 1) % NA>(t_nxt, ja - steps_per_unit_);
+              if (ja < steps_per_unit_) load_alpha.template operator()<(U + NA - 1) % NA>(t_cur, ja, ti_cur.y);
+              else if (t_nxt >= 0)
+                load_alpha.template operator()<(U + NA - 1) % NA>(t_nxt, ja - steps_per_unit_, ti_nxt.y);
+            }
+            if constexpr (MIXED && U == 4) {
+              if (o1 > o0 && o1 <= p.nnz) {
+                oe[0] = __ldg(p.oent + o0);
+                if (o1 > o0 + 1u) oe[1] = __ldg(p.oent + o0 + 1u);
+              }
             }
 
             // Pieces of a whole stage (CH steps) come out of the ring at its
             // first step; the stage is refilled (S copies ahead) right away, so
             // S full copies are in flight while the steps are computed.
             if constexpr (U % CH == 0) {
-              const bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8u * st, ph));
+              const bool ok = __all_sync(0xffffffffu, p.stall_test ? mbar_wait(dead_bar, 0u, 1000000ull)
+                                                                   : mbar_wait(bars + 8u * st, ph));
               if (!ok) {
                 failed = true;
                 if (lane == 0) atomicOr(p.status, kStatusTimeout);
@@ -525,15 +589,15 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
               for (int h = 0; h < CH; ++h)
 #pragma unroll
                 for (int i = 0; i < SP; ++i) {
-                  const bool live = !MULTI || (pg * 4 + i < p.q);
+                  const bool live = (!MULTI || (pg * 4 + i < p.q)) && (!MIXED || (uint32_t)i < ti_cur.y);
                   wst[h][i] = live ? lds128(src + (uint32_t)h * STEP_BYTES + 512u * i) : make_uint4(0, 0, 0, 0);
                 }
               __syncwarp();
               const int cn = j / CH + S;       // chunk to fetch into the freed stage
               if (cn < chunks_per_unit) {
-                if (lane == 0) issue(t_cur, cn, st);
+                if (lane == 0) issue(t_cur, ti_cur, cn, st);
               } else if (t_nxt >= 0) {
-                if (lane == 0) issue(t_nxt, cn - chunks_per_unit, st);
+                if (lane == 0) issue(t_nxt, ti_nxt, cn - chunks_per_unit, st);
               } else {
                 --outstanding;
               }
@@ -548,6 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
 #pragma unroll
             for (int i = 0; i < Q; ++i) {
               if (MULTI && pg * 4 + i >= p.q) continue;
+              if (MIXED && (uint32_t)i >= ti_cur.y) continue;
               const uint4 w4 = wv[i];
               if constexpr (RUN == 16) {
                 float acc0 = 0.f, acc1 = 0.f;
@@ -614,6 +679,25 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           }
         }
         if (failed) break;
+        // Mixed storage: the row's outliers in this slice, in entry order.
+        if constexpr (MIXED) {
+          if (o1 != o0) {
+            if (o1 < o0 || o1 > p.nnz) {
+              atomicOr(p.status, kStatusFormat);
+            } else {
+              const unsigned short* xb = reinterpret_cast<const unsigned short*>(p.x) + (size_t)b * p.n;
+              for (uint32_t e = o0; e < o1; ++e) {
+                const uint32_t v = e < o0 + 2u ? oe[e - o0] : __ldg(p.oent + e);
+                const uint32_t k = (uint32_t)s * kSliceInputs + (v & 0xFFFFu);
+                if ((v & 0xFFFFu) >= (uint32_t)kSliceInputs || k >= (uint32_t)p.n) {
+                  atomicOr(p.status, kStatusFormat);
+                  continue;
+                }
+                yacc = fmaf(h2f((uint16_t)(v >> 16)), h2f(__ldg(xb + k)), yacc);
+              }
+            }
+          }
+        }
         // One slice: the row's sum is y.  Several: this slice's partial, summed
         // over slices by the split-K reduce kernel that follows.
         if (p.ns == 1) {
@@ -630,6 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         if (t_nxt < 0) break;
         if constexpr (AHEAD1) {
           t_cur = t_nxt;
+          ti_cur = ti_nxt;
           continue;
         }
         int t_after = -1;
@@ -648,6 +733,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         }
         t_cur = t_nxt;
         t_nxt = t_after;
+        ti_cur = ti_nxt;
+        if (t_nxt >= 0) ti_nxt = tile_info(t_nxt);
       }
     }
   }

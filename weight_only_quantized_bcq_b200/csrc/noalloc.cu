@@ -10,7 +10,8 @@
 // The scratch is a file-scope __device__ array: every GPU on which the library
 // is loaded holds its LUTGEMM_NOALLOC_SCRATCH_BYTES until the process exits.
 // Layout (fixed, independent of the problem size):
-//   [0, 256)              status word (sticky internal-error bits)
+//   [0, 256)              status word (sticky error bits, read and cleared
+//                         with lutgemm_library_status)
 //   [256, +4 KB)          per-segment tile counters, zero between calls
 //   [.., end)             split-K partial sums, written before they are read
 // The counters sit at a fixed place so that they are never overlaid by
@@ -29,6 +30,7 @@ namespace lutgemm {
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
                            float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
                            cudaStream_t stream);
+cudaError_t tc_status_address(unsigned** out);
 int tc_plan(int m, int n, int batch, int q, int max_split);
 }  // namespace lutgemm
 
@@ -69,10 +71,10 @@ RunKernel pick_kernel(int q, int g, bool has_offset, bool packed) {
 }
 
 // Once per device, with that device current: look up the scratch array's
-// device address and zero its status word and counters on the caller's
-// stream (ordered before the first launch).  Then, once per kernel and
-// device, opt the kernel into its shared-memory size.
-cudaError_t prepare(RunKernel kernel, cudaStream_t stream, DeviceScratch* out) {
+// device address (the host-side name g_scratch is not a device address) and
+// zero its status word and counters on the caller's stream, ordered before
+// the first launch that uses them.
+cudaError_t scratch_setup(cudaStream_t stream, DeviceScratch* out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -83,32 +85,42 @@ cudaError_t prepare(RunKernel kernel, cudaStream_t stream, DeviceScratch* out) {
     void* ptr = nullptr;
     err = cudaGetSymbolAddress(&ptr, g_scratch);
     if (err != cudaSuccess) return err;
-    int sms = 0, reserved = 0, optin = 0;
+    int sms = 0;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
-    if ((err = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess)
-      return err;
-    if ((err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
-      return err;
-    if ((unsigned)reserved != kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
     err = cudaMemsetAsync(ptr, 0, kPartOff, stream);
     if (err != cudaSuccess) return err;
     d.base = static_cast<unsigned char*>(ptr);
     d.sm_count = sms;
     d.ready = true;
   }
-  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
-  if (g_smem_done.find(key) == g_smem_done.end()) {
-    // Static shared memory would move the dynamic window off kTableBase.
-    cudaFuncAttributes fa;
-    err = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
-    if (err != cudaSuccess) return err;
-    if (fa.sharedSizeBytes != 0) return cudaErrorInvalidConfiguration;
-    err = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (err != cudaSuccess) return err;
-    g_smem_done.insert(key);
-  }
   *out = d;
+  return cudaSuccess;
+}
+
+// Once per kernel and device: the shared-memory window check and opt-in.
+cudaError_t kernel_setup(RunKernel kernel) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  if (g_smem_done.find(key) != g_smem_done.end()) return cudaSuccess;
+  int reserved = 0, optin = 0;
+  if ((err = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess)
+    return err;
+  if ((err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+    return err;
+  // The tables sit at a fixed window address right after the reserved region,
+  // and static shared memory would move the dynamic window off it.
+  if ((unsigned)reserved != kTableBase || optin < kSmemBytes) return cudaErrorInvalidConfiguration;
+  cudaFuncAttributes fa;
+  err = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
+  if (err != cudaSuccess) return err;
+  if (fa.sharedSizeBytes != 0) return cudaErrorInvalidConfiguration;
+  err = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes);
+  if (err != cudaSuccess) return err;
+  g_smem_done.insert(key);
   return cudaSuccess;
 }
 
@@ -121,34 +133,43 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   if (q < 1 || q > 8 || m < 1 || n < 8 || n % 8 != 0 || g < 8 || g % 8 != 0 || n % g != 0 || batch < 1)
     return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_ALLOW_TENSOR_CORES)) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_ALLOW_TENSOR_CORES | LUTGEMM_TEST_STALL)) != 0u)
+    return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
+  const bool stall = (flags & LUTGEMM_TEST_STALL) != 0u;
   if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
   if (!aligned(packed, 16) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(offset, 4) ||
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;
-  // The tensor-core path needs no scratch at all (same rule as lutgemm_run).
-  // (one K split: no scratch)
-  if ((flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && batch >= 8 && !scales_packed && n % 128 == 0 && g % 64 == 0 &&
-      tc_plan(m, n, batch, q, 1) > 0) {
-    const cudaError_t e = launch_tc_gemm(packed, alpha_ptr_h(alpha), offset, reinterpret_cast<const __half*>(x), y,
-                                         nullptr, 1, m, n, batch, q, g, y_f16 ? 1 : 0, nullptr,
-                                         reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
-  }
   const int ns = ceil_div(n, kSliceInputs);
   const int mt = ceil_div(m, kTileRows);
-  const size_t partials = (size_t)batch * ns * mt * kTileRows * sizeof(float);
-  if (partials > kScratchBytes - kPartOff) return LUTGEMM_ERR_WORKSPACE;
+  // Split-K partials exist only with several slices; one slice writes y directly.
+  const size_t partials = ns > 1 ? (size_t)batch * ns * mt * kTileRows * sizeof(float) : 0;
+  const bool fits = partials <= kScratchBytes - kPartOff;
+  // The tensor-core path with one K split needs no scratch.  It runs where
+  // lutgemm_run would pick it, and also where the lookup kernel's partials
+  // would not fit the scratch.
+  const bool tc_ok = (flags & LUTGEMM_ALLOW_TENSOR_CORES) != 0u && !stall && batch >= 8 && !scales_packed &&
+                     n % 128 == 0 && g % 64 == 0;
+  const bool use_tc = tc_ok && (tc_plan(m, n, batch, q, 1) > 0 || !fits);
+  if (!use_tc && !fits) return LUTGEMM_ERR_WORKSPACE;
 
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceScratch d;
+  if (scratch_setup(st, &d) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  unsigned* const status = reinterpret_cast<unsigned*>(d.base + kStatusOff);
+  if (use_tc) {
+    const cudaError_t e = launch_tc_gemm(packed, alpha_ptr_h(alpha), offset, reinterpret_cast<const __half*>(x), y,
+                                         nullptr, 1, m, n, batch, q, g, y_f16 ? 1 : 0, status, st);
+    return e == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+  }
+
   const RunKernel kernel = pick_kernel(q, g, offset != nullptr, scales_packed);
   if (kernel == nullptr) return LUTGEMM_ERR_VALUE;
-  DeviceScratch d;
-  if (prepare(kernel, st, &d) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  if (kernel_setup(kernel) != cudaSuccess) return LUTGEMM_ERR_CUDA;
 
-  RunParams p;
+  RunParams p = {};
   p.packed = packed;
   p.alpha = reinterpret_cast<const __half*>(alpha);
   p.offset = offset;
@@ -156,7 +177,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   p.y = y;
   p.part = reinterpret_cast<float*>(d.base + kPartOff);
   p.tile_cnt = reinterpret_cast<unsigned*>(d.base + kTileCounterOff);
-  p.status = reinterpret_cast<unsigned*>(d.base + kStatusOff);
+  p.status = status;
   p.m = m;
   p.n = n;
   p.batch = batch;
@@ -166,6 +187,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   p.mt = mt;
   p.ng = n / g;
   p.y_f16 = y_f16 ? 1 : 0;
+  p.stall_test = stall ? 1 : 0;
   p.total_units = (long long)batch * ns * mt;
   long long grid = 0;
   choose_launch(d.sm_count, (long long)batch * ns, mt, &grid, &p.seg_aligned);
@@ -182,5 +204,28 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   if (cudaLaunchKernelEx(&cfg, kernel, p) != cudaSuccess) return LUTGEMM_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return LUTGEMM_ERR_CUDA;
   if (p.ns > 1 && launch_splitk_reduce(p, st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  return LUTGEMM_OK;
+}
+
+// The status words of the calls that run without a caller workspace, on the
+// current device: the no-alloc scratch's and the tensor-core path's own.
+extern "C" int lutgemm_library_status(uint32_t* status, int clear, void* stream) {
+  if (!status) return LUTGEMM_ERR_NULL;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceScratch d;
+  if (scratch_setup(st, &d) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  unsigned* tc = nullptr;
+  if (tc_status_address(&tc) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  unsigned* const words[2] = {reinterpret_cast<unsigned*>(d.base + kStatusOff), tc};
+  unsigned v[2] = {0u, 0u};
+  for (int k = 0; k < 2; ++k)
+    if (cudaMemcpyAsync(&v[k], words[k], sizeof(unsigned), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return LUTGEMM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  *status = v[0] | v[1];
+  if (clear) {
+    for (int k = 0; k < 2; ++k)
+      if (v[k] != 0u && cudaMemsetAsync(words[k], 0, sizeof(unsigned), st) != cudaSuccess) return LUTGEMM_ERR_CUDA;
+  }
   return LUTGEMM_OK;
 }

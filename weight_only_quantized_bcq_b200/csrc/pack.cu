@@ -64,6 +64,52 @@ __global__ void pack_signs_kernel(const int8_t* __restrict__ signs, int q, int m
   if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_SIGN);
 }
 
+// Mixed storage: block (s, R) holds q_b = block_off[u+1] - block_off[u]
+// planes (u = s*mt + R) from byte 4096 * block_off[u]; its chunk (U, i) sits
+// at (U * q_b + i) * 512, with the byte map of the uniform layout.  One
+// thread per (block, U, plane i < q_max, lane); threads of planes the block
+// does not store return.  A table entry that would write past the buffer is
+// flagged and its block left unwritten.
+__global__ void pack_signs_mixed_kernel(const int8_t* __restrict__ signs, const uint32_t* __restrict__ block_off,
+                                        int q_max, int m, int n, int mt, long long nthreads, size_t packed_bytes,
+                                        uint8_t* __restrict__ packed, int32_t* flags) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nthreads) return;
+  const long long chunk = tid >> 5;          // ((s*mt + R)*8 + U)*q_max + i
+  const int l = (int)(tid & 31);
+  const int i = (int)(chunk % q_max);
+  const long long sRU = chunk / q_max;
+  const int U = (int)(sRU & 7);
+  const long long u = sRU >> 3;
+  const int R = (int)(u % mt);
+  const int s = (int)(u / mt);
+  const uint32_t b0 = block_off[u], b1 = block_off[u + 1];
+  const uint32_t qb = b1 - b0;
+  if (b1 < b0 || qb < 1u || qb > (uint32_t)q_max || (size_t)b1 * kBlockBytes > packed_bytes) {
+    if (flags && i == 0 && U == 0 && l == 0) atomicOr(flags, LUTGEMM_FLAG_BAD_BLOCK);
+    return;
+  }
+  if ((uint32_t)i >= qb) return;
+  const int r = R * kTileRows + l;
+  const int P = piece_of(U, l);
+  uint32_t words[4] = {0u, 0u, 0u, 0u};
+  bool bad = false;
+  if (r < m) {
+    const int8_t* rowp = signs + ((size_t)i * m + r) * (size_t)n;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int k0 = s * kSliceInputs + 128 * P + 8 * run_of(j, l);
+      if (k0 < n) {
+        const uint2 v = *reinterpret_cast<const uint2*>(rowp + k0);
+        words[j >> 2] |= sign_byte(v, bad) << (8 * (j & 3));
+      }
+    }
+  }
+  const size_t dst = (size_t)b0 * kBlockBytes + ((size_t)U * qb + i) * 512 + (size_t)l * 16;
+  *reinterpret_cast<uint4*>(packed + dst) = make_uint4(words[0], words[1], words[2], words[3]);
+  if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_SIGN);
+}
+
 // Plane i of a uniform code is bit i of the code (0-based, least significant first).
 __global__ void pack_codes_kernel(const uint8_t* __restrict__ codes, int q, int m, int n, int mt,
                                   long long nthreads, uint8_t* __restrict__ packed, int32_t* flags) {
@@ -186,6 +232,18 @@ cudaError_t launch_pack_signs(const int8_t* signs, int q, int m, int n, uint8_t*
   const int block = 256;
   const long long grid = (nthreads + block - 1) / block;
   pack_signs_kernel<<<(unsigned)grid, block, 0, stream>>>(signs, q, m, n, mt, nthreads, packed, flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_signs_mixed(const int8_t* signs, const uint32_t* block_off, int q_max, int m, int n,
+                                    uint8_t* packed, size_t packed_bytes, int32_t* flags, cudaStream_t stream) {
+  const int mt = (m + kTileRows - 1) / kTileRows;
+  const int ns = (n + kSliceInputs - 1) / kSliceInputs;
+  const long long nthreads = (long long)ns * mt * q_max * 256;
+  const int block = 256;
+  const long long grid = (nthreads + block - 1) / block;
+  pack_signs_mixed_kernel<<<(unsigned)grid, block, 0, stream>>>(signs, block_off, q_max, m, n, mt, nthreads,
+                                                                packed_bytes, packed, flags);
   return cudaGetLastError();
 }
 

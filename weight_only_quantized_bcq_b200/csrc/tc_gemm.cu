@@ -810,6 +810,16 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const float* o
 
 }  // namespace
 
+// Device address of the tensor-core path's own status word on the current
+// device (used when the caller gives none).
+cudaError_t tc_status_address(unsigned** out) {
+  void* sp = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&sp, g_tc_status);
+  if (e != cudaSuccess) return e;
+  *out = static_cast<unsigned*>(sp);
+  return cudaSuccess;
+}
+
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
                            float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
                            cudaStream_t stream) {

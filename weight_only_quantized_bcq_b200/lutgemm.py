@@ -17,9 +17,12 @@ LIB_PATH = os.path.join(_HERE, "liblutgemm.so")
 
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_VALUE, ERR_CUDA = range(7)
 FLAG_BAD_SIGN, FLAG_BAD_CODE, FLAG_BAD_ZERO = 1, 2, 4
+STATUS_WINDOW, STATUS_TIMEOUT, STATUS_FORMAT = 1, 2, 4
+FLAG_BAD_BLOCK = 8
 Y_F16 = 1
 SCALES_PACKED = 2
 ALLOW_TENSOR_CORES = 4
+TEST_STALL = 0x80000000
 
 _lib = None
 
@@ -42,6 +45,14 @@ _SIGNATURES = {
                      _vp], _c_int),
     "lutgemm_run_noalloc": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_uint, _vp],
                             _c_int),
+    "lutgemm_workspace_status": ([_vp, _c_size, _vp, _c_int, _vp], _c_int),
+    "lutgemm_mixed_offsets": ([_vp, _c_int, _c_int, _c_int, _vp], _c_int),
+    "lutgemm_pack_outliers": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
+    "lutgemm_pack_bcq_mixed": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp], _c_int),
+    "lutgemm_run_mixed": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp, _vp, _vp, _c_int, _vp,
+                           _vp, _c_uint, _vp, _c_size, _vp], _c_int),
+    "lutgemm_library_status": ([_vp, _c_int, _vp], _c_int),
+    "lutgemm_launch_plan": ([_c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
 }
 
 
@@ -65,6 +76,17 @@ def lib() -> ctypes.CDLL:
             fn.restype = res
         _lib = handle
     return _lib
+
+
+class LutgemmDeviceError(RuntimeError):
+    """A kernel failed while it ran: its sticky status word has bits set."""
+
+    def __init__(self, bits: int, where: str):
+        self.bits = bits
+        names = [n for b, n in ((STATUS_WINDOW, "shared-memory window"), (STATUS_TIMEOUT, "wait timed out"),
+                                (STATUS_FORMAT, "mixed-storage entry out of range")) if bits & b]
+        super().__init__(f"{where}: device status 0x{bits:x} ({', '.join(names) or 'unknown bits'}): "
+                         "the outputs are not valid")
 
 
 def status_string(status: int) -> str:
@@ -128,6 +150,40 @@ def _batch_of(x, n: int) -> int:
     if x.dim() not in (1, 2) or x.shape[-1] != n:
         raise ValueError(f"x must be [n] or [batch][n] with n = {n}; got {tuple(x.shape)}")
     return x.shape[0] if x.dim() == 2 else 1
+
+
+def workspace_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
+    """The LUTGEMM_STATUS_* bits of a lutgemm_run workspace (waits for the
+    stream's work so far); cleared afterwards when ``clear``."""
+    _need(workspace, torch.uint8, "workspace")
+    _one_device(stream, workspace=workspace)
+    v = ctypes.c_uint32(0)
+    _check(lib().lutgemm_workspace_status(_ptr(workspace), workspace.numel(), ctypes.byref(v), int(clear),
+                                          _stream(stream)),
+           "lutgemm_workspace_status")
+    return int(v.value)
+
+
+def library_status(clear: bool = True, stream=None) -> int:
+    """The LUTGEMM_STATUS_* bits of the words lutgemm_run_tc and
+    lutgemm_run_noalloc use on the current device; cleared when ``clear``."""
+    v = ctypes.c_uint32(0)
+    _check(lib().lutgemm_library_status(ctypes.byref(v), int(clear), _stream(stream)), "lutgemm_library_status")
+    return int(v.value)
+
+
+def launch_plan(m: int, n: int, batch: int, sm_count: int):
+    """(grid, seg_aligned, dynamic_tiles) of the lookup kernel, as lutgemm_run chooses it."""
+    grid, aligned, dyn = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().lutgemm_launch_plan(m, n, batch, sm_count, ctypes.byref(grid), ctypes.byref(aligned),
+                                     ctypes.byref(dyn)),
+           "lutgemm_launch_plan")
+    return grid.value, aligned.value, dyn.value
+
+
+def _raise_if_bits(bits: int, where: str):
+    if bits:
+        raise LutgemmDeviceError(bits, where)
 
 
 @functools.lru_cache(maxsize=256)
@@ -266,25 +322,30 @@ def _check_product_args(packed, alpha, x, offset, y, workspace, m, n, q, g, y_f1
 def run(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
         offset: torch.Tensor = None, y: torch.Tensor = None, workspace: torch.Tensor = None,
         y_f16: bool = False, scales_packed: bool = False, allow_tensor_cores: bool = False,
-        stream=None) -> torch.Tensor:
+        check: bool = False, stream=None, _flags: int = 0) -> torch.Tensor:
     """y[b] = W x[b] for a packed BCQ weight W (m x n), computed by lutgemm_run.
     With ``scales_packed`` alpha is the output of ``pack_scales``; with
-    ``allow_tensor_cores`` the library may take the tensor-core path (batch >= 8)."""
+    ``allow_tensor_cores`` the library may take the tensor-core path (batch >= 8).
+    With ``check`` the call waits for the kernels and raises LutgemmDeviceError
+    if the workspace's status word has bits set (and clears them)."""
     batch = _check_product_args(packed, alpha, x, offset, y, workspace, m, n, q, g, y_f16, scales_packed, stream)
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     if workspace is None:
         workspace = new_workspace(m, n, batch, q, g, device=x.device)
     flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0) | \
-        (ALLOW_TENSOR_CORES if allow_tensor_cores else 0)
+        (ALLOW_TENSOR_CORES if allow_tensor_cores else 0) | _flags
     _check(lib().lutgemm_run(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
                              flags, _ptr(workspace), workspace.numel(), _stream(stream)),
            "lutgemm_run")
+    if check:
+        _raise_if_bits(workspace_status(workspace, clear=True, stream=stream), "lutgemm_run")
     return y
 
 
 def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
-           y: torch.Tensor = None, y_f16: bool = False, offset: torch.Tensor = None, stream=None) -> torch.Tensor:
+           y: torch.Tensor = None, y_f16: bool = False, offset: torch.Tensor = None, check: bool = False,
+           stream=None) -> torch.Tensor:
     """``run`` on the tensor cores (lutgemm_run_tc), for large batches;
     n % 128 == 0 and g % 64 == 0, [q][n/g][m] scales, optional fp32 offsets."""
     batch = _check_product_args(packed, alpha, x, offset, y, None, m, n, q, g, y_f16, False, stream)
@@ -293,12 +354,15 @@ def run_tc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n
     _check(lib().lutgemm_run_tc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x), _ptr(y),
                                 Y_F16 if y_f16 else 0, _stream(stream)),
            "lutgemm_run_tc")
+    if check:
+        _raise_if_bits(library_status(clear=True, stream=stream), "lutgemm_run_tc")
     return y
 
 
 def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int, q: int, g: int,
                 offset: torch.Tensor = None, y: torch.Tensor = None, y_f16: bool = False,
-                scales_packed: bool = False, allow_tensor_cores: bool = False, stream=None) -> torch.Tensor:
+                scales_packed: bool = False, allow_tensor_cores: bool = False, check: bool = False,
+                stream=None, _flags: int = 0) -> torch.Tensor:
     """``run`` through lutgemm_run_noalloc, for callers that cannot allocate a
     workspace: the library uses its own fixed 16 MiB device scratch instead.
     Only ``y`` is allocated here, and only when the caller passes none.  Calls
@@ -307,8 +371,95 @@ def run_noalloc(packed: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: i
     if y is None:
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0) | \
-        (ALLOW_TENSOR_CORES if allow_tensor_cores else 0)
+        (ALLOW_TENSOR_CORES if allow_tensor_cores else 0) | _flags
     _check(lib().lutgemm_run_noalloc(m, n, batch, q, g, _ptr(packed), _ptr(alpha), _ptr(offset), _ptr(x),
                                      _ptr(y), flags, _stream(stream)),
            "lutgemm_run_noalloc")
+    if check:
+        _raise_if_bits(library_status(clear=True, stream=stream), "lutgemm_run_noalloc")
+    return y
+
+
+# ---------------------------------------------------------------------------
+# Mixed storage (2/4/16-bit in one matrix): per-block plane counts, sparse
+# fp16 outliers.  The format is described in include/lutgemm.h.
+# ---------------------------------------------------------------------------
+def mixed_offsets(block_planes: torch.Tensor, q_max: int, m: int, n: int) -> torch.Tensor:
+    """Host uint8 plane counts [ceil(n/1024)][ceil(m/32)] -> the block table
+    (exclusive prefix sums, 4096-byte units) as a host int32 tensor holding
+    the uint32 values, by lutgemm_mixed_offsets."""
+    ns, mt = -(-n // 1024), -(-m // 32)
+    bp = block_planes.contiguous()
+    if bp.dtype != torch.uint8 or bp.is_cuda or tuple(bp.shape) != (ns, mt):
+        raise ValueError(f"block_planes must be a host uint8 tensor [{ns}][{mt}]")
+    out = torch.empty(ns * mt + 1, dtype=torch.int32)
+    _check(lib().lutgemm_mixed_offsets(_ptr(bp), q_max, m, n, _ptr(out)), "lutgemm_mixed_offsets")
+    return out
+
+
+def pack_outliers(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, m: int, n: int):
+    """Host row-CSR outliers (int32 row_ptr [m+1], int32 col, fp16 val) ->
+    (optr, oent) host int32 tensors holding the kernel's uint32 layout."""
+    rp, c, v = row_ptr.contiguous(), col.contiguous(), val.contiguous()
+    if rp.dtype != torch.int32 or c.dtype != torch.int32 or v.dtype != torch.float16 or rp.numel() != m + 1 \
+            or rp.is_cuda or c.is_cuda or v.is_cuda or c.numel() != v.numel():
+        raise ValueError("outliers must be host tensors: int32 row_ptr [m+1], int32 col [nnz], fp16 val [nnz]")
+    nnz = c.numel()
+    optr = torch.empty(-(-n // 1024) * m + 1, dtype=torch.int32)
+    oent = torch.empty(max(nnz, 1), dtype=torch.int32)
+    _check(lib().lutgemm_pack_outliers(_ptr(rp), _ptr(c), _ptr(v), m, n, nnz, _ptr(optr), _ptr(oent)),
+           "lutgemm_pack_outliers")
+    return optr, oent[:nnz]
+
+
+def pack_bcq_mixed(signs: torch.Tensor, block_off: torch.Tensor, status_flags: torch.Tensor = None,
+                   stream=None) -> torch.Tensor:
+    """int8 signs [q_max][m][n] and the block table (int32, on the device) ->
+    the mixed packed planes, by lutgemm_pack_bcq_mixed."""
+    _need(signs, torch.int8, "signs")
+    q_max, m, n = signs.shape
+    _need(block_off, torch.int32, "block_off", -(-n // 1024) * -(-m // 32) + 1)
+    if status_flags is not None:
+        _need(status_flags, torch.int32, "status_flags", 1)
+    _one_device(stream, signs=signs, block_off=block_off, status_flags=status_flags)
+    nbytes = int(block_off[-1].item()) * 4096
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=signs.device)
+    _check(lib().lutgemm_pack_bcq_mixed(_ptr(signs), _ptr(block_off), q_max, m, n, _ptr(packed), nbytes,
+                                        _ptr(status_flags), _stream(stream)),
+           "lutgemm_pack_bcq_mixed")
+    return packed
+
+
+def run_mixed(packed: torch.Tensor, block_off: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int,
+              q_max: int, g: int, optr: torch.Tensor = None, oent: torch.Tensor = None, y: torch.Tensor = None,
+              workspace: torch.Tensor = None, y_f16: bool = False, check: bool = False, stream=None,
+              _flags: int = 0) -> torch.Tensor:
+    """y[b] = W x[b] for a mixed matrix, by lutgemm_run_mixed (outliers optional)."""
+    batch = _batch_of(x, n)
+    _need(packed, torch.uint8, "packed")
+    _need(block_off, torch.int32, "block_off", -(-n // 1024) * -(-m // 32) + 1)
+    _need(alpha, torch.float16, "alpha", q_max * _groups(n, g) * m)
+    _need(x, torch.float16, "x")
+    nnz = 0
+    if oent is not None:
+        _need(oent, torch.int32, "oent")
+        _need(optr, torch.int32, "optr", -(-n // 1024) * m + 1)
+        nnz = oent.numel()
+    if y is not None:
+        _need(y, torch.float16 if y_f16 else torch.float32, "y", batch * m)
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+    _one_device(stream, x=x, packed=packed, block_off=block_off, alpha=alpha, optr=optr, oent=oent, y=y,
+                workspace=workspace)
+    if y is None:
+        y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
+    if workspace is None:
+        workspace = new_workspace(m, n, batch, q_max, g, device=x.device)
+    flags = (Y_F16 if y_f16 else 0) | _flags
+    _check(lib().lutgemm_run_mixed(m, n, batch, q_max, g, _ptr(packed), packed.numel(), _ptr(block_off),
+                                   _ptr(alpha), _ptr(optr) if nnz else None, _ptr(oent) if nnz else None, nnz,
+                                   _ptr(x), _ptr(y), flags, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "lutgemm_run_mixed")
+    if check:
+        _raise_if_bits(workspace_status(workspace, clear=True, stream=stream), "lutgemm_run_mixed")
     return y

@@ -27,3 +27,27 @@ def algorithmic_bytes(m: int, n: int, q: int, g: int, batch: int = 1,
 def lookups(m: int, n: int, q: int, batch: int = 1) -> int:
     """Table reads of one matmul: one per (plane, row, 8-input run, batch column)."""
     return q * m * (n // 8) * batch
+
+
+def mixed_algorithmic_bytes(block_planes, m: int, n: int, g: int, batch: int = 1, nnz: int = 0,
+                            y_bytes: int = 4) -> int:
+    """Bytes one product in mixed storage cannot avoid moving: the stored
+    planes (4096 bytes per plane of every 32-row x 1024-input block), the fp16
+    scales of the stored planes (one per plane, row and group of g inputs
+    inside the block), the block table (4 bytes per block + 1), the outlier
+    pointers (4 bytes per (slice, row) + 1) and entries (4 bytes each) when
+    there are outliers, x and y.  block_planes: [n_s][m_t] plane counts."""
+    ns, mt = -(-n // 1024), -(-m // 32)
+    planes = 0
+    scales = 0
+    for s in range(ns):
+        k0, k1 = 1024 * s, min(n, 1024 * (s + 1))
+        groups = len(range(k0 // g, (k1 - 1) // g + 1))       # groups that meet this slice
+        for R in range(mt):
+            qb = int(block_planes[s][R])
+            rows = min(m, 32 * (R + 1)) - 32 * R
+            planes += 4096 * qb
+            scales += 2 * qb * rows * groups
+    table = 4 * (ns * mt + 1)
+    outl = (4 * (ns * m + 1) + 4 * nnz) if nnz > 0 else 0
+    return planes + scales + table + outl + 2 * batch * n + y_bytes * batch * m

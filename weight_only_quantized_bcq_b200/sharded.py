@@ -155,6 +155,22 @@ class ShardedLinear:
         self.alpha = alpha
         self.workspace = lutgemm.new_workspace(self.m, self.n, batch, plan.q, plan.g, device=signs.device)
 
+    @classmethod
+    def from_packed(cls, plan: ShardPlan, packed: torch.Tensor, alpha: torch.Tensor, group=None, batch: int = 1):
+        """A shard whose planes are already packed (``lutgemm.pack_bcq`` layout of
+        the local [q][m'][n'] matrix); alpha is [q][n'/g][m'] fp16."""
+        from . import lutgemm
+        self = cls.__new__(cls)
+        self.plan, self.group = plan, group
+        self.m, self.n = plan.local_m, plan.local_n
+        if self.m < 1 or self.n < 8:
+            raise ValueError("empty shard: use fewer ranks for this matrix")
+        if packed.numel() < lutgemm.packed_bytes(plan.q, self.m, self.n):
+            raise ValueError("packed buffer smaller than the shard's packed size")
+        self.packed, self.alpha = packed, alpha
+        self.workspace = lutgemm.new_workspace(self.m, self.n, batch, plan.q, plan.g, device=packed.device)
+        return self
+
     def local_product(self, x_local: torch.Tensor) -> torch.Tensor:
         from . import lutgemm
         b = x_local.shape[0]
