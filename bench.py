@@ -1022,6 +1022,26 @@ SWEEP = [("opt175b_qkv", 36864, 12288, 3, 128, (1, 2, 4, 8, 16, 32)),
          ("llama70b_down", 8192, 28672, 2, 64, (1, 2, 4, 8))]
 
 
+def _graph_us(fn, calls: int, stream, replays: int = 3) -> float:
+    """Microseconds per call of fn(0), fn(1), ..., fn(calls-1) captured in one
+    CUDA graph and replayed back to back: the device time of consecutive
+    launches, with no host launch overhead between them."""
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(calls):
+            fn(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(replays):
+        graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    del graph
+    return t0.elapsed_time(t1) * 1e3 / (calls * replays)
+
+
 def run_sweep(args):
     from weight_only_quantized_bcq_b200 import lutgemm
     torch.cuda.set_device(0)
@@ -1034,7 +1054,7 @@ def run_sweep(args):
         reps = 3   # distinct weight copies: consecutive launches miss L2
         bufs = [S.draw_random_bytes(gen, lutgemm.packed_bytes(q, m, n)).cuda() for _ in range(reps)]
         alpha = S.draw_alpha(gen, q, m, n, g, 0.02).cuda()
-        packed_scales = g % 128 == 0
+        packed_scales = g % 128 == 0 or g == 64
         scales = lutgemm.pack_scales(alpha, m, n, g) if packed_scales else alpha
         for b in batches:
             x = S.draw_x(gen, b, n).cuda()
@@ -1054,20 +1074,17 @@ def run_sweep(args):
                 b_.record(stream)
             torch.cuda.synchronize()
             iso = statistics.median(a_.elapsed_time(b_) for a_, b_ in ev) * 1e3
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for i in range(30):
-                run(i)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            b2b = e0.elapsed_time(e1) * 1e3 / 30
+            b2b = _graph_us(run, 30, stream)
             nbytes = algorithmic_bytes(m, n, q, g, b)
             # Lookups: q*m*n/8 table reads per batch column; one conflict-free
             # wavefront (32 reads) per clock per SM at the measured clock.
             lookups = q * m * n // 8 * b
             smem_floor = lookups / 32 / sm / 1.965e3
             line = {"config": name, "m": m, "n": n, "q": q, "g": g, "batch": b,
+                    "scales": "unit-major" if packed_scales else "[q][n/g][m]",
                     "us_isolated": round(iso, 1), "us_back_to_back": round(b2b, 1),
+                    "note": "isolated: events around one eager launch (includes launch latency); back to back: "
+                            "30 launches in a CUDA graph, three weight copies in turn",
                     "gbs_back_to_back": round(nbytes / (b2b * 1e-6) / 1e9, 1),
                     "hbm_floor_us": round(nbytes / (peak * 1e3), 1),
                     "smem_floor_us": round(smem_floor, 1),
@@ -1078,13 +1095,7 @@ def run_sweep(args):
                     lutgemm.run_tc(bufs[i % reps], alpha, x, m, n, q, g, y=y, stream=stream)
                 for i in range(3):
                     run_tc(i)
-                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                t0.record(stream)
-                for i in range(30):
-                    run_tc(i)
-                t1.record(stream)
-                torch.cuda.synchronize()
-                line["us_tensor_cores_back_to_back"] = round(t0.elapsed_time(t1) * 1e3 / 30, 1)
+                line["us_tensor_cores_back_to_back"] = round(_graph_us(run_tc, 30, stream), 1)
                 # lutgemm_run with LUTGEMM_ALLOW_TENSOR_CORES: the library's own choice
                 # (lookups, or tensor cores with K splits and the reduce).
                 def run_auto(i):
@@ -1092,12 +1103,7 @@ def run_sweep(args):
                                 stream=stream)
                 for i in range(3):
                     run_auto(i)
-                t0.record(stream)
-                for i in range(30):
-                    run_auto(i)
-                t1.record(stream)
-                torch.cuda.synchronize()
-                line["us_auto_back_to_back"] = round(t0.elapsed_time(t1) * 1e3 / 30, 1)
+                line["us_auto_back_to_back"] = round(_graph_us(run_auto, 30, stream), 1)
             print(json.dumps(line), flush=True)
 
 
@@ -1188,9 +1194,22 @@ def run_parallel(args):
 
     for _ in range(args.warmup):
         parallel_step(args.parallel, lins, x_in)
+    # The step as a CUDA graph (shard products and the NCCL collective), so
+    # the host's launch overhead is not timed; --graph-steps 0: eager.
+    graph = None
+    if args.graph_steps > 0:
+        side = torch.cuda.Stream(device=device)
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            y_graph = parallel_step(args.parallel, lins, x_in)
+        stream.wait_stream(side)
+        graph.replay()
+        barrier()
+    step_fn = graph.replay if graph is not None else (lambda: parallel_step(args.parallel, lins, x_in))
     with ClockSampler(torch.cuda.current_device()) as clocks:
-        region_ms = timed(lambda: parallel_step(args.parallel, lins, x_in), args.steps)
-    y = parallel_step(args.parallel, lins, x_in)
+        region_ms = timed(step_fn, args.steps)
+    y = y_graph if graph is not None else parallel_step(args.parallel, lins, x_in)
 
     # The products alone (no exchange), to give the collective's share.
     def products_only():
@@ -1208,6 +1227,8 @@ def run_parallel(args):
         y_host.copy_(parallel_step(args.parallel, lins, xi), non_blocking=True)
     e2e_ms = timed(e2e_step, args.steps)
 
+    if graph is not None:
+        del graph          # a graph holding NCCL work is released before the group is destroyed
     whole, mine = parallel_bytes(plans, batch)
     value = whole * args.steps / (region_ms * 1e-3) / 1e9
     peak, peak_kind = _peaks()
@@ -1224,7 +1245,9 @@ def run_parallel(args):
                        "bytes_per_step_whole": whole, "bytes_per_step_rank0": mine,
                        "l2": "no flush: every step streams each shard's weights once; a shard below 126 MB "
                              "may stay in L2 at large N",
-                       "launch": "eager launches; collectives by torch.distributed (NCCL)"},
+                       "launch": ("each step a CUDA graph replay (shard products + NCCL collective)"
+                                  if args.graph_steps > 0 else "eager launches") +
+                                 "; collectives by torch.distributed (NCCL)"},
             "products_ms_per_step": round(prod_ms / args.steps, 5),
             "collective_share": round(max(0.0, 1.0 - prod_ms / region_ms), 4),
             "roofline": {"bound": "hbm", "achieved": round(mine * args.steps / (region_ms * 1e-3) / 1e9, 1),
@@ -1317,17 +1340,38 @@ def run_mixed_workload(args):
     for k in range(args.warmup):
         step(k)
     barrier()
+    # The timed steps are replays of a CUDA graph of `per_graph` steps (the
+    # weight copies alternate inside it), as in the layer bench.
+    per_graph = args.graph_steps if args.graph_steps > 0 and args.steps % args.graph_steps == 0 else 0
+    graph = None
+    if per_graph:
+        if per_graph % reps:
+            per_graph = reps * max(1, per_graph // reps)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for k in range(per_graph):
+                step(k)
+        graph.replay()
+        barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_steps = args.steps if not per_graph else (args.steps // per_graph) * per_graph
     with ClockSampler(torch.cuda.current_device()) as clocks:
         barrier()
         t0.record(stream)
-        for k in range(args.steps):
-            step(k)
+        if graph is not None:
+            for _ in range(n_steps // per_graph):
+                graph.replay()
+        else:
+            for k in range(n_steps):
+                step(k)
         t1.record(stream)
         barrier()
     region_ms = max_over_ranks(pg, t0.elapsed_time(t1), device)
-    k_last = args.steps - 1
+    if graph is not None:
+        del graph
+    k_last = (per_graph - 1) if per_graph else (n_steps - 1)
     y_timed = [mt["y"].cpu().clone() for mt in mats]
+    b2b_us = {mt["name"]: _graph_us(lambda i, mt=mt: one(mt, i), 10, stream) for mt in mats}
     status = [lutgemm.workspace_status(mt["ws"]) for mt in mats]
     ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in mats]
           for _ in range(args.steps)]
@@ -1349,12 +1393,12 @@ def run_mixed_workload(args):
     barrier()
     e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1), device)
     step_bytes = sum(mt["bytes"] for mt in mats)
-    value = step_bytes * args.steps * world / (region_ms * 1e-3) / 1e9
+    value = step_bytes * n_steps * world / (region_ms * 1e-3) / 1e9
     peak, peak_kind = _peaks()
     if rank == 0:
         out = {
             "metric": MIXED_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(region_ms / args.steps, 5),
+            "steps": n_steps, "warmup": args.warmup, "ms_per_step": round(region_ms / n_steps, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "LLaMA-70B-shaped linears (8192x8192, 28672x8192, 8192x28672), mixed storage: "
                                    f"2-plane blocks, {args.mixed_hi:.3f} of blocks at 4 planes, "
@@ -1366,17 +1410,20 @@ def run_mixed_workload(args):
                              "(> 126 MB L2)",
                        "parallelism": "replicas" if world == 1 else f"replicas{world}"},
             "us_per_matmul": {k: round(v, 2) for k, v in us_per.items()},
-            "us_per_matmul_note": "median of isolated launches (events around each launch)",
-            "gbs_per_matmul": {mt["name"]: round(mt["bytes"] / (us_per[mt["name"]] * 1e-6) / 1e9, 1) for mt in mats},
+            "us_per_matmul_note": "median of isolated launches (events around each eager launch)",
+            "us_per_matmul_back_to_back": {k: round(v, 2) for k, v in b2b_us.items()},
+            "gbs_per_matmul_back_to_back": {mt["name"]: round(mt["bytes"] / (b2b_us[mt["name"]] * 1e-6) / 1e9, 1)
+                                            for mt in mats},
             "hbm_floor_us": {mt["name"]: round(mt["bytes"] / (peak * 1e3), 2) for mt in mats},
-            "roofline": {"bound": "hbm", "achieved": round(step_bytes * args.steps / (region_ms * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "hbm", "achieved": round(step_bytes * n_steps / (region_ms * 1e-3) / 1e9, 1),
                          "peak": peak, "unit": "GB/s",
-                         "frac": round(step_bytes * args.steps / (region_ms * 1e-3) / 1e9 / peak, 4),
+                         "frac": round(step_bytes * n_steps / (region_ms * 1e-3) / 1e9 / peak, 4),
                          "traffic": None, "peak_kind": peak_kind, "kernel": "lut_gemm_kernel (mixed)"},
             "e2e": {"value": round(step_bytes * args.steps * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": sum(mt["x_host"].numel() * 2 for mt in mats),
                     "d2h_bytes_per_step": sum(mt["y_host"].numel() * 4 for mt in mats)},
-            "gpu_launches": args.steps * len(mats) * 2,
+            "gpu_launches": n_steps * sum(1 + (mt["n"] > 1024) for mt in mats),
+            "gpu_launches_note": "lookup kernel and split-K reduce per call",
             "device_status": status,
             "clocks": clocks.summary(),
         }

@@ -62,18 +62,21 @@
  *   the q * 512 bytes a warp reads per step.
  *
  * Unit-major scale layout (produced by lutgemm_pack_scales, consumed by
- * lutgemm_run with LUTGEMM_SCALES_PACKED; only for g % 128 == 0, where every
- * 128-input piece has one scale per plane).  The pages fix no layout; this
- * one gives each lane the scales of a whole (slice, row tile) in 16*SP
+ * lutgemm_run with LUTGEMM_SCALES_PACKED; for g % 128 == 0, where every
+ * 128-input piece has one scale per plane, H = 1, and for g == 64, where it
+ * has two, one per 64-input half, H = 2).  The pages fix no layout; this one
+ * gives each lane the scales of a whole (slice, row tile) in 16*SP*H
  * contiguous bytes, so they arrive in a few 16-byte loads one tile ahead.
  *   SP = min(q, 4) planes per step, n_pg = ceil(q/4) plane groups.
- *   Element (s, R, pg, l, U, e) (pg < n_pg, l < 32, U < 8, e < SP) is the
- *   fp16 at element index ((((s * m_t + R) * n_pg + pg) * 32 + l) * 8 + U) * SP + e
+ *   Element (s, R, pg, l, U, e, h) (pg < n_pg, l < 32, U < 8, e < SP, h < H)
+ *   is the fp16 at element index
+ *   (((((s * m_t + R) * n_pg + pg) * 32 + l) * 8 + U) * SP + e) * H + h
  *   and holds alpha[4*pg + e][G][32*R + l] with
- *   G = (1024*s + 128*P) / g, P = U xor (4 * (l / 16)) (the piece lane l
- *   reads at step U).  It is 0 when 4*pg + e >= q, 32*R + l >= m or
- *   1024*s + 128*P >= n.  Size: n_s * m_t * n_pg * 512 * SP bytes (equal to
- *   the [q][n/g][m] array when g == 128, m % 32 == 0 and n % 1024 == 0).
+ *   G = (1024*s + 128*P + 64*h) / g, P = U xor (4 * (l / 16)) (the piece
+ *   lane l reads at step U).  It is 0 when 4*pg + e >= q, 32*R + l >= m or
+ *   1024*s + 128*P + 64*h >= n.  Size: n_s * m_t * n_pg * 512 * SP * H bytes
+ *   (equal to the [q][n/g][m] array when g is 128 or 64, m % 32 == 0 and
+ *   n % 1024 == 0).
  *
  * Other layouts (row-major, innermost last):
  *   signs  int8   [q][m][n]     each -1 or +1
@@ -122,7 +125,7 @@ extern "C" {
 
 /* Flags of lutgemm_run. */
 #define LUTGEMM_Y_F16          1u /* write y as fp16 (round to nearest even of the fp32 sum) */
-#define LUTGEMM_SCALES_PACKED  2u /* alpha is in the unit-major scale layout (g % 128 == 0) */
+#define LUTGEMM_SCALES_PACKED  2u /* alpha is in the unit-major scale layout (g % 128 == 0 or g == 64) */
 #define LUTGEMM_ALLOW_TENSOR_CORES 4u /* lutgemm_run may compute on the tensor cores (see there) */
 /* Test hook of lutgemm_run and lutgemm_run_noalloc, for checking error
  * reporting: every warp of the lookup kernel makes its first weight wait on
@@ -144,8 +147,9 @@ const char* lutgemm_status_string(int status);
 size_t lutgemm_packed_bytes(int q, int m, int n);
 
 /* Bytes of the unit-major scale buffer for (q, m, n, g):
- * ceil(n/1024) * ceil(m/32) * ceil(q/4) * 512 * min(q, 4).  Returns 0 for
- * invalid shapes and when g % 128 != 0.  Pure host function. */
+ * ceil(n/1024) * ceil(m/32) * ceil(q/4) * 512 * min(q, 4) * H, H = 2 for
+ * g == 64 and 1 otherwise.  Returns 0 for invalid shapes and unless
+ * g % 128 == 0 or g == 64.  Pure host function. */
 size_t lutgemm_scales_bytes(int q, int m, int n, int g);
 
 /* Bytes of the lutgemm_run workspace: [status word, 256 B | per-segment tile
@@ -284,10 +288,11 @@ int lutgemm_fit_bcq_grid(const uint16_t* w, int q, int m, int n, int g, int iter
  * are those of the BCQ format (LUT-GEMM card, Summary: q binary planes, each
  * with a scale per group of g inputs).
  *   alpha        dev fp16 [q][n/g][m], 2-byte aligned
- *   q, m, n, g   1 <= q <= 8, m >= 1, n % 8 == 0, g % 128 == 0, n % g == 0
+ *   q, m, n, g   1 <= q <= 8, m >= 1, n % 8 == 0, g % 128 == 0 or g == 64,
+ *                n % g == 0
  *   scales       dev, lutgemm_scales_bytes(q,m,n,g) bytes, 16-byte aligned
  *                (output, fully written)
- * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also for g % 128 != 0),
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also for other g),
  * ERR_ALIGN or ERR_CUDA. */
 int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
                         uint16_t* scales, void* stream);
@@ -305,7 +310,7 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *   packed     dev, packed layout above, 16-byte aligned
  *   alpha      dev fp16 [q][n/g][m], 2-byte aligned; with
  *              LUTGEMM_SCALES_PACKED the lutgemm_pack_scales output instead
- *              (16-byte aligned; g % 128 == 0), which gives the same bits
+ *              (16-byte aligned; g % 128 == 0 or g == 64), which gives the same bits
  *   offset     dev fp32 [n/g][m] or NULL (pure BCQ), 4-byte aligned
  *   x          dev fp16 [batch][n], 16-byte aligned
  *   y          dev [batch][m] fp32 (4-byte aligned) or, with LUTGEMM_Y_F16,
@@ -314,7 +319,7 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *   sums to the workspace and a reduce kernel adds them in slice order.
  *   flags      OR of LUTGEMM_Y_F16, LUTGEMM_SCALES_PACKED and
  *              LUTGEMM_ALLOW_TENSOR_CORES; other bits, or
- *              LUTGEMM_SCALES_PACKED with g % 128 != 0, give ERR_VALUE.
+ *              LUTGEMM_SCALES_PACKED with another g, give ERR_VALUE.
  *              With LUTGEMM_ALLOW_TENSOR_CORES the call computes the product
  *              on the tensor cores as lutgemm_run_tc does (same result within
  *              the same tolerance, not the same bits) when that path takes
@@ -328,8 +333,9 @@ int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g,
  *              counters are not touched.  Otherwise the flag changes
  *              nothing.
  *   workspace  dev, >= lutgemm_workspace_size(m,n,batch,q,g) bytes,
- *              16-byte aligned, zero-filled before its first use; left
- *              zero-filled by every successful call.  Calls that share a
+ *              16-byte aligned, zero-filled before its first use; its
+ *              counters are left zero by every call, its status word keeps
+ *              its bits until lutgemm_workspace_status clears them.  Calls that share a
  *              workspace must not overlap on the device.
  * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE or
  * ERR_CUDA. */
@@ -380,9 +386,13 @@ int lutgemm_run_tc(int m, int n, int batch, int q, int g,
  *     in (s, R) order, in 4096-byte units (lutgemm_mixed_offsets); the last
  *     entry is the total, and the packed buffer holds 4096 * total bytes;
  *   - packed planes: block (s, R) occupies q_b * 4096 bytes from byte
- *     4096 * table[s*m_t + R]; inside it chunk (U, i) (U < 8, i < q_b)
- *     sits at (U * q_b + i) * 512, with the byte map of the uniform layout
- *     (so all q_b = q gives lutgemm_pack_bcq's buffer);
+ *     4096 * table[s*m_t + R], its planes in pairs: pair h holds planes 2h
+ *     and 2h+1 (2h alone when q_b = 2h+1), e_h planes, from byte 8192 * h of
+ *     the block, and chunk (U, i') (U < 8, plane 2h + i') of the pair sits
+ *     at (U * e_h + i') * 512 from there, with the byte map of the uniform
+ *     layout (so blocks of at most two planes are laid out as
+ *     lutgemm_pack_bcq lays them out; the kernel streams a block one pair,
+ *     that is one pass, at a time);
  *   - alpha fp16 [q_max][n/g][m]: entries of planes a block does not store
  *     are never read;
  *   - outliers, as the caller gives them: row CSR, row_ptr int32 [m+1],
@@ -456,9 +466,12 @@ int lutgemm_run_mixed(int m, int n, int batch, int q_max, int g, const uint8_t* 
  *   Arguments, layouts and results are those of lutgemm_run, without the
  *   workspace.  Returns LUTGEMM_ERR_WORKSPACE when the problem needs more
  *   scratch than the array holds: more than 16 MiB - 4 KiB - 256 B of
- *   split-K partial sums (batch * ceil(n/1024) * ceil(m/32) * 128 bytes when
- *   n > 1024); a call that LUTGEMM_ALLOW_TENSOR_CORES sends to the tensor
- *   cores needs no scratch.  Other statuses as for lutgemm_run.
+ *   split-K partial sums (batch * ceil(n/1024) * ceil(m/32) * 128 bytes
+ *   when n > 1024; with one slice none are needed).  With
+ *   LUTGEMM_ALLOW_TENSOR_CORES a problem the tensor-core path takes runs
+ *   there with one K split, which needs no scratch, when lutgemm_run would
+ *   take that path or when the partials would not fit.  Other statuses as
+ *   for lutgemm_run.
  *   The first call on a device does a one-time set-up on that device (looks
  *   up the array's device address and zeroes its counters on `stream`); make
  *   that first call before any stream capture.  Every call shares the one

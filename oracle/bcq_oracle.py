@@ -262,21 +262,24 @@ def packed_row_tiles(packed, q: int, m: int, n: int, R0: int, R1: int):
 
 # ---------------------------------------------------------------------------
 # Unit-major scale layout (this library's own; defined in include/lutgemm.h).
-# Only for g % 128 == 0.  SP = min(q, 4), n_pg = ceil(q / 4).  Element
-# (s, R, pg, l, U, e) sits at index
-#   ((((s * m_t + R) * n_pg + pg) * 32 + l) * 8 + U) * SP + e
-# and holds alpha[4*pg + e][G][32*R + l], G = (1024*s + 128*P) // g,
-# P = U xor (4 * (l // 16)); 0 when the plane, row or piece is out of range.
+# For g % 128 == 0 (one scale per 128-input piece, H = 1) and g == 64 (two,
+# one per 64-input half of a piece, H = 2).  SP = min(q, 4), n_pg = ceil(q/4).
+# Element (s, R, pg, l, U, e, h) sits at index
+#   (((((s * m_t + R) * n_pg + pg) * 32 + l) * 8 + U) * SP + e) * H + h
+# and holds alpha[4*pg + e][G][32*R + l], G = (1024*s + 128*P + 64*h) // g,
+# P = U xor (4 * (l // 16)); 0 when the plane, row or piece half is out of
+# range.
 # ---------------------------------------------------------------------------
 def _scale_dims(q: int, m: int, n: int, g: int):
-    if g % PIECE != 0 or n % g != 0:
-        raise ValueError("the unit-major scale layout needs g % 128 == 0 and n % g == 0")
-    return math.ceil(n / SLICE), math.ceil(m / TILE_ROWS), min(q, 4), math.ceil(q / 4)
+    if not (g % PIECE == 0 or g == PIECE // 2) or n % g != 0:
+        raise ValueError("the unit-major scale layout needs g % 128 == 0 or g == 64, and n % g == 0")
+    return (math.ceil(n / SLICE), math.ceil(m / TILE_ROWS), min(q, 4), math.ceil(q / 4),
+            2 if g == PIECE // 2 else 1)
 
 
 def scales_nbytes(q: int, m: int, n: int, g: int) -> int:
-    ns, mt, sp, npg = _scale_dims(q, m, n, g)
-    return ns * mt * npg * 512 * sp
+    ns, mt, sp, npg, H = _scale_dims(q, m, n, g)
+    return ns * mt * npg * 512 * sp * H
 
 
 def pack_scales(alpha, g: int) -> np.ndarray:
@@ -284,26 +287,27 @@ def pack_scales(alpha, g: int) -> np.ndarray:
     a = np.asarray(alpha, dtype=np.float16)
     q, ng, m = a.shape
     n = ng * g
-    ns, mt, sp, npg = _scale_dims(q, m, n, g)
-    out = np.zeros((ns, mt, npg, TILE_ROWS, 8, sp), dtype=np.float16)
+    ns, mt, sp, npg, H = _scale_dims(q, m, n, g)
+    out = np.zeros((ns, mt, npg, TILE_ROWS, 8, sp, H), dtype=np.float16)
     for s_ in range(ns):
         for U in range(8):
             for half in range(2):                       # l // 16
                 P = U ^ (4 * half)
-                k0 = SLICE * s_ + PIECE * P
-                if k0 >= n:
-                    continue                            # piece beyond n: stays 0
-                G = k0 // g
-                for pg in range(npg):
-                    for e in range(sp):
-                        i = 4 * pg + e
-                        if i >= q:
-                            continue                    # padding plane: stays 0
-                        col = np.zeros(mt * TILE_ROWS, dtype=np.float16)
-                        col[:m] = a[i, G, :]
-                        col = col.reshape(mt, TILE_ROWS)
-                        lanes = slice(16 * half, 16 * half + 16)
-                        out[s_, :, pg, lanes, U, e] = col[:, lanes]
+                for h in range(H):
+                    k0 = SLICE * s_ + PIECE * P + (PIECE // 2) * h
+                    if k0 >= n:
+                        continue                        # beyond n: stays 0
+                    G = k0 // g
+                    for pg in range(npg):
+                        for e in range(sp):
+                            i = 4 * pg + e
+                            if i >= q:
+                                continue                # padding plane: stays 0
+                            col = np.zeros(mt * TILE_ROWS, dtype=np.float16)
+                            col[:m] = a[i, G, :]
+                            col = col.reshape(mt, TILE_ROWS)
+                            lanes = slice(16 * half, 16 * half + 16)
+                            out[s_, :, pg, lanes, U, e, h] = col[:, lanes]
     return out.reshape(-1)
 
 
@@ -312,27 +316,28 @@ def unpack_scales(scales, q: int, m: int, n: int, g: int) -> np.ndarray:
 
     A group wider than one piece appears once per piece; every copy must agree.
     """
-    ns, mt, sp, npg = _scale_dims(q, m, n, g)
-    buf = np.asarray(scales, dtype=np.float16).reshape(ns, mt, npg, TILE_ROWS, 8, sp)
+    ns, mt, sp, npg, H = _scale_dims(q, m, n, g)
+    buf = np.asarray(scales, dtype=np.float16).reshape(ns, mt, npg, TILE_ROWS, 8, sp, H)
     ng = n // g
     out = np.full((q, ng, m), np.nan, dtype=np.float64)
     for s_ in range(ns):
         for U in range(8):
             for l in range(TILE_ROWS):
                 P = U ^ (4 * (l // 16))
-                k0 = SLICE * s_ + PIECE * P
-                if k0 >= n:
-                    continue
-                G = k0 // g
-                rows = np.arange(mt) * TILE_ROWS + l
-                ok = rows < m
-                for i in range(q):
-                    v = buf[s_, :, i // 4, l, U, i % 4].astype(np.float64)[ok]
-                    prev = out[i, G, rows[ok]]
-                    seen = ~np.isnan(prev)
-                    if np.any(prev[seen] != v[seen]):
-                        raise ValueError("copies of one group scale disagree")
-                    out[i, G, rows[ok]] = v
+                for h in range(H):
+                    k0 = SLICE * s_ + PIECE * P + (PIECE // 2) * h
+                    if k0 >= n:
+                        continue
+                    G = k0 // g
+                    rows = np.arange(mt) * TILE_ROWS + l
+                    ok = rows < m
+                    for i in range(q):
+                        v = buf[s_, :, i // 4, l, U, i % 4, h].astype(np.float64)[ok]
+                        prev = out[i, G, rows[ok]]
+                        seen = ~np.isnan(prev)
+                        if np.any(prev[seen] != v[seen]):
+                            raise ValueError("copies of one group scale disagree")
+                        out[i, G, rows[ok]] = v
     if np.isnan(out).any():
         raise ValueError("some scale never appears in the buffer")
     return out.astype(np.float16)
@@ -601,9 +606,13 @@ def fit_bcq_grid_trace(w, q: int, g: int, iters: int):
 #     position out; a fitter stores the outlier's residual);
 #   * packed planes: blocks in (s, R) order, block (s, R) holds q_b * 4096
 #     bytes from byte 4096 * off[s * m_t + R], off the exclusive prefix sum
-#     of q_b in that order; inside a block, chunk (U, i) sits at
-#     (U * q_b + i) * 512 with the byte map of the uniform layout (so with
-#     q_b = q everywhere the buffer equals pack_bcq's);
+#     of q_b in that order; inside a block the planes are stored in pairs:
+#     pair h holds planes 2h and 2h+1 (only 2h when q_b = 2h + 1), e_h of
+#     them, from byte 8192 * h of the block, and its chunk (U, i') (plane
+#     2h + i') sits at (U * e_h + i') * 512 from there, with the byte map of
+#     the uniform layout (so a block of at most two planes is laid out as
+#     pack_bcq lays it out; pairs let the kernel move two planes per copy
+#     whatever the block's count);
 #   * outliers for the kernel: slice-major CSR, the entries of (slice s,
 #     row r) at [optr[s * m + r], optr[s * m + r + 1]), sorted by input, each
 #     a uint32 (k - 1024 s) | (fp16 bits << 16).
@@ -631,10 +640,16 @@ def mixed_packed_nbytes(block_planes) -> int:
     return int(np.asarray(block_planes, dtype=np.int64).sum()) * BLOCK_BYTES
 
 
+def _plane_pairs(qb: int):
+    """(first plane, planes) of each stored pair of a block with qb planes."""
+    return [(2 * h, min(2, qb - 2 * h)) for h in range((qb + 1) // 2)]
+
+
 def pack_mixed(signs, block_planes) -> np.ndarray:
     """int8 signs [q_max][m][n] -> the mixed packed buffer.  Block (s, R)
-    stores planes 0 .. q_b - 1 of its rows and inputs, packed as a one-tile,
-    one-slice matrix by ``pack_bcq``; planes from q_b on are not stored."""
+    stores planes 0 .. q_b - 1 of its rows and inputs, pair by pair, each
+    pair packed as a one-tile, one-slice matrix by ``pack_bcq``; planes from
+    q_b on are not stored."""
     sg = np.asarray(signs)
     q_max, m, n = sg.shape
     bp = _check_blocks(block_planes, m, n)
@@ -645,8 +660,9 @@ def pack_mixed(signs, block_planes) -> np.ndarray:
     for s_ in range(ns):
         for R in range(mt):
             qb = int(bp[s_, R])
-            blk = sg[:qb, TILE_ROWS * R: TILE_ROWS * (R + 1), SLICE * s_: SLICE * (s_ + 1)]
-            parts.append(pack_bcq(blk))
+            for i0, e in _plane_pairs(qb):
+                blk = sg[i0: i0 + e, TILE_ROWS * R: TILE_ROWS * (R + 1), SLICE * s_: SLICE * (s_ + 1)]
+                parts.append(pack_bcq(blk))
     return np.concatenate(parts)
 
 
@@ -665,8 +681,10 @@ def unpack_mixed(packed, block_planes, q_max: int, m: int, n: int) -> np.ndarray
             qb = int(bp[s_, R])
             r0, k0 = TILE_ROWS * R, SLICE * s_
             mr, nk = min(m, r0 + TILE_ROWS) - r0, min(n, k0 + SLICE) - k0
-            blk = pk[int(off[u]) * BLOCK_BYTES: int(off[u + 1]) * BLOCK_BYTES]
-            out[:qb, r0: r0 + mr, k0: k0 + nk] = unpack_bcq_vec(blk, qb, mr, nk)
+            base = int(off[u]) * BLOCK_BYTES
+            for i0, e in _plane_pairs(qb):
+                blk = pk[base + i0 * BLOCK_BYTES: base + (i0 + e) * BLOCK_BYTES]
+                out[i0: i0 + e, r0: r0 + mr, k0: k0 + nk] = unpack_bcq_vec(blk, e, mr, nk)
     return out
 
 
@@ -765,8 +783,10 @@ def mixed_matmul_tiles(x, packed, block_planes, alpha, g: int, m: int, n: int, t
             qb = int(bp[s_, R])
             k0 = SLICE * s_
             nk = min(n, k0 + SLICE) - k0
-            blk = pk[int(off[u]) * BLOCK_BYTES: int(off[u + 1]) * BLOCK_BYTES]
-            signs[:qb, r0: r0 + mr, k0: k0 + nk] = unpack_bcq_vec(blk, qb, mr, nk)
+            base = int(off[u]) * BLOCK_BYTES
+            for i0, e in _plane_pairs(qb):
+                blk = pk[base + i0 * BLOCK_BYTES: base + (i0 + e) * BLOCK_BYTES]
+                signs[i0: i0 + e, r0: r0 + mr, k0: k0 + nk] = unpack_bcq_vec(blk, e, mr, nk)
         r0 += mr
     sub = None
     if outliers is not None:

@@ -112,17 +112,19 @@ def test_run_rejects_bad_flags_and_small_workspace(L):
     assert _run(L, flags=8) == L.ERR_VALUE
     assert _run(L, flags=16 | L.Y_F16) == L.ERR_VALUE
     assert _run(L, flags=8 | L.ALLOW_TENSOR_CORES) == L.ERR_VALUE
-    # Unit-major scales need g % 128 == 0 and a 16-byte aligned scale buffer.
-    assert _run(L, n=1024, g=64, flags=L.SCALES_PACKED) == L.ERR_VALUE
+    # Unit-major scales need g % 128 == 0 or g == 64 and a 16-byte aligned scale buffer.
+    assert _run(L, n=1024, g=32, flags=L.SCALES_PACKED) == L.ERR_VALUE
+    assert _run(L, n=1024, g=64, flags=L.SCALES_PACKED, alpha=FAKE + 2) == L.ERR_ALIGN
     assert _run(L, alpha=FAKE + 2, flags=L.SCALES_PACKED) == L.ERR_ALIGN
     need = L.workspace_size(64, 1024, 1, 3, 128)
     assert _run(L, ws_bytes=need - 1) == L.ERR_WORKSPACE
 
 
 def test_scales_bytes(L):
-    for q, m, n, g in [(3, 40, 2048, 128), (5, 70, 2048, 256), (2, 33, 640, 128), (8, 1, 1024, 1024)]:
+    for q, m, n, g in [(3, 40, 2048, 128), (5, 70, 2048, 256), (2, 33, 640, 128), (8, 1, 1024, 1024),
+                       (2, 40, 2048, 64), (6, 33, 640, 64)]:
         assert L.scales_bytes(q, m, n, g) == O.scales_nbytes(q, m, n, g)
-    assert L.scales_bytes(3, 64, 1024, 64) == 0        # g % 128 != 0
+    assert L.scales_bytes(3, 64, 1024, 32) == 0        # neither g % 128 == 0 nor g == 64
     assert L.scales_bytes(3, 64, 1000, 128) == 0       # n % g != 0
     assert L.scales_bytes(9, 64, 1024, 128) == 0
 
@@ -194,7 +196,7 @@ def test_pack_scales_validation(L):
     lib = L.lib()
     assert lib.lutgemm_pack_scales(None, 3, 32, 1024, 128, FAKE, None) == L.ERR_NULL
     assert lib.lutgemm_pack_scales(FAKE, 3, 32, 1024, 128, None, None) == L.ERR_NULL
-    assert lib.lutgemm_pack_scales(FAKE, 3, 32, 1024, 64, FAKE, None) == L.ERR_SHAPE
+    assert lib.lutgemm_pack_scales(FAKE, 3, 32, 1024, 32, FAKE, None) == L.ERR_SHAPE
     assert lib.lutgemm_pack_scales(FAKE, 0, 32, 1024, 128, FAKE, None) == L.ERR_SHAPE
     assert lib.lutgemm_pack_scales(FAKE + 1, 3, 32, 1024, 128, FAKE, None) == L.ERR_ALIGN
     assert lib.lutgemm_pack_scales(FAKE, 3, 32, 1024, 128, FAKE + 8, None) == L.ERR_ALIGN

@@ -225,7 +225,8 @@ def test_full_size_sampled(L, name, m, n, q, g, batch, sigma, outl, seed):
 # with packed scales gives the same bits as a run with the [q][n/g][m] array.
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("q,m,n,g", [(1, 32, 1024, 128), (3, 40, 2048, 128), (2, 33, 640, 128),
-                                     (4, 100, 3072, 384), (5, 70, 2048, 256), (8, 33, 1152, 128)])
+                                     (4, 100, 3072, 384), (5, 70, 2048, 256), (8, 33, 1152, 128),
+                                     (2, 40, 2048, 64), (3, 33, 640, 64), (6, 64, 1024, 64)])
 def test_pack_scales_bit_exact(L, q, m, n, g):
     alpha = S.draw_alpha(S.generator(300 + q), q, m, n, g, 0.02)
     scales = L.pack_scales(alpha.to(DEV), m, n, g)
@@ -244,6 +245,10 @@ PACKED_CASES = [
     (4, 130, 4096, 512, 4, False, False),
     (5, 70, 2048, 256, 1, False, False),
     (8, 129, 3072, 128, 2, True, True),
+    (2, 300, 3072, 64, 1, False, False),      # g = 64: two scales per piece
+    (2, 257, 2560, 64, 3, True, False),
+    (3, 97, 640, 64, 2, False, True),
+    (5, 70, 2048, 64, 1, True, False),
 ]
 
 
@@ -287,11 +292,32 @@ def test_packed_scales_full_size_fc1(L):
 
 
 def test_packed_scales_rejected_for_small_groups(L):
-    signs, alpha, x = _problem(88, 3, 64, 1024, 64, 1)
+    signs, alpha, x = _problem(88, 3, 64, 1024, 32, 1)
     packed = L.pack_bcq(signs.to(DEV))
     with pytest.raises(L.LutgemmError) as e:
-        L.run(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 64, scales_packed=True)
+        L.run(packed, alpha.to(DEV), x.to(DEV), 64, 1024, 3, 32, scales_packed=True)
     assert e.value.status == L.ERR_VALUE
+
+
+def test_packed_scales_full_size_llama_up_g64(L):
+    """LLaMA-70B up-projection shape (28672 x 8192, q = 2, g = 64) with the
+    g = 64 unit-major scales at batch 1: the same bits as the [q][n/g][m]
+    scales, and sampled rows against the oracle."""
+    m, n, q, g, seed = 28672, 8192, 2, 64, 3
+    gen = S.generator(seed)
+    packed = S.draw_random_bytes(gen, O.packed_nbytes(q, m, n)).to(DEV)
+    alpha = S.draw_alpha(gen, q, m, n, g, 0.03)
+    x = S.draw_x(gen, 1, n, outlier_frac=0.001)
+    scales = L.pack_scales(alpha.to(DEV), m, n, g)
+    y_pk = L.run(packed, scales, x.to(DEV), m, n, q, g, scales_packed=True, check=True)
+    y_raw = L.run(packed, alpha.to(DEV), x.to(DEV), m, n, q, g, check=True)
+    assert torch.equal(y_pk, y_raw)
+    rows = _sample_rows(m, seed=seed)
+    s_rows = O.unpack_rows(packed.cpu().numpy(), q, m, n, rows)
+    a_rows = alpha.numpy()[:, :, rows]
+    ok, st = compare(y_pk.cpu().numpy()[:, rows], O.bcq_matmul_rows(x.numpy(), s_rows, a_rows, g), a_rows,
+                     x.numpy(), n)
+    assert ok, st
 
 
 # ---------------------------------------------------------------------------

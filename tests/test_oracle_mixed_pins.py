@@ -44,6 +44,18 @@ def pin_layout_golden(pack_mixed, offsets) -> bool:
     return np.array_equal(np.asarray(pack_mixed(_layout_signs(c), bp)), want)
 
 
+def pin_pairs_golden(pack_mixed) -> bool:
+    """Blocks of three and four planes: the planes are stored in pairs."""
+    for c in _gold()["pairs_cases"]:
+        bp = np.array(c["block_planes"], dtype=np.uint8)
+        want = np.zeros(c["total_bytes"], dtype=np.uint8)
+        for off, v in c["nonzero"].items():
+            want[int(off)] = v
+        if not np.array_equal(np.asarray(pack_mixed(_layout_signs(c), bp)), want):
+            return False
+    return True
+
+
 def pin_unpack_golden(unpack_mixed) -> bool:
     c = _gold()["layout_case"]
     bp = np.array(c["block_planes"], dtype=np.uint8)
@@ -137,7 +149,14 @@ def pin_bruteforce(matmul) -> bool:
 # ---------------------------------------------------------------------------
 def test_mixed_layout_pins():
     assert pin_layout_golden(O.pack_mixed, O.mixed_block_offsets)
+    assert pin_pairs_golden(O.pack_mixed)
     assert pin_unpack_golden(O.unpack_mixed)
+    for c in _gold()["pairs_cases"]:
+        bp = np.array(c["block_planes"], dtype=np.uint8)
+        buf = np.zeros(c["total_bytes"], dtype=np.uint8)
+        for off, v in c["nonzero"].items():
+            buf[int(off)] = v
+        assert np.array_equal(O.unpack_mixed(buf, bp, c["q_max"], c["m"], c["n"]), _layout_signs(c))
 
 
 def test_mixed_value_pins():
@@ -151,12 +170,14 @@ def test_outlier_layout_pin():
 
 @pytest.mark.parametrize("q,m,n,g", [(3, 45, 2056, 8), (2, 70, 3000, 40), (4, 33, 1032, 8)])
 def test_equal_plane_counts_reduce_to_plain_bcq(q, m, n, g):
-    """Every block at q planes and no outliers: the buffer is pack_bcq's and
-    the product is bcq_matmul's."""
+    """Every block at q planes and no outliers: the product is bcq_matmul's,
+    and with at most two planes the buffer is pack_bcq's."""
     signs, alpha, _, _, x = _random_mixed(q + m, q, m, n, g)
     bp = np.full((-(-n // 1024), -(-m // 32)), q, dtype=np.uint8)
-    assert np.array_equal(O.pack_mixed(signs, bp), O.pack_bcq(signs))
     assert np.array_equal(O.mixed_matmul(x, signs, alpha, bp, g), O.bcq_matmul(x, signs, alpha, g))
+    s2 = signs[:2]
+    bp2 = np.full_like(bp, 2)
+    assert np.array_equal(O.pack_mixed(s2, bp2), O.pack_bcq(s2))
 
 
 def test_outliers_alone_are_the_sparse_product():
@@ -265,9 +286,21 @@ def _pack_plane_major(signs, bp):
     return np.concatenate(out)
 
 
+def _pack_unpaired(signs, bp):
+    # All of a block's planes in one chunk sequence: chunk (U, i) at (U*q_b + i)*512.
+    out = []
+    bp = np.asarray(bp)
+    for s_ in range(bp.shape[0]):
+        for R in range(bp.shape[1]):
+            qb = int(bp[s_, R])
+            out.append(O.pack_bcq(signs[:qb, 32 * R: 32 * R + 32, 1024 * s_: 1024 * s_ + 1024]))
+    return np.concatenate(out)
+
+
 def test_layout_pins_catch_mistakes():
     assert not pin_layout_golden(O.pack_mixed, _offsets_inclusive)
-    assert not pin_layout_golden(_pack_plane_major, O.mixed_block_offsets)
+    assert not (pin_layout_golden(_pack_plane_major, O.mixed_block_offsets) and pin_pairs_golden(_pack_plane_major))
+    assert not pin_pairs_golden(_pack_unpaired)
 
 
 def _outliers_absolute_k(rp, col, val, m, n):

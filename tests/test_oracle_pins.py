@@ -526,7 +526,8 @@ def test_scales_pins():
 
 
 @pytest.mark.parametrize("q,m,n,g", [(1, 32, 1024, 128), (3, 40, 2048, 128), (4, 100, 3072, 384),
-                                     (5, 70, 2048, 256), (8, 33, 1152, 128), (2, 33, 640, 128)])
+                                     (5, 70, 2048, 256), (8, 33, 1152, 128), (2, 33, 640, 128),
+                                     (2, 40, 2048, 64), (3, 33, 640, 64), (6, 64, 1024, 64)])
 def test_scales_roundtrip(q, m, n, g):
     alpha = _distinct_alpha(q, n // g, m)
     packed = O.pack_scales(alpha, g)
@@ -537,12 +538,14 @@ def test_scales_roundtrip(q, m, n, g):
     # once per piece of its group that lies inside n.
     vals = packed.view(np.uint16)
     counts = np.bincount(vals, minlength=alpha.size + 1)
-    assert np.all(counts[1:] == g // 128)
+    assert np.all(counts[1:] == max(1, g // 128))
 
 
-def test_scales_reject_groups_below_a_piece():
+def test_scales_reject_groups_below_half_a_piece():
     with pytest.raises(ValueError):
-        O.scales_nbytes(3, 32, 1024, 64)
+        O.scales_nbytes(3, 32, 1024, 32)
+    with pytest.raises(ValueError):
+        O.scales_nbytes(3, 32, 1024, 192)
 
 
 def _scales_pieces_not_swapped(alpha, g):
@@ -601,7 +604,15 @@ def _scales_group_per_run(alpha, g):
     return out.reshape(-1)
 
 
-@pytest.mark.parametrize("mutant", [_scales_pieces_not_swapped, _scales_step_major, _scales_planes_reversed,
+def _scales_halves_swapped(alpha, g):
+    # g = 64: the two halves of a piece in the wrong order.
+    out = O.pack_scales(alpha, g)
+    if g == 64:
+        out = out.reshape(-1, 2)[:, ::-1].reshape(-1).copy()
+    return out
+
+
+@pytest.mark.parametrize("mutant", [_scales_halves_swapped, _scales_pieces_not_swapped, _scales_step_major, _scales_planes_reversed,
                                     _scales_group_per_run])
 def test_scales_pins_catch_mistakes(mutant):
     assert not pin_scales_golden(mutant)

@@ -126,6 +126,15 @@ def _rank_main(rank, world, port, outdir):
         s, a = T.take_shard(pr, signs, alpha)
         y = T.gather_rows(pr, _oracle(x, s, a, g), None)
         res["rows"] = float((y - full).abs().max() / full.abs().max())
+        # Rows, one batch column and equal ranges: the direct gather.
+        m_eq = 64 * world
+        s_eq, a_eq, x_eq = _problem(q, m_eq, n, g, 1, seed=8)
+        pe = T.plan_rows(m_eq, n, q, g, world, rank)
+        assert pe.m == pe.world * pe.span
+        se, ae = T.take_shard(pe, s_eq, a_eq)
+        ye = T.gather_rows(pe, _oracle(x_eq, se, ae, g), None)
+        full_eq = _oracle(x_eq, s_eq, a_eq, g)
+        res["rows_eq"] = float((ye - full_eq).abs().max() / full_eq.abs().max())
         # Inputs: each rank's partial product over its groups, summed.
         pi = T.plan_inputs(m, n, q, g, world, rank)
         s, a = T.take_shard(pi, signs, alpha)
@@ -165,6 +174,7 @@ def test_sharded_products_equal_the_whole_matrix(tmp_path, world):
         res = json.load(open(tmp_path / f"rank{r}.json"))
         # FP64 on both sides: only the summation order differs.
         assert res["rows"] < 1e-13, res
+        assert res["rows_eq"] < 1e-13, res
         assert res["inputs"] < 1e-13, res
         assert res["scatter"] < 1e-13, res
         assert res["paired"] < 1e-12, res

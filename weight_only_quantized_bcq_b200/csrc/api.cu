@@ -231,9 +231,10 @@ size_t lutgemm_packed_bytes(int q, int m, int n) {
 }
 
 size_t lutgemm_scales_bytes(int q, int m, int n, int g) {
-  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g % 128 != 0) return 0;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || !(g % 128 == 0 || g == 64)) return 0;
   const size_t sp = q < 4 ? (size_t)q : 4u;
-  return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * ceil_div(q, 4) * 512u * sp;
+  const size_t halves = g == 64 ? 2u : 1u;
+  return (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * ceil_div(q, 4) * 512u * sp * halves;
 }
 
 int lutgemm_run_tc(int m, int n, int batch, int q, int g, const uint8_t* packed, const uint16_t* alpha,
@@ -279,7 +280,7 @@ int lutgemm_fit_bcq_grid(const uint16_t* w, int q, int m, int n, int g, int iter
 
 int lutgemm_pack_scales(const uint16_t* alpha, int q, int m, int n, int g, uint16_t* scales, void* stream) {
   if (!alpha || !scales) return LUTGEMM_ERR_NULL;
-  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || g % 128 != 0) return LUTGEMM_ERR_SHAPE;
+  if (!valid_matrix(q, m, n) || !valid_groups(n, g) || !(g % 128 == 0 || g == 64)) return LUTGEMM_ERR_SHAPE;
   if (!aligned(alpha, 2) || !aligned(scales, 16)) return LUTGEMM_ERR_ALIGN;
   const cudaError_t err = launch_pack_scales(reinterpret_cast<const __half*>(alpha), q, m, n, g, scales,
                                              reinterpret_cast<cudaStream_t>(stream));
@@ -367,7 +368,7 @@ int lutgemm_run(int m, int n, int batch, int q, int g, const uint8_t* packed, co
   const bool stall = (flags & LUTGEMM_TEST_STALL) != 0u;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
-  if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
+  if (scales_packed && !(g % 128 == 0 || g == 64)) return LUTGEMM_ERR_VALUE;
   if (!aligned(packed, 16) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(offset, 4) ||
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
     return LUTGEMM_ERR_ALIGN;

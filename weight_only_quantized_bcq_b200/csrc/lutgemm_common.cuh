@@ -148,6 +148,17 @@ using RunKernel = void (*)(RunParams);
 // the run kernel when ns > 1 (programmatic launch: it waits for the run).
 cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream);
 
+// The fixed order in which the reduce kernel adds a row's slice partials: 2^L slice lanes, the
+// smallest power of two (at most 32) that leaves each lane at most two
+// slices; lane l adds slices l*per .. l*per + per - 1 (per = ceil(ns / 2^L))
+// in order, in batches of 8 padded with +0, and the lane sums are added in
+// lane order.
+__host__ __device__ inline int reduce_lanes_log2(int ns) {
+  int sl_log2 = 0;
+  while (sl_log2 < 5 && ((ns + (1 << sl_log2) - 1) >> sl_log2) > 2) ++sl_log2;
+  return sl_log2;
+}
+
 constexpr unsigned kStatusWindow = 1u;
 constexpr unsigned kStatusTimeout = 2u;
 constexpr unsigned kStatusFormat = 4u;   // a mixed-storage block or outlier entry out of range

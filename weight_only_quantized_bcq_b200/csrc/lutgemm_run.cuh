@@ -232,9 +232,11 @@ __device__ __forceinline__ void static_for(std::integer_sequence<int, Is...>, F&
 
 }  // namespace detail
 
-// MIXED: mixed storage (lutgemm_run_mixed).  Every (slice, row tile) block
-// holds its own number of planes, 1..Q, at the offset p.block_off gives, and
-// sparse fp16 outliers (slice-major CSR) are added to each row's sum.
+// MIXED: mixed storage (lutgemm_run_mixed), with Q = 2.  Every (slice, row
+// tile) block holds its own number of planes, 1..4, at the offset
+// p.block_off gives, stored in pairs; a block is one pass per pair (one or
+// two), each pass moving two planes per step like the q = 2 kernel.  Sparse
+// fp16 outliers (slice-major CSR) are added to each row's sum.
 template <int Q, int MODE, bool MULTI, bool HAS_OFF, bool PK, bool MIXED = false>
 __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p) {
   using namespace detail;
@@ -244,9 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr uint32_t STEP_BYTES = 512u * SP;
   constexpr uint32_t STAGE_BYTES = STEP_BYTES * CH;
   static_assert(!MULTI || CH == 1, "plane groups are fetched one step at a time");
-  static_assert(!MIXED || (Q <= 4 && !MULTI && !HAS_OFF && !PK), "mixed storage: up to 4 planes, [q][n/g][m] scales");
+  static_assert(!MIXED || (Q == 2 && !MULTI && !HAS_OFF && !PK), "mixed storage: plane pairs, [q][n/g][m] scales");
+  constexpr uint32_t QB_MAX = MIXED ? 4u : (uint32_t)Q;   // planes of one mixed block
   static_assert(S >= 2 && S <= 7, "weight ring of 2..7 stages (barrier slot 7 is the test hook's)");
-  constexpr int NPG = MULTI ? 2 : 1;                   // plane groups of a unit
+  constexpr int NPG = (MULTI || MIXED) ? 2 : 1;        // plane groups of a unit (at most)
+  constexpr int GP = MIXED ? 2 : 4;                    // planes per plane group
 
   extern __shared__ __align__(16) unsigned char smem[];
   // Let the next kernel in the stream start on SMs as they free up; it waits
@@ -266,8 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr int APP = RUN >= 8 ? 16 / RUN : 1;      // prefetched scales per piece
   constexpr bool PRE_ALPHA = RUN >= 8;
   // Scales in the unit-major layout: p.alpha holds, for every (slice, row
-  // tile, plane group, lane), the 8 x SP scales of that lane's pass.
-  static_assert(!PK || RUN == 16, "unit-major scales need one scale per piece");
+  // tile, plane group, lane), the 8 x SP x HPK scales of that lane's pass
+  // (HPK = 2 when g = 64: one per half of each piece).
+  static_assert(!PK || RUN >= 8, "unit-major scales need one or two scales per piece");
+  constexpr int HPK = RUN == 8 ? 2 : 1;
   // Register stages of prefetched scales: step j's are loaded NA-1 steps
   // ahead (7 with one scale per piece, 3 with two, to bound registers); the
   // scales come from HBM and their latency under full load is microseconds.
@@ -358,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   }
 
   uint16_t ab[NA][Q][APP];
-  uint4 sc_cur[PK ? SP : 1], sc_nxt[PK ? SP : 1];   // unit-major scales of this pass and the next
+  uint4 sc_cur[PK ? SP * HPK : 1], sc_nxt[PK ? SP * HPK : 1];   // unit-major scales of this pass and the next
   float ob[NA][APP];
   uint4 wst[CH][SP];       // the pieces of the current ring stage
 
@@ -405,7 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     int t_nxt = static_tile(1);
     const bool busy = t_cur >= 0;
     constexpr int CPT = 8 / CH;                      // ring chunks per unit and plane group
-    const int chunks_per_unit = CPT * npg;
+    // Mixed storage: one pass per plane pair of the tile (npg_t, set per tile).
+    int npg_t = npg;
+    int chunks_per_unit = CPT * npg_t;
 
     // Mixed storage: (first 4096-byte block, planes) of row tile R_ of this
     // slice, from the block table.  An entry outside the packed buffer or
@@ -416,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         const uint32_t* bo = p.block_off + (size_t)s * p.mt + R_;
         const uint32_t b0 = __ldg(bo), b1 = __ldg(bo + 1);
         const uint32_t qb = b1 - b0;
-        if (b1 < b0 || qb < 1u || qb > (uint32_t)Q || b1 > p.packed_blocks) {
+        if (b1 < b0 || qb < 1u || qb > QB_MAX || b1 > p.packed_blocks) {
           if (lane == 0) atomicOr(p.status, kStatusFormat);
           return make_uint2(0u, 0u);
         }
@@ -436,13 +444,28 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bars + 8u * stage) : "memory");
           return;
         }
-        const uint8_t* src = p.packed + (size_t)ti.x * kBlockBytes + (size_t)U_ * ti.y * 512;
-        tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * ti.y * CH, bars + 8u * stage, wpol);
+        // Pair pg_ of the block: e planes from byte 8192 * pg_, CH steps of e * 512.
+        const uint32_t e = min(2u, ti.y - 2u * (uint32_t)pg_);
+        const uint8_t* src = p.packed + (size_t)ti.x * kBlockBytes + (size_t)pg_ * 2 * kBlockBytes + (size_t)U_ * e * 512;
+        tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * e * CH, bars + 8u * stage, wpol);
       } else {
         const int planes = MULTI ? min(4, p.q - 4 * pg_) : Q;
         const uint8_t* src = slice_base + (size_t)R_ * unit_bytes + ((size_t)U_ * p.q + 4 * pg_) * 512;
         tma_load(ring + (uint32_t)stage * STAGE_BYTES, src, 512u * planes * CH, bars + 8u * stage, wpol);
       }
+    };
+
+    // Mixed storage: each lane's outlier range [o0, o1) in row tile R_ of
+    // this slice (rows past m: empty), read a tile ahead of its use.
+    auto outlier_range = [&](int R_) -> uint2 {
+      uint2 r = make_uint2(0u, 0u);
+      if constexpr (MIXED) {
+        if (p.optr != nullptr && R_ >= 0 && R_ * kTileRows + lane < p.m) {
+          const uint32_t* op = p.optr + (size_t)s * p.m + (size_t)R_ * kTileRows + lane;
+          r = make_uint2(__ldg(op), __ldg(op + 1));
+        }
+      }
+      return r;
     };
 
     // Per-piece scales (and offsets) of step j of row tile R into register
@@ -463,8 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           if constexpr (!PK) {
 #pragma unroll
             for (int i = 0; i < Q; ++i) {
-              const bool live = (!MULTI || (pg_ * 4 + i < p.q)) && (!MIXED || (uint32_t)i < planes);
-              ab[SLOT][i][r] = (ok && live) ? ld_u16(ap + (size_t)(pg_ * 4 + i) * plane_stride) : (uint16_t)0;
+              const int plane = pg_ * GP + i;
+              const bool live = (!MULTI || (plane < p.q)) && (!MIXED || (uint32_t)plane < planes);
+              ab[SLOT][i][r] = (ok && live) ? ld_u16(ap + (size_t)plane * plane_stride) : (uint16_t)0;
             }
           }
           if constexpr (HAS_OFF) ob[SLOT][r] = (ok && pg_ == 0) ? __ldg(p.offset + (size_t)G * p.m + row) : 0.f;
@@ -474,6 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
 
     uint2 ti_cur = busy ? tile_info(t_cur) : make_uint2(0u, 0u);
     uint2 ti_nxt = t_nxt >= 0 ? tile_info(t_nxt) : make_uint2(0u, 0u);
+    uint2 or_cur = busy ? outlier_range(t_cur) : make_uint2(0u, 0u);
+    uint2 or_nxt = outlier_range(t_nxt);
     // The first S copies of the first tile go out before the tables are built.
     if (busy && lane == 0) {
       int st2 = st;
@@ -490,13 +516,13 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     __syncthreads();  // every warp is done with the previous segment's tables
     build_tables<RUN, HAS_OFF>(p, b, s, chunk_sum, run_sum);
 
-    // Unit-major scales of pass pg_ of row tile R_ (SP 16-byte loads).
-    auto load_scales = [&](int R_, int pg_, uint4 (&dst)[PK ? SP : 1]) {
+    // Unit-major scales of pass pg_ of row tile R_ (SP * HPK 16-byte loads).
+    auto load_scales = [&](int R_, int pg_, uint4 (&dst)[PK ? SP * HPK : 1]) {
       if constexpr (PK) {
         const uint4* src = reinterpret_cast<const uint4*>(p.alpha) +
-                           ((((size_t)s * p.mt + R_) * npg + pg_) * kTileRows + lane) * SP;
+                           ((((size_t)s * p.mt + R_) * npg + pg_) * kTileRows + lane) * (SP * HPK);
 #pragma unroll
-        for (int e = 0; e < SP; ++e) dst[e] = __ldg(src + e);
+        for (int e = 0; e < SP * HPK; ++e) dst[e] = __ldg(src + e);
       }
     };
 
@@ -505,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
       static_for(std::make_integer_sequence<int, NA - 1>{}, [&]<int D>() {
         load_alpha.template operator()<D>(t_cur, D, ti_cur.y);
       });
-      const int steps_per_unit_ = steps_per_unit;
+      int steps_per_unit_ = steps_per_unit;
       bool more = dyn;        // grabs may still succeed
       unsigned pend = 0;      // lane 0: raw count returned by the pending grab
       bool nxt_pending = false;
@@ -525,20 +551,48 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           grabbing = dyn && more && t_nxt >= 0;
         }
         if (grabbing && lane == 0) pend = atomicAdd(tile_ctr, 1u);
+        if constexpr (MIXED) {
+          npg_t = (int)((ti_cur.y + 1u) >> 1);
+          steps_per_unit_ = 8 * npg_t;
+          chunks_per_unit = CPT * npg_t;
+        }
         const int R = t_cur;
         const int row = R * kTileRows + lane;
         float yacc = 0.f;
-        // Mixed storage: this row's outliers in this slice, [o0, o1) of the
-        // entries; the first two are fetched mid-unit.
-        uint32_t o0 = 0u, o1 = 0u, oe[2] = {0u, 0u};
+        // Mixed storage: this lane's row's outliers in this slice are the
+        // entries [o0, o1), in input order.  The first six are pipelined over
+        // the steps of the first pass (entry t read at step t, its x at step
+        // t + 2, added at step t + 3), the rest follow the pass.  w * x is
+        // exact in fp32, and the sum runs in entry order.
+        uint32_t o0 = or_cur.x, o1 = or_cur.y;
+        uint32_t oq[6] = {0u, 0u, 0u, 0u, 0u, 0u};   // entries, then (w bits << 16) | x bits
+        float osum = 0.f;
         if constexpr (MIXED) {
-          if (p.optr != nullptr && row < p.m) {
-            const uint32_t* op = p.optr + (size_t)s * p.m + row;
-            o0 = __ldg(op);
-            o1 = __ldg(op + 1);
+          if (o1 < o0 || o1 > p.nnz) {
+            atomicOr(p.status, kStatusFormat);
+            o1 = o0;
           }
         }
-        for (int pg = 0; pg < npg && !failed; ++pg) {
+        auto outlier_x = [&](uint32_t v) -> uint32_t {
+          const uint32_t kin = v & 0xFFFFu, k = (uint32_t)s * kSliceInputs + kin;
+          if (kin >= (uint32_t)kSliceInputs || k >= (uint32_t)p.n) {
+            atomicOr(p.status, kStatusFormat);
+            return 0u;
+          }
+          const uint32_t xb = __ldg(reinterpret_cast<const unsigned short*>(p.x) + (size_t)b * p.n + k);
+          return (v & 0xFFFF0000u) | xb;
+        };
+        auto outlier_add = [&](uint32_t wx) {
+          osum = fmaf(h2f((uint16_t)(wx >> 16)), h2f((uint16_t)(wx & 0xFFFFu)), osum);
+        };
+        // Mixed storage: the tile after next, settled at step 4 of the first
+        // pass (its grab went out at the top of this tile), so that its
+        // block-table entry and outlier range are read a whole tile before
+        // its copies are issued.
+        int t_aft = -1;
+        bool aft_known = false;
+        uint2 ti_aft = make_uint2(0u, 0u), or_aft = make_uint2(0u, 0u);
+        for (int pg = 0; pg < npg_t && !failed; ++pg) {
           static_for(std::make_integer_sequence<int, 8>{}, [&]<int U>() {
             if (failed) return;
             const int j = pg * 8 + U;          // step within the unit
@@ -566,10 +620,37 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
               else if (t_nxt >= 0)
                 load_alpha.template operator()<(U + NA - 1) % NA>(t_nxt, ja - steps_per_unit_, ti_nxt.y);
             }
-            if constexpr (MIXED && U == 4) {
-              if (o1 > o0 && o1 <= p.nnz) {
-                oe[0] = __ldg(p.oent + o0);
-                if (o1 > o0 + 1u) oe[1] = __ldg(p.oent + o0 + 1u);
+            if constexpr (MIXED) {
+              if (pg == 0) {
+                if constexpr (U <= 5) {
+                  if (o0 + U < o1) oq[U] = __ldg(p.oent + o0 + U);
+                }
+                if constexpr (U >= 2 && U - 2 <= 5) {
+                  if (o0 + (U - 2) < o1) oq[U - 2] = outlier_x(oq[U - 2]);
+                }
+                if constexpr (U >= 3 && U - 3 <= 5) {
+                  if (o0 + (U - 3) < o1) outlier_add(oq[U - 3]);
+                }
+                if constexpr (U == 4) {
+                  if (dyn) {
+                    if (grabbing) {
+                      int tile = -1;
+                      if (lane == 0) {
+                        const long long t = dyn_base + pend;
+                        tile = t < p.mt ? (int)t : -1;
+                      }
+                      t_aft = __shfl_sync(0xffffffffu, tile, 0);
+                      more = t_aft >= 0;
+                    }
+                  } else {
+                    t_aft = static_tile(k + 2);
+                  }
+                  if (t_aft >= 0) {
+                    ti_aft = tile_info(t_aft);
+                    or_aft = outlier_range(t_aft);
+                  }
+                  aft_known = true;
+                }
               }
             }
 
@@ -585,12 +666,16 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
                 return;
               }
               const uint32_t src = ring + (uint32_t)st * STAGE_BYTES + (uint32_t)lane * 16u;
+              // A mixed pass with one plane packs its steps 512 bytes apart.
+              const uint32_t step_stride =
+                  MIXED ? 512u * min(2u, ti_cur.y - 2u * (uint32_t)pg) : STEP_BYTES;
 #pragma unroll
               for (int h = 0; h < CH; ++h)
 #pragma unroll
                 for (int i = 0; i < SP; ++i) {
-                  const bool live = (!MULTI || (pg * 4 + i < p.q)) && (!MIXED || (uint32_t)i < ti_cur.y);
-                  wst[h][i] = live ? lds128(src + (uint32_t)h * STEP_BYTES + 512u * i) : make_uint4(0, 0, 0, 0);
+                  const bool live =
+                      (!MULTI || (pg * 4 + i < p.q)) && (!MIXED || (uint32_t)(pg * GP + i) < ti_cur.y);
+                  wst[h][i] = live ? lds128(src + (uint32_t)h * step_stride + 512u * i) : make_uint4(0, 0, 0, 0);
                 }
               __syncwarp();
               const int cn = j / CH + S;       // chunk to fetch into the freed stage
@@ -612,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
 #pragma unroll
             for (int i = 0; i < Q; ++i) {
               if (MULTI && pg * 4 + i >= p.q) continue;
-              if (MIXED && (uint32_t)i >= ti_cur.y) continue;
+              if (MIXED && (uint32_t)(pg * GP + i) >= ti_cur.y) continue;
               const uint4 w4 = wv[i];
               if constexpr (RUN == 16) {
                 float acc0 = 0.f, acc1 = 0.f;
@@ -633,11 +718,21 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
                   float acc0 = 0.f, acc1 = 0.f;
                   lookup_word<IMM>(word_of(w4, 2 * r), colb[u2][2 * r], acc0, acc1);
                   lookup_word<IMM>(word_of(w4, 2 * r + 1), colb[u2][2 * r + 1], acc0, acc1);
-                  yacc = fmaf(h2f(ab[U % NA][i][r]), acc0 + acc1, yacc);
+                  float al;
+                  if constexpr (PK) {
+                    // Both halves of (step U, plane i) share one 32-bit word;
+                    // run pair r of this lane is half r xor (lam >> 3).
+                    const int wi = U * SP + i;   // unrolled: a constant
+                    const uint32_t w2 = word_of(sc_cur[wi / 4], wi % 4);
+                    al = h2f((uint16_t)(((uint32_t)r ^ (lam >> 3)) ? (w2 >> 16) : (w2 & 0xffffu)));
+                  } else {
+                    al = h2f(ab[U % NA][i][r]);
+                  }
+                  yacc = fmaf(al, acc0 + acc1, yacc);
                 }
               } else {
                 // One scale per run: group of run c is (1024 s + 8 c) / g.
-                const __half* ap = p.alpha + (size_t)(pg * 4 + i) * plane_stride + row;
+                const __half* ap = p.alpha + (size_t)(pg * GP + i) * plane_stride + row;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                   float v[4];
@@ -675,29 +770,19 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           });
           if constexpr (PK) {
 #pragma unroll
-            for (int e = 0; e < SP; ++e) sc_cur[e] = sc_nxt[e];
+            for (int e = 0; e < SP * HPK; ++e) sc_cur[e] = sc_nxt[e];
           }
-        }
-        if (failed) break;
-        // Mixed storage: the row's outliers in this slice, in entry order.
-        if constexpr (MIXED) {
-          if (o1 != o0) {
-            if (o1 < o0 || o1 > p.nnz) {
-              atomicOr(p.status, kStatusFormat);
-            } else {
-              const unsigned short* xb = reinterpret_cast<const unsigned short*>(p.x) + (size_t)b * p.n;
-              for (uint32_t e = o0; e < o1; ++e) {
-                const uint32_t v = e < o0 + 2u ? oe[e - o0] : __ldg(p.oent + e);
-                const uint32_t k = (uint32_t)s * kSliceInputs + (v & 0xFFFFu);
-                if ((v & 0xFFFFu) >= (uint32_t)kSliceInputs || k >= (uint32_t)p.n) {
-                  atomicOr(p.status, kStatusFormat);
-                  continue;
-                }
-                yacc = fmaf(h2f((uint16_t)(v >> 16)), h2f(__ldg(xb + k)), yacc);
-              }
+          if constexpr (MIXED) {
+            // Entries beyond the pipelined ones, after the first pass.
+            if (pg == 0 && !failed) {
+              if (o0 + 5u < o1) outlier_add(oq[5]);
+              for (uint32_t e = o0 + 6u; e < o1; ++e) outlier_add(outlier_x(__ldg(p.oent + e)));
             }
           }
         }
+        if (failed) break;
+        // Mixed storage: the row's outliers, after its planes.
+        if constexpr (MIXED) yacc += osum;
         // One slice: the row's sum is y.  Several: this slice's partial, summed
         // over slices by the split-K reduce kernel that follows.
         if (p.ns == 1) {
@@ -715,10 +800,13 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         if constexpr (AHEAD1) {
           t_cur = t_nxt;
           ti_cur = ti_nxt;
+          or_cur = or_nxt;
           continue;
         }
         int t_after = -1;
-        if (dyn) {
+        if (MIXED && aft_known) {
+          t_after = t_aft;
+        } else if (dyn) {
           if (grabbing) {
             int tile = -1;
             if (lane == 0) {
@@ -734,7 +822,14 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
         t_cur = t_nxt;
         t_nxt = t_after;
         ti_cur = ti_nxt;
-        if (t_nxt >= 0) ti_nxt = tile_info(t_nxt);
+        or_cur = or_nxt;
+        if (MIXED && aft_known) {
+          ti_nxt = ti_aft;
+          or_nxt = or_aft;
+        } else if (t_nxt >= 0) {
+          ti_nxt = tile_info(t_nxt);
+          or_nxt = outlier_range(t_nxt);
+        }
       }
     }
   }
@@ -764,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
 }
 
 // Kernel for (mode, offsets, unit-major scales); unit-major scales exist
-// only for the one-scale-per-piece modes (g % 128 == 0).
+// for the modes with one or two scales per piece (g % 128 == 0, g == 64).
 #define LUTGEMM_RUN_SELECT_OFF(Qv, MULTIv, OFFv)                                   \
   switch (mode) {                                                                  \
     case kG128:                                                                    \
@@ -773,7 +868,9 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     case kG128x:                                                                   \
       return packed ? lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv, true>              \
                     : lut_gemm_kernel<Qv, kG128x, MULTIv, OFFv, false>;            \
-    case kG64: return packed ? nullptr : lut_gemm_kernel<Qv, kG64, MULTIv, OFFv, false>; \
+    case kG64:                                                                     \
+      return packed ? lut_gemm_kernel<Qv, kG64, MULTIv, OFFv, true>                \
+                    : lut_gemm_kernel<Qv, kG64, MULTIv, OFFv, false>;              \
     case kG8: return packed ? nullptr : lut_gemm_kernel<Qv, kG8, MULTIv, OFFv, false>;   \
     default: return packed ? nullptr : lut_gemm_kernel<Qv, kGAny, MULTIv, OFFv, false>;  \
   }

@@ -138,7 +138,7 @@ extern "C" int lutgemm_run_noalloc(int m, int n, int batch, int q, int g, const 
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
   const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
   const bool stall = (flags & LUTGEMM_TEST_STALL) != 0u;
-  if (scales_packed && g % 128 != 0) return LUTGEMM_ERR_VALUE;
+  if (scales_packed && !(g % 128 == 0 || g == 64)) return LUTGEMM_ERR_VALUE;
   if (!aligned(packed, 16) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(offset, 4) ||
       !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4))
     return LUTGEMM_ERR_ALIGN;

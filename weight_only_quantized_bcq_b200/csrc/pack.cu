@@ -65,8 +65,10 @@ __global__ void pack_signs_kernel(const int8_t* __restrict__ signs, int q, int m
 }
 
 // Mixed storage: block (s, R) holds q_b = block_off[u+1] - block_off[u]
-// planes (u = s*mt + R) from byte 4096 * block_off[u]; its chunk (U, i) sits
-// at (U * q_b + i) * 512, with the byte map of the uniform layout.  One
+// planes (u = s*mt + R) from byte 4096 * block_off[u], in pairs: pair h
+// (planes 2h and 2h+1, or 2h alone when q_b = 2h+1; e planes) from byte
+// 8192 * h of the block, its chunk (U, i') at (U * e + i') * 512, with the
+// byte map of the uniform layout.  One
 // thread per (block, U, plane i < q_max, lane); threads of planes the block
 // does not store return.  A table entry that would write past the buffer is
 // flagged and its block left unwritten.
@@ -105,7 +107,9 @@ __global__ void pack_signs_mixed_kernel(const int8_t* __restrict__ signs, const 
       }
     }
   }
-  const size_t dst = (size_t)b0 * kBlockBytes + ((size_t)U * qb + i) * 512 + (size_t)l * 16;
+  const uint32_t h = (uint32_t)i >> 1, e = min(2u, qb - 2u * h);
+  const size_t dst = (size_t)b0 * kBlockBytes + (size_t)h * 2 * kBlockBytes + ((size_t)U * e + (i & 1)) * 512 +
+                     (size_t)l * 16;
   *reinterpret_cast<uint4*>(packed + dst) = make_uint4(words[0], words[1], words[2], words[3]);
   if (bad && flags) atomicOr(flags, LUTGEMM_FLAG_BAD_SIGN);
 }
@@ -176,7 +180,7 @@ __global__ void uniform_scales_kernel(const __half* __restrict__ scale, const ui
 // alpha[4*pg + e][(1024*s + 128*P) / g][32*R + l], P = U xor 4*(l/16), or 0
 // for a plane, row or piece out of range.
 __global__ void pack_scales_kernel(const __half* __restrict__ alpha, int q, int m, int n, int g, int mt,
-                                   int npg, int sp, long long nthreads, uint4* __restrict__ out) {
+                                   int npg, int sp, int halves, long long nthreads, uint4* __restrict__ out) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid >= nthreads) return;
   const int l = (int)(tid & 31);
@@ -187,26 +191,30 @@ __global__ void pack_scales_kernel(const __half* __restrict__ alpha, int q, int 
   const int s = (int)(sR / mt);
   const int row = R * kTileRows + l;
   const int ng = n / g;
-  uint32_t words[16];
+  uint32_t words[32];
 #pragma unroll
-  for (int w = 0; w < 16; ++w) words[w] = 0u;
+  for (int w = 0; w < 32; ++w) words[w] = 0u;
 #pragma unroll
   for (int U = 0; U < 8; ++U) {
     const int P = U ^ (4 * (l >> 4));
-    const int k0 = s * kSliceInputs + 128 * P;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = 4 * pg + e;
-      if (e < sp && i < q && row < m && k0 < n) {
-        const uint32_t h = __ldg(reinterpret_cast<const unsigned short*>(alpha) +
-                                 ((size_t)i * ng + k0 / g) * (size_t)m + row);
-        const int idx = U * sp + e;
-        words[idx >> 1] |= h << (16 * (idx & 1));
+    for (int h = 0; h < 2; ++h) {
+      const int k0 = s * kSliceInputs + 128 * P + 64 * h;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * pg + e;
+        if (h < halves && e < sp && i < q && row < m && k0 < n) {
+          const uint32_t v = __ldg(reinterpret_cast<const unsigned short*>(alpha) +
+                                   ((size_t)i * ng + k0 / g) * (size_t)m + row);
+          const int idx = (U * sp + e) * halves + h;
+          words[idx >> 1] |= v << (16 * (idx & 1));
+        }
       }
     }
   }
-  uint4* dst = out + (size_t)tid * sp;
-  for (int v = 0; v < sp; ++v) dst[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
+  uint4* dst = out + (size_t)tid * sp * halves;
+  for (int v = 0; v < sp * halves; ++v)
+    dst[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
 }
 
 }  // namespace
@@ -217,10 +225,11 @@ cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, 
   const int ns = (n + kSliceInputs - 1) / kSliceInputs;
   const int npg = (q + 3) / 4;
   const int sp = q < 4 ? q : 4;
+  const int halves = g == 64 ? 2 : 1;
   const long long nthreads = (long long)ns * mt * npg * 32;
   const int block = 256;
   pack_scales_kernel<<<(unsigned)((nthreads + block - 1) / block), block, 0, stream>>>(
-      alpha, q, m, n, g, mt, npg, sp, nthreads, reinterpret_cast<uint4*>(scales));
+      alpha, q, m, n, g, mt, npg, sp, halves, nthreads, reinterpret_cast<uint4*>(scales));
   return cudaGetLastError();
 }
 

@@ -74,8 +74,7 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const flo
 cudaError_t launch_splitk_reduce(const RunParams& p, cudaStream_t stream) {
   // Slice lanes per quad: the smallest power of two that leaves each lane at
   // most two slices, up to 32 lanes.
-  int sl_log2 = 0;
-  while (sl_log2 < 5 && ((p.ns + (1 << sl_log2) - 1) >> sl_log2) > 2) ++sl_log2;
+  const int sl_log2 = reduce_lanes_log2(p.ns);
   const int qpb = kReduceThreads >> sl_log2;
   const long long quads = (long long)p.mt * (kTileRows / 4);
   const long long blocks = (long long)p.batch * ((quads + qpb - 1) / qpb);

@@ -214,13 +214,13 @@ def new_workspace(m: int, n: int, batch: int, q: int, g: int, device=None) -> to
 
 @functools.lru_cache(maxsize=256)
 def scales_bytes(q: int, m: int, n: int, g: int) -> int:
-    """Bytes of the unit-major scale buffer (0 when g % 128 != 0 or the shape is invalid)."""
+    """Bytes of the unit-major scale buffer (0 unless g % 128 == 0 or g == 64, or for an invalid shape)."""
     return lib().lutgemm_scales_bytes(q, m, n, g)
 
 
 def pack_scales(alpha: torch.Tensor, m: int, n: int, g: int, stream=None) -> torch.Tensor:
     """fp16 alpha [q][n/g][m] on the GPU -> unit-major scales (fp16, 1-D), for
-    ``run(..., scales_packed=True)``; needs g % 128 == 0."""
+    ``run(..., scales_packed=True)``; needs g % 128 == 0 or g == 64."""
     q = alpha.shape[0] if alpha.dim() else 0
     _need(alpha, torch.float16, "alpha", q * _groups(n, g) * m)
     _one_device(stream, alpha=alpha)

@@ -105,6 +105,12 @@ def gather_rows(plan: ShardPlan, y_local: torch.Tensor, group=None) -> torch.Ten
     range so that the collective moves equal blocks, and the padding is dropped."""
     import torch.distributed as dist
     b = y_local.shape[0]
+    if b == 1 and plan.m == plan.world * plan.span and y_local.is_contiguous():
+        # One batch column, equal ranges: the ranks' rows are consecutive
+        # blocks of y as they stand, so they are gathered straight into y.
+        out = y_local.new_empty((1, plan.m))
+        dist.all_gather_into_tensor(out.view(-1), y_local.view(-1), group=group)
+        return out
     block = y_local.new_zeros((plan.span, b))
     block[: y_local.shape[1]] = y_local.t()
     out = y_local.new_empty((plan.world * plan.span, b))
