@@ -62,7 +62,7 @@ __all__ = [
     "fit_bcq_grid", "fit_bcq_grid_trace", "nearest_grid_codes",
     "mixed_block_offsets", "mixed_packed_nbytes", "pack_mixed", "unpack_mixed",
     "mixed_weights", "mixed_matmul", "pack_outliers", "unpack_outliers", "outlier_dense",
-    "mixed_matmul_tiles",
+    "mixed_matmul_tiles", "mixed_scales_nbytes", "pack_mixed_scales", "unpack_mixed_scales",
 ]
 
 
@@ -801,3 +801,91 @@ def mixed_matmul_tiles(x, packed, block_planes, alpha, g: int, m: int, n: int, t
     # plane counts are those columns of block_planes.
     y = mixed_matmul(x, signs, a[:, :, rows], bp[:, tiles], g, sub)
     return y, rows
+
+
+# ---------------------------------------------------------------------------
+# Unit-major scales of mixed storage (this library's own layout, defined in
+# include/lutgemm.h): the scales of the planes each block stores, in the
+# order the kernel's lanes read them.  For g % 128 == 0 (H = 1) and g == 64
+# (H = 2).  Block u = s * m_t + R with table entry off[u] starts at element
+# off[u] * 256 * H; its pair h (planes 2h and 2h+1, or 2h alone; e_h planes)
+# at + h * 512 * H; lane l's pass at + l * 8 * e_h * H; element
+# (U * e_h + e) * H + hh of it holds alpha[2h + e][G][32R + l] with
+# G = (1024 s + 128 P + 64 hh) // g, P = U xor 4 * (l // 16); 0 for rows >= m
+# or inputs >= n.  With every block at q <= 2 planes this is pack_scales's
+# buffer for those q planes.
+# ---------------------------------------------------------------------------
+def mixed_scales_nbytes(block_planes, g: int) -> int:
+    H = 2 if g == PIECE // 2 else 1
+    return int(np.asarray(block_planes, dtype=np.int64).sum()) * 512 * H
+
+
+def pack_mixed_scales(alpha, block_planes, g: int) -> np.ndarray:
+    """fp16 alpha [q_max][n/g][m] -> fp16 unit-major mixed scale buffer (1-D)."""
+    a = np.asarray(alpha, dtype=np.float16)
+    q_max, ng, m = a.shape
+    n = ng * g
+    if not (g % PIECE == 0 or g == PIECE // 2):
+        raise ValueError("unit-major scales need g % 128 == 0 or g == 64")
+    H = 2 if g == PIECE // 2 else 1
+    bp = _check_blocks(block_planes, m, n)
+    off = mixed_block_offsets(bp)
+    ns, mt = bp.shape
+    out = np.zeros(int(off[-1]) * 256 * H, dtype=np.float16)
+    for s_ in range(ns):
+        for R in range(mt):
+            u = s_ * mt + R
+            base = int(off[u]) * 256 * H
+            for i0, e_h in _plane_pairs(int(bp[s_, R])):
+                h = i0 // 2
+                for l in range(TILE_ROWS):
+                    row = TILE_ROWS * R + l
+                    if row >= m:
+                        continue
+                    for U in range(8):
+                        P = U ^ (4 * (l // 16))
+                        for hh in range(H):
+                            k0 = SLICE * s_ + PIECE * P + (PIECE // 2) * hh
+                            if k0 >= n:
+                                continue
+                            for e in range(e_h):
+                                idx = base + h * 512 * H + l * 8 * e_h * H + (U * e_h + e) * H + hh
+                                out[idx] = a[i0 + e, k0 // g, row]
+    return out
+
+
+def unpack_mixed_scales(scales, block_planes, q_max: int, m: int, n: int, g: int) -> np.ndarray:
+    """Inverse of ``pack_mixed_scales``: alpha [q_max][n/g][m] with the scales
+    the blocks store (a group wider than a piece appears once per piece; the
+    copies must agree) and 0 for planes no block of the group stores."""
+    H = 2 if g == PIECE // 2 else 1
+    bp = _check_blocks(block_planes, m, n)
+    off = mixed_block_offsets(bp)
+    buf = np.asarray(scales, dtype=np.float16)
+    ns, mt = bp.shape
+    out = np.zeros((q_max, n // g, m), dtype=np.float64)
+    seen = np.zeros(out.shape, dtype=bool)
+    for s_ in range(ns):
+        for R in range(mt):
+            u = s_ * mt + R
+            base = int(off[u]) * 256 * H
+            for i0, e_h in _plane_pairs(int(bp[s_, R])):
+                h = i0 // 2
+                for l in range(TILE_ROWS):
+                    row = TILE_ROWS * R + l
+                    if row >= m:
+                        continue
+                    for U in range(8):
+                        P = U ^ (4 * (l // 16))
+                        for hh in range(H):
+                            k0 = SLICE * s_ + PIECE * P + (PIECE // 2) * hh
+                            if k0 >= n:
+                                continue
+                            for e in range(e_h):
+                                v = float(buf[base + h * 512 * H + l * 8 * e_h * H + (U * e_h + e) * H + hh])
+                                G = k0 // g
+                                if seen[i0 + e, G, row] and out[i0 + e, G, row] != v:
+                                    raise ValueError("copies of one group scale disagree")
+                                out[i0 + e, G, row] = v
+                                seen[i0 + e, G, row] = True
+    return out.astype(np.float16)

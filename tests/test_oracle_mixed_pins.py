@@ -144,6 +144,24 @@ def pin_bruteforce(matmul) -> bool:
     return bool(np.all(np.abs(y - want) <= 1e-12 * (np.abs(want) + 1.0)))
 
 
+def _distinct(q, ng, m):
+    return np.arange(1, q * ng * m + 1, dtype=np.uint16).reshape(q, ng, m).view(np.float16)
+
+
+def pin_mixed_scales_golden(pack) -> bool:
+    for c in _gold()["scales_cases"]:
+        a = _distinct(c["q_max"], c["n"] // c["g"], c["m"])
+        out = np.asarray(pack(a, np.array(c["block_planes"], dtype=np.uint8), c["g"]), dtype=np.float16)
+        if out.size != c["nelem"]:
+            return False
+        bits = out.view(np.uint16)
+        for e in c["entries"]:
+            want = 0 if e[1] is None else int(a.view(np.uint16)[e[1], e[2], e[3]])
+            if int(bits[e[0]]) != want:
+                return False
+    return True
+
+
 # ---------------------------------------------------------------------------
 # The pins on the real oracle.
 # ---------------------------------------------------------------------------
@@ -213,6 +231,56 @@ def test_tile_rows_equal_the_whole_product(tiles):
     full = O.mixed_matmul(x, signs, alpha, bp, 84, outl)
     assert np.array_equal(rows, np.concatenate([np.arange(32 * t, min(100, 32 * t + 32)) for t in tiles]))
     assert np.allclose(y, full[:, rows], rtol=1e-13, atol=1e-13)
+
+
+def test_mixed_scales_pins():
+    assert pin_mixed_scales_golden(O.pack_mixed_scales)
+
+
+@pytest.mark.parametrize("q,m,n,g", [(2, 40, 2048, 64), (1, 33, 1152, 128), (2, 64, 3072, 256)])
+def test_mixed_scales_reduce_to_unit_major_scales(q, m, n, g):
+    """Every block at q <= 2 planes: the buffer is pack_scales's."""
+    a = _distinct(q, n // g, m)
+    bp = np.full((-(-n // 1024), -(-m // 32)), q, dtype=np.uint8)
+    assert np.array_equal(O.pack_mixed_scales(a, bp, g).view(np.uint16), O.pack_scales(a, g).view(np.uint16))
+
+
+@pytest.mark.parametrize("q_max,m,n,g", [(4, 70, 3072, 64), (3, 33, 2048, 128), (4, 64, 2048, 256)])
+def test_mixed_scales_roundtrip(q_max, m, n, g):
+    rng = np.random.default_rng(q_max + m)
+    bp = rng.integers(1, q_max + 1, (-(-n // 1024), -(-m // 32))).astype(np.uint8)
+    a = _distinct(q_max, n // g, m)
+    buf = O.pack_mixed_scales(a, bp, g)
+    assert buf.size * 2 == O.mixed_scales_nbytes(bp, g)
+    back = O.unpack_mixed_scales(buf, bp, q_max, m, n, g)
+    # Each (plane, group, row) comes back where its block stores the plane, else 0.
+    for s_ in range(bp.shape[0]):
+        for R in range(bp.shape[1]):
+            rows = slice(32 * R, min(m, 32 * R + 32))
+            groups = sorted({k // g for k in range(1024 * s_, min(n, 1024 * s_ + 1024))})
+            for G in groups:
+                qb = int(bp[s_, R])
+                assert np.array_equal(back[:qb, G, rows].view(np.uint16), a[:qb, G, rows].view(np.uint16))
+
+
+def _mixed_scales_pairs_swapped(alpha, bp, g):
+    # Pair 1 of each 3- or 4-plane block stored before pair 0.
+    out = O.pack_mixed_scales(alpha, bp, g).copy()
+    H = 2 if g == 64 else 1
+    off = O.mixed_block_offsets(bp)
+    for u, qb in enumerate(np.asarray(bp).reshape(-1)):
+        if qb >= 3:
+            base = int(off[u]) * 256 * H
+            p0 = out[base: base + 512 * H].copy()
+            e1 = int(qb) - 2
+            p1 = out[base + 512 * H: base + 512 * H + 256 * H * e1].copy()
+            out[base: base + p1.size] = p1
+            out[base + p1.size: base + p1.size + p0.size] = p0
+    return out
+
+
+def test_mixed_scales_pins_catch_mistakes():
+    assert not pin_mixed_scales_golden(_mixed_scales_pairs_swapped)
 
 
 def test_mixed_rejects_bad_inputs():
