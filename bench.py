@@ -1274,7 +1274,7 @@ MIXED_METRIC = "Mixed 2/4/16-bit LUT-GEMM (lutgemm_run_mixed): achieved HBM GB/s
 MIXED_SHAPES = (("llama70b_qkvo", 8192, 8192), ("llama70b_up", 28672, 8192), ("llama70b_down", 8192, 28672))
 
 
-def _mixed_layer(q_max, g, batch, frac_hi, density, seed, device, reps):
+def _mixed_layer(q_max, g, batch, frac_hi, density, seed, device, reps, packed_scales=True):
     from weight_only_quantized_bcq_b200 import lutgemm
     from weight_only_quantized_bcq_b200.roofline import mixed_algorithmic_bytes
     gen = S.generator(seed)
@@ -1288,9 +1288,13 @@ def _mixed_layer(q_max, g, batch, frac_hi, density, seed, device, reps):
         x_h = S.draw_x(gen, batch, n, outlier_frac=0.001).pin_memory()
         rp, col, val = S.draw_outliers(gen, m, n, density)
         optr, oent = lutgemm.pack_outliers(rp, col, val, m, n)
-        mats.append({"name": name, "m": m, "n": n, "bp": bp, "boff": boff_h.to(device),
+        boff_d = boff_h.to(device)
+        alpha_d = alpha_h.to(device)
+        if packed_scales:
+            alpha_d = lutgemm.pack_scales_mixed(alpha_d, boff_d, m, n, g)
+        mats.append({"name": name, "m": m, "n": n, "bp": bp, "boff": boff_d,
                      "copies": [c.to(device) for c in copies_h], "packed_host": copies_h[-1],
-                     "alpha": alpha_h.to(device), "alpha_host": alpha_h, "x_host": x_h, "x": x_h.to(device),
+                     "alpha": alpha_d, "alpha_host": alpha_h, "x_host": x_h, "x": x_h.to(device),
                      "outliers_host": (rp, col, val), "optr": optr.to(device), "oent": oent.to(device),
                      "y": torch.empty((batch, m), dtype=torch.float32, device=device),
                      "y_host": torch.empty((batch, m), dtype=torch.float32).pin_memory(),
@@ -1315,13 +1319,16 @@ def run_mixed_workload(args):
         pg = dist
     q_max, g, batch = 4, 64, args.batch
     reps = 2      # weight copies used in turn: consecutive steps miss L2
-    mats = _mixed_layer(q_max, g, batch, args.mixed_hi, args.mixed_outliers, rank_seed(rank), device, reps)
+    packed_scales = args.scales == "packed"
+    mats = _mixed_layer(q_max, g, batch, args.mixed_hi, args.mixed_outliers, rank_seed(rank), device, reps,
+                        packed_scales)
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)
 
     def one(mt, k):
         lutgemm.run_mixed(mt["copies"][k % reps], mt["boff"], mt["alpha"], mt["x"], mt["m"], mt["n"], q_max, g,
-                          optr=mt["optr"], oent=mt["oent"], y=mt["y"], workspace=mt["ws"], stream=stream)
+                          optr=mt["optr"], oent=mt["oent"], y=mt["y"], workspace=mt["ws"],
+                          scales_packed=packed_scales, stream=stream)
 
     def step(k, events=None):
         for i, mt in enumerate(mats):
@@ -1405,6 +1412,8 @@ def run_mixed_workload(args):
                                    f"{100 * args.mixed_outliers:.2f}% fp16 outliers, g={g}, batch {batch}",
                        "q_max": q_max, "g": g, "batch": batch, "frac_4plane_blocks": args.mixed_hi,
                        "outlier_density": args.mixed_outliers, "bytes_per_step": step_bytes,
+                       "scales": ("unit-major mixed layout, reordered once at load time (lutgemm_pack_scales_mixed)"
+                                  if packed_scales else "[q_max][n/g][m]"),
                        "avg_planes": {mt["name"]: round(mt["avg_planes"], 3) for mt in mats},
                        "l2": f"two weight copies used in turn: {2 * step_bytes / 1e6:.0f} MB between reuses "
                              "(> 126 MB L2)",

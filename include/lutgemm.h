@@ -433,10 +433,34 @@ int lutgemm_pack_bcq_mixed(const int8_t* signs, const uint32_t* block_off, int q
 int lutgemm_pack_outliers(const int32_t* row_ptr, const int32_t* col, const uint16_t* val, int m, int n, int nnz,
                           uint32_t* optr, uint32_t* oent);
 
+/* Unit-major scales of a mixed matrix (for g % 128 == 0, H = 1, or g == 64,
+ * H = 2): the scales of the planes each block stores, in the order the
+ * lookup kernel's lanes read them, so that a lane's scales for a pass arrive
+ * in a few 16-byte loads a pass ahead.  Block (s, R) with table entry t
+ * starts at element t * 256 * H; its pair h (planes 2h and 2h+1, or 2h
+ * alone; e_h planes) at + h * 512 * H; lane l's pass at + l * 8 * e_h * H;
+ * element (U * e_h + e) * H + hh of it holds alpha[2h + e][G][32R + l],
+ * G = (1024 s + 128 P + 64 hh) / g, P = U xor (4 * (l / 16)); 0 for rows
+ * >= m or inputs >= n.  Size: 512 * H * (the table's last entry) bytes.
+ *   alpha         dev fp16 [q_max][n/g][m], 2-byte aligned
+ *   block_off     dev uint32 block table, 4-byte aligned
+ *   scales        dev, scales_bytes = 512 * H * (table's last entry),
+ *                 16-byte aligned (output; every element of a stored plane
+ *                 is written)
+ *   status_flags  dev int32 or NULL: LUTGEMM_FLAG_BAD_BLOCK for a table
+ *                 entry out of range (that block is not written)
+ * Returns LUTGEMM_OK, ERR_NULL, ERR_SHAPE (also for other g), ERR_ALIGN,
+ * ERR_VALUE (scales_bytes not a multiple of 512 * H or below one plane per
+ * block) or ERR_CUDA. */
+int lutgemm_pack_scales_mixed(const uint16_t* alpha, const uint32_t* block_off, int q_max, int m, int n, int g,
+                              uint16_t* scales, size_t scales_bytes, int32_t* status_flags, void* stream);
+
 /* y = W x for a mixed matrix, by the lookup kernel: the same tables, with
  * each block's own plane count, and each row's outliers added after its
  * planes (w * x in fp32, in entry order), so repeated calls give identical
- * bits.  Operands as described above; x, y, flags (LUTGEMM_Y_F16, or the
+ * bits.  Operands as described above; x, y, flags (LUTGEMM_Y_F16,
+ * LUTGEMM_SCALES_PACKED: alpha is the lutgemm_pack_scales_mixed output,
+ * 16-byte aligned, g % 128 == 0 or g == 64, which gives the same bits; or the
  * test hook LUTGEMM_TEST_STALL) and workspace (lutgemm_workspace_size with
  * q = q_max) as lutgemm_run.  optr and oent may be NULL when nnz == 0.
  * The kernel checks every block-table and outlier entry it uses against

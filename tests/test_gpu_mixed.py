@@ -214,3 +214,68 @@ def test_mixed_stall_hook_reports_timeout(L):
     L.run_mixed(packed, boff, alpha.to(DEV), x.to(DEV), m, n, q_max, g, optr=optr, oent=oent, workspace=ws,
                 _flags=L.TEST_STALL)
     assert L.workspace_status(ws) == L.STATUS_TIMEOUT
+
+
+# ---------------------------------------------------------------------------
+# Unit-major scales of mixed storage: bit-exact packing, and the product with
+# them gives the bits of the product with [q_max][n/g][m] scales.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("q_max,m,n,g,lo", [(4, 100, 3072, 64, 1), (3, 70, 2048, 128, 1), (4, 64, 2048, 256, 2),
+                                            (2, 33, 1152, 128, 1), (4, 40, 1024, 64, 3)])
+def test_pack_scales_mixed_bit_exact(L, q_max, m, n, g, lo):
+    gen = S.generator(600 + q_max * 7 + m)
+    bp = S.draw_block_planes(gen, m, n, 0.4, lo=lo, hi=q_max)
+    alpha = S.draw_alpha(gen, q_max, m, n, g, 0.03)
+    boff = L.mixed_offsets(bp, q_max, m, n).to(DEV)
+    flags = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sc = L.pack_scales_mixed(alpha.to(DEV), boff, m, n, g, status_flags=flags)
+    torch.cuda.synchronize()
+    want = O.pack_mixed_scales(alpha.numpy(), bp.numpy(), g)
+    assert int(flags.item()) == 0
+    assert sc.numel() == want.size
+    assert np.array_equal(sc.cpu().numpy().view(np.uint16), want.view(np.uint16))
+
+
+@pytest.mark.parametrize("q_max,m,n,g,batch,lo,density", [
+    (4, 512, 2048, 64, 1, 2, 0.005),
+    (3, 257, 4096, 128, 3, 1, 0.0),       # 1- and 3-plane blocks: one-plane passes
+    (4, 2048, 4096, 64, 37, 1, 0.005),    # counter-taken tiles, every plane count
+    (2, 300, 2048, 256, 2, 1, 0.01),
+])
+def test_run_mixed_packed_scales_same_bits(L, q_max, m, n, g, batch, lo, density):
+    bp, signs, alpha, x, outl = _problem(700 + q_max + m, q_max, m, n, g, batch, 0.4, density, lo=lo)
+    boff, packed, optr, oent = _device(L, bp, signs, outl, m, n)
+    a_d, x_d = alpha.to(DEV), x.to(DEV)
+    sc = L.pack_scales_mixed(a_d, boff, m, n, g)
+    y_raw = L.run_mixed(packed, boff, a_d, x_d, m, n, q_max, g, optr=optr, oent=oent, check=True)
+    y_pk = L.run_mixed(packed, boff, sc, x_d, m, n, q_max, g, optr=optr, oent=oent, scales_packed=True, check=True)
+    assert torch.equal(y_raw, y_pk)
+    o = None if outl is None else tuple(t.numpy() for t in outl)
+    y_ref = O.mixed_matmul(x.numpy(), signs.numpy(), alpha.numpy(), bp.numpy(), g, o)
+    ok, st = compare(y_pk.cpu().numpy(), y_ref, _effective_alpha(alpha, bp.numpy(), m, n, g), x.numpy(), n)
+    assert ok, st
+
+
+def test_full_size_llama_up_packed_scales(L):
+    """The bench's configuration: LLaMA-70B up-projection, 2/4-plane blocks,
+    0.5 % outliers, unit-major scales, batch 1; 48 row tiles against the oracle."""
+    q_max, m, n, g = 4, 28672, 8192, 64
+    gen = S.generator(4141)
+    bp = S.draw_block_planes(gen, m, n, 0.125)
+    boff_h = L.mixed_offsets(bp, q_max, m, n)
+    packed = S.draw_random_bytes(gen, int(boff_h[-1]) * 4096)
+    alpha = S.draw_alpha(gen, q_max, m, n, g, 0.03)
+    x = S.draw_x(gen, 1, n, outlier_frac=0.001)
+    rp, col, val = S.draw_outliers(gen, m, n, 0.005)
+    optr, oent = L.pack_outliers(rp, col, val, m, n)
+    boff = boff_h.to(DEV)
+    sc = L.pack_scales_mixed(alpha.to(DEV), boff, m, n, g)
+    y = L.run_mixed(packed.to(DEV), boff, sc, x.to(DEV), m, n, q_max, g, optr=optr.to(DEV), oent=oent.to(DEV),
+                    scales_packed=True, check=True)
+    mt = m // 32
+    tiles = np.unique(np.r_[0, mt - 1, np.random.default_rng(6).choice(mt, 46, replace=False)])
+    y_ref, rows = O.mixed_matmul_tiles(x.numpy(), packed.numpy(), bp.numpy(), alpha.numpy(), g, m, n, tiles,
+                                       (rp.numpy(), col.numpy(), val.numpy()))
+    a_eff = _effective_alpha(torch.from_numpy(alpha.numpy()[:, :, rows]), bp.numpy()[:, tiles], rows.size, n, g)
+    ok, st = compare(y.cpu().numpy()[:, rows], y_ref, a_eff, x.numpy(), n)
+    assert ok, st

@@ -89,7 +89,9 @@ def test_run_mixed_validation(L):
     assert _run_mixed(L, q_max=5) == L.ERR_SHAPE
     assert _run_mixed(L, q_max=0) == L.ERR_SHAPE
     assert _run_mixed(L, g=100) == L.ERR_SHAPE
-    assert _run_mixed(L, flags=L.SCALES_PACKED) == L.ERR_VALUE
+    assert _run_mixed(L, flags=8) == L.ERR_VALUE                       # no such flag
+    assert _run_mixed(L, g=32, flags=L.SCALES_PACKED) == L.ERR_VALUE   # unit-major scales need g % 128 == 0 or 64
+    assert _run_mixed(L, alpha=FAKE + 2, flags=L.SCALES_PACKED) == L.ERR_ALIGN
     assert _run_mixed(L, pbytes=8191) == L.ERR_VALUE
     assert _run_mixed(L, boff=FAKE + 2) == L.ERR_ALIGN
     assert _run_mixed(L, x=FAKE + 8) == L.ERR_ALIGN
@@ -102,3 +104,13 @@ def test_pack_mixed_validation(L):
     assert lib.lutgemm_pack_bcq_mixed(FAKE, FAKE, 5, 64, 1024, FAKE, 8192, None, None) == L.ERR_SHAPE
     assert lib.lutgemm_pack_bcq_mixed(FAKE, FAKE, 4, 64, 1024, FAKE + 8, 8192, None, None) == L.ERR_ALIGN
     assert lib.lutgemm_pack_bcq_mixed(FAKE, FAKE, 4, 64, 1024, FAKE, 4096, None, None) == L.ERR_VALUE
+
+
+def test_pack_scales_mixed_validation(L):
+    lib = L.lib()
+    assert lib.lutgemm_pack_scales_mixed(None, FAKE, 4, 64, 1024, 128, FAKE, 8192, None, None) == L.ERR_NULL
+    assert lib.lutgemm_pack_scales_mixed(FAKE, FAKE, 4, 64, 1024, 32, FAKE, 8192, None, None) == L.ERR_SHAPE
+    assert lib.lutgemm_pack_scales_mixed(FAKE, FAKE, 5, 64, 1024, 128, FAKE, 8192, None, None) == L.ERR_SHAPE
+    assert lib.lutgemm_pack_scales_mixed(FAKE, FAKE, 4, 64, 1024, 128, FAKE + 8, 8192, None, None) == L.ERR_ALIGN
+    assert lib.lutgemm_pack_scales_mixed(FAKE, FAKE, 4, 64, 1024, 128, FAKE, 8000, None, None) == L.ERR_VALUE
+    assert lib.lutgemm_pack_scales_mixed(FAKE, FAKE, 4, 64, 1024, 128, FAKE, 512, None, None) == L.ERR_VALUE

@@ -19,6 +19,8 @@ cudaError_t launch_pack_scales(const __half* alpha, int q, int m, int n, int g, 
                                cudaStream_t stream);
 cudaError_t launch_pack_signs_mixed(const int8_t* signs, const uint32_t* block_off, int q_max, int m, int n,
                                     uint8_t* packed, size_t packed_bytes, int32_t* flags, cudaStream_t stream);
+cudaError_t launch_pack_scales_mixed(const __half* alpha, const uint32_t* block_off, int q_max, int m, int n, int g,
+                                     uint16_t* scales, size_t scales_bytes, int32_t* flags, cudaStream_t stream);
 cudaError_t launch_tc_gemm(const uint8_t* packed, const __half* alpha, const float* offset, const __half* x, void* y,
                            float* part, int nsplit, int m, int n, int batch, int q, int g, int y_f16, unsigned* status,
                            cudaStream_t stream);
@@ -478,6 +480,23 @@ int lutgemm_pack_bcq_mixed(const int8_t* signs, const uint32_t* block_off, int q
   return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
 }
 
+int lutgemm_pack_scales_mixed(const uint16_t* alpha, const uint32_t* block_off, int q_max, int m, int n, int g,
+                              uint16_t* scales, size_t scales_bytes, int32_t* status_flags, void* stream) {
+  if (!alpha || !block_off || !scales) return LUTGEMM_ERR_NULL;
+  if (q_max < 1 || q_max > 4 || !valid_matrix(q_max, m, n) || !valid_groups(n, g) || !(g % 128 == 0 || g == 64))
+    return LUTGEMM_ERR_SHAPE;
+  if (!aligned(alpha, 2) || !aligned(block_off, 4) || !aligned(scales, 16) || !aligned(status_flags, 4))
+    return LUTGEMM_ERR_ALIGN;
+  const size_t per_plane = g == 64 ? 1024u : 512u;
+  if (scales_bytes % per_plane != 0 ||
+      scales_bytes < (size_t)ceil_div(n, kSliceInputs) * ceil_div(m, kTileRows) * per_plane)
+    return LUTGEMM_ERR_VALUE;
+  const cudaError_t err = launch_pack_scales_mixed(reinterpret_cast<const __half*>(alpha), block_off, q_max, m, n, g,
+                                                   scales, scales_bytes, status_flags,
+                                                   reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? LUTGEMM_OK : LUTGEMM_ERR_CUDA;
+}
+
 int lutgemm_run_mixed(int m, int n, int batch, int q_max, int g, const uint8_t* packed, size_t packed_bytes,
                       const uint32_t* block_off, const uint16_t* alpha, const uint32_t* optr, const uint32_t* oent,
                       int nnz, const uint16_t* x, void* y, unsigned flags, void* workspace, size_t workspace_bytes,
@@ -487,10 +506,12 @@ int lutgemm_run_mixed(int m, int n, int batch, int q_max, int g, const uint8_t* 
   if (q_max < 1 || q_max > 4 || !valid_matrix(q_max, m, n) || !valid_groups(n, g) || batch < 1 || nnz < 0)
     return LUTGEMM_ERR_SHAPE;
   if ((long long)batch * ceil_div(n, kSliceInputs) >= (1ll << 31)) return LUTGEMM_ERR_SHAPE;
-  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_TEST_STALL)) != 0u) return LUTGEMM_ERR_VALUE;
+  if ((flags & ~(LUTGEMM_Y_F16 | LUTGEMM_SCALES_PACKED | LUTGEMM_TEST_STALL)) != 0u) return LUTGEMM_ERR_VALUE;
   const bool y_f16 = (flags & LUTGEMM_Y_F16) != 0u;
+  const bool scales_packed = (flags & LUTGEMM_SCALES_PACKED) != 0u;
+  if (scales_packed && !(g % 128 == 0 || g == 64)) return LUTGEMM_ERR_VALUE;
   if (packed_bytes % kBlockBytes != 0 || packed_bytes / kBlockBytes > 0xFFFFFFFFull) return LUTGEMM_ERR_VALUE;
-  if (!aligned(packed, 16) || !aligned(block_off, 4) || !aligned(alpha, 2) || !aligned(optr, 4) ||
+  if (!aligned(packed, 16) || !aligned(block_off, 4) || !aligned(alpha, scales_packed ? 16 : 2) || !aligned(optr, 4) ||
       !aligned(oent, 4) || !aligned(x, 16) || !aligned(y, y_f16 ? 2 : 4) || !aligned(workspace, 16))
     return LUTGEMM_ERR_ALIGN;
   if (workspace_bytes < lutgemm_workspace_size(m, n, batch, q_max, g)) return LUTGEMM_ERR_WORKSPACE;
@@ -512,7 +533,8 @@ int lutgemm_run_mixed(int m, int n, int batch, int q_max, int g, const uint8_t* 
   p.optr = nnz > 0 ? optr : nullptr;
   p.oent = nnz > 0 ? oent : nullptr;
   p.nnz = (uint32_t)nnz;
-  return launch_lookup(p, run_kernel_mixed(group_mode(g)), workspace, reinterpret_cast<cudaStream_t>(stream));
+  return launch_lookup(p, run_kernel_mixed(group_mode(g), scales_packed), workspace,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -170,6 +170,6 @@ RunKernel run_kernel_q2(int mode, bool has_offset, bool packed);
 RunKernel run_kernel_q3(int mode, bool has_offset, bool packed);
 RunKernel run_kernel_q4(int mode, bool has_offset, bool packed);
 RunKernel run_kernel_q8(int mode, bool has_offset, bool packed);   // 5 <= q <= 8, planes in groups of four
-RunKernel run_kernel_mixed(int mode);   // mixed storage: 1..4 planes per block, sparse outliers
+RunKernel run_kernel_mixed(int mode, bool packed);   // mixed storage: 1..4 planes per block, sparse outliers
 
 }  // namespace lutgemm

@@ -225,6 +225,29 @@ __device__ __forceinline__ void build_tables(const RunParams& p, int b, int s, f
   }
 }
 
+// A one-plane pass of mixed-storage scales (8 * H halves, in the order
+// (step, half)) moved into the two-plane order (step, plane, half) with
+// plane 1 zero.  H = 1: half U goes to element 2U; H = 2: the word of step U
+// goes to word 2U.
+template <int H, int N>
+__device__ __forceinline__ void spread_scales(uint4 (&sc)[N]) {
+  static_assert(N == 1 || N == 2 * H, "a pass holds 2 * H words");
+  if constexpr (N == 1) {
+    return;                       // no unit-major scales: nothing to move
+  } else if constexpr (H == 1) {
+    uint32_t w[4] = {sc[0].x, sc[0].y, sc[0].z, sc[0].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o[k] = (w[k >> 1] >> (16 * (k & 1))) & 0xffffu;
+    sc[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    sc[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  } else {
+    const uint32_t r[8] = {sc[0].x, sc[0].y, sc[0].z, sc[0].w, sc[1].x, sc[1].y, sc[1].z, sc[1].w};
+#pragma unroll
+    for (int v = 0; v < 4; ++v) sc[v] = make_uint4(r[2 * v], 0u, r[2 * v + 1], 0u);
+  }
+}
+
 template <int... Is, class F>
 __device__ __forceinline__ void static_for(std::integer_sequence<int, Is...>, F&& f) {
   (f.template operator()<Is>(), ...);
@@ -246,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
   constexpr uint32_t STEP_BYTES = 512u * SP;
   constexpr uint32_t STAGE_BYTES = STEP_BYTES * CH;
   static_assert(!MULTI || CH == 1, "plane groups are fetched one step at a time");
-  static_assert(!MIXED || (Q == 2 && !MULTI && !HAS_OFF && !PK), "mixed storage: plane pairs, [q][n/g][m] scales");
+  static_assert(!MIXED || (Q == 2 && !MULTI && !HAS_OFF), "mixed storage: plane pairs, no offsets");
   constexpr uint32_t QB_MAX = MIXED ? 4u : (uint32_t)Q;   // planes of one mixed block
   static_assert(S >= 2 && S <= 7, "weight ring of 2..7 stages (barrier slot 7 is the test hook's)");
   constexpr int NPG = (MULTI || MIXED) ? 2 : 1;        // plane groups of a unit (at most)
@@ -517,17 +540,28 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     build_tables<RUN, HAS_OFF>(p, b, s, chunk_sum, run_sum);
 
     // Unit-major scales of pass pg_ of row tile R_ (SP * HPK 16-byte loads).
-    auto load_scales = [&](int R_, int pg_, uint4 (&dst)[PK ? SP * HPK : 1]) {
+    // Mixed storage: the pass of pair pg_ of the tile's block (table entry
+    // ti_.x) holds e planes, so a lane loads e * HPK of them; a one-plane pass
+    // is spread to the two-plane order when it starts (spread_scales).
+    auto load_scales = [&](int R_, uint2 ti_, int pg_, uint4 (&dst)[PK ? SP * HPK : 1]) {
       if constexpr (PK) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.alpha) +
-                           ((((size_t)s * p.mt + R_) * npg + pg_) * kTileRows + lane) * (SP * HPK);
+        if constexpr (MIXED) {
+          const uint32_t e = ti_.y > 2u * (uint32_t)pg_ ? min(2u, ti_.y - 2u * (uint32_t)pg_) : 0u;
+          const uint4* src = reinterpret_cast<const uint4*>(p.alpha) +
+                             ((size_t)ti_.x * 32 + (size_t)pg_ * 64 + (size_t)lane * e) * HPK;
 #pragma unroll
-        for (int e = 0; e < SP * HPK; ++e) dst[e] = __ldg(src + e);
+          for (int v = 0; v < SP * HPK; ++v) dst[v] = (uint32_t)v < e * HPK ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(p.alpha) +
+                             ((((size_t)s * p.mt + R_) * npg + pg_) * kTileRows + lane) * (SP * HPK);
+#pragma unroll
+          for (int e = 0; e < SP * HPK; ++e) dst[e] = __ldg(src + e);
+        }
       }
     };
 
     if (busy) {
-      load_scales(t_cur, 0, sc_cur);
+      load_scales(t_cur, ti_cur, 0, sc_cur);
       static_for(std::make_integer_sequence<int, NA - 1>{}, [&]<int D>() {
         load_alpha.template operator()<D>(t_cur, D, ti_cur.y);
       });
@@ -611,8 +645,13 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
             if constexpr (PK && U == 0) {
               // Scales of the next pass: this tile's next plane group, or the
               // next tile's first.
-              if (pg + 1 < npg) load_scales(t_cur, pg + 1, sc_nxt);
-              else if (t_nxt >= 0) load_scales(t_nxt, 0, sc_nxt);
+              if (pg + 1 < npg_t) load_scales(t_cur, ti_cur, pg + 1, sc_nxt);
+              else if (t_nxt >= 0) load_scales(t_nxt, ti_nxt, 0, sc_nxt);
+              // Mixed storage: a pass with one plane came as 8 * HPK scales;
+              // place them where the two-plane order reads plane 0.
+              if constexpr (MIXED) {
+                if (ti_cur.y - 2u * (uint32_t)pg == 1u) spread_scales<HPK>(sc_cur);
+              }
             }
             {
               const int ja = j + NA - 1;       // scales NA-1 steps ahead

@@ -256,6 +256,66 @@ cudaError_t launch_pack_signs_mixed(const int8_t* signs, const uint32_t* block_o
   return cudaGetLastError();
 }
 
+// Unit-major scales of mixed storage: one thread per (block, pair, lane)
+// writes the lane's pass, e * H 16-byte words from element
+// table[u] * 256 * H + pair * 512 * H + lane * 8 * e * H (layout in
+// include/lutgemm.h).  Threads of pairs a block does not store return; a
+// table entry past the buffer is flagged and not written.
+__global__ void pack_scales_mixed_kernel(const __half* __restrict__ alpha, const uint32_t* __restrict__ block_off,
+                                         int q_max, int m, int n, int g, int mt, int halves, long long nthreads,
+                                         size_t out_elems, uint16_t* __restrict__ out, int32_t* flags) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nthreads) return;
+  const int l = (int)(tid & 31);
+  const int h = (int)((tid >> 5) & 1);
+  const long long u = tid >> 6;
+  const int R = (int)(u % mt);
+  const int s = (int)(u / mt);
+  const uint32_t b0 = block_off[u], b1 = block_off[u + 1];
+  const uint32_t qb = b1 - b0;
+  if (b1 < b0 || qb < 1u || qb > (uint32_t)q_max || (size_t)b1 * 256 * halves > out_elems) {
+    if (flags && h == 0 && l == 0) atomicOr(flags, LUTGEMM_FLAG_BAD_BLOCK);
+    return;
+  }
+  if (2u * (uint32_t)h >= qb) return;
+  const uint32_t e_h = min(2u, qb - 2u * (uint32_t)h);
+  const int row = R * kTileRows + l;
+  const int ng = n / g;
+  uint32_t words[16];
+#pragma unroll
+  for (int w = 0; w < 16; ++w) words[w] = 0u;
+  for (int U = 0; U < 8; ++U) {
+    const int P = U ^ (4 * (l >> 4));
+    for (int hh = 0; hh < halves; ++hh) {
+      const int k0 = s * kSliceInputs + 128 * P + 64 * hh;
+      for (uint32_t e = 0; e < e_h; ++e) {
+        if (row < m && k0 < n) {
+          const uint32_t v = __ldg(reinterpret_cast<const unsigned short*>(alpha) +
+                                   ((size_t)(2 * h + e) * ng + k0 / g) * (size_t)m + row);
+          const int idx = (int)((U * e_h + e) * halves + hh);
+          words[idx >> 1] |= v << (16 * (idx & 1));
+        }
+      }
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out + (size_t)b0 * 256 * halves + (size_t)h * 512 * halves +
+                                        (size_t)l * 8 * e_h * halves);
+  for (uint32_t v = 0; v < e_h * halves; ++v)
+    dst[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
+}
+
+cudaError_t launch_pack_scales_mixed(const __half* alpha, const uint32_t* block_off, int q_max, int m, int n, int g,
+                                     uint16_t* scales, size_t scales_bytes, int32_t* flags, cudaStream_t stream) {
+  const int mt = (m + kTileRows - 1) / kTileRows;
+  const int ns = (n + kSliceInputs - 1) / kSliceInputs;
+  const int halves = g == 64 ? 2 : 1;
+  const long long nthreads = (long long)ns * mt * 64;
+  const int block = 256;
+  pack_scales_mixed_kernel<<<(unsigned)((nthreads + block - 1) / block), block, 0, stream>>>(
+      alpha, block_off, q_max, m, n, g, mt, halves, nthreads, scales_bytes / 2, scales, flags);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_uniform_to_bcq(const uint8_t* codes, const __half* scale, const uint8_t* zero, int q,
                                   int m, int n, int g, uint8_t* packed, __half* alpha, float* offset,
                                   int32_t* flags, cudaStream_t stream) {

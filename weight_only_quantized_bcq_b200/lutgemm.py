@@ -49,6 +49,7 @@ _SIGNATURES = {
     "lutgemm_mixed_offsets": ([_vp, _c_int, _c_int, _c_int, _vp], _c_int),
     "lutgemm_pack_outliers": ([_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lutgemm_pack_bcq_mixed": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp], _c_int),
+    "lutgemm_pack_scales_mixed": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp], _c_int),
     "lutgemm_run_mixed": ([_c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp, _vp, _vp, _vp, _c_int, _vp,
                            _vp, _c_uint, _vp, _c_size, _vp], _c_int),
     "lutgemm_library_status": ([_vp, _c_int, _vp], _c_int),
@@ -430,15 +431,36 @@ def pack_bcq_mixed(signs: torch.Tensor, block_off: torch.Tensor, status_flags: t
     return packed
 
 
+def pack_scales_mixed(alpha: torch.Tensor, block_off: torch.Tensor, m: int, n: int, g: int,
+                      status_flags: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """fp16 alpha [q_max][n/g][m] and the block table (device) -> the unit-major
+    mixed scales (fp16, 1-D), for ``run_mixed(..., scales_packed=True)``;
+    needs g % 128 == 0 or g == 64."""
+    q_max = alpha.shape[0] if alpha.dim() else 0
+    _need(alpha, torch.float16, "alpha", q_max * _groups(n, g) * m)
+    _need(block_off, torch.int32, "block_off", -(-n // 1024) * -(-m // 32) + 1)
+    if status_flags is not None:
+        _need(status_flags, torch.int32, "status_flags", 1)
+    _one_device(stream, alpha=alpha, block_off=block_off, status_flags=status_flags)
+    nbytes = int(block_off[-1].item()) * (1024 if g == 64 else 512)
+    scales = torch.empty(max(nbytes // 2, 8), dtype=torch.float16, device=alpha.device)
+    _check(lib().lutgemm_pack_scales_mixed(_ptr(alpha), _ptr(block_off), q_max, m, n, g, _ptr(scales), nbytes,
+                                           _ptr(status_flags), _stream(stream)),
+           "lutgemm_pack_scales_mixed")
+    return scales
+
+
 def run_mixed(packed: torch.Tensor, block_off: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, m: int, n: int,
               q_max: int, g: int, optr: torch.Tensor = None, oent: torch.Tensor = None, y: torch.Tensor = None,
-              workspace: torch.Tensor = None, y_f16: bool = False, check: bool = False, stream=None,
-              _flags: int = 0) -> torch.Tensor:
-    """y[b] = W x[b] for a mixed matrix, by lutgemm_run_mixed (outliers optional)."""
+              workspace: torch.Tensor = None, y_f16: bool = False, scales_packed: bool = False, check: bool = False,
+              stream=None, _flags: int = 0) -> torch.Tensor:
+    """y[b] = W x[b] for a mixed matrix, by lutgemm_run_mixed (outliers optional;
+    with ``scales_packed`` alpha is the output of ``pack_scales_mixed``)."""
     batch = _batch_of(x, n)
     _need(packed, torch.uint8, "packed")
     _need(block_off, torch.int32, "block_off", -(-n // 1024) * -(-m // 32) + 1)
-    _need(alpha, torch.float16, "alpha", q_max * _groups(n, g) * m)
+    _need(alpha, torch.float16, "alpha",
+          (packed.numel() // 4096) * (512 if g == 64 else 256) if scales_packed else q_max * _groups(n, g) * m)
     _need(x, torch.float16, "x")
     nnz = 0
     if oent is not None:
@@ -455,7 +477,7 @@ def run_mixed(packed: torch.Tensor, block_off: torch.Tensor, alpha: torch.Tensor
         y = torch.empty((batch, m), dtype=torch.float16 if y_f16 else torch.float32, device=x.device)
     if workspace is None:
         workspace = new_workspace(m, n, batch, q_max, g, device=x.device)
-    flags = (Y_F16 if y_f16 else 0) | _flags
+    flags = (Y_F16 if y_f16 else 0) | (SCALES_PACKED if scales_packed else 0) | _flags
     _check(lib().lutgemm_run_mixed(m, n, batch, q_max, g, _ptr(packed), packed.numel(), _ptr(block_off),
                                    _ptr(alpha), _ptr(optr) if nnz else None, _ptr(oent) if nnz else None, nnz,
                                    _ptr(x), _ptr(y), flags, _ptr(workspace), workspace.numel(), _stream(stream)),
