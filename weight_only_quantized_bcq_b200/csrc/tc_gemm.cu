@@ -27,7 +27,10 @@
 //     tensor memory (row r in lane r, inputs 2c and 2c+1 in column c: the
 //     layout the tensor cores read an A operand from); in a group, warp w
 //     takes rows 32(w mod 4)..+31 (the lanes it may access) and the
-//     64-input half (w / 4) mod 2.  A never touches shared memory.
+//     64-input half (w / 4) mod 2.  A never touches shared memory.  A warp
+//     visits only its group's steps; a unit slot is released by the MMA
+//     warp's commit alone (that commit follows its waits for every step of
+//     the unit, and each step's barrier is arrived after the reads).
 //   warp 20 (MMA): the converged warp runs the loop and one elected lane
 //     issues the 8 tcgen05.mma (K = 16 each, A from tensor memory, B from
 //     shared memory) per plane and the commits that free A stages, units
@@ -39,8 +42,9 @@
 // Accumulation: the tensor cores add into their fp32 accumulator with
 // truncation, so an error of up to an ulp per MMA step would build up over
 // the q * n / 16 steps of a long row.  Each K block therefore accumulates in
-// fresh tensor-memory buffers (two per K block at BN <= 64, even and odd K
-// steps, so consecutive MMAs are independent; ping-pong between K blocks),
+// fresh tensor-memory buffers (two per K block at BN = 64, even and odd K
+// steps, so consecutive MMAs are independent; one at BN = 32 and 128;
+// ping-pong between K blocks),
 // and warps 16-19 add them into fp32 running sums (round to nearest) as soon
 // as the block's MMAs complete; warp 16+w owns accumulator lanes
 // 32w..32w+31 = tile rows, keeps the running sums (in registers at BN = 32,
@@ -205,6 +209,25 @@ struct UnitIter {
   }
 };
 
+// Position in a ring of n slots: the slot and the parity of the pass over
+// the ring (the mbarrier phase of the slot's current use).  Advanced one use
+// at a time, so no division by a run-time ring size is needed.
+struct RingPos {
+  int n, slot;
+  uint32_t phase;
+  __device__ __forceinline__ void init(int n_) {
+    n = n_;
+    slot = 0;
+    phase = 0;
+  }
+  __device__ __forceinline__ void next() {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 struct TcLayout {
   uint32_t slot_bytes;     // one unit: x tiles, chunk groups, scale rows (multiple of 1024)
   uint32_t bits_off;       // 8 chunk groups of q * 512 bytes: (row tile, half) = 2 wq + h
@@ -221,12 +244,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kBTile = (uint32_t)BN * kTcBK * 2;   // x tile: BN rows x 128 inputs
   // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128.
   constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
-  // MMAs that add into one accumulator wait on each other; with two
-  // accumulator sets (even and odd K steps of every plane, summed when the K
-  // block is flushed) consecutive MMAs are independent and the tensor pipe
-  // stays full.  At BN = 128 an MMA takes longer than that dependency, and
-  // tensor memory holds one set only.
-  constexpr int kSets = BN <= 64 ? 2 : 1;
+  // Accumulator sets per K block.  At BN = 64 two sets (even and odd K steps
+  // of every plane, summed when the K block is flushed) keep consecutive MMAs
+  // independent.  At BN = 32 the 24 dependent MMAs of a K block into one set
+  // issue at the same rate (measured), and one set leaves a seventh A stage
+  // and halves the flush; at BN = 128 an MMA takes longer than the
+  // dependency, and tensor memory holds one set only.
+  constexpr int kSets = BN == 64 ? 2 : 1;
   // At BN = 32 the accumulate warps keep the running sums in registers (32
   // per thread); wider tiles keep them in tensor memory.
   constexpr bool kRunRegs = BN <= 32;
@@ -237,17 +261,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kRunCol = 2u * kSets * BN;
   constexpr int kACol0 = ((2 * kSets + (kRunRegs ? 0 : 1)) * BN + 63) / 64 * 64;
-  constexpr int kSA = (512 - kACol0) / 64 < 6 ? (512 - kACol0) / 64 : 6;
+  constexpr int kSA = (512 - kACol0) / 64 < 7 ? (512 - kACol0) / 64 : 7;
   static_assert(kSA >= 2, "at least two A stages must fit tensor memory");
 
   extern __shared__ __align__(1024) unsigned char tc_smem_raw[];
   const uint32_t raw = (uint32_t)__cvta_generic_to_shared(tc_smem_raw);
   const uint32_t ring = (raw + 1023u) & ~1023u;
   const uint32_t bars = ring + (uint32_t)L.nu * L.slot_bytes;
-  const uint32_t fullU = bars, emptyU = bars + 64, fullA = bars + 128, emptyA = bars + 176;
-  const uint32_t accFull = bars + 224, accFree = bars + 240, done = bars + 256;
-  const uint32_t tmem_slot = bars + 264;
-  const uint32_t flag_slot = bars + 268;                     // CTA failure flag (shared)
+  // mbarriers: 8 unit slots, 8 A stages, 2 accumulator buffers each.
+  const uint32_t fullU = bars, emptyU = bars + 64, fullA = bars + 128, emptyA = bars + 192;
+  const uint32_t accFull = bars + 256, accFree = bars + 272, done = bars + 288;
+  const uint32_t tmem_slot = bars + 296;
+  const uint32_t flag_slot = bars + 300;                     // CTA failure flag (shared)
 
   const int tid = threadIdx.x;
   // Broadcast from lane 0 so that the compiler knows the warp index, and all
@@ -270,9 +295,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < L.nu; ++s) {
       bar_init(fullU + 8 * s, 1);
-      // dequant warps + the MMA commit (+ the accumulate warps, which read the
-      // x tiles for the offset term)
-      bar_init(emptyU + 8 * s, kTcDequantWarps + 1 + (HAS_OFF ? 4 : 0));
+      // The MMA commit (+ the accumulate warps, which read the x tiles for the
+      // offset term).  The commit follows the MMA warp's waits for every plane
+      // step of the unit, each arrived after the dequant warps' reads of the
+      // unit's bits and scales, so no dequant warp needs to arrive here.
+      bar_init(emptyU + 8 * s, 1 + (HAS_OFF ? 4 : 0));
     }
     for (int s = 0; s < kSA; ++s) {
       bar_init(fullA + 8 * s, kTcDequantWarps / 2);       // one group of dequant warps per step
@@ -333,74 +360,94 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t a_tm = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)kACol0 + (uint32_t)(32 * hsel);
     const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * 2 * q * 512 + lane * 16 + h8 * 8);
     const uint32_t alpha_lane = L.alpha_off + (uint32_t)((wq * 32 + lane) * 2);
+    // The group's plane steps are ai = grp, grp + 2, ...; the warp visits
+    // only those, carrying the unit, the K block in the unit (w), the plane
+    // (i) and the A stage along, and waits for a unit only when its next step
+    // lies there.
     UnitIter it;
     it.init(n, s_begin, s_end);
-    int ai = 0;                                              // plane step (A stage sequence)
+    RingPos ur, ar;                                          // unit slot, A stage
+    ur.init(L.nu);
+    ar.init(kSA);
+    int ai = 0, w = 0, i = 0;
+    bool need_unit = true;                                   // the unit changed since the last wait
+    // Moves the step position d plane steps on.
+    auto advance = [&](int d) {
+      ai += d;
+      for (int k = 0; k < d; ++k) ar.next();
+      i += d;
+      while (i >= q && it.valid()) {
+        i -= q;
+        if (++w >= it.count()) {
+          w = 0;
+          it.next();
+          ur.next();
+          need_unit = true;
+        }
+      }
+    };
+    advance(grp);
+    uint32_t slot = 0;
     bool go = true;
-    for (int u = 0; it.valid() && go; it.next(), ++u) {
-      const int sl = u % L.nu;
-      const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
-      if (!__all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)))) {
+    while (it.valid() && go) {
+      if (need_unit) {
+        slot = ring + (uint32_t)ur.slot * L.slot_bytes;
+        if (!__all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * ur.slot, ur.phase))) {
+          if (lane == 0) fail();
+          break;
+        }
+        if (__any_sync(0xffffffffu, failed())) break;
+        need_unit = false;
+      }
+      const int st = ar.slot;
+      const uint32_t bsrc = slot + bits_lane + (uint32_t)(((half_sel ^ w) * q + i) * 512);
+      const uint32_t asrc = slot + alpha_lane + (uint32_t)(((w * q + i) * 2 + (apb == 2 ? hsel : 0)) * 256);
+      uint32_t b0w, b1w, ah;
+      asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0w), "=r"(b1w) : "r"(bsrc) : "memory");
+      asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc) : "memory");
+      const uint32_t w0 = __byte_perm(b0w, b1w, sel0);       // runs 0..3 of the half, in order
+      const uint32_t w1 = __byte_perm(b0w, b1w, sel1);       // runs 4..7
+      // Element pair (2e, 2e+1) of a run byte rb8: the product rb8 *
+      // (2^(15-2e) + 2^(30-2e)) puts bit 2e at bit 15 and bit 2e+1 at bit 31
+      // (the two fp16 sign bits), with no carries between the two copies.  A
+      // clear bit (beta = -1) sets the sign of +alpha.
+      const uint32_t a2 = (ah | (ah << 16)) & row_mask;
+      uint32_t v[32];
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const uint32_t rb8 = __byte_perm(cc < 4 ? w0 : w1, 0u, 0x4440u | (uint32_t)(cc & 3));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t t = rb8 * ((1u << (15 - 2 * e)) + (1u << (30 - 2 * e)));
+          v[4 * cc + e] = a2 ^ (~t & 0x80008000u);
+        }
+      }
+      // The stage's previous use (one pass back) must have been consumed.
+      if (ai >= kSA && !__all_sync(0xffffffffu, bar_wait_sleep(emptyA + 8 * st, ar.phase ^ 1u))) {
         if (lane == 0) fail();
         break;
       }
-      go = !__any_sync(0xffffffffu, failed());
-      const int cnt = it.count();
-      for (int w = 0; w < cnt && go; ++w) {
-        const uint32_t bsrc = slot + bits_lane + (uint32_t)((half_sel ^ w) * q * 512);
-        const uint32_t asrc = slot + alpha_lane + (uint32_t)((w * q * 2 + (apb == 2 ? hsel : 0)) * 256);
-        for (int i = 0; i < q; ++i, ++ai) {
-          if ((ai & 1) != grp) continue;
-          const int st = ai % kSA;
-          uint32_t b0w, b1w, ah;
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0w), "=r"(b1w) : "r"(bsrc + (uint32_t)(i * 512))
-                       : "memory");
-          asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc + (uint32_t)(i * 512)) : "memory");
-          const uint32_t w0 = __byte_perm(b0w, b1w, sel0);   // runs 0..3 of the half, in order
-          const uint32_t w1 = __byte_perm(b0w, b1w, sel1);   // runs 4..7
-          // Element pair (2e, 2e+1) of a run byte b: the product b * (2^(15-2e)
-          // + 2^(30-2e)) puts bit 2e at bit 15 and bit 2e+1 at bit 31 (the two
-          // fp16 sign bits), with no carries between the two copies.  A clear
-          // bit (beta = -1) sets the sign of +alpha.
-          const uint32_t a2 = (ah | (ah << 16)) & row_mask;
-          uint32_t v[32];
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const uint32_t b = __byte_perm(cc < 4 ? w0 : w1, 0u, 0x4440u | (uint32_t)(cc & 3));
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t t = b * ((1u << (15 - 2 * e)) + (1u << (30 - 2 * e)));
-              v[4 * cc + e] = a2 ^ (~t & 0x80008000u);
-            }
-          }
-          if (ai >= kSA &&
-              !__all_sync(0xffffffffu, bar_wait_sleep(emptyA + 8 * st, (uint32_t)(((ai - kSA) / kSA) & 1)))) {
-            if (lane == 0) fail();
-            go = false;
-            break;
-          }
-          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          tmem_st32(a_tm + (uint32_t)(st * 64), v);
-          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-          asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) bar_arrive(fullA + 8 * st);
-        }
-      }
-      // This warp has read all it needs from the unit.
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      tmem_st32(a_tm + (uint32_t)(st * 64), v);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
-      if (lane == 0) bar_arrive(emptyU + 8 * sl);
+      if (lane == 0) bar_arrive(fullA + 8 * st);
+      advance(2);
     }
   } else if (warp == kTcProdWarp) {
     // ---- Producer: one unit of x tiles, chunk groups and scale rows per ring slot.
     const int rows_here = m - rb * kTcBM < kTcBM ? m - rb * kTcBM : kTcBM;
     UnitIter it;
     it.init(n, s_begin, s_end);
-    for (int u = 0; it.valid(); it.next(), ++u) {
-      const int sl = u % L.nu;
+    RingPos ur;
+    ur.init(L.nu);
+    for (int u = 0; it.valid(); it.next(), ++u, ur.next()) {
+      const int sl = ur.slot;
       const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
       const uint32_t bar = fullU + 8 * sl;
-      if (u >= L.nu && !__all_sync(0xffffffffu, bar_wait_sleep(emptyU + 8 * sl, (uint32_t)(((u / L.nu) - 1) & 1)))) {
+      // The slot's previous use (one pass back) must have been released.
+      if (u >= L.nu && !__all_sync(0xffffffffu, bar_wait_sleep(emptyU + 8 * sl, ur.phase ^ 1u))) {
         if (lane == 0) fail();
         break;
       }
@@ -486,12 +533,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // commit.
     UnitIter it;
     it.init(n, s_begin, s_end);
-    int ai = 0, j = 0;                                       // plane step, K block (processing order)
+    int j = 0;                                               // K block (processing order)
+    RingPos ur, ar;                                          // unit slot, A stage
+    ur.init(L.nu);
+    ar.init(kSA);
     bool ok = true;
-    for (int u = 0; it.valid() && ok; it.next(), ++u) {
-      const int sl = u % L.nu;
+    for (; it.valid() && ok; it.next(), ur.next()) {
+      const int sl = ur.slot;
       const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
-      if (!__all_sync(0xffffffffu, bar_wait(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)))) {
+      if (!__all_sync(0xffffffffu, bar_wait(fullU + 8 * sl, ur.phase))) {
         ok = false;
         break;
       }
@@ -505,9 +555,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         const uint64_t db0 = smem_desc(slot + (uint32_t)w * kBTile);
-        for (int i = 0; i < q; ++i, ++ai) {
-          const int st = ai % kSA;
-          if (!__all_sync(0xffffffffu, bar_wait(fullA + 8 * st, (uint32_t)((ai / kSA) & 1)))) {
+        for (int i = 0; i < q; ++i, ar.next()) {
+          const int st = ar.slot;
+          if (!__all_sync(0xffffffffu, bar_wait(fullA + 8 * st, ar.phase))) {
             ok = false;
             break;
           }
@@ -621,16 +671,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           uint32_t a[kPiece], b[kPiece];
           if constexpr (kPiece == 16) {
             tmem_ld16(acc_tm + (uint32_t)c0, a);
-            tmem_ld16(acc_tm + (uint32_t)(BN + c0), b);
+            if constexpr (kSets == 2) tmem_ld16(acc_tm + (uint32_t)(BN + c0), b);
           } else {
             tmem_ld8(acc_tm + (uint32_t)c0, a);
-            tmem_ld8(acc_tm + (uint32_t)(BN + c0), b);
+            if constexpr (kSets == 2) tmem_ld8(acc_tm + (uint32_t)(BN + c0), b);
           }
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
           for (int jj = 0; jj < kPiece; ++jj) {
-            const float f = __uint_as_float(a[jj]) + __uint_as_float(b[jj]);
-            float r = j > 0 ? __uint_as_float(run[c0 + jj]) + f : f;
+            const float f = kSets == 2 ? __uint_as_float(a[jj]) + __uint_as_float(b[jj]) : __uint_as_float(a[jj]);
+            float r = __uint_as_float(run[c0 + jj]) + f;       // the sums start at +0
             if constexpr (HAS_OFF) {
               r = fmaf(offr[0], __shfl_sync(0xffffffffu, sx[0][0], c0 + jj), r);
               r = fmaf(offr[1], __shfl_sync(0xffffffffu, sx[1][0], c0 + jj), r);
@@ -672,10 +722,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       UnitIter it;
       it.init(n, s_begin, s_end);
       int j = 0;
-      for (int u = 0; it.valid() && ok; it.next(), ++u) {
-        const int sl = u % L.nu;
+      RingPos ur;
+      ur.init(L.nu);
+      for (; it.valid() && ok; it.next(), ur.next()) {
+        const int sl = ur.slot;
         const uint32_t slot = ring + (uint32_t)sl * L.slot_bytes;
-        ok = __all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * sl, (uint32_t)((u / L.nu) & 1)));
+        ok = __all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * sl, ur.phase));
         if (!ok) break;
         const int cnt = it.count();
         for (int w = 0; w < cnt && ok; ++w, ++j) {
