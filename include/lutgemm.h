@@ -195,7 +195,7 @@ int lutgemm_launch_plan(int m, int n, int batch, int sm_count, int* grid, int* s
  * 8 and max_split), or 0 when its cost model expects the lookup kernel to
  * be faster (always 0 below batch 8).  The model is fitted to B200
  * measurements of both paths: tensor cores ~ waves x (K blocks per split x
- * 1900 / 2170 / 2700 cycles at 32 / 64 / 128 batch columns per tile + 12k)
+ * 1650 / 1860 / 2480 cycles at 32 / 64 / 128 batch columns per tile + 14k)
  * + 15k (+ the reduce when split); lookups ~ q m n batch / 8 table reads at
  * 0.62 of a 32-read wavefront per clock per SM + 15k.  lutgemm_run passes
  * ceil(n / 1024) and the device's SM count.  A pure host function (whether

@@ -32,10 +32,11 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
 // lookup kernel is expected to be faster.  A cost model fitted to B200
 // measurements of both paths (OPT-175B and LLaMA-70B linears, batch 8-32,
 // isolated back-to-back launches):
-//   tensor cores: waves x (K blocks per split x c(BN) + 12k) + 15k cycles, with
+//   tensor cores: waves x (K blocks per split x c(BN) + 14k) + 15k cycles, with
 //     waves = ceil(ceil(m/128) * ceil(batch/BN) * splits / SMs) and
-//     c = 1900 / 2170 / 2700 cycles per 128-input block at BN = 32 / 64 / 128
-//     (nearly independent of q: the per-block hand-offs dominate); a split
+//     c = 1650 / 1860 / 2480 cycles per 128-input block at BN = 32 / 64 / 128
+//     (nearly independent of q at q <= 3: the tensor-memory stores of the A
+//     tiles and the per-block hand-offs dominate); a split
 //     run adds the fp32 partials' reduce (launch + bytes at HBM speed);
 //   lookups: q m n batch / 8 table reads at 0.62 of one 32-read wavefront per
 //     clock per SM, + 15k cycles.
@@ -48,7 +49,7 @@ int tc_plan_for(int m, int n, int batch, int q, int max_split, int sm_count) {
   if (m < 1 || n < 128 || batch < 8 || q < 1 || max_split < 1 || sm_count < 1) return 0;
   const double sms = sm_count;
   const int bn = batch <= 32 ? 32 : (batch <= 64 ? 64 : 128);
-  const double block_cycles = bn == 32 ? 1900.0 : (bn == 64 ? 2170.0 : 2700.0);
+  const double block_cycles = bn == 32 ? 1650.0 : (bn == 64 ? 1860.0 : 2480.0);
   const double ctas = (double)((m + 127) / 128) * (double)((batch + bn - 1) / bn);
   const int s_all = (n + 1023) / 1024;
   const int nkb = n / 128;
@@ -59,7 +60,7 @@ int tc_plan_for(int m, int n, int batch, int q, int max_split, int sm_count) {
     const int spz = (s_all + sp - 1) / sp;
     if ((s_all + spz - 1) / spz != sp) continue;          // would leave a split empty
     const double kb = (double)(8 * spz < nkb ? 8 * spz : nkb);
-    double t = std::ceil(ctas * sp / sms) * (kb * block_cycles + 12000.0) + 15000.0;
+    double t = std::ceil(ctas * sp / sms) * (kb * block_cycles + 14000.0) + 15000.0;
     if (sp > 1) t += 4000.0 + ((double)batch * mt32 * sp * 4.0 + (double)batch * m * 4.0) / 6.4e12 * 1.965e9;
     if (sp == 1) unsplit = t;
     if (best_s == 0 || t < best) {

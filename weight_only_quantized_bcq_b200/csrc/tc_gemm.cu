@@ -166,6 +166,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&v)[16]
       : "memory");
 }
 
+// Orders the computation of v before the following volatile asm statements
+// (an empty statement that takes the 32 values as operands).
+__device__ __forceinline__ void pin32(const uint32_t (&v)[32]) {
+  asm volatile("" ::"r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+               "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+               "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+               "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]));
+}
+
 // tcgen05.commit from one elected lane of a converged warp: the mbarrier
 // arrives once all tensor-core work this thread issued before has completed.
 __device__ __forceinline__ void commit_one(uint32_t bar) {
@@ -389,8 +398,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     advance(grp);
     uint32_t slot = 0;
     bool go = true;
+    // The stage whose store is still in flight (-1: none).  With enough A
+    // stages (kDefer) a step's store is completed and its stage handed to the
+    // MMA warp only after the warp has expanded its next step, so the store's
+    // latency overlaps that work (FC1 at batch 32: 275 -> 268 us); with two
+    // or three stages, holding a stage longer costs more than it hides.
+    constexpr bool kDefer = kSA >= 4;
+    int pend = -1;
+    auto hand_over = [&]() {
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) bar_arrive(fullA + 8 * pend);
+      pend = -1;
+    };
     while (it.valid() && go) {
       if (need_unit) {
+        // A store still in flight is handed over before waiting for a new
+        // unit: the slot's refill may need the MMAs of that very step.
+        if (pend >= 0) hand_over();
         slot = ring + (uint32_t)ur.slot * L.slot_bytes;
         if (!__all_sync(0xffffffffu, bar_wait_sleep(fullU + 8 * ur.slot, ur.phase))) {
           if (lane == 0) fail();
@@ -422,6 +448,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           v[4 * cc + e] = a2 ^ (~t & 0x80008000u);
         }
       }
+      if (pend >= 0) {
+        pin32(v);
+        hand_over();
+      }
       // The stage's previous use (one pass back) must have been consumed.
       if (ai >= kSA && !__all_sync(0xffffffffu, bar_wait_sleep(emptyA + 8 * st, ar.phase ^ 1u))) {
         if (lane == 0) fail();
@@ -429,12 +459,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       tmem_st32(a_tm + (uint32_t)(st * 64), v);
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) bar_arrive(fullA + 8 * st);
+      pend = st;
+      if constexpr (!kDefer) hand_over();
       advance(2);
     }
+    if (pend >= 0) hand_over();
+    // No store of this warp is in flight when tensor memory is released.
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   } else if (warp == kTcProdWarp) {
     // ---- Producer: one unit of x tiles, chunk groups and scale rows per ring slot.
     const int rows_here = m - rb * kTcBM < kTcBM ? m - rb * kTcBM : kTcBM;
