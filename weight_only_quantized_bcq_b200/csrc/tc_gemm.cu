@@ -239,15 +239,16 @@ struct RingPos {
 
 struct TcLayout {
   uint32_t slot_bytes;     // one unit: x tiles, chunk groups, scale rows (multiple of 1024)
-  uint32_t bits_off;       // 8 chunk groups of q * 512 bytes: (row tile, half) = 2 wq + h
-  uint32_t alpha_off;      // 2 x q x 2 scale rows of 128 fp16: (which, plane, K half)
+  uint32_t bits_off;       // 8 chunk groups of q * 512 bytes: (half, row tile) = 4 h + wq
+  uint32_t alpha_off;      // 2 x 2 x q scale rows of 128 fp16: (which, K half, plane)
   int nu;                  // ring depth in units
   int alpha_bulk;          // scale rows by bulk copy (16-byte aligned rows) or by lane loads
 };
 
 template <int BN, bool HAS_OFF>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed,
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
+                   const __grid_constant__ CUtensorMap amap, const uint8_t* __restrict__ packed,
                    const __half* __restrict__ alpha, const float* __restrict__ offset, void* y, float* part,
                    int spz, int m, int n, int batch, int q, int g, int mt, int y_f16, unsigned* status, TcLayout L) {
   constexpr uint32_t kBTile = (uint32_t)BN * kTcBK * 2;   // x tile: BN rows x 128 inputs
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     const uint32_t row_mask = row < m ? 0xFFFFFFFFu : 0u;   // rows past m get a zero scale
     const uint32_t a_tm = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)kACol0 + (uint32_t)(32 * hsel);
-    const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * 2 * q * 512 + lane * 16 + h8 * 8);
+    const uint32_t bits_lane = L.bits_off + (uint32_t)(wq * q * 512 + lane * 16 + h8 * 8);
     const uint32_t alpha_lane = L.alpha_off + (uint32_t)((wq * 32 + lane) * 2);
     // The group's plane steps are ai = grp, grp + 2, ...; the warp visits
     // only those, carrying the unit, the K block in the unit (w), the plane
@@ -426,8 +427,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         need_unit = false;
       }
       const int st = ar.slot;
-      const uint32_t bsrc = slot + bits_lane + (uint32_t)(((half_sel ^ w) * q + i) * 512);
-      const uint32_t asrc = slot + alpha_lane + (uint32_t)(((w * q + i) * 2 + (apb == 2 ? hsel : 0)) * 256);
+      const uint32_t bsrc = slot + bits_lane + (uint32_t)(((half_sel ^ w) * 4 * q + i) * 512);
+      const uint32_t asrc = slot + alpha_lane + (uint32_t)(((w * 2 + (apb == 2 ? hsel : 0)) * q + i) * 256);
       uint32_t b0w, b1w, ah;
       asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0w), "=r"(b1w) : "r"(bsrc) : "memory");
       asm volatile("ld.shared.u16 %0, [%1];" : "=r"(ah) : "r"(asrc) : "memory");
@@ -468,7 +469,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   } else if (warp == kTcProdWarp) {
     // ---- Producer: one unit of x tiles, chunk groups and scale rows per ring slot.
-    const int rows_here = m - rb * kTcBM < kTcBM ? m - rb * kTcBM : kTcBM;
     UnitIter it;
     it.init(n, s_begin, s_end);
     RingPos ur;
@@ -486,51 +486,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int cnt = it.count();
       {
         // The whole warp computes the copies; one elected lane issues each.
-        uint32_t bytes = (uint32_t)cnt * kBTile;
-        for (int wq = 0; wq < 4; ++wq)
-          if (rb * 4 + wq < mt) bytes += 2u * (uint32_t)q * 512u;
-        if (L.alpha_bulk) bytes += (uint32_t)(cnt * q * apb * rows_here * 2);
+        // Per K block one x tile (both 64-input halves); per chunk group
+        // (P, P ^ 4) the q planes of the 4 row tiles; per K block and scale
+        // group the q planes' scale rows.  Rows and row tiles past m are
+        // filled with zeros and counted.
+        uint32_t bytes = (uint32_t)cnt * kBTile + 8u * (uint32_t)q * 512u;
+        if (L.alpha_bulk) bytes += (uint32_t)(cnt * apb * q * kTcBM * 2);
         asm volatile(
             "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
             " @e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n}" ::"r"(bar),
             "r"(bytes)
             : "memory");
-        for (int w = 0; w < cnt; ++w) {
-          const int kb = it.kb(w);
+        for (int w = 0; w < cnt; ++w)
+          asm volatile(
+              "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+              " @e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+              "[%5];\n}" ::"r"(slot + (uint32_t)w * kBTile),
+              "l"(&xmap), "r"(0), "r"(b0), "r"(2 * it.kb(w)), "r"(bar)
+              : "memory");
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            asm volatile(
-                "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-                " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-                "[%4];\n}" ::"r"(slot + (uint32_t)w * kBTile + (uint32_t)h * (kBTile / 2)),
-                "l"(&xmap), "r"(kb * kTcBK + 64 * h), "r"(b0), "r"(bar)
-                : "memory");
-        }
-        for (int wq = 0; wq < 4; ++wq) {
-          const int R = rb * 4 + wq;
-          if (R >= mt) continue;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint8_t* src = packed + (((size_t)it.s * mt + R) * 8 + (size_t)(it.P ^ (4 * h))) * q * 512;
-            asm volatile(
-                "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-                " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
-                    slot + L.bits_off + (uint32_t)((wq * 2 + h) * q * 512)),
-                "l"(src), "r"(q * 512), "r"(bar)
-                : "memory");
-          }
-        }
+        for (int h = 0; h < 2; ++h)
+          asm volatile(
+              "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+              " @e cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], "
+              "[%1, {%2, %3, %4, %5, %6}], [%7];\n}" ::"r"(slot + L.bits_off + (uint32_t)(h * 4 * q * 512)),
+              "l"(&bmap), "r"(0), "r"(0), "r"(it.P ^ (4 * h)), "r"(rb * 4), "r"(it.s), "r"(bar)
+              : "memory");
         if (L.alpha_bulk) {
           for (int w = 0; w < cnt; ++w)
             for (int h = 0; h < apb; ++h) {
               const int G = (2 * it.kb(w) + h) / halves_per_g;
-              for (int i = 0; i < q; ++i)
-                asm volatile(
-                    "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-                    " @e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
-                        slot + L.alpha_off + (uint32_t)(((w * q + i) * 2 + h) * 256)),
-                    "l"(alpha + ((size_t)i * ng + G) * m + (size_t)rb * kTcBM), "r"(rows_here * 2), "r"(bar)
-                    : "memory");
+              asm volatile(
+                  "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+                  " @e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], "
+                  "[%1, {%2, %3, %4}], [%5];\n}" ::"r"(slot + L.alpha_off + (uint32_t)((w * 2 + h) * q * 256)),
+                  "l"(&amap), "r"(rb * kTcBM), "r"(G), "r"(0), "r"(bar)
+                  : "memory");
             }
         }
       }
@@ -548,7 +539,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 v[k] = r < m ? (uint32_t)__ldg(src + r) : 0u;
               }
               asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(
-                               slot + L.alpha_off + (uint32_t)(((w * q + i) * 2 + h) * 256 + lane * 8)),
+                               slot + L.alpha_off + (uint32_t)(((w * 2 + h) * q + i) * 256 + lane * 8)),
                            "r"(v[0] | (v[1] << 16)), "r"(v[2] | (v[3] << 16))
                            : "memory");
             }
@@ -848,18 +839,49 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const float* o
                       cudaStream_t stream) {
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
+  // x as [n/64][batch][64] fp16: one box is the two 64-input halves of a K
+  // block for BN batch rows (128-byte swizzle, K-major).
   CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)batch};
-  const cuuint64_t strides[1] = {(cuuint64_t)n * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)BN};
-  const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(x), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  // Scale rows go by bulk copy when every row segment of a tile starts on a
-  // 16-byte boundary; otherwise the producer warp loads them.
+  {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)batch, (cuuint64_t)n / 64};
+    const cuuint64_t strides[2] = {(cuuint64_t)n * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)BN, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<__half*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  // The packed planes as [slice][row tile][chunk group U][plane][256] uint16
+  // (512-byte pieces): one box is the q pieces of the 4 row tiles of a
+  // 128-row block for one chunk group; row tiles past m are zero-filled.
+  CUtensorMap bmap;
+  {
+    const cuuint64_t mt = (cuuint64_t)((m + kTileRows - 1) / kTileRows);
+    const cuuint64_t dims[5] = {256, (cuuint64_t)q, 8, mt, (cuuint64_t)((n + kSliceInputs - 1) / kSliceInputs)};
+    const cuuint64_t strides[4] = {512, (cuuint64_t)q * 512, (cuuint64_t)q * 4096, mt * q * 4096};
+    const cuuint32_t box[5] = {256, (cuuint32_t)q, 1, 4, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (enc(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 5, const_cast<uint8_t*>(packed), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  // Scale rows by tensor copy when every row of the [q][n/g][m] scales starts
+  // on a 16-byte boundary (one box: 128 rows of one group, all q planes,
+  // rows past m zero-filled); otherwise the producer warp loads them.
   const bool alpha_bulk = m % 8 == 0 && (reinterpret_cast<uintptr_t>(alpha) % 16) == 0;
+  CUtensorMap amap = map;
+  if (alpha_bulk) {
+    const cuuint64_t dims[3] = {(cuuint64_t)m, (cuuint64_t)(n / g), (cuuint64_t)q};
+    const cuuint64_t strides[2] = {(cuuint64_t)m * 2, (cuuint64_t)(n / g) * (cuuint64_t)m * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kTcBM, 1, (cuuint32_t)q};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<__half*>(alpha), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   const TcLayout L = tc_layout<BN>(q, alpha_bulk);
   if (L.nu < 2) return cudaErrorInvalidValue;
   const size_t smem = tc_smem_bytes(L);
@@ -886,8 +908,8 @@ cudaError_t launch_bn(const uint8_t* packed, const __half* alpha, const float* o
   const int spz = (s_all + nsplit - 1) / nsplit;
   if (nsplit < 1 || (s_all + spz - 1) / spz != nsplit) return cudaErrorInvalidValue;
   dim3 grid((unsigned)((m + kTcBM - 1) / kTcBM), (unsigned)((batch + BN - 1) / BN), (unsigned)nsplit);
-  tc_gemm_kernel<BN, HAS_OFF><<<grid, kTcThreads, smem, stream>>>(map, packed, alpha, offset, y, part, spz, m, n,
-                                                                   batch, q, g, mt, y_f16, status, L);
+  tc_gemm_kernel<BN, HAS_OFF><<<grid, kTcThreads, smem, stream>>>(map, bmap, amap, packed, alpha, offset, y, part,
+                                                                   spz, m, n, batch, q, g, mt, y_f16, status, L);
   return cudaGetLastError();
 }
 
