@@ -195,9 +195,9 @@ int lutgemm_launch_plan(int m, int n, int batch, int sm_count, int* grid, int* s
  * 8 and max_split), or 0 when its cost model expects the lookup kernel to
  * be faster (always 0 below batch 8).  The model is fitted to B200
  * measurements of both paths: tensor cores ~ waves x (K blocks per split x
- * 1650 / 1860 / 2480 cycles at 32 / 64 / 128 batch columns per tile + 14k)
- * + 15k (+ the reduce when split); lookups ~ q m n batch / 8 table reads at
- * 0.62 of a 32-read wavefront per clock per SM + 15k.  lutgemm_run passes
+ * q/3 x 1600 / 1870 / 2450 cycles at 32 / 64 / 128 batch columns per tile +
+ * 14k) + 15k (+ the reduce when split); lookups ~ q m n batch / 8 table reads
+ * at 0.39 + 0.092 q of a 32-read wavefront per clock per SM + 20k.  lutgemm_run passes
  * ceil(n / 1024) and the device's SM count.  A pure host function (whether
  * the operands suit the tensor-core path -- n % 128, g % 64, scale layout --
  * is checked by lutgemm_run, not here). */

@@ -239,16 +239,17 @@ def test_tensor_core_plan_matches_the_measured_choices(L):
     """lutgemm_tc_plan on 148 SMs picks, for each measured (shape, batch), the
     path and split count that measured fastest on a B200 (OPT-175B and
     LLaMA-70B linears; see the config sweep): QKV and FC1 one split, out-proj
-    and FC2 three, the LLaMA-70B linears at batch 8 the lookup kernel."""
+    and FC2 three; at batch 8 the LLaMA-70B up-projection one split and its
+    8192-wide q/k/v/o and down projections two."""
     sms = 148
     want = {  # (m, n, q): {batch: splits}
         (36864, 12288, 3): {8: 1, 16: 1, 32: 1, 256: 1},
         (49152, 12288, 3): {8: 1, 16: 1, 32: 1, 256: 1},
         (12288, 49152, 3): {8: 3, 16: 3, 32: 3, 256: 3},
         (12288, 12288, 3): {256: 3},
-        (8192, 8192, 2): {8: 0},
-        (28672, 8192, 2): {8: 0},
-        (8192, 28672, 2): {8: 0},
+        (8192, 8192, 2): {8: 2},
+        (28672, 8192, 2): {8: 1},
+        (8192, 28672, 2): {8: 2},
     }
     for (m, n, q), cases in want.items():
         for batch, splits in cases.items():

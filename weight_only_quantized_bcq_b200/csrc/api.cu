@@ -1,6 +1,7 @@
 // C ABI of the LUT-GEMM library: argument validation, workspace sizing and
 // kernel launches on the caller's stream.  Declarations and the contract of
 // every call are in include/lutgemm.h.
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 #include <set>
@@ -32,14 +33,14 @@ cudaError_t launch_fit_bcq(const __half* w, int q, int m, int n, int g, int iter
 // lookup kernel is expected to be faster.  A cost model fitted to B200
 // measurements of both paths (OPT-175B and LLaMA-70B linears, batch 8-32,
 // isolated back-to-back launches):
-//   tensor cores: waves x (K blocks per split x c(BN) + 14k) + 15k cycles, with
+//   tensor cores: waves x (K blocks per split x c + 14k) + 15k cycles, with
 //     waves = ceil(ceil(m/128) * ceil(batch/BN) * splits / SMs) and
-//     c = 1650 / 1860 / 2480 cycles per 128-input block at BN = 32 / 64 / 128
-//     (nearly independent of q at q <= 3: the tensor-memory stores of the A
-//     tiles and the per-block hand-offs dominate); a split
+//     c = q/3 x 1600 / 1870 / 2450 cycles per 128-input block at BN = 32 /
+//     64 / 128 (the A-tile stores and expansion scale with the planes); a split
 //     run adds the fp32 partials' reduce (launch + bytes at HBM speed);
-//   lookups: q m n batch / 8 table reads at 0.62 of one 32-read wavefront per
-//     clock per SM, + 15k cycles.
+//   lookups: q m n batch / 8 table reads at e(q) = 0.39 + 0.092 q of one
+//     32-read wavefront per clock per SM (0.57 at q = 2, 0.67 at q = 3:
+//     per-unit costs are shared by the planes), + 20k cycles.
 // It picks the faster path (and split count) for the 12 measured (shape,
 // batch >= 8) cases and the batch-256 layer: FC2- and out-proj-like matrices
 // (few 128-row blocks, long K) take 3 splits, QKV and FC1 none, LLaMA-70B at
@@ -49,7 +50,7 @@ int tc_plan_for(int m, int n, int batch, int q, int max_split, int sm_count) {
   if (m < 1 || n < 128 || batch < 8 || q < 1 || max_split < 1 || sm_count < 1) return 0;
   const double sms = sm_count;
   const int bn = batch <= 32 ? 32 : (batch <= 64 ? 64 : 128);
-  const double block_cycles = bn == 32 ? 1650.0 : (bn == 64 ? 1860.0 : 2480.0);
+  const double block_cycles = (bn == 32 ? 1600.0 : (bn == 64 ? 1870.0 : 2450.0)) * q / 3.0;
   const double ctas = (double)((m + 127) / 128) * (double)((batch + bn - 1) / bn);
   const int s_all = (n + 1023) / 1024;
   const int nkb = n / 128;
@@ -73,7 +74,8 @@ int tc_plan_for(int m, int n, int batch, int q, int max_split, int sm_count) {
     best = unsplit;
     best_s = 1;
   }
-  const double t_lut = (double)q * m * n * batch / 8.0 / (sms * 32.0) / 0.62 + 15000.0;
+  const double e_lut = std::min(0.39 + 0.092 * q, 0.85);
+  const double t_lut = (double)q * m * n * batch / 8.0 / (sms * 32.0) / e_lut + 20000.0;
   return best_s > 0 && best < t_lut ? best_s : 0;
 }
 
