@@ -17,11 +17,13 @@
 //     units.  A unit is the K-block pair (P, P ^ 4) of one 1024-input slice:
 //     those two blocks read the same two chunk groups of the packed layout
 //     (lanes 0-15 of a row tile hold piece P in chunk P, lanes 16-31 in
-//     chunk P ^ 4), so one bulk copy per chunk group and row tile serves
-//     both.  Each unit holds the two x tiles (TMA, 128-byte swizzle,
-//     K-major), the 8 chunk groups of the tile's 4 row tiles and the scale
-//     rows of the tile (per K block and plane one row, or one per 64-input
-//     half when g = 64).
+//     chunk P ^ 4), so one copy per chunk group serves both.  Each unit
+//     holds the two x tiles (128-byte swizzle, K-major), the 8 chunk groups
+//     of the tile's 4 row tiles and the scale rows of the tile (per K block
+//     and plane one row, or one per 64-input half when g = 64), fetched by
+//     4-6 TMA tensor copies: one per x tile (both 64-input halves), one per
+//     chunk group (all planes of the 4 row tiles), one per K block and scale
+//     group (all planes).
 //   warps 0-15 (dequant, two groups of 8 taking alternate plane steps):
 //     expand a plane's bits for the tile into a 128 x 128 fp16 A tile in
 //     tensor memory (row r in lane r, inputs 2c and 2c+1 in column c: the
