@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
       // v_i = sum_k beta_ik * w_k; on a grid also M_iq = 2 #(beta_i = +1) - g,
       // M_qq = g and v_q = sum_k w_k.
       int diff[Q * (Q - 1) / 2 + 1];
-      int plus[Q];
+      int plus[Q] = {};
       float v[D];
 #pragma unroll
       for (int i = 0; i < Q; ++i) {
@@ -270,7 +270,6 @@ __global__ void __launch_bounds__(kFitWarps * 32) fit_bcq_kernel(const __half* _
         if (i < Q) return (i == k) ? (float)g : (float)(g - 2 * diff[i * (i - 1) / 2 + k]);
         return (k < Q) ? (float)(2 * plus[k] - g) : (float)g;
       };
-      (void)plus;
       // Cholesky of M (every lane, same arithmetic), then two triangular solves.
       float L[D][D];
       bool ok = true;

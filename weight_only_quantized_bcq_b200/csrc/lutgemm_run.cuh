@@ -495,7 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
     // stage SLOT; `planes` of them (the tile's plane count in mixed storage).
     auto load_alpha = [&]<int SLOT>(int R_, int j, uint32_t planes) {
       if constexpr (PRE_ALPHA) {
-        const int pg_ = j >> 3, U_ = j & 7;
+        [[maybe_unused]] const int pg_ = j >> 3;
+        const int U_ = j & 7;
         const int row = R_ * kTileRows + lane;
         const int P = U_ ^ (int)(4 * a);
 #pragma unroll
@@ -504,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
           if constexpr (MODE == kG128) G = 8 * s + P;
           else if constexpr (MODE == kG128x) G = (8 * s + P) / (p.g >> 7);
           else G = 16 * s + 2 * P + (r ^ (int)(lam >> 3));
-          const bool ok = row < p.m && G < p.ng;
-          const __half* ap = p.alpha + (size_t)G * p.m + row;
+          [[maybe_unused]] const bool ok = row < p.m && G < p.ng;
+          [[maybe_unused]] const __half* ap = p.alpha + (size_t)G * p.m + row;
           if constexpr (!PK) {
 #pragma unroll
             for (int i = 0; i < Q; ++i) {
@@ -732,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_gemm_kernel(const RunParams p
 
             constexpr uint32_t IMM = step_imm<U>();
             constexpr int u2 = U >> 2;
-            const int P = U ^ (int)(4 * a);
+            [[maybe_unused]] const int P = U ^ (int)(4 * a);
 #pragma unroll
             for (int i = 0; i < Q; ++i) {
               if (MULTI && pg * 4 + i >= p.q) continue;
